@@ -1,0 +1,43 @@
+"""Plant plausible mistakes in copies of the oracle source and check that the pin
+suite catches every one of them (CPU only; the real oracle is untouched)."""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "ternmoe_oracle.c")
+
+MUTANTS = {
+    "code_01_is_minus": ("case 1: return 1;", "case 1: return -1;"),
+    "big_endian_in_byte": ("(row[k / 4] >> (2 * (k % 4)))", "(row[k / 4] >> (2 * (3 - k % 4)))"),
+    "dropped_minus_term": ("return plus - minus;", "return plus;"),
+    "ties_to_higher_index": ("l[e] > l[best]", "l[e] >= l[best]"),
+    "gates_not_renormalised": ("gates[t * k + i] = ev[i] / z;", "gates[t * k + i] = ev[i];"),
+    "silu_dropped": ("return g / (1.0 + exp(-g)) * u;", "return g * u;"),
+    "down_scale_dropped": ("tern_dot_f64(drow, hd, f, &bad, &unchecked) * (double)sd",
+                           "tern_dot_f64(drow, hd, f, &bad, &unchecked)"),
+    "rms_sum_not_mean": ("sqrt(ss / (double)d + eps)", "sqrt(ss + eps)"),
+    "quant_truncates": ("float r = rintf(p);", "float r = truncf(p);"),
+    "residual_dropped": ("f64_to_bf16(bf16_to_f64(x[i]) + bf16_to_f64(y[i]))", "y[i]"),
+    "gate_up_swapped": ("h[j] = (float)silu_times(g, u);", "h[j] = (float)silu_times(u, g);"),
+    "int8_scale_order": ("g = g * sg;\n                    g = g * sx;", "g = g * sx;\n                    g = g * sx;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) >= 1, "mutation site vanished: " + name
+    mut = tmp_path / "mut.c"
+    mut.write_text(src.replace(old, new))
+    so = tmp_path / "mut.so"
+    subprocess.check_call(["gcc", "-O2", "-std=gnu11", "-fPIC", "-shared", "-ffp-contract=off",
+                           "-o", str(so), str(mut), "-lm"])
+    env = dict(os.environ, TERNMOE_ORACLE_LIB=str(so))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, "pins did not catch mutant " + name + "\n" + r.stdout[-2000:]
