@@ -1,0 +1,192 @@
+/*
+ * ternmoe.h -- C ABI of libternmoe.so: ternary-weight mixture-of-experts FFN decode on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (from the web pages on the Maple-Preview model):
+ *   - weights are ternary, every weight -1, 0 or +1 ("How a 20B Model Hits 120 tok/s on an
+ *     iPhone", lead and "Why the number is plausible"), packed four 2-bit codes per byte
+ *     and used without unpacking ("A 20B AI Model Trained in Ternary Just Hit 218
+ *     Tokens/Second on a $599 Mac Mini", "What Ternary Actually Means" and "The
+ *     Architecture: Designed for the Hardware"), so a dot product is adds and subtracts of
+ *     activations followed by one per-row scale;
+ *   - batch-1 decode is a sequence of matrix-vector products bound by memory bandwidth
+ *     (same page, "What Ternary Actually Means");
+ *   - a learned router picks 8 of 256 experts per token ("iPhone Runs a 20B Model at 120
+ *     tok/s", "MoE Is the Other Half of the Story Behind the 20B Figure"; "A 20B AI Model...",
+ *     "The Architecture: Designed for the Hardware"), 24 layers deep.
+ *
+ * Packed format (the pages leave the encoding undisclosed -- "iPhone Runs a 20B Model...",
+ * "What a Credible Reproduction Report Should Disclose"; this library fixes it):
+ *   code 00 -> 0, 01 -> +1, 10 -> -1 (11 is never written and reads as 0);
+ *   weight k of row m is in bits 2(k%4)..2(k%4)+1 of byte m*(K/4) + k/4;
+ *   one fp32 scale per output row.
+ *
+ * Conventions for every call below
+ *   - All array pointers are DEVICE pointers owned by the caller; the library never frees
+ *     them.  bf16 values travel as uint16_t bit patterns.  Row-major layouts.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Calls
+ *     enqueue work and return without waiting, except tern_pack / tern_unpack (they wait
+ *     for their own kernel to report invalid codes) and tern_stream_status.
+ *   - Arguments are checked on the host before anything is enqueued; a failed check returns
+ *     TERN_EINVAL / TERN_EALIGN / TERN_EWORKSPACE and enqueues nothing.  A CUDA launch
+ *     error returns TERN_ECUDA.  No C++ exception crosses the ABI.
+ *   - K (the reduction length of a ternary matrix) must be a multiple of 64 so packed rows
+ *     are whole 16-byte vectors; K <= 2048, or a multiple of 2048 up to 16384.  Packed
+ *     arrays and activations must be 16-byte aligned, scales 4-byte aligned.
+ *   - The library allocates no device memory on these paths: scratch space is the
+ *     caller's `workspace`.  A workspace must be zero-filled once before its first use
+ *     (cudaMemset); every successful call leaves its control words zero again.  Calls that
+ *     share a workspace must not overlap on the GPU.
+ */
+#ifndef TERNMOE_H
+#define TERNMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TERNMOE_ABI_VERSION 1
+
+typedef enum {
+    TERN_OK = 0,
+    TERN_EINVAL = 1,      /* bad shape, null pointer, k > E, unsupported size */
+    TERN_EALIGN = 2,      /* pointer not aligned as required */
+    TERN_ECODE = 3,       /* pack: weight outside {-1,0,1}; unpack: code 11 present */
+    TERN_ECUDA = 4,       /* a CUDA runtime call or launch failed */
+    TERN_ETIMEOUT = 5,    /* a bounded in-kernel wait gave up (device status word) */
+    TERN_EWORKSPACE = 6,  /* workspace null or smaller than the query says */
+    TERN_EUNSUPPORTED = 7 /* valid request this build does not implement */
+} tern_status;
+
+typedef enum {
+    TERN_ACT_BF16 = 0, /* bf16 activations; exact integer dot on a 24-bit fixed-point grid */
+    TERN_ACT_INT8 = 1  /* int8 activations (per-vector absmax quantisation), int32 accumulate */
+} tern_act;
+
+/* One MoE FFN layer (device pointers). E experts, each a SwiGLU expert with ternary gate and
+ * up matrices [f][d] and a ternary down matrix [d][f]; router W_g [E][d] in bf16.
+ * The pages do not describe the expert body; this library takes the SwiGLU reading. */
+typedef struct {
+    const uint8_t *gate;       /* [E][f][d/4] packed */
+    const uint8_t *up;         /* [E][f][d/4] packed */
+    const uint8_t *down;       /* [E][d][f/4] packed */
+    const float *gate_scale;   /* [E][f] */
+    const float *up_scale;     /* [E][f] */
+    const float *down_scale;   /* [E][d] */
+    const uint16_t *router;    /* [E][d] bf16 */
+    int64_t d, f;              /* hidden and expert width; multiples of 64 */
+    int32_t E, k;              /* experts, experts per token: 1 <= k <= 8, k <= E <= 1024 */
+} tern_moe_layer;
+
+/* Byte offsets, inside the workspace of moe_ffn_decode, of the intermediates the last call
+ * left there (for inspection and parity checks; -1 = not produced on this path). */
+typedef struct {
+    int64_t logits;   /* double [T][E] router logits */
+    int64_t idx;      /* int32 [T][k] selected experts, descending logit, ties -> lower index */
+    int64_t gates64;  /* double [T][k] renormalised gates */
+    int64_t gates32;  /* float [T][k] the same rounded to fp32 */
+    int64_t h;        /* float [T][k][f] SwiGLU output of each (token, slot) */
+    int64_t qx;       /* int8 [T][d] quantised layer input (int8 path) */
+    int64_t sx;       /* float [T] its scale (int8 path) */
+    int64_t qh;       /* int8 [T][k][f] quantised h (int8 path) */
+    int64_t sh;       /* float [T][k] its scale (int8 path) */
+    int64_t acc_g;    /* int32 [T][k][f] gate accumulators (int8 path) */
+    int64_t acc_u;    /* int32 [T][k][f] up accumulators (int8 path) */
+    int64_t acc_d;    /* int32 [T][k][d] down accumulators (int8 path) */
+    int64_t ye;       /* double [T][k][d] expert outputs before the gate */
+    int64_t n_unique; /* int32: number of distinct experts selected by the step */
+    int64_t total;    /* bytes needed */
+} tern_ffn_layout;
+
+/* Human-readable name of a status code (static string). */
+const char *tern_status_str(tern_status s);
+
+/* TERNMOE_ABI_VERSION of the loaded library. */
+int32_t tern_abi_version(void);
+
+/* Pack int8 weights w [M][K] (values -1, 0, +1) into packed [M][K/4].
+ * Waits for its kernel; returns TERN_ECODE if any weight is outside {-1,0,1} (that weight
+ * is written as code 00).  K % 4 == 0. */
+tern_status tern_pack(const int8_t *w, int64_t M, int64_t K, uint8_t *packed, void *stream);
+
+/* Unpack packed [M][K/4] into int8 w [M][K].  Waits; returns TERN_ECODE if a code 11 was
+ * found (written as 0).  K % 4 == 0. */
+tern_status tern_unpack(const uint8_t *packed, int64_t M, int64_t K, int8_t *w, void *stream);
+
+/* Ternary GEMV for T tokens:  S[t,m] = sum_k w[m,k] x[t,k]  (adds/subtracts only), then
+ *   act = TERN_ACT_INT8: x is int8 [T][K]; acc[t,m] = S (int32, exact; acc may be NULL);
+ *        y[t,m] = ((float)S * row_scale[m]) * x_scale[t]   (x_scale may be NULL: no factor);
+ *   act = TERN_ACT_BF16: x is bf16 [T][K]; y[t,m] = row_scale[m] * S, where S is summed
+ *        exactly on a 24-bit fixed-point grid per token (every bf16 within 2^15 of the
+ *        token's absmax is exact; smaller ones round to the grid), scaled in fp64 and
+ *        rounded to fp32; acc must be NULL.
+ * Wp [M][K/4], row_scale [M], y [T][M].  1 <= T <= 64. */
+tern_status tern_gemv(const uint8_t *Wp, const float *row_scale, int64_t M, int64_t K, tern_act act,
+                      const void *x, const float *x_scale, int64_t T, int32_t *acc, float *y,
+                      void *stream);
+
+/* Per-vector absmax int8 quantisation of bf16 rows x [T][n]:  s[t] = absmax/127,
+ * q = clamp(rint(x * (127/absmax)), -127, 127) in fp32, ties to even; a zero row gives
+ * q = 0, s = 0.  (The pages are silent on activation precision; this is the int8 reading.) */
+tern_status tern_quant_absmax(const uint16_t *x, int64_t T, int64_t n, int8_t *q, float *s,
+                              void *stream);
+
+/* Router: logits[t,e] = sum_k Wg[e,k] x[t,k] accumulated in fp64 (every bf16 x bf16 product
+ * is exact); top-k by logit descending, ties to the lower expert index; gates renormalised
+ * over the selected experts, g_i = exp(l_i - l_max) / sum_j exp(l_j - l_max), in fp64 and
+ * written as fp32.  Wg [E][d] bf16, x [T][d] bf16, topk_idx [T][k], topk_gate [T][k],
+ * logits [T][E] (may be NULL).  1 <= T <= 64, 1 <= k <= 8, k <= E <= 1024, d % 8 == 0. */
+size_t moe_route_workspace_bytes(int64_t T, int32_t E);
+tern_status moe_route_topk(const uint16_t *Wg, const uint16_t *x, int64_t T, int64_t d, int32_t E,
+                           int32_t k, int32_t *topk_idx, float *topk_gate, double *logits,
+                           void *workspace, size_t ws_bytes, void *stream);
+
+/* One MoE FFN layer for T tokens (decode):
+ *   route (as moe_route_topk) -> group the (token, slot) pairs by expert so every selected
+ *   expert's packed weights stream from memory once per call -> for each pair
+ *   h = silu(s_g * (G x)) * (s_u * (U x)) -> y_e = s_d * (D h) -> y[t] = sum over the k
+ *   slots in top-k order of gate * y_e, in fp64, written as bf16 (nearest even) and, if
+ *   y_f32 != NULL, as fp32.
+ *   act = TERN_ACT_BF16: x and h enter the dots on a 24-bit fixed-point grid (see tern_gemv).
+ *   act = TERN_ACT_INT8: x is absmax-quantised per token and h per (token, slot); the dots
+ *     are exact int32; g = ((float)acc_g * s_g) * s_x, u likewise, h = fp32 of the fp64
+ *     SwiGLU, y_e = ((float)acc_d * s_d) * s_h.
+ * x [T][d] bf16, y [T][d] bf16, y_f32 [T][d] or NULL.  1 <= T <= T_max <= 64. */
+size_t moe_ffn_workspace_bytes(const tern_moe_layer *L, int64_t T_max, tern_act act);
+tern_status moe_ffn_workspace_layout(const tern_moe_layer *L, int64_t T_max, tern_act act,
+                                     tern_ffn_layout *out);
+tern_status moe_ffn_decode(const tern_moe_layer *L, const uint16_t *x, int64_t T, tern_act act,
+                           uint16_t *y, float *y_f32, void *workspace, size_t ws_bytes,
+                           void *stream);
+
+/* A stack of n_layers residual MoE FFN layers, applied in place to x [T][d] (bf16):
+ *   n = bf16(x / sqrt(mean(x^2) + rms_eps))   (fp64, no learned gain)
+ *   x = bf16(x + moe_ffn_decode(n))            (exact sum, one rounding)
+ * All layers must share d, f, E, k.  1 <= n_layers <= 64.  For T == 1 the whole stack runs
+ * as ONE persistent kernel (one CTA per SM, in-kernel grid barriers with bounded waits);
+ * otherwise layer by layer.  A timed-out in-kernel wait sets the device status word to
+ * TERN_ETIMEOUT (read it with tern_stream_status) and the workspace must be zero-filled
+ * again before reuse. */
+size_t moe_stack_workspace_bytes(const tern_moe_layer *L0, int64_t T_max, tern_act act);
+tern_status moe_stack_decode(const tern_moe_layer *layers, int32_t n_layers, uint16_t *x, int64_t T,
+                             float rms_eps, tern_act act, void *workspace, size_t ws_bytes,
+                             void *stream);
+
+/* Waits for `stream`, then returns and clears the device status word of the current device
+ * (TERN_OK, or TERN_ETIMEOUT if an in-kernel bounded wait gave up since the last read), or
+ * TERN_ECUDA if the wait itself failed. */
+tern_status tern_stream_status(void *stream);
+
+/* Test hook for the bounded waits: launches one block that waits on a flag nobody sets,
+ * for at most `spin_limit` polls, then sets TERN_ETIMEOUT in the device status word and
+ * returns.  `flag` is a device int the caller owns (must stay 0). */
+tern_status tern_test_bounded_wait(int32_t *flag, int64_t spin_limit, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TERNMOE_H */

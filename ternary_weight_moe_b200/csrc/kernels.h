@@ -1,0 +1,71 @@
+// kernels.h -- host-side launchers of the sm_100a kernels (internal to libternmoe).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/ternmoe.h"
+
+namespace tern {
+
+// ---- format
+cudaError_t launch_pack(const int8_t *w, int64_t M, int64_t K, uint8_t *packed, unsigned long long *bad,
+                        cudaStream_t s);
+cudaError_t launch_unpack(const uint8_t *p, int64_t M, int64_t K, int8_t *w, unsigned long long *bad,
+                          cudaStream_t s);
+cudaError_t launch_quant_absmax(const uint16_t *x, int64_t T, int64_t n, int8_t *q, float *sc,
+                                cudaStream_t s);
+
+// ---- ternary GEMV
+cudaError_t launch_gemv(const uint8_t *Wp, const float *rs, int64_t M, int64_t K, tern_act act,
+                        const void *x, const float *xs, int64_t T, int32_t *acc, float *y, cudaStream_t s);
+
+// ---- MoE layer, general T (kernel-per-stage path)
+struct FfnWs {           // device pointers carved from the caller's workspace
+    unsigned int *ctrl;  // [0] route arrival counter
+    double *logits;      // [T][E]
+    int32_t *idx;        // [T][k]
+    double *g64;         // [T][k]
+    float *g32;          // [T][k]
+    int32_t *n_unique;   // [1]
+    int32_t *uexp;       // [E]
+    int32_t *uoff;       // [E+1]
+    int32_t *ent;        // [T*k]
+    uint32_t *xw;        // [T][NL][d/4] activation limb words
+    float *xsc;          // [T] int8 scale, or shift (as int bits) on the bf16 path
+    float *h;            // [T*k][f]
+    uint32_t *hw;        // [T*k][NL][f/4]
+    float *hsc;          // [T*k]
+    int32_t *acc_g, *acc_u, *acc_d;  // int8 path traces
+    double *ye;          // [T*k][d]
+};
+
+cudaError_t launch_route(const uint16_t *Wg, const uint16_t *x, int T, int d, int E, int k, double *logits,
+                         int32_t *idx, float *g32, double *g64, unsigned int *counter, bool dispatch,
+                         int32_t *n_unique, int32_t *uexp, int32_t *uoff, int32_t *ent, cudaStream_t s);
+
+cudaError_t launch_ffn_stages(const tern_moe_layer *L, const uint16_t *x, int T, tern_act act, const FfnWs &w,
+                              uint16_t *y, float *y_f32, const uint16_t *residual, uint16_t *x_out,
+                              cudaStream_t s);
+
+cudaError_t launch_rmsnorm(const uint16_t *x, int T, int d, double eps, uint16_t *n, cudaStream_t s);
+
+// ---- persistent whole-stack decode, T == 1
+struct StackLayerDev {
+    const uint8_t *gate, *up, *down;
+    const float *sg, *su, *sd;
+    const uint16_t *router;
+};
+size_t stack_persistent_ws_bytes(const tern_moe_layer *L0);
+void stack_persistent_offsets(const tern_moe_layer *L0, int64_t *hist, int64_t *idx_hist, int64_t *gate_hist);
+tern_status launch_stack_persistent(const tern_moe_layer *layers, int n_layers, uint16_t *x, float eps,
+                                    tern_act act, void *ws, size_t ws_bytes, int *status, cudaStream_t s);
+
+// ---- bounded-wait test hook
+cudaError_t launch_test_wait(int32_t *flag, long long limit, int *status, cudaStream_t s);
+
+// address of the device status word on the current device
+int *status_word();
+
+}  // namespace tern

@@ -1,0 +1,364 @@
+// tern_common.cuh -- device helpers shared by the sm_100a kernels of libternmoe.
+//
+// Ternary decode without unpacking: a packed byte holds four 2-bit codes (00 -> 0,
+// 01 -> +1, 10 -> -1, little-endian along K).  Each byte is turned into four signed int8
+// lanes by ONE shared-memory table read (a 256-entry table replicated per lane so every
+// lane reads its own bank), and the four products with activations happen in ONE dp4a.
+// This is the integer-unit form of "negate, zero, or pass through" ("A 20B AI Model Trained
+// in Ternary Just Hit 218 Tokens/Second on a $599 Mac Mini", "What Ternary Actually
+// Means"): the weights are never widened to bf16 and no floating-point multiply is issued
+// per weight.
+//
+// Activations enter as integer "limbs":
+//   int8 path: one signed limb (the quantised value);
+//   bf16/fp32 path: a 24-bit fixed-point value x_int = rint(x * 2^s) with s chosen per
+//     vector so that |x_int| < 2^23, split into hi (signed 8 bit), mid and lo (unsigned
+//     8 bit): x_int = hi*65536 + mid*256 + lo.  The dot is then exact in integers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/ternmoe.h"
+
+namespace tern {
+
+constexpr int kWarp = 32;
+
+// ------------------------------------------------------------------ device status word
+// A per-device int owned by the library (first error wins; read and cleared by
+// tern_stream_status()); kernels receive its address.
+__device__ __forceinline__ void set_status(int *st, int code) {
+    if (st) atomicCAS(st, 0, code);
+}
+
+// ---------------------------------------------------------------------------- bf16 / fp64
+__device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+
+// nearest bf16 (ties to even) of a finite double, directly from the fp64 bits
+__device__ __forceinline__ uint16_t f64_to_bf16_rne(double v) {
+    unsigned long long u = (unsigned long long)__double_as_longlong(v);
+    const uint32_t sign = (uint32_t)(u >> 63) << 15;
+    u &= 0x7FFFFFFFFFFFFFFFull;
+    if (u == 0) return (uint16_t)sign;
+    int e = (int)(u >> 52) - 1023;            // unbiased exponent (inputs are normal fp64)
+    unsigned long long m = (u & 0xFFFFFFFFFFFFFull) | (1ull << 52);  // 53-bit significand
+    int keep;                                  // significand bits kept in bf16 at this exponent
+    if (e >= -126) keep = 8;
+    else keep = 8 - (-126 - e);                // bf16 subnormal range
+    if (keep <= 0) {
+        // below half the smallest subnormal (or exactly half: ties to even -> 0)
+        if (keep == 0 && m > (1ull << 52)) return (uint16_t)(sign | 1);
+        return (uint16_t)sign;
+    }
+    const int drop = 53 - keep;
+    unsigned long long q = m >> drop;
+    const unsigned long long rem = m & ((1ull << drop) - 1);
+    const unsigned long long half = 1ull << (drop - 1);
+    if (rem > half || (rem == half && (q & 1))) q++;
+    // q has `keep` (or keep+1 after carry) significant bits; rebuild the bf16 value
+    if (e >= -126) {
+        if (q == (1ull << 8)) { q >>= 1; e++; }
+        if (e > 127) return (uint16_t)(sign | 0x7F80u);
+        return (uint16_t)(sign | ((uint32_t)(e + 127) << 7) | (uint32_t)(q & 0x7F));
+    }
+    // subnormal: value = q * 2^-133 ; if q reached 2^7 it becomes the smallest normal
+    return (uint16_t)(sign | (uint32_t)q);
+}
+
+// ---------------------------------------------------------------------------- dp4a
+__device__ __forceinline__ int dp4a_ss(uint32_t a, uint32_t b, int c) {
+    return __dp4a((int)a, (int)b, c);
+}
+// a: signed int8x4 (ternary weights), b: unsigned 8-bit limbs
+__device__ __forceinline__ int dp4a_su(uint32_t a, uint32_t b, int c) {
+    int d;
+    asm("dp4a.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// -------------------------------------------------------------------- decode table
+// lut[b * 32 + lane] = the four weights of byte b as signed int8 lanes (byte j = code j).
+constexpr int kLutWords = 256 * kWarp;
+constexpr int kLutBytes = kLutWords * 4;
+
+__device__ __forceinline__ uint32_t decode_byte(uint32_t b) {
+    uint32_t out = 0;
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        const uint32_t c = (b >> (2 * j)) & 3u;
+        const uint32_t v = (c == 1u) ? 0x01u : (c == 2u) ? 0xFFu : 0x00u;
+        out |= v << (8 * j);
+    }
+    return out;
+}
+
+__device__ __forceinline__ void lut_fill(uint32_t *lut) {
+    for (int i = threadIdx.x; i < kLutWords; i += blockDim.x) lut[i] = decode_byte((uint32_t)i >> 5);
+}
+
+// ------------------------------------------------------------------- segment dot
+// A "segment" is 64 consecutive codes = 16 packed bytes (one uint4).  xw[l][b] holds limb l
+// of the four activations that meet byte b of the segment.
+template <int NL>
+struct SegX {
+    uint32_t w[NL][16];
+};
+
+template <int NL>
+__device__ __forceinline__ void seg_dot(const uint4 wb, const SegX<NL> &x, const uint32_t *lut_lane,
+                                        int (&acc)[NL]) {
+    const uint32_t words[4] = {wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+    for (int q = 0; q < 4; q++) {
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const uint32_t byte = (words[q] >> (8 * i)) & 0xFFu;
+            const uint32_t wv = lut_lane[byte << 5];
+            const int b = 4 * q + i;
+            if (NL == 1) {
+                acc[0] = dp4a_ss(wv, x.w[0][b], acc[0]);
+            } else {
+                acc[0] = dp4a_ss(wv, x.w[0][b], acc[0]);   // hi limb: signed
+                acc[1] = dp4a_su(wv, x.w[1][b], acc[1]);   // mid limb: unsigned
+                acc[2] = dp4a_su(wv, x.w[2][b], acc[2]);   // lo limb: unsigned
+            }
+        }
+    }
+}
+
+// load the limbs of one segment from a limb-word array laid out [NL][n/4] (u32 words)
+template <int NL>
+__device__ __forceinline__ void seg_load_x(SegX<NL> &x, const uint32_t *limbw, int64_t words_per_limb,
+                                           int64_t seg) {
+#pragma unroll
+    for (int l = 0; l < NL; l++) {
+        const uint4 *p = reinterpret_cast<const uint4 *>(limbw + (int64_t)l * words_per_limb + seg * 16);
+#pragma unroll
+        for (int v = 0; v < 4; v++) {
+            const uint4 t = __ldg(p + v);
+            x.w[l][4 * v + 0] = t.x;
+            x.w[l][4 * v + 1] = t.y;
+            x.w[l][4 * v + 2] = t.z;
+            x.w[l][4 * v + 3] = t.w;
+        }
+    }
+}
+
+// same, from shared memory
+template <int NL>
+__device__ __forceinline__ void seg_load_x_smem(SegX<NL> &x, const uint32_t *limbw, int words_per_limb, int seg) {
+#pragma unroll
+    for (int l = 0; l < NL; l++) {
+        const uint4 *p = reinterpret_cast<const uint4 *>(limbw + l * words_per_limb + seg * 16);
+#pragma unroll
+        for (int v = 0; v < 4; v++) {
+            const uint4 t = p[v];
+            x.w[l][4 * v + 0] = t.x;
+            x.w[l][4 * v + 1] = t.y;
+            x.w[l][4 * v + 2] = t.z;
+            x.w[l][4 * v + 3] = t.w;
+        }
+    }
+}
+
+// Per-lane partial sums -> at most two int32 for the cross-lane reduction.
+// NL == 3: hi stays separate, (mid*256 + lo) is combined; both fit int32 for <= 256 codes
+// per lane and 32 lanes.
+template <int NL>
+__device__ __forceinline__ void acc_to_pair(const int (&acc)[NL], int &a, int &b) {
+    if (NL == 1) {
+        a = acc[0];
+        b = 0;
+    } else {
+        a = acc[0];
+        b = acc[1] * 256 + acc[2];
+    }
+}
+
+__device__ __forceinline__ long long pair_value(int NLv, int a, int b) {
+    return NLv == 1 ? (long long)a : (long long)a * 65536ll + (long long)b;
+}
+
+// xor-reduce within aligned groups of G lanes
+template <int G>
+__device__ __forceinline__ int group_sum(int v) {
+#pragma unroll
+    for (int o = G / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ double warp_sum_f64(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ float warp_max_f32(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+    return v;
+}
+
+// block-wide max of non-negative floats (all threads get the result); red >= 32 floats
+__device__ __forceinline__ float block_max_f32(float v, float *red) {
+    v = warp_max_f32(v);
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    __syncthreads();
+    if (l == 0) red[w] = v;
+    __syncthreads();
+    const int nw = (blockDim.x + 31) >> 5;
+    float r = (l < nw) ? red[l] : 0.0f;
+    r = warp_max_f32(r);
+    return r;
+}
+
+// ------------------------------------------------------- fixed-point activation limbs
+// Shift s such that |x| * 2^s < 2^23 for every element (s = 22 - floor(log2(absmax))).
+__device__ __forceinline__ int fixed_shift(float absmax) {
+    if (!(absmax > 0.0f)) return 0;
+    return 22 - ilogbf(absmax);
+}
+
+// x_int = rint(x * 2^s) split into three bytes: hi (signed), mid, lo (unsigned)
+__device__ __forceinline__ void fixed_limbs(float x, int s, uint32_t &hi, uint32_t &mid, uint32_t &lo) {
+    const int xi = __float2int_rn(scalbnf(x, s));
+    hi = (uint32_t)(xi >> 16) & 0xFFu;
+    mid = (uint32_t)(xi >> 8) & 0xFFu;
+    lo = (uint32_t)xi & 0xFFu;
+}
+
+// ---------------------------------------------------------------------------- top-k
+// One warp selects the top k of E fp64 logits: descending value, ties to the lower index.
+// Lane l owns experts l, l+32, ...; selected entries are set to -inf (logits are finite).
+template <int J>
+__device__ __forceinline__ void warp_topk(const double *lg, int E, int k, int32_t *idx_out, double *g64, float *g32) {
+    const int lane = threadIdx.x & 31;
+    double v[J];
+#pragma unroll
+    for (int j = 0; j < J; j++) {
+        const int e = lane + 32 * j;
+        v[j] = (e < E) ? lg[e] : -INFINITY;
+    }
+    double selv[8];
+    int seli[8];
+    for (int r = 0; r < k; r++) {
+        double bv = -INFINITY;
+        int bi = 0x7FFFFFFF;
+#pragma unroll
+        for (int j = 0; j < J; j++) {
+            const int e = lane + 32 * j;
+            if (e < E && (v[j] > bv || (v[j] == bv && e < bi))) {
+                bv = v[j];
+                bi = e;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const double ov = __shfl_xor_sync(0xFFFFFFFFu, bv, o);
+            const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
+            if (ov > bv || (ov == bv && oi < bi)) {
+                bv = ov;
+                bi = oi;
+            }
+        }
+        selv[r] = bv;
+        seli[r] = bi;
+        if ((bi & 31) == lane) {
+#pragma unroll
+            for (int j = 0; j < J; j++)
+                if (j == (bi >> 5)) v[j] = -INFINITY;
+        }
+    }
+    if (lane == 0) {
+        const double l0 = selv[0];
+        double ev[8];
+        double z = 0.0;
+        for (int r = 0; r < k; r++) {
+            ev[r] = exp(selv[r] - l0);
+            z += ev[r];
+        }
+        for (int r = 0; r < k; r++) {
+            idx_out[r] = seli[r];
+            const double g = ev[r] / z;
+            if (g64) g64[r] = g;
+            if (g32) g32[r] = (float)g;
+        }
+    }
+}
+
+// ----------------------------------------------------------- absmax int8 quantisation
+// q = clamp(rint(x * (127/absmax)), -127, 127) in fp32, ties to even; s = absmax/127
+__device__ __forceinline__ float quant_inv(float absmax) { return __fdiv_rn(127.0f, absmax); }
+__device__ __forceinline__ int quant_one(float x, float inv) {
+    int q = __float2int_rn(__fmul_rn(x, inv));
+    return q > 127 ? 127 : (q < -127 ? -127 : q);
+}
+
+// ----------------------------------------------------------------- SwiGLU epilogue
+__device__ __forceinline__ float swiglu_f32(double g, double u) {
+    return (float)(g / (1.0 + exp(-g)) * u);
+}
+
+// --------------------------------------------------------- bounded grid-wide barrier
+// Monotonic arrival counter: barrier number n waits until the counter reaches n * nblocks.
+// The counter is reset to zero by the last block to leave the kernel (see grid_exit), so it
+// is zero at every launch.  Waits give up after `limit` polls: the status word is set to
+// TERN_ETIMEOUT and false is returned; the caller then leaves the kernel.
+struct GridSync {
+    unsigned int *arrive;   // monotonic arrivals
+    unsigned int *leave;    // blocks that finished
+    int *status;            // device status word
+    unsigned int nblocks;
+    unsigned int epoch;     // barriers passed by this block
+    long long limit;
+};
+
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int *p) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void red_release_gpu_add(unsigned int *p, unsigned int v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// returns false on timeout (all threads of the block get the same answer)
+__device__ __forceinline__ bool grid_sync(GridSync &gs, int *flag_smem) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        gs.epoch++;
+        const unsigned int target = gs.epoch * gs.nblocks;
+        red_release_gpu_add(gs.arrive, 1u);
+        long long n = 0;
+        int ok = 1;
+        while ((int)(ld_acquire_gpu(gs.arrive) - target) < 0) {
+            if (++n > gs.limit) {
+                ok = 0;
+                set_status(gs.status, TERN_ETIMEOUT);
+                break;
+            }
+        }
+        *flag_smem = ok;
+    }
+    __syncthreads();
+    const bool ok = *flag_smem != 0;
+    __syncthreads();
+    if (threadIdx.x != 0) gs.epoch++;
+    return ok;
+}
+
+// last block out resets both counters so the next launch starts from zero
+__device__ __forceinline__ void grid_exit(GridSync &gs) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const unsigned int n = atomicAdd(gs.leave, 1u);
+        if (n == gs.nblocks - 1) {
+            atomicExch(gs.arrive, 0u);
+            atomicExch(gs.leave, 0u);
+        }
+    }
+}
+
+}  // namespace tern

@@ -1,0 +1,83 @@
+"""The C-ABI library: it loads without a GPU, exports every function the header declares,
+and rejects bad arguments on the host before touching CUDA."""
+import ctypes
+
+import pytest
+
+import ternary_weight_moe_b200 as tm
+
+
+def test_library_exports_every_header_function():
+    names = tm.header_functions()
+    assert len(names) >= 15
+    L = tm.lib()
+    for n in names:
+        assert hasattr(L, n), n
+    assert tm.abi_version() == 1
+
+
+def test_status_strings():
+    assert tm.status_str(0) == "TERN_OK"
+    for c in range(1, 8):
+        assert tm.status_str(c).startswith(tm.STATUS[c])
+
+
+def _fake_layer(d=2048, f=512, E=256, k=8, misalign=0):
+    base = 1 << 40
+    return tm.MoELayerC(base + misalign, base + 4096, base + 8192, base + 12288, base + 16384, base + 20480,
+                        base + 24576, d, f, E, k)
+
+
+def test_workspace_queries_are_host_only():
+    L = _fake_layer()
+    n1 = tm.lib().moe_ffn_workspace_bytes(ctypes.byref(L), 1, tm.TERN_ACT_BF16)
+    n64 = tm.lib().moe_ffn_workspace_bytes(ctypes.byref(L), 64, tm.TERN_ACT_BF16)
+    assert 0 < n1 < n64
+    assert tm.lib().moe_ffn_workspace_bytes(ctypes.byref(L), 65, tm.TERN_ACT_BF16) == 0
+    assert tm.lib().moe_stack_workspace_bytes(ctypes.byref(L), 1, tm.TERN_ACT_INT8) > 0
+    out = tm.FfnLayoutC()
+    assert tm.lib().moe_ffn_workspace_layout(ctypes.byref(L), 4, tm.TERN_ACT_INT8, ctypes.byref(out)) == 0
+    assert out.total == tm.lib().moe_ffn_workspace_bytes(ctypes.byref(L), 4, tm.TERN_ACT_INT8)
+    assert out.acc_g >= 0 and out.qx >= 0
+    assert tm.lib().moe_ffn_workspace_layout(ctypes.byref(L), 4, tm.TERN_ACT_BF16, ctypes.byref(out)) == 0
+    assert out.acc_g == -1 and out.qx == -1
+    assert tm.lib().moe_route_workspace_bytes(1, 256) > 256 * 8
+
+
+@pytest.mark.parametrize("bad", [dict(d=100), dict(f=0), dict(E=0), dict(k=9), dict(k=300, E=256), dict(E=2000),
+                                 dict(d=4096)])
+def test_layer_validation(bad):
+    L = _fake_layer(**bad)
+    assert tm.lib().moe_ffn_workspace_bytes(ctypes.byref(L), 1, tm.TERN_ACT_BF16) == 0
+
+
+def test_argument_checks_before_any_launch():
+    L = tm.lib()
+    p = ctypes.c_void_p(1 << 40)
+    # K not a multiple of 64
+    assert L.tern_gemv(p, p, 16, 100, 0, p, None, 1, None, p, None) == 1
+    # T out of range
+    assert L.tern_gemv(p, p, 16, 512, 0, p, None, 0, None, p, None) == 1
+    assert L.tern_gemv(p, p, 16, 512, 0, p, None, 65, None, p, None) == 1
+    # bf16 path takes no accumulator output
+    assert L.tern_gemv(p, p, 16, 512, 0, p, None, 1, p, p, None) == 1
+    # misaligned packed weights
+    q = ctypes.c_void_p((1 << 40) + 4)
+    assert L.tern_gemv(q, p, 16, 512, 1, p, None, 1, None, p, None) == 2
+    # K = 3072 is neither <= 2048 nor a multiple of 2048
+    assert L.tern_gemv(p, p, 16, 3072, 1, p, None, 1, None, p, None) == 1
+    # null workspace
+    Lc = _fake_layer()
+    assert L.moe_ffn_decode(ctypes.byref(Lc), p, 1, 0, p, None, None, 0, None) == 6
+    # misaligned expert weights
+    Lm = _fake_layer(misalign=8)
+    assert L.moe_ffn_decode(ctypes.byref(Lm), p, 1, 0, p, None, p, 1 << 30, None) == 2
+    # route: k > E
+    assert L.moe_route_topk(p, p, 1, 2048, 4, 8, p, p, None, p, 1 << 20, None) == 1
+    # pack: K not a multiple of 4
+    assert L.tern_pack(p, 4, 6, p, None) == 1
+    # stack: too many layers / negative eps
+    arr = (tm.MoELayerC * 1)(Lc)
+    assert L.moe_stack_decode(arr, 0, p, 1, 1e-6, 0, p, 1 << 30, None) == 1
+    assert L.moe_stack_decode(arr, 1, p, 1, -1.0, 0, p, 1 << 30, None) == 1
+    assert L.tern_test_bounded_wait(None, 10, None) == 1
