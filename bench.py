@@ -1,0 +1,418 @@
+"""Benchmark: ternary MoE FFN decode, batch 1, through a 24-layer stack on B200.
+
+Workload: 24 residual MoE FFN layers (d=2048, 256 SwiGLU experts of 512x2048 / 2048x512,
+ternary weights packed 2 bits per code, per-row fp32 scales, bf16 router, top-8), about
+4.93 GB resident in HBM; each step decodes ONE token through all 24 layers with
+x <- x + FFN(RMSNorm(x)) in bf16.  Synthetic seeded data (no trained weights exist here).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--act bf16|int8] [--impl reference]
+
+Timing: W warm-up steps, then K timed steps.  The L2 cache (126 MB) is flushed before every
+timed step by writing a 256 MB buffer; each step is bracketed by CUDA events on the stream
+the library launches on, and the device time of a step excludes the flush.  `value` is
+tokens/s over all ranks (one independent replica per GPU, no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ternary MoE FFN decode tokens/s @batch1; achieved HBM GB/s vs B200 peak"
+UNIT = "tokens/s"
+N_LAYERS = 24
+WID = 5
+BYTES_PER_LAYER_TOKEN = 8 * (786432 + 12288) + 1048576   # experts' packed codes + scales, router
+BYTES_PER_TOKEN = N_LAYERS * BYTES_PER_LAYER_TOKEN       # 178,520,064 B
+WORKLOAD = ("24-layer ternary MoE FFN stack, batch-1 decode: d=2048, E=256 SwiGLU experts "
+            "512x2048/2048x512, top-8, 2-bit packed ternary weights, bf16 router")
+
+
+def _config(act_name, world, l2):
+    return {"workload": WORKLOAD, "layers": N_LAYERS, "batch": 1, "d": 2048, "f": 512, "experts": 256,
+            "top_k": 8, "activations": act_name, "resident_bytes": 4932501504,
+            "weight_bytes_per_token": BYTES_PER_TOKEN, "parallelism": f"replicas{world}", "l2": l2}
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            p = json.load(fh)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ rank plumbing
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def aggregate(values, op, world, backend_device=None):
+    """max/sum of a per-rank float over all ranks (identity when world == 1)."""
+    if world == 1:
+        return float(values)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(values)], dtype=torch.float64, device=backend_device or "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i in range(4) if r[i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ model
+
+def device_layer(layer, shape, dev):
+    """One synthetic layer generated on the device and packed by the library's packer."""
+    import torch
+
+    import synth
+    import ternary_weight_moe_b200 as tm
+
+    E, d, f = shape.E, shape.d, shape.f
+    gc, uc, dc = synth.layer_codes_torch(WID, layer, shape, dev)
+    gate = tm.tern_pack(gc.view(E * f, d)).view(E, f, d // 4)
+    up = tm.tern_pack(uc.view(E * f, d)).view(E, f, d // 4)
+    down = tm.tern_pack(dc.view(E * d, f)).view(E, d, f // 4)
+    del gc, uc, dc
+    sg, su, sd = synth.layer_scales(WID, layer, shape)
+    router = synth.layer_router(WID, layer, shape)
+    return tm.MoELayer(gate, up, down, torch.from_numpy(sg).to(dev), torch.from_numpy(su).to(dev),
+                       torch.from_numpy(sd).to(dev), torch.from_numpy(router.view(np.int16)).to(dev), k=shape.k)
+
+
+def build_stack(dev):
+    import synth
+    import ternary_weight_moe_b200 as tm
+
+    shape = synth.MoEShape()
+    layers = [device_layer(l, shape, dev) for l in range(N_LAYERS)]
+    return shape, layers, tm.Stack(layers)
+
+
+def cpu_baseline(act_oracle, budget_s=12.0, max_tokens=4):
+    """The oracle (single-threaded C, fp64/exact) decoding whole tokens through the same
+    24-layer stack; experts are regenerated on the host outside the timed region."""
+    import oracle
+    import synth
+    from tests.gpu_cases import HostLayer
+
+    shape = synth.MoEShape()
+    hosts = [HostLayer(WID, l, shape) for l in range(N_LAYERS)]
+    spent, tokens = 0.0, 0
+    while tokens < max_tokens and (spent < budget_s or tokens == 0):
+        x = synth.tokens_bf16(WID, 50000 + tokens, 1, shape.d)
+        for l in range(N_LAYERS):
+            n, _ = oracle.rmsnorm(x, 1e-6)
+            _, idx, _, _ = hosts[l].route(n)
+            hosts[l].fill(idx)
+            L = hosts[l].oracle_layer()
+            t0 = time.perf_counter()
+            x = oracle.stack_layer(L, x, eps=1e-6, act=act_oracle)["x_out"]
+            spent += time.perf_counter() - t0
+        tokens += 1
+    return {"value": tokens / spent, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{tokens} tokens x {N_LAYERS} layers through the CPU oracle (C, fp64/exact, one thread); "
+                      "host expert regeneration excluded"}
+
+
+PHASES = [("norm", 0, 1), ("router", 1, 2), ("barrier1_wait", 2, 3), ("topk", 3, 4), ("issue", 4, 5),
+          ("scales", 5, 6), ("wait_gate_up_rows", 6, 7), ("gate_up", 7, 8), ("barrier2_wait", 8, 9),
+          ("h_limbs", 9, 10), ("wait_down_rows", 10, 11), ("down", 11, 12), ("combine", 12, 13)]
+
+
+def phase_summary(tr):
+    """Median over CTAs and layers of each phase (us), the last-arrival -> first-departure
+    latency of the three grid barriers, and the mean layer time."""
+    d = lambda a, b: np.median((tr[:, :, b] - tr[:, :, a]).astype(np.float64)) / 1e3
+    out = {name: round(float(d(a, b)), 3) for name, a, b in PHASES}
+    b1 = np.median(tr[:, :, 3].min(1) - tr[:, :, 2].max(1)) / 1e3
+    b2 = np.median(tr[:, :, 9].min(1) - tr[:, :, 8].max(1)) / 1e3
+    b3 = np.median(tr[1:, :, 0].min(1) - tr[:-1, :, 13].max(1)) / 1e3
+    out["barrier_propagation"] = [round(float(b1), 3), round(float(b2), 3), round(float(b3), 3)]
+    out["layer_total"] = round(float(np.median(np.diff(tr[:, :, 0].min(1)))) / 1e3, 3)
+    return out
+
+
+def run_reference(args):
+    """--impl reference: the CPU oracle as the reference arm (rank 0 only)."""
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    import synth
+    from tests.gpu_cases import HostLayer
+
+    act = oracle.ACT_INT8 if args.act == "int8" else oracle.ACT_BF16
+    shape = synth.MoEShape()
+    hosts = [HostLayer(WID, l, shape) for l in range(N_LAYERS)]
+    # one step = one layer of one token (1/24 of a token); tokens cycle over a small set so
+    # the host copies of the experts stay bounded
+    ntok = 2
+    chain = {}
+
+    def step(i):
+        t = (i // N_LAYERS) % ntok
+        l = i % N_LAYERS
+        x = chain.get((t, l))
+        if x is None:
+            x = synth.tokens_bf16(WID, 60000 + t, 1, shape.d) if l == 0 else chain[(t, l - 1, "out")]
+            chain[(t, l)] = x
+        n, _ = oracle.rmsnorm(x, 1e-6)
+        _, idx, _, _ = hosts[l].route(n)
+        hosts[l].fill(idx)
+        L = hosts[l].oracle_layer()
+        t0 = time.perf_counter()
+        out = oracle.stack_layer(L, x, eps=1e-6, act=act)["x_out"]
+        dt = time.perf_counter() - t0
+        chain[(t, l, "out")] = out
+        return dt
+
+    for i in range(args.warmup):
+        step(i)
+    spent = sum(step(args.warmup + i) for i in range(args.steps))
+    tokens = args.steps / N_LAYERS
+    value = tokens / spent
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": spent / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": _config(args.act, world, "n/a (CPU)"), "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": f"{args.steps} layer-token steps (one layer of one token each) through "
+                                       "the CPU oracle (C, fp64/exact, one thread)"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--act", choices=["bf16", "int8"], default="bf16")
+    ap.add_argument("--impl", default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=N_LAYERS,
+                    help="profiling only: a shorter stack (the benchmark line is the 24-layer stack)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+
+    import ternary_weight_moe_b200 as tm
+    import synth
+
+    def dev_u16(a, device):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device)
+
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    act = tm.TERN_ACT_INT8 if args.act == "int8" else tm.TERN_ACT_BF16
+
+    global N_LAYERS, BYTES_PER_TOKEN
+    if args.layers != N_LAYERS:
+        N_LAYERS = args.layers
+        BYTES_PER_TOKEN = N_LAYERS * BYTES_PER_LAYER_TOKEN
+    shape, layers, stack = build_stack(dev)
+    ws = tm.workspace(tm.moe_stack_workspace_bytes(layers[0], 1, act), dev)
+    lay = tm.moe_stack_workspace_layout(layers[0], 1, act)
+    launches = tm.moe_stack_kernel_launches(layers[0], N_LAYERS, 1, act)
+    K, W = args.steps, args.warmup
+    xs_host = synth.tokens_bf16(WID, 70000 + 100000 * rank, K + W, shape.d)
+    xs = dev_u16(xs_host, dev)                       # inputs resident in HBM before timing
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    for i in range(W):
+        tm.moe_stack_decode(stack, xs[i:i + 1], act=act, ws=ws)
+    torch.cuda.synchronize(dev)
+    if tm.tern_stream_status() != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    trace_t = []
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        t_wall0 = time.perf_counter()
+        torch.cuda.nvtx.range_push("timed")
+        for i in range(K):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            tm.moe_stack_decode(stack, xs[W + i:W + i + 1], act=act, ws=ws)
+            ev[i][1].record(stream)
+        torch.cuda.nvtx.range_pop()
+        torch.cuda.synchronize(dev)
+        t_wall = time.perf_counter() - t_wall0
+    if tm.tern_stream_status() != 0:
+        raise RuntimeError("device status set during the timed region")
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    dev_ms = sum(step_ms)
+    # phase stamps of the last step: every CTA, every layer (ns, %globaltimer)
+    P = torch.cuda.get_device_properties(dev).multi_processor_count
+    tr = ws[lay["trace"]:lay["trace"] + N_LAYERS * P * 16 * 8].view(torch.int64).view(N_LAYERS, P, 16).cpu().numpy()
+    phases = phase_summary(tr) if launches == 1 else None
+    try:
+        os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+        np.save(os.path.join(ROOT, "gpurun_out", f"trace_{args.act}_rank{rank}.npy"), tr)
+    except OSError:
+        pass
+
+    # back-to-back throughput without flushes (context)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(K):
+        tm.moe_stack_decode(stack, xs[W + i:W + i + 1], act=act, ws=ws)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    b2b_ms = e0.elapsed_time(e1)
+
+    # end to end through the public call with host buffers: pinned H2D of the token, the
+    # stack, D2H of the result, and a host wait per token (the next token needs it)
+    hx = torch.from_numpy(xs_host.view(np.int16)).pin_memory()
+    hy = torch.empty_like(hx).pin_memory()
+    xd = torch.empty((1, shape.d), dtype=torch.int16, device=dev)
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e2.record(stream)
+    for i in range(K):
+        xd.copy_(hx[W + i:W + i + 1], non_blocking=True)
+        tm.moe_stack_decode(stack, xd, act=act, ws=ws)
+        hy[W + i:W + i + 1].copy_(xd, non_blocking=True)
+        stream.synchronize()
+    e3.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e2.elapsed_time(e3)
+
+    dev_ms_max = aggregate(dev_ms, "max", world, dev)
+    e2e_ms_max = aggregate(e2e_ms, "max", world, dev)
+    b2b_ms_max = aggregate(b2b_ms, "max", world, dev)
+    tokens_all = K * world
+    value = tokens_all / (dev_ms_max / 1e3)
+    peak, peak_kind = peaks()
+    avg_launch_ms = dev_ms / K / max(launches, 1)
+    achieved = BYTES_PER_TOKEN / launches / (avg_launch_ms * 1e-3) / 1e9
+    traffic = None
+    tfile = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tfile):
+        try:
+            tj = json.load(open(tfile))
+            key = f"stack_kernel_{args.act}"
+            if key in tj and tj[key].get("valid", False):
+                traffic = tj[key]["bytes_per_launch"]
+        except Exception:
+            traffic = None
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": dev_ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8" if args.act == "int8" else "bf16-in/int-limbs/f64-epilogue", "data": "synthetic",
+        "config": dict(_config(args.act, world, "flushed before every timed step (256 MB write, not timed)"),
+                       layers=N_LAYERS),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic, "kernel": f"stack_kernel<{1 if args.act == 'int8' else 3}>",
+                     "bytes_per_launch": BYTES_PER_TOKEN // launches, "peak_kind": peak_kind},
+        "e2e": {"value": tokens_all / (e2e_ms_max / 1e3), "unit": UNIT, "h2d_bytes_per_step": 2 * shape.d,
+                "d2h_bytes_per_step": 2 * shape.d},
+        "gpu_launches": int(launches * K),
+        "clocks": clk.summary(),
+        "back_to_back_tokens_per_s": tokens_all / (b2b_ms_max / 1e3),
+        "step_ms_p10_p50_p90": [float(np.percentile(step_ms, q)) for q in (10, 50, 90)],
+        "layer_phase_us": phases,
+        "wall_s_timed_region": t_wall,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        from oracle import ACT_BF16, ACT_INT8
+
+        result["cpu_baseline"] = cpu_baseline(ACT_INT8 if args.act == "int8" else ACT_BF16)
+    if world > 1:
+        torch.distributed.barrier()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

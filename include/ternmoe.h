@@ -175,6 +175,26 @@ tern_status moe_stack_decode(const tern_moe_layer *layers, int32_t n_layers, uin
                              float rms_eps, tern_act act, void *workspace, size_t ws_bytes,
                              void *stream);
 
+/* Where, inside a moe_stack_decode workspace, a T == 1 call (the persistent kernel) leaves
+ * its per-layer record, for inspection and parity checks (byte offsets):
+ *   hist    uint16 [n_layers+1][d]  bf16 x entering each layer, and the final x;
+ *   idx     int32  [n_layers][k]    experts chosen at each layer (descending logit);
+ *   gates64 double [n_layers][k]    their renormalised gates;
+ *   trace   uint64 [n_layers][P][16] %globaltimer (ns) stamped by each of the P CTAs (one per
+ *           SM, P <= 256) at phase boundaries: 0 layer start, 1 RMSNorm done, 2 logits stored,
+ *           3 past barrier 1, 4 top-k done, 5 copies issued, 6 scales loaded, 7 gate/up rows
+ *           landed, 8 h stored, 9 past barrier 2, 10 h limbs built, 11 down rows landed,
+ *           12 down done, 13 x' stored. */
+typedef struct {
+    int64_t hist, idx, gates64, trace, total;
+} tern_stack_layout;
+tern_status moe_stack_workspace_layout(const tern_moe_layer *L0, int64_t T_max, tern_act act,
+                                       tern_stack_layout *out);
+
+/* Number of kernel launches one moe_stack_decode call with these arguments makes on the
+ * current device (1 on the persistent T == 1 path), or -1 if the arguments are invalid. */
+int32_t moe_stack_kernel_launches(const tern_moe_layer *L0, int32_t n_layers, int64_t T, tern_act act);
+
 /* Waits for `stream`, then returns and clears the device status word of the current device
  * (TERN_OK, or TERN_ETIMEOUT if an in-kernel bounded wait gave up since the last read), or
  * TERN_ECUDA if the wait itself failed. */

@@ -49,6 +49,10 @@ class FfnLayoutC(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int64) for n in _LAYOUT_FIELDS]
 
 
+class StackLayoutC(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in ("hist", "idx", "gates64", "trace", "total")]
+
+
 _lib = None
 
 
@@ -81,6 +85,8 @@ def lib():
             "moe_ffn_decode": (st, [ctypes.POINTER(MoELayerC), vp, i64, st, vp, vp, vp, sz, vp]),
             "moe_stack_workspace_bytes": (sz, [ctypes.POINTER(MoELayerC), i64, st]),
             "moe_stack_decode": (st, [ctypes.POINTER(MoELayerC), i32, vp, i64, ctypes.c_float, st, vp, sz, vp]),
+            "moe_stack_workspace_layout": (st, [ctypes.POINTER(MoELayerC), i64, st, ctypes.POINTER(StackLayoutC)]),
+            "moe_stack_kernel_launches": (i32, [ctypes.POINTER(MoELayerC), i32, i64, st]),
             "tern_stream_status": (st, [vp]),
             "tern_test_bounded_wait": (st, [vp, i64, vp]),
         }
@@ -289,6 +295,17 @@ def moe_stack_decode(stack: Stack, x, eps=1e-6, act=TERN_ACT_BF16, ws=None, stre
     _check(lib().moe_stack_decode(stack.c, len(stack.layers), _ptr(xb), T, float(eps), act, _ptr(ws), ws.numel(),
                                   _stream(stream)), "moe_stack_decode")
     return x
+
+
+def moe_stack_workspace_layout(layer0: MoELayer, T_max: int = 1, act=TERN_ACT_BF16) -> dict:
+    out = StackLayoutC()
+    _check(lib().moe_stack_workspace_layout(ctypes.byref(layer0.c), T_max, act, ctypes.byref(out)),
+           "moe_stack_workspace_layout")
+    return {n: int(getattr(out, n)) for n in ("hist", "idx", "gates64", "trace", "total")}
+
+
+def moe_stack_kernel_launches(layer0: MoELayer, n_layers: int, T: int, act=TERN_ACT_BF16) -> int:
+    return int(lib().moe_stack_kernel_launches(ctypes.byref(layer0.c), n_layers, T, act))
 
 
 def tern_stream_status(stream=None) -> int:

@@ -285,6 +285,28 @@ tern_status moe_stack_decode(const tern_moe_layer *layers, int32_t n_layers, uin
     return TERN_OK;
 }
 
+tern_status moe_stack_workspace_layout(const tern_moe_layer *L0, int64_t T_max, tern_act act, tern_stack_layout *out) {
+    tern_status st = check_layer(L0);
+    if (st != TERN_OK) return st;
+    if (!out || T_max < 1 || T_max > kMaxT) return TERN_EINVAL;
+    const Layout o = make_layout(L0->d, L0->f, L0->E, L0->k, T_max, act);
+    const int64_t base = o.total + up256(T_max * L0->d * 2);
+    int64_t hist, idx, g, tr;
+    stack_persistent_offsets(L0, &hist, &idx, &g, &tr);
+    out->hist = base + hist;
+    out->idx = base + idx;
+    out->gates64 = base + g;
+    out->trace = base + tr;
+    out->total = (int64_t)moe_stack_workspace_bytes(L0, T_max, act);
+    return TERN_OK;
+}
+
+int32_t moe_stack_kernel_launches(const tern_moe_layer *L0, int32_t n_layers, int64_t T, tern_act act) {
+    if (check_layer(L0) != TERN_OK || n_layers < 1 || n_layers > kMaxLayers || T < 1 || T > kMaxT) return -1;
+    if (T == 1 && stack_persistent_supported(L0, n_layers, act)) return 1;
+    return 7 * n_layers;
+}
+
 tern_status tern_stream_status(void *stream) {
     if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return TERN_ECUDA;
     int h = 0;

@@ -58,7 +58,9 @@ struct StackLayerDev {
     const uint16_t *router;
 };
 size_t stack_persistent_ws_bytes(const tern_moe_layer *L0);
-void stack_persistent_offsets(const tern_moe_layer *L0, int64_t *hist, int64_t *idx_hist, int64_t *gate_hist);
+bool stack_persistent_supported(const tern_moe_layer *L0, int n_layers, tern_act act);
+void stack_persistent_offsets(const tern_moe_layer *L0, int64_t *hist, int64_t *idx_hist, int64_t *gate_hist,
+                              int64_t *ttrace);
 tern_status launch_stack_persistent(const tern_moe_layer *layers, int n_layers, uint16_t *x, float eps,
                                     tern_act act, void *ws, size_t ws_bytes, int *status, cudaStream_t s);
 

@@ -38,6 +38,7 @@ constexpr int kStackWarps = 16;
 constexpr int kStackThreads = kStackWarps * 32;
 constexpr int kMaxStackLayers = 64;
 constexpr int kSK = 8;  // max experts per token on this path
+constexpr int kMaxTraceCtas = 256;
 
 struct StackParams {
     StackLayerDev layer[kMaxStackLayers];
@@ -52,6 +53,7 @@ struct StackParams {
     double *gate_hist;    // [n_layers][k]
     int *status;
     long long limit_ns;   // bound on every in-kernel wait
+    unsigned long long *ttrace;  // [n_layers][P][16] %globaltimer stamps of every CTA at phase boundaries
     // static work split (host computed)
     int P;                // CTAs
     int rb_rows;          // max router rows per CTA
@@ -153,7 +155,7 @@ __device__ __forceinline__ float block_max_nonneg(float v, float *red) {
 // Shared memory map (bytes): lut | router rows | gate rows | up rows | down rows | x | n |
 // h limbs | small arrays.  D = d elements, F = f elements.
 struct SmemMap {
-    uint32_t lut, rbuf, gbuf, ubuf, dbuf, xs, ns, hl, total;
+    uint32_t lut, rbuf, gbuf, ubuf, dbuf, xs, ns, xl, hl, total;
 };
 
 __host__ __device__ inline uint32_t align128(uint32_t v) { return (v + 127u) & ~127u; }
@@ -175,8 +177,10 @@ __host__ __device__ inline SmemMap smem_map(int d, int f, int k, int rb_rows, in
     p = align128(p + (uint32_t)d * 2);
     m.ns = p;
     p = align128(p + (uint32_t)d * 2);
+    m.xl = p;
+    p = align128(p + (uint32_t)NL * (d / 64) * kSegPad * 4);
     m.hl = p;
-    p = align128(p + (uint32_t)k * NL * f);
+    p = align128(p + (uint32_t)k * NL * (f / 64) * kSegPad * 4);
     m.total = p;
     return m;
 }
@@ -194,6 +198,8 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
     __shared__ int s_hshift[kSK];
     __shared__ float s_hscale[kSK];
     __shared__ double s_ye[64][kSK];
+    __shared__ float s_sg[64], s_su[64], s_sd[kSK * 64];
+    __shared__ unsigned int s_hmax[kSK];
     __shared__ int s_ok;
     __shared__ double s_r;
     __shared__ float s_nscale;  // int8: s_x ; bf16: shift as int bits
@@ -209,7 +215,10 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
     uint8_t *dbuf = smem + sm.dbuf;
     uint16_t *xs = reinterpret_cast<uint16_t *>(smem + sm.xs);
     uint16_t *ns = reinterpret_cast<uint16_t *>(smem + sm.ns);
+    uint32_t *xl = reinterpret_cast<uint32_t *>(smem + sm.xl);
     uint32_t *hl = reinterpret_cast<uint32_t *>(smem + sm.hl);
+    const int xlp = (d / 64) * kSegPad;  // padded words per limb of n
+    const int hlp = (f / 64) * kSegPad;  // padded words per limb of one slot's h
 
     // static shares of this CTA
     const int nr = (E - c + P - 1) / P;                        // router rows: c, c+P, ...
@@ -220,6 +229,11 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
     const long long lim = p.limit_ns;
     unsigned int bar_target = 0;
     bool alive = true;
+    unsigned int n_rt = 0, n_gu = 0, n_dn = 0;  // phases issued per mbarrier (thread 0)
+
+    unsigned long long *tt = (tid == 0) ? p.ttrace : nullptr;
+#define TSTAMP(l, ph) \
+    if (tt) tt[((size_t)(l) * P + c) * 16 + (ph)] = gtimer();
 
     lut_fill(lut);
     if (tid == 0) {
@@ -232,6 +246,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
     // router rows of layer 0
     if (tid == 0 && nr > 0) {
         mbar_expect_tx(&mb_router, (uint32_t)(nr * d * 2));
+        n_rt++;
         for (int r = 0; r < nr; r++)
             bulk_g2s(rbuf + (size_t)r * d, p.layer[0].router + (size_t)(c + r * P) * d, (uint32_t)(d * 2), &mb_router);
     }
@@ -241,12 +256,18 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
         const uint32_t par = (uint32_t)(l & 1);
         const uint16_t *xin = (l == 0) ? p.x : p.hist + (size_t)l * d;
         // ---------------------------------------------------------------- A: norm + router
+        TSTAMP(l, 0)
         double ss = 0.0;
-        for (int i = tid; i < d; i += kStackThreads) {
-            const uint16_t b = __ldcg(xin + i);
-            xs[i] = b;
-            const double v = (double)bf16_to_f32(b);
-            ss = fma(v, v, ss);
+        for (int i4 = tid; i4 < d / 4; i4 += kStackThreads) {
+            const uint2 v4 = __ldcg(reinterpret_cast<const uint2 *>(xin) + i4);
+            reinterpret_cast<uint2 *>(xs)[i4] = v4;
+            const uint16_t bb[4] = {(uint16_t)(v4.x & 0xFFFFu), (uint16_t)(v4.x >> 16), (uint16_t)(v4.y & 0xFFFFu),
+                                    (uint16_t)(v4.y >> 16)};
+#pragma unroll
+            for (int e = 0; e < 4; e++) {
+                const double v = (double)bf16_to_f32(bb[e]);
+                ss = fma(v, v, ss);
+            }
         }
         ss = block_sum_f64(ss, s_red);
         if (tid == 0) s_r = sqrt(ss / (double)d + p.eps);
@@ -261,13 +282,15 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             amax = fmaxf(amax, fabsf(bf16_to_f32(nb)));
         }
         amax = block_max_nonneg(amax, s_redf);
+        TSTAMP(l, 1)
         if (tid == 0) {
             if (NL == 1) s_nscale = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
             else s_nscale = __int_as_float(fixed_shift(amax));
         }
         // router rows (prefetched): each row split over kStackWarps / rb_rows warps
         if (nr > 0) {
-            if (!mbar_wait(&mb_router, par, lim, p.status)) alive = false;
+            const bool okw = mbar_wait(&mb_router, par, lim, p.status);
+            alive = __syncthreads_and(okw ? 1 : 0) && alive;
             const int wpr = kStackWarps / p.rb_rows;  // warps per row (rb_rows <= 16)
             const int rr = warp / wpr, part = warp % wpr;
             double acc = 0.0;
@@ -291,16 +314,19 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
         // prefetch the next layer's router rows into the now free buffer
         if (tid == 0 && nr > 0 && l + 1 < p.n_layers) {
             mbar_expect_tx(&mb_router, (uint32_t)(nr * d * 2));
+            n_rt++;
             for (int q = 0; q < nr; q++)
                 bulk_g2s(rbuf + (size_t)q * d, p.layer[l + 1].router + (size_t)(c + q * P) * d, (uint32_t)(d * 2),
                          &mb_router);
         }
+        TSTAMP(l, 2)
         bar_target += (unsigned)P;
         if (!stack_grid_sync(p.bar, bar_target, lim, p.status, &s_ok) || !alive) {
             alive = false;
             break;
         }
         // ---------------------------------------------------------------- B: top-k, issue copies
+        TSTAMP(l, 3)
         for (int e = tid; e < E; e += kStackThreads) s_logit[e] = __ldcg(p.logits + e);
         __syncthreads();
         if (warp == 0) {
@@ -314,10 +340,12 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                 }
         }
         __syncthreads();
+        TSTAMP(l, 4)
         if (tid == 0) {
             // gate/up rows of this CTA's (slot,row) pairs, then its down rows for every slot
             const uint32_t rowb = (uint32_t)(d / 4);
             mbar_expect_tx(&mb_gu, (uint32_t)(2 * (p1 - p0)) * rowb);
+            n_gu++;
             int q = 0;
             for (int pp = p0; pp < p1;) {
                 const int s = pp / f, j = pp % f;
@@ -330,22 +358,35 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             }
             const uint32_t rowd = (uint32_t)(f / 4);
             mbar_expect_tx(&mb_dn, (uint32_t)(k * nrows) * rowd);
+            n_dn++;
             for (int s = 0; s < k; s++)
                 bulk_g2s(dbuf + (size_t)s * p.dn_rows * rowd, Ly.down + ((size_t)s_idx[s] * d + i0) * rowd,
                          (uint32_t)nrows * rowd, &mb_dn);
         }
-        // activation limbs of n for this lane's segment (G = d/64 lanes per row)
-        SegX<NL> X;
+        TSTAMP(l, 5)
+        // per-row scales of this CTA's rows, fetched while the weight copies are in flight
+        for (int q = tid; q < p1 - p0; q += kStackThreads) {
+            const int pp = p0 + q, s2 = pp / f, j = pp % f;
+            const size_t o = (size_t)s_idx[s2] * f + j;
+            s_sg[q] = __ldg(Ly.sg + o);
+            s_su[q] = __ldg(Ly.su + o);
+        }
+        for (int q = tid; q < k * nrows; q += kStackThreads)
+            s_sd[q] = __ldg(Ly.sd + (size_t)s_idx[q / nrows] * d + i0 + q % nrows);
+        TSTAMP(l, 6)
+        // activation limbs of n: one word (4 elements) per thread into the padded layout,
+        // then every lane loads the limbs of its segment (G = d/64 lanes per row)
         {
-            const int gl = lane % (d / 64);
             const int sh = __float_as_int(s_nscale);
             const float inv = (NL == 1 && amax > 0.0f) ? quant_inv(amax) : 0.0f;
-#pragma unroll
-            for (int b = 0; b < 16; b++) {
+            for (int w = tid; w < d / 4; w += kStackThreads) {
+                const uint2 v4 = reinterpret_cast<const uint2 *>(ns)[w];
+                const uint16_t bb[4] = {(uint16_t)(v4.x & 0xFFFFu), (uint16_t)(v4.x >> 16), (uint16_t)(v4.y & 0xFFFFu),
+                                        (uint16_t)(v4.y >> 16)};
                 uint32_t w0 = 0, w1 = 0, w2 = 0;
 #pragma unroll
                 for (int e = 0; e < 4; e++) {
-                    const float v = bf16_to_f32(ns[gl * 64 + 4 * b + e]);
+                    const float v = bf16_to_f32(bb[e]);
                     if (NL == 1) {
                         w0 |= ((uint32_t)(amax > 0.0f ? quant_one(v, inv) : 0) & 0xFFu) << (8 * e);
                     } else {
@@ -356,21 +397,26 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                         w2 |= lo << (8 * e);
                     }
                 }
-                X.w[0][b] = w0;
+                const int pw = padded_word(w);
+                xl[pw] = w0;
                 if (NL > 1) {
-                    X.w[NL > 1 ? 1 : 0][b] = w1;
-                    X.w[NL > 2 ? 2 : 0][b] = w2;
+                    xl[xlp + pw] = w1;
+                    xl[2 * xlp + pw] = w2;
                 }
             }
         }
+        __syncthreads();
+        SegX<NL> X;
+        seg_load_x_padded<NL>(X, xl, xlp, lane % (d / 64));
         // ---------------------------------------------------------------- C: gate/up -> h
         if (p1 > p0) {
-            if (!mbar_wait(&mb_gu, par, lim, p.status)) alive = false;
+            const bool okw = mbar_wait(&mb_gu, par, lim, p.status);
+            alive = __syncthreads_and(okw ? 1 : 0) && alive;
+            TSTAMP(l, 7)
             const uint32_t *lut_lane = lut + lane;
             const int rowb = d / 4;
             for (int q = warp; q < p1 - p0; q += kStackWarps) {
                 const int pp = p0 + q, s = pp / f, j = pp % f;
-                const int e = s_idx[s];
                 const uint4 wg = *reinterpret_cast<const uint4 *>(gbuf + (size_t)q * rowb + lane * 16);
                 const uint4 wu = *reinterpret_cast<const uint4 *>(ubuf + (size_t)q * rowb + lane * 16);
                 int ag[NL], au[NL];
@@ -389,7 +435,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                 }
                 if (lane == 0) {
                     const long long Sg = pair_value(NL, ga, gb2), Su = pair_value(NL, ua, ub);
-                    const float sg = __ldg(Ly.sg + (size_t)e * f + j), su = __ldg(Ly.su + (size_t)e * f + j);
+                    const float sg = s_sg[q], su = s_su[q];
                     float hv;
                     if (NL == 1) {
                         const float gv = __fmul_rn(__fmul_rn(__int2float_rn((int)Sg), sg), s_nscale);
@@ -403,6 +449,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                 }
             }
         }
+        TSTAMP(l, 8)
         bar_target += (unsigned)P;
         if (!stack_grid_sync(p.bar, bar_target, lim, p.status, &s_ok) || !alive) {
             alive = false;
@@ -410,16 +457,25 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
         }
         // ---------------------------------------------------------------- D: down + combine + residual
         {
-            // limbs of every slot's h (each warp pair handles one slot)
-            const int s = warp >> 1;
-            float m = 0.0f;
-            if (s < k)
-                for (int j = (warp & 1) * 32 + lane; j < f; j += 64) m = fmaxf(m, fabsf(__ldcg(p.H + (size_t)s * f + j)));
-            m = warp_max_f32(m);
-            if (lane == 0) s_redf[warp] = m;
+            // every slot's h, read once from L2; per-slot absmax via shared atomics
+            TSTAMP(l, 9)
+            const int wpl = f / 4;  // float4 (= limb words) per slot
+            constexpr int kMaxV = 8;
+            float4 hv[kMaxV];
+            if (tid < kSK) s_hmax[tid] = 0u;
+            __syncthreads();
+#pragma unroll
+            for (int j = 0; j < kMaxV; j++) {
+                const int w = tid + j * kStackThreads;
+                if (w < k * wpl) {
+                    hv[j] = __ldcg(reinterpret_cast<const float4 *>(p.H) + w);
+                    const float m4 = fmaxf(fmaxf(fabsf(hv[j].x), fabsf(hv[j].y)), fmaxf(fabsf(hv[j].z), fabsf(hv[j].w)));
+                    atomicMax(&s_hmax[w / wpl], __float_as_uint(m4));
+                }
+            }
             __syncthreads();
             if (tid < k) {
-                const float a = fmaxf(s_redf[2 * tid], s_redf[2 * tid + 1]);
+                const float a = __uint_as_float(s_hmax[tid]);
                 if (NL == 1) {
                     s_hscale[tid] = a > 0.0f ? __fdiv_rn(a, 127.0f) : 0.0f;
                     s_hshift[tid] = __float_as_int(a);  // keep absmax for the quantiser
@@ -428,18 +484,19 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                 }
             }
             __syncthreads();
-            const int wpl = f / 4;  // words per limb per slot
-            for (int w = tid; w < k * wpl; w += kStackThreads) {
+#pragma unroll
+            for (int j = 0; j < kMaxV; j++) {
+                const int w = tid + j * kStackThreads;
+                if (w >= k * wpl) continue;
                 const int ss2 = w / wpl, b = w % wpl;
-                const float4 hv = __ldcg(reinterpret_cast<const float4 *>(p.H + (size_t)ss2 * f) + b);
-                const float vv[4] = {hv.x, hv.y, hv.z, hv.w};
+                const float vv[4] = {hv[j].x, hv[j].y, hv[j].z, hv[j].w};
                 uint32_t w0 = 0, w1 = 0, w2 = 0;
                 if (NL == 1) {
                     const float a = __int_as_float(s_hshift[ss2]);
                     const float inv = a > 0.0f ? quant_inv(a) : 0.0f;
 #pragma unroll
                     for (int e = 0; e < 4; e++) w0 |= ((uint32_t)(a > 0.0f ? quant_one(vv[e], inv) : 0) & 0xFFu) << (8 * e);
-                    hl[(size_t)ss2 * wpl + b] = w0;
+                    hl[(size_t)ss2 * hlp + padded_word(b)] = w0;
                 } else {
 #pragma unroll
                     for (int e = 0; e < 4; e++) {
@@ -449,13 +506,18 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                         w1 |= mi << (8 * e);
                         w2 |= lo << (8 * e);
                     }
-                    hl[((size_t)ss2 * NL + 0) * wpl + b] = w0;
-                    hl[((size_t)ss2 * NL + (NL > 1 ? 1 : 0)) * wpl + b] = w1;
-                    hl[((size_t)ss2 * NL + (NL > 2 ? 2 : 0)) * wpl + b] = w2;
+                    hl[((size_t)ss2 * NL + 0) * hlp + padded_word(b)] = w0;
+                    hl[((size_t)ss2 * NL + (NL > 1 ? 1 : 0)) * hlp + padded_word(b)] = w1;
+                    hl[((size_t)ss2 * NL + (NL > 2 ? 2 : 0)) * hlp + padded_word(b)] = w2;
                 }
             }
             __syncthreads();
-            if (nrows > 0 && !mbar_wait(&mb_dn, par, lim, p.status)) alive = false;
+            TSTAMP(l, 10)
+            if (nrows > 0) {
+                const bool okw = mbar_wait(&mb_dn, par, lim, p.status);
+                alive = __syncthreads_and(okw ? 1 : 0) && alive;
+            }
+            TSTAMP(l, 11)
             // (row, slot) pairs, G = f/64 lanes each; 512-wide rows -> 8 lanes, 4 pairs per warp pass
             const int G = f / 64;
             const int ppw = 32 / G;
@@ -467,7 +529,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                 const bool valid = pi < npairs;
                 const int rrow = valid ? pi / k : 0, sl = valid ? pi % k : 0;
                 SegX<NL> Hx;
-                seg_load_x_smem<NL>(Hx, hl + (size_t)sl * NL * wpl, wpl, gl);
+                seg_load_x_padded<NL>(Hx, hl + (size_t)sl * NL * hlp, hlp, gl);
                 int acc[NL];
 #pragma unroll
                 for (int z = 0; z < NL; z++) acc[z] = 0;
@@ -482,8 +544,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                 }
                 if (valid && gl == 0) {
                     const long long S = pair_value(NL, a, b);
-                    const int i = i0 + rrow;
-                    const float sd = __ldg(Ly.sd + (size_t)s_idx[sl] * d + i);
+                    const float sd = s_sd[sl * nrows + rrow];
                     double v;
                     if (NL == 1) v = (double)__fmul_rn(__fmul_rn(__int2float_rn((int)S), sd), s_hscale[sl]);
                     else v = ldexp((double)S, -s_hshift[sl]) * (double)sd;
@@ -491,6 +552,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                 }
             }
             __syncthreads();
+            TSTAMP(l, 12)
             const bool last = (l + 1 == p.n_layers);
             if (tid < nrows) {
                 double y = 0.0;
@@ -501,6 +563,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                 p.hist[(size_t)(l + 1) * d + i] = xo;
                 if (last) p.x[i] = xo;
             }
+            TSTAMP(l, 13)
             if (!last) {
                 bar_target += (unsigned)P;
                 if (!stack_grid_sync(p.bar, bar_target, lim, p.status, &s_ok) || !alive) {
@@ -509,6 +572,13 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                 }
             }
         }
+    }
+#undef TSTAMP
+    // after a timeout, let this CTA's own copies in flight land (bounded) before leaving
+    if (!alive && tid == 0) {
+        if (n_rt) mbar_wait(&mb_router, (n_rt - 1) & 1u, lim, p.status);
+        if (n_gu) mbar_wait(&mb_gu, (n_gu - 1) & 1u, lim, p.status);
+        if (n_dn) mbar_wait(&mb_dn, (n_dn - 1) & 1u, lim, p.status);
     }
     // leave: the last CTA out resets the barrier counters for the next launch
     __syncthreads();
@@ -526,7 +596,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
 // Persistent-path workspace: barrier words, logits [E], H [k][f], x history
 // [(kMaxStackLayers+1)][d], routing history [kMaxStackLayers][k] (int32 + fp64).
 struct StackWs {
-    int64_t bar, logits, H, hist, idx_hist, gate_hist, total;
+    int64_t bar, logits, H, hist, idx_hist, gate_hist, ttrace, total;
 };
 
 static inline int64_t up256_(int64_t v) { return (v + 255) & ~int64_t(255); }
@@ -545,17 +615,20 @@ static StackWs stack_ws_layout(const tern_moe_layer *L0) {
     o.hist = take((int64_t)(kMaxStackLayers + 1) * L0->d * 2);
     o.idx_hist = take((int64_t)kMaxStackLayers * L0->k * 4);
     o.gate_hist = take((int64_t)kMaxStackLayers * L0->k * 8);
+    o.ttrace = take((int64_t)kMaxStackLayers * kMaxTraceCtas * 16 * 8);
     o.total = p;
     return o;
 }
 
 size_t stack_persistent_ws_bytes(const tern_moe_layer *L0) { return (size_t)stack_ws_layout(L0).total; }
 
-void stack_persistent_offsets(const tern_moe_layer *L0, int64_t *hist, int64_t *idx_hist, int64_t *gate_hist) {
+void stack_persistent_offsets(const tern_moe_layer *L0, int64_t *hist, int64_t *idx_hist, int64_t *gate_hist,
+                              int64_t *ttrace) {
     const StackWs o = stack_ws_layout(L0);
     *hist = o.hist;
     *idx_hist = o.idx_hist;
     *gate_hist = o.gate_hist;
+    *ttrace = o.ttrace;
 }
 
 static int sm_count() {
@@ -565,20 +638,48 @@ static int sm_count() {
     return n;
 }
 
+struct StackPlan {
+    int P, rb_rows, gu_pairs, dn_rows;
+    SmemMap sm;
+    const void *fn;
+};
+
+static tern_status stack_plan(const tern_moe_layer &L0, int n_layers, tern_act act, StackPlan &pl) {
+    if (n_layers > kMaxStackLayers || L0.d != 2048 || L0.k > kSK || L0.f % 64 || L0.f > 2048) return TERN_EUNSUPPORTED;
+    const int64_t g = L0.f / 64;
+    if ((g & (g - 1)) != 0) return TERN_EUNSUPPORTED;
+    pl.P = sm_count();
+    if (pl.P <= 0) return TERN_ECUDA;
+    if (pl.P > kMaxTraceCtas) pl.P = kMaxTraceCtas;
+    pl.rb_rows = (L0.E + pl.P - 1) / pl.P;
+    pl.gu_pairs = (int)((L0.k * L0.f + pl.P - 1) / pl.P);
+    pl.dn_rows = (int)((L0.d + pl.P - 1) / pl.P);
+    if (pl.rb_rows > kStackWarps || pl.dn_rows > 64 || pl.gu_pairs > 64 || L0.k * L0.f > 8 * 4 * kStackThreads)
+        return TERN_EUNSUPPORTED;
+    const int NL = act == TERN_ACT_INT8 ? 1 : 3;
+    pl.sm = smem_map((int)L0.d, (int)L0.f, L0.k, pl.rb_rows, pl.gu_pairs, pl.dn_rows, NL);
+    pl.fn = act == TERN_ACT_INT8 ? (const void *)stack_kernel<1> : (const void *)stack_kernel<3>;
+    if (cudaFuncSetAttribute(pl.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.sm.total) != cudaSuccess)
+        return TERN_ECUDA;
+    int nb = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, pl.fn, kStackThreads, pl.sm.total) != cudaSuccess)
+        return TERN_ECUDA;
+    if (nb < 1) return TERN_EUNSUPPORTED;
+    return TERN_OK;
+}
+
+bool stack_persistent_supported(const tern_moe_layer *L0, int n_layers, tern_act act) {
+    StackPlan pl;
+    return stack_plan(*L0, n_layers, act, pl) == TERN_OK;
+}
+
 tern_status launch_stack_persistent(const tern_moe_layer *layers, int n_layers, uint16_t *x, float eps, tern_act act,
                                     void *ws, size_t ws_bytes, int *status, cudaStream_t s) {
     const tern_moe_layer &L0 = layers[0];
-    if (n_layers > kMaxStackLayers || L0.d != 2048 || L0.k > kSK || L0.f % 64 || L0.f > 2048) return TERN_EUNSUPPORTED;
-    {
-        const int64_t g = L0.f / 64;
-        if ((g & (g - 1)) != 0) return TERN_EUNSUPPORTED;
-    }
-    const int P = sm_count();
-    if (P <= 0) return TERN_ECUDA;
-    const int rb_rows = (L0.E + P - 1) / P;
-    const int gu_pairs = (int)((L0.k * L0.f + P - 1) / P);
-    const int dn_rows = (int)((L0.d + P - 1) / P);
-    if (rb_rows > kStackWarps || dn_rows > 64) return TERN_EUNSUPPORTED;
+    StackPlan pl;
+    const tern_status pst = stack_plan(L0, n_layers, act, pl);
+    if (pst != TERN_OK) return pst;
+    const int P = pl.P, rb_rows = pl.rb_rows, gu_pairs = pl.gu_pairs, dn_rows = pl.dn_rows;
     const StackWs o = stack_ws_layout(&L0);
     if (ws_bytes < (size_t)o.total) return TERN_EWORKSPACE;
     if (!status) return TERN_ECUDA;
@@ -608,6 +709,7 @@ tern_status launch_stack_persistent(const tern_moe_layer *layers, int n_layers, 
     prm.hist = reinterpret_cast<uint16_t *>(b + o.hist);
     prm.idx_hist = reinterpret_cast<int32_t *>(b + o.idx_hist);
     prm.gate_hist = reinterpret_cast<double *>(b + o.gate_hist);
+    prm.ttrace = reinterpret_cast<unsigned long long *>(b + o.ttrace);
     prm.status = status;
     prm.limit_ns = 1000000000ll;  // every in-kernel wait gives up after one second
     prm.P = P;
@@ -615,14 +717,8 @@ tern_status launch_stack_persistent(const tern_moe_layer *layers, int n_layers, 
     prm.gu_pairs = gu_pairs;
     prm.dn_rows = dn_rows;
 
-    const int NL = act == TERN_ACT_INT8 ? 1 : 3;
-    const SmemMap sm = smem_map(prm.d, prm.f, prm.k, rb_rows, gu_pairs, dn_rows, NL);
-    const void *fn = act == TERN_ACT_INT8 ? (const void *)stack_kernel<1> : (const void *)stack_kernel<3>;
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm.total) != cudaSuccess)
-        return TERN_ECUDA;
-    int nb = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, kStackThreads, sm.total) != cudaSuccess) return TERN_ECUDA;
-    if (nb < 1) return TERN_EUNSUPPORTED;
+    const SmemMap sm = pl.sm;
+    const void *fn = pl.fn;
     void *args[] = {&prm};
     const cudaError_t e = cudaLaunchCooperativeKernel(fn, dim3(P), dim3(kStackThreads), args, sm.total, s);
     return e == cudaSuccess ? TERN_OK : TERN_ECUDA;

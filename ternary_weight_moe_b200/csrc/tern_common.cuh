@@ -162,6 +162,28 @@ __device__ __forceinline__ void seg_load_x_smem(SegX<NL> &x, const uint32_t *lim
     }
 }
 
+// Padded limb layout in shared memory: the 16 words of segment g start at word 20*g, so the
+// 128-bit loads of 8 lanes reading 8 different segments fall in 8 different bank groups.
+constexpr int kSegPad = 20;
+__device__ __forceinline__ int padded_word(int w) { return (w >> 4) * kSegPad + (w & 15); }
+
+template <int NL>
+__device__ __forceinline__ void seg_load_x_padded(SegX<NL> &x, const uint32_t *limbw, int words_per_limb_padded,
+                                                  int seg) {
+#pragma unroll
+    for (int l = 0; l < NL; l++) {
+        const uint4 *p = reinterpret_cast<const uint4 *>(limbw + l * words_per_limb_padded + seg * kSegPad);
+#pragma unroll
+        for (int v = 0; v < 4; v++) {
+            const uint4 t = p[v];
+            x.w[l][4 * v + 0] = t.x;
+            x.w[l][4 * v + 1] = t.y;
+            x.w[l][4 * v + 2] = t.z;
+            x.w[l][4 * v + 3] = t.w;
+        }
+    }
+}
+
 // Per-lane partial sums -> at most two int32 for the cross-lane reduction.
 // NL == 3: hi stays separate, (mid*256 + lo) is combined; both fit int32 for <= 256 codes
 // per lane and 32 lanes.
@@ -231,59 +253,66 @@ __device__ __forceinline__ void fixed_limbs(float x, int s, uint32_t &hi, uint32
 // ---------------------------------------------------------------------------- top-k
 // One warp selects the top k of E fp64 logits: descending value, ties to the lower index.
 // Lane l owns experts l, l+32, ...; selected entries are set to -inf (logits are finite).
+// Order-preserving 64-bit key of a finite double (larger double -> larger unsigned key;
+// -0.0 and +0.0 map to the same key).
+__device__ __forceinline__ unsigned long long f64_order_key(double v) {
+    if (v == 0.0) v = 0.0;  // fold -0.0 into +0.0
+    const unsigned long long u = (unsigned long long)__double_as_longlong(v);
+    return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+}
+
+// One warp selects the top k (k <= 8) of E fp64 logits: descending value, ties to the lower
+// index.  Lane l owns experts l, l+32, ...  Each round reduces the lanes' best 64-bit keys
+// with the single-instruction warp max (__reduce_max_sync) on the high word, then the low
+// word, then the index.  Gates: lanes 0..k-1 each compute one exp(l_i - l_0) in fp64; lane 0
+// sums them in top-k order.  Outputs (written by lanes 0..k-1): idx_out, g64, g32 (either
+// gate pointer may be null).
 template <int J>
 __device__ __forceinline__ void warp_topk(const double *lg, int E, int k, int32_t *idx_out, double *g64, float *g32) {
     const int lane = threadIdx.x & 31;
-    double v[J];
+    unsigned long long key[J];
 #pragma unroll
     for (int j = 0; j < J; j++) {
         const int e = lane + 32 * j;
-        v[j] = (e < E) ? lg[e] : -INFINITY;
+        key[j] = (e < E) ? f64_order_key(lg[e]) : 0ull;  // 0 = below every finite logit
     }
-    double selv[8];
-    int seli[8];
+    int sel_e = 0;
     for (int r = 0; r < k; r++) {
-        double bv = -INFINITY;
-        int bi = 0x7FFFFFFF;
+        // lane-local best (largest key, then lowest index = lowest j)
+        unsigned long long bk = 0ull;
+        int bj = 0;
 #pragma unroll
-        for (int j = 0; j < J; j++) {
-            const int e = lane + 32 * j;
-            if (e < E && (v[j] > bv || (v[j] == bv && e < bi))) {
-                bv = v[j];
-                bi = e;
+        for (int j = 0; j < J; j++)
+            if (key[j] > bk) {
+                bk = key[j];
+                bj = j;
             }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const double ov = __shfl_xor_sync(0xFFFFFFFFu, bv, o);
-            const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
-            if (ov > bv || (ov == bv && oi < bi)) {
-                bv = ov;
-                bi = oi;
-            }
-        }
-        selv[r] = bv;
-        seli[r] = bi;
-        if ((bi & 31) == lane) {
+        const unsigned hi = (unsigned)(bk >> 32), lo = (unsigned)bk;
+        const unsigned mhi = __reduce_max_sync(0xFFFFFFFFu, hi);
+        const unsigned mlo = __reduce_max_sync(0xFFFFFFFFu, hi == mhi ? lo : 0u);
+        const bool cand = (hi == mhi) && (lo == mlo);
+        const int e = lane + 32 * bj;
+        const unsigned wi = __reduce_min_sync(0xFFFFFFFFu, cand ? (unsigned)e : 0xFFFFFFFFu);
+        int win = (int)wi;
+        if (win < 0 || win >= E) win = r;  // NaN inputs must still not index out of range
+        if (win == e && cand) {
 #pragma unroll
             for (int j = 0; j < J; j++)
-                if (j == (bi >> 5)) v[j] = -INFINITY;
+                if (j == bj) key[j] = 0ull;
         }
+        if (lane == r) sel_e = win;
     }
-    if (lane == 0) {
-        const double l0 = selv[0];
-        double ev[8];
-        double z = 0.0;
-        for (int r = 0; r < k; r++) {
-            ev[r] = exp(selv[r] - l0);
-            z += ev[r];
-        }
-        for (int r = 0; r < k; r++) {
-            idx_out[r] = seli[r];
-            const double g = ev[r] / z;
-            if (g64) g64[r] = g;
-            if (g32) g32[r] = (float)g;
-        }
+    // gates: lane r < k holds expert sel_e; logit of the top-1 broadcast from lane 0
+    const double lsel = (lane < k) ? lg[sel_e] : 0.0;
+    const double l0 = __shfl_sync(0xFFFFFFFFu, lsel, 0);
+    const double ev = (lane < k) ? exp(lsel - l0) : 0.0;
+    double z = 0.0;
+    for (int r = 0; r < k; r++) z += __shfl_sync(0xFFFFFFFFu, ev, r);  // top-k order
+    if (lane < k) {
+        idx_out[lane] = sel_e;
+        const double g = ev / z;
+        if (g64) g64[lane] = g;
+        if (g32) g32[lane] = (float)g;
     }
 }
 

@@ -159,7 +159,7 @@ def test_stack_teacher_forced_per_layer(stack3, act):
     dev = layers[0].gate.device
     x = synth.tokens_bf16(WID_STACK, 7, 1, shape.d)
     xd = dev_u16(x, dev)
-    # the full stack in one call
+    # the full stack in one call (T = 1: the persistent kernel)
     full = xd.clone()
     tm.moe_stack_decode(tm.Stack(layers), full, eps=1e-6, act=act)
     # layer by layer on the GPU, each compared with the oracle on the GPU's own input
@@ -178,3 +178,67 @@ def test_stack_teacher_forced_per_layer(stack3, act):
         mismatched += int((got != ref["x_out"]).sum())
     assert mismatched <= 3 * 2048 * 5e-3
     assert torch.equal(full.view(torch.int16), cur.view(torch.int16))
+
+
+def test_persistent_matches_stage_path_bit_exact(stack3):
+    """The one-launch T=1 stack and the kernel-per-stage path (taken for T=2) do the same
+    arithmetic in the same order, so a token gives identical bits on both."""
+    shape, layers, hosts = stack3
+    dev = layers[0].gate.device
+    st = tm.Stack(layers)
+    for act in (tm.TERN_ACT_BF16, tm.TERN_ACT_INT8):
+        assert tm.moe_stack_kernel_launches(layers[0], 3, 1, act) == 1
+        assert tm.moe_stack_kernel_launches(layers[0], 3, 2, act) == 21
+        x = synth.tokens_bf16(WID_STACK, 8, 1, shape.d)
+        one = dev_u16(x, dev)
+        two = dev_u16(np.concatenate([x, x]), dev)
+        tm.moe_stack_decode(st, one, act=act)
+        tm.moe_stack_decode(st, two, act=act)
+        assert tm.tern_stream_status() == 0
+        assert torch.equal(one.view(torch.int16)[0], two.view(torch.int16)[0])
+        assert torch.equal(two.view(torch.int16)[0], two.view(torch.int16)[1])
+
+
+@pytest.fixture(scope="module")
+def stack24(cuda_dev):
+    shape = synth.MoEShape()
+    layers = [device_layer(WID_STACK, l, shape, cuda_dev) for l in range(24)]
+    return shape, layers
+
+
+@pytest.mark.parametrize("act,steps", [(tm.TERN_ACT_BF16, (0, 1)), (tm.TERN_ACT_INT8, (2,))])
+def test_stack24_persistent_teacher_forced(stack24, act, steps):
+    """The 24-layer stack, one launch per token (the benchmark's configuration): every
+    layer's output checked against the oracle run on the kernel's own input to that layer."""
+    shape, layers = stack24
+    dev = layers[0].gate.device
+    st = tm.Stack(layers)
+    ws = tm.workspace(tm.moe_stack_workspace_bytes(layers[0], 1, act), dev)
+    lay = tm.moe_stack_workspace_layout(layers[0], 1, act)
+    k, d = shape.k, shape.d
+    hosts = [HostLayer(WID_STACK, l, shape) for l in range(24)]
+    for step in steps:
+        x = synth.tokens_bf16(WID_STACK, 1000 + step, 1, d)
+        xd = dev_u16(x, dev)
+        tm.moe_stack_decode(st, xd, eps=1e-6, act=act, ws=ws)
+        assert tm.tern_stream_status() == 0
+        hist = host_u16(ws_view(ws, lay["hist"], torch.int16, 25 * d).view(25, d))
+        idx = ws_view(ws, lay["idx"], torch.int32, 24 * k).view(24, k).cpu().numpy()
+        g64 = ws_view(ws, lay["gates64"], torch.float64, 24 * k).view(24, k).cpu().numpy()
+        assert (hist[0] == x[0]).all()
+        assert (hist[24] == host_u16(xd)[0]).all()
+        mism = 0
+        for l in range(24):
+            n, _ = oracle.rmsnorm(hist[l], 1e-6)
+            _, idx_ref, _, _ = hosts[l].route(n)
+            hosts[l].fill(idx_ref)
+            ref = oracle.stack_layer(hosts[l].oracle_layer(), hist[l], eps=1e-6, act=act)
+            assert (idx[l] == ref["idx"][0]).all(), l
+            assert np.abs(g64[l] - ref["gates"][0]).max() <= 1e-12
+            close = _bf16_ulp_close(hist[l + 1], ref["x_out"][0])
+            assert close.all(), (l, np.argwhere(~close)[:5])
+            mism += int((hist[l + 1] != ref["x_out"][0]).sum())
+        assert mism <= 24 * d * 5e-3
+        # and the whole chain stays finite and of sane size
+        xf = synth.bf16_bits_to_f64(hist)
+        assert np.isfinite(xf).all() and np.abs(xf).max() < 1e3
