@@ -183,9 +183,10 @@ def cpu_baseline(act_oracle, budget_s=12.0, max_tokens=4):
                       "host expert regeneration excluded"}
 
 
-PHASES = [("norm", 0, 1), ("router", 1, 2), ("barrier1_wait", 2, 3), ("topk", 3, 4), ("issue", 4, 5),
-          ("scales", 5, 6), ("wait_gate_up_rows", 6, 7), ("gate_up", 7, 8), ("barrier2_wait", 8, 9),
-          ("h_limbs", 9, 10), ("wait_down_rows", 10, 11), ("down", 11, 12), ("combine", 12, 13)]
+PHASES = [("x_wait", 0, 1), ("norm_limbs", 1, 2), ("router", 2, 3), ("logits_wait", 3, 4), ("topk", 4, 5),
+          ("issue", 5, 6), ("gate_up_rows_wait", 6, 7), ("gate_up_dots", 7, 8), ("swiglu", 8, 9),
+          ("h_wait", 9, 10), ("h_limbs", 10, 11), ("down_rows_wait", 11, 12), ("down_dots", 12, 13),
+          ("combine", 13, 14)]
 
 
 def phase_summary(tr):
@@ -193,10 +194,11 @@ def phase_summary(tr):
     latency of the three grid barriers, and the mean layer time."""
     d = lambda a, b: np.median((tr[:, :, b] - tr[:, :, a]).astype(np.float64)) / 1e3
     out = {name: round(float(d(a, b)), 3) for name, a, b in PHASES}
-    b1 = np.median(tr[:, :, 3].min(1) - tr[:, :, 2].max(1)) / 1e3
-    b2 = np.median(tr[:, :, 9].min(1) - tr[:, :, 8].max(1)) / 1e3
-    b3 = np.median(tr[1:, :, 0].min(1) - tr[:-1, :, 13].max(1)) / 1e3
-    out["barrier_propagation"] = [round(float(b1), 3), round(float(b2), 3), round(float(b3), 3)]
+    # exchange latency: last producer's publish -> first consumer's receipt
+    e_log = np.median(tr[:, :, 4].min(1) - tr[:, :, 3].max(1)) / 1e3
+    e_h = np.median(tr[:, :, 10].min(1) - tr[:, :, 9].max(1)) / 1e3
+    e_x = np.median(tr[1:, :, 1].min(1) - tr[:-1, :, 14].max(1)) / 1e3
+    out["exchange_latency"] = {"logits": round(float(e_log), 3), "h": round(float(e_h), 3), "x": round(float(e_x), 3)}
     out["layer_total"] = round(float(np.median(np.diff(tr[:, :, 0].min(1)))) / 1e3, 3)
     return out
 
@@ -253,6 +255,7 @@ def run_reference(args):
 
 
 def main():
+    global N_LAYERS, BYTES_PER_TOKEN
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=400)
@@ -288,7 +291,6 @@ def main():
     torch.cuda.set_device(dev)
     act = tm.TERN_ACT_INT8 if args.act == "int8" else tm.TERN_ACT_BF16
 
-    global N_LAYERS, BYTES_PER_TOKEN
     if args.layers != N_LAYERS:
         N_LAYERS = args.layers
         BYTES_PER_TOKEN = N_LAYERS * BYTES_PER_LAYER_TOKEN
@@ -328,8 +330,13 @@ def main():
         raise RuntimeError("device status set during the timed region")
     step_ms = [a.elapsed_time(b) for a, b in ev]
     dev_ms = sum(step_ms)
-    # phase stamps of the last step: every CTA, every layer (ns, %globaltimer)
+    # one extra, traced step (outside the timed region): every CTA stamps every phase
     P = torch.cuda.get_device_properties(dev).multi_processor_count
+    os.environ["TERNMOE_TRACE"] = "1"
+    flush.fill_(1)
+    tm.moe_stack_decode(stack, xs[W:W + 1].clone(), act=act, ws=ws)
+    torch.cuda.synchronize(dev)
+    os.environ["TERNMOE_TRACE"] = "0"
     tr = ws[lay["trace"]:lay["trace"] + N_LAYERS * P * 16 * 8].view(torch.int64).view(N_LAYERS, P, 16).cpu().numpy()
     phases = phase_summary(tr) if launches == 1 else None
     try:
@@ -398,7 +405,7 @@ def main():
         "clocks": clk.summary(),
         "back_to_back_tokens_per_s": tokens_all / (b2b_ms_max / 1e3),
         "step_ms_p10_p50_p90": [float(np.percentile(step_ms, q)) for q in (10, 50, 90)],
-        "layer_phase_us": phases,
+        "layer_phase_us_traced_step": phases,
         "wall_s_timed_region": t_wall,
     }
     if rank == 0 and not args.no_cpu_baseline:

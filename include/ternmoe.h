@@ -181,10 +181,12 @@ tern_status moe_stack_decode(const tern_moe_layer *layers, int32_t n_layers, uin
  *   idx     int32  [n_layers][k]    experts chosen at each layer (descending logit);
  *   gates64 double [n_layers][k]    their renormalised gates;
  *   trace   uint64 [n_layers][P][16] %globaltimer (ns) stamped by each of the P CTAs (one per
- *           SM, P <= 256) at phase boundaries: 0 layer start, 1 RMSNorm done, 2 logits stored,
- *           3 past barrier 1, 4 top-k done, 5 copies issued, 6 scales loaded, 7 gate/up rows
- *           landed, 8 h stored, 9 past barrier 2, 10 h limbs built, 11 down rows landed,
- *           12 down done, 13 x' stored. */
+ *           SM, P <= 256) at phase boundaries, written only when the environment variable
+ *           TERNMOE_TRACE is "1" at the time of the call (the stamps cost time): 0 layer start, 1 x received, 2 n and limbs
+ *           ready, 3 own logits published, 4 all logits received, 5 top-k done, 6 copies
+ *           issued, 7 gate/up rows landed, 8 gate/up dots done, 9 h published, 10 all h
+ *           received, 11 h limbs built, 12 down rows landed, 13 down dots done,
+ *           14 x' published. */
 typedef struct {
     int64_t hist, idx, gates64, trace, total;
 } tern_stack_layout;

@@ -6,27 +6,30 @@
 // Ternary Actually Means").  At d = 2048 one layer moves only 7.4 MB, about a microsecond of
 // HBM time on a B200, so the chain router -> top-k -> expert rows -> h -> down -> residual
 // is bound by latency, not by bytes.  This kernel therefore:
-//   * runs the whole stack in ONE launch: one CTA per SM, co-resident (cooperative launch),
-//     three bounded grid barriers per layer (after the router logits, after h, after x');
+//   * runs the whole stack in ONE launch: one CTA per SM, all co-resident (cooperative
+//     launch), no kernel boundary between layers;
+//   * exchanges data between CTAs with flag-carrying 64-bit words: {32-bit payload, 32-bit
+//     tag}, written and read as single 64-bit accesses (single-copy atomic), where the tag
+//     names the launch and the layer.  A consumer polls the data itself, so each exchange
+//     costs one L2 round trip instead of a barrier plus a read, and no arrival counter has
+//     to be reset between launches;
 //   * gives every CTA a fixed share of each layer's bytes and moves it with TMA bulk copies
-//     (cp.async.bulk, global -> shared, mbarrier completion), issued as early as the data
-//     dependencies allow: the next layer's router rows during the current layer, and a
-//     CTA's gate/up AND down rows together as soon as top-k is known -- the down rows do not
-//     depend on h, so they land while gate/up is computed;
+//     (cp.async.bulk global -> shared, mbarrier completion) as early as the dependencies
+//     allow: the next layer's router rows during the current layer; a CTA's gate/up AND down
+//     rows together as soon as top-k is known (the down rows do not depend on h);
 //   * decodes the packed bytes in registers (one table read + one dp4a per limb per byte).
 //
-// Per layer l (x_l in global memory, bf16):
-//   A  every CTA: n = bf16(x / sqrt(mean x^2 + eps)) (fp64), its router rows -> logits (fp64)
-//   -- grid barrier --
-//   B  every CTA: top-k + gates (identical in every CTA), issue its TMA copies
-//   C  its (slot, row) pairs of gate/up -> h = silu(g) * u (fp64 epilogue) -> global
-//   -- grid barrier --
-//   D  every CTA: limbs of all h; its output rows: down for every slot, gate-weighted sum in
-//      top-k order (fp64), bf16, residual add -> x_{l+1}
-//   -- grid barrier --
-#include <cooperative_groups.h>
+// Per layer l, in every CTA (P = #SMs CTAs):
+//   A  x_l (exchange) -> sum of squares and absmax in one block reduction -> n = bf16(x/r),
+//      activation limbs; its router rows (prefetched) -> logits -> exchange
+//   B  all logits -> top-k + gates -> TMA copies of its gate/up pairs and down rows
+//   C  its (slot,row) gate/up pairs -> h = silu(g) * u (fp64 epilogue, one thread per row)
+//      -> exchange
+//   D  all h -> limbs; its output rows: down for every slot, gate-weighted sum in top-k order
+//      (fp64), bf16, residual add -> x_{l+1} -> exchange
 #include <cuda_runtime.h>
 #include <math.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include "kernels.h"
@@ -44,21 +47,21 @@ struct StackParams {
     StackLayerDev layer[kMaxStackLayers];
     int n_layers, d, f, E, k;
     double eps;
-    uint16_t *x;          // [d] in/out
-    unsigned int *bar;    // [0] arrivals, [1] leavers
-    double *logits;       // [E]
-    float *H;             // [k][f]
-    uint16_t *hist;       // [n_layers+1][d]  x before each layer and after the last
-    int32_t *idx_hist;    // [n_layers][k]
-    double *gate_hist;    // [n_layers][k]
+    uint16_t *x;                  // [d] in/out
+    unsigned int *ctl;            // [0] CTAs that left this launch, [1] launch epoch
+    unsigned long long *xll;      // [d/2]  {two bf16 of x_{l}, tag}
+    unsigned long long *lll;      // [2E]   {high / low word of the fp64 logit, tag}
+    unsigned long long *hll;      // [k*f]  {fp32 h, tag}
+    uint16_t *hist;               // [n_layers+1][d]  x before each layer and after the last
+    int32_t *idx_hist;            // [n_layers][k]
+    double *gate_hist;            // [n_layers][k]
     int *status;
-    long long limit_ns;   // bound on every in-kernel wait
-    unsigned long long *ttrace;  // [n_layers][P][16] %globaltimer stamps of every CTA at phase boundaries
-    // static work split (host computed)
-    int P;                // CTAs
-    int rb_rows;          // max router rows per CTA
-    int gu_pairs;         // max gate/up pairs per CTA
-    int dn_rows;          // max output rows per CTA
+    long long limit_ns;           // bound on every in-kernel wait
+    unsigned long long *ttrace;   // [n_layers][P][16] %globaltimer stamps of every CTA
+    int P;                        // CTAs
+    int rb_rows;                  // max router rows per CTA
+    int gu_pairs;                 // max gate/up pairs per CTA
+    int dn_rows;                  // max output rows per CTA (even)
 };
 
 // ------------------------------------------------------------------ PTX helpers
@@ -105,55 +108,47 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, long l
     return true;
 }
 
-// bounded grid barrier on a monotonic arrival counter (zero at launch, reset by the last
-// CTA to leave).  Returns false on timeout.
-__device__ __forceinline__ bool stack_grid_sync(unsigned int *arrive, unsigned int target, long long limit_ns,
-                                                int *status, int *s_ok) {
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        red_release_gpu_add(arrive, 1u);
-        int ok = 1;
-        if ((int)(ld_acquire_gpu(arrive) - target) < 0) {
-            const unsigned long long t0 = gtimer();
-            while ((int)(ld_acquire_gpu(arrive) - target) < 0) {
-                if ((long long)(gtimer() - t0) > limit_ns) {
-                    ok = 0;
-                    set_status(status, TERN_ETIMEOUT);
-                    break;
+// ---- flag-carrying words: one 64-bit access carries payload and tag together
+__device__ __forceinline__ void ll_store(unsigned long long *p, uint32_t val, uint32_t tag) {
+    const unsigned long long w = ((unsigned long long)tag << 32) | (unsigned long long)val;
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+}
+__device__ __forceinline__ unsigned long long ll_load(const unsigned long long *p) {
+    unsigned long long w;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
+    return w;
+}
+// Poll n words p[0..n) (n <= 8) until every tag equals `tag`; payloads into out[].
+// False on timeout (status set).
+template <int N>
+__device__ __forceinline__ bool ll_poll(const unsigned long long *p, int n, uint32_t tag, uint32_t (&out)[N],
+                                        long long limit_ns, int *status) {
+    unsigned pending = (n >= 32) ? 0xFFFFFFFFu : ((1u << n) - 1u);
+    unsigned long long t0 = 0;
+    bool started = false;
+    while (true) {
+#pragma unroll
+        for (int i = 0; i < N; i++) {
+            if (pending & (1u << i)) {
+                const unsigned long long w = ll_load(p + i);
+                if ((uint32_t)(w >> 32) == tag) {
+                    out[i] = (uint32_t)w;
+                    pending &= ~(1u << i);
                 }
             }
         }
-        *s_ok = ok;
+        if (!pending) return true;
+        if (!started) {
+            t0 = gtimer();
+            started = true;
+        } else if ((long long)(gtimer() - t0) > limit_ns) {
+            set_status(status, TERN_ETIMEOUT);
+            return false;
+        }
     }
-    __syncthreads();
-    return *s_ok != 0;
 }
 
-__device__ __forceinline__ double block_sum_f64(double v, double *red) {
-    v = warp_sum_f64(v);
-    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-    if (l == 0) red[w] = v;
-    __syncthreads();
-    double r = (l < kStackWarps) ? red[l] : 0.0;
-    r = warp_sum_f64(r);
-    __syncthreads();
-    return r;
-}
-
-__device__ __forceinline__ float block_max_nonneg(float v, float *red) {
-    v = warp_max_f32(v);
-    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-    if (l == 0) red[w] = v;
-    __syncthreads();
-    float r = (l < kStackWarps) ? red[l] : 0.0f;
-    r = warp_max_f32(r);
-    __syncthreads();
-    return r;
-}
-
-// ------------------------------------------------------------------ the kernel
-// Shared memory map (bytes): lut | router rows | gate rows | up rows | down rows | x | n |
-// h limbs | small arrays.  D = d elements, F = f elements.
+// ------------------------------------------------------------------ shared memory map
 struct SmemMap {
     uint32_t lut, rbuf, gbuf, ubuf, dbuf, xs, ns, xl, hl, total;
 };
@@ -185,24 +180,42 @@ __host__ __device__ inline SmemMap smem_map(int d, int f, int k, int rb_rows, in
     return m;
 }
 
+// limb words of four consecutive values v[0..3] (one word per limb)
+template <int NL>
+__device__ __forceinline__ void limb_words(const float (&v)[4], int sh_or_unused, float inv, bool nonzero,
+                                           uint32_t (&w)[3]) {
+    w[0] = w[1] = w[2] = 0;
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+        if (NL == 1) {
+            w[0] |= ((uint32_t)(nonzero ? quant_one(v[e], inv) : 0) & 0xFFu) << (8 * e);
+        } else {
+            uint32_t h, m, lo;
+            fixed_limbs(v[e], sh_or_unused, h, m, lo);
+            w[0] |= h << (8 * e);
+            w[1] |= m << (8 * e);
+            w[2] |= lo << (8 * e);
+        }
+    }
+}
+
+// ------------------------------------------------------------------ the kernel
 template <int NL>
 __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_constant__ StackParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t mb_router, mb_gu, mb_dn;
-    __shared__ double s_red[32];
-    __shared__ float s_redf[32];
+    __shared__ double s_red[kStackWarps];
+    __shared__ float s_redf[kStackWarps];
     __shared__ double s_part[kStackWarps][kStackWarps];
-    __shared__ double s_logit[1024];
+    __shared__ double s_logit[256];
     __shared__ int s_idx[kSK];
     __shared__ double s_gate[kSK];
     __shared__ int s_hshift[kSK];
     __shared__ float s_hscale[kSK];
+    __shared__ unsigned int s_hmax[kSK];
+    __shared__ long long s_S[64][2];
     __shared__ double s_ye[64][kSK];
     __shared__ float s_sg[64], s_su[64], s_sd[kSK * 64];
-    __shared__ unsigned int s_hmax[kSK];
-    __shared__ int s_ok;
-    __shared__ double s_r;
-    __shared__ float s_nscale;  // int8: s_x ; bf16: shift as int bits
 
     const int d = p.d, f = p.f, E = p.E, k = p.k, P = p.P;
     const int c = blockIdx.x;
@@ -221,13 +234,13 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
     const int hlp = (f / 64) * kSegPad;  // padded words per limb of one slot's h
 
     // static shares of this CTA
-    const int nr = (E - c + P - 1) / P;                        // router rows: c, c+P, ...
+    const int nr = (E - c + P - 1) / P;  // router rows: c, c+P, ...
     const int NPt = k * f;
     const int p0 = (int)((long long)c * NPt / P), p1 = (int)((long long)(c + 1) * NPt / P);
-    const int i0 = (int)((long long)c * d / P), i1 = (int)((long long)(c + 1) * d / P);
+    const int i0 = 2 * (int)((long long)c * (d / 2) / P), i1 = 2 * (int)((long long)(c + 1) * (d / 2) / P);
     const int nrows = i1 - i0;
     const long long lim = p.limit_ns;
-    unsigned int bar_target = 0;
+    const uint32_t ep = ld_acquire_gpu(p.ctl + 1);  // launch epoch, advanced by the previous launch
     bool alive = true;
     unsigned int n_rt = 0, n_gu = 0, n_dn = 0;  // phases issued per mbarrier (thread 0)
 
@@ -243,8 +256,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
         fence_mbar_init();
     }
     __syncthreads();
-    // router rows of layer 0
-    if (tid == 0 && nr > 0) {
+    if (tid == 0 && nr > 0) {  // router rows of layer 0
         mbar_expect_tx(&mb_router, (uint32_t)(nr * d * 2));
         n_rt++;
         for (int r = 0; r < nr; r++)
@@ -254,44 +266,89 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
     for (int l = 0; l < p.n_layers && alive; l++) {
         const StackLayerDev &Ly = p.layer[l];
         const uint32_t par = (uint32_t)(l & 1);
-        const uint16_t *xin = (l == 0) ? p.x : p.hist + (size_t)l * d;
-        // ---------------------------------------------------------------- A: norm + router
+        const uint32_t tag = (ep << 7) | (uint32_t)(l + 1);  // never 0 (a zeroed workspace holds 0)
         TSTAMP(l, 0)
-        double ss = 0.0;
-        for (int i4 = tid; i4 < d / 4; i4 += kStackThreads) {
-            const uint2 v4 = __ldcg(reinterpret_cast<const uint2 *>(xin) + i4);
-            reinterpret_cast<uint2 *>(xs)[i4] = v4;
-            const uint16_t bb[4] = {(uint16_t)(v4.x & 0xFFFFu), (uint16_t)(v4.x >> 16), (uint16_t)(v4.y & 0xFFFFu),
-                                    (uint16_t)(v4.y >> 16)};
+        // ------------------------------------------------------------ A: x_l, norm, limbs
+        // thread t owns elements 4t..4t+3 (d = 2048 = 4 * 512)
+        float xv[4];
+        {
+            bool ok = true;
+            uint32_t pr[2] = {0, 0};
+            if (l == 0) {
+                const uint2 v4 = __ldcg(reinterpret_cast<const uint2 *>(p.x) + tid);
+                pr[0] = v4.x;
+                pr[1] = v4.y;
+            } else {
+                ok = ll_poll<2>(p.xll + 2 * tid, 2, tag, pr, lim, p.status);
+            }
+            alive = __syncthreads_and(ok ? 1 : 0) && alive;
+            reinterpret_cast<uint2 *>(xs)[tid] = make_uint2(pr[0], pr[1]);
+            xv[0] = bf16_to_f32((uint16_t)(pr[0] & 0xFFFFu));
+            xv[1] = bf16_to_f32((uint16_t)(pr[0] >> 16));
+            xv[2] = bf16_to_f32((uint16_t)(pr[1] & 0xFFFFu));
+            xv[3] = bf16_to_f32((uint16_t)(pr[1] >> 16));
+        }
+        TSTAMP(l, 1)
+        if (l == 0 && c == 0) reinterpret_cast<uint2 *>(p.hist)[tid] = reinterpret_cast<const uint2 *>(xs)[tid];
+        double r;
+        float amax_n;
+        {
+            double ss = 0.0;
+            float am = 0.0f;
 #pragma unroll
             for (int e = 0; e < 4; e++) {
-                const double v = (double)bf16_to_f32(bb[e]);
+                const double v = (double)xv[e];
                 ss = fma(v, v, ss);
+                am = fmaxf(am, fabsf(xv[e]));
+            }
+            ss = warp_sum_f64(ss);
+            am = warp_max_f32(am);
+            if (lane == 0) {
+                s_red[warp] = ss;
+                s_redf[warp] = am;
+            }
+            __syncthreads();
+            // every thread folds the 16 warp partials in the same order: same r everywhere
+            double ts = 0.0;
+            float ta = 0.0f;
+#pragma unroll
+            for (int w = 0; w < kStackWarps; w++) {
+                ts += s_red[w];
+                ta = fmaxf(ta, s_redf[w]);
+            }
+            r = sqrt(ts / (double)d + p.eps);
+            // rounding is monotone, so max |bf16(x_k / r)| = bf16(max |x_k| / r)
+            amax_n = bf16_to_f32(f64_to_bf16_rne((double)ta / r));
+        }
+        const float s_nq = (NL == 1) ? (amax_n > 0.0f ? __fdiv_rn(amax_n, 127.0f) : 0.0f) : 0.0f;
+        const int sh_n = (NL == 1) ? 0 : fixed_shift(amax_n);
+        {
+            float nv[4];
+            uint16_t nb[4];
+#pragma unroll
+            for (int e = 0; e < 4; e++) {
+                nb[e] = f64_to_bf16_rne((double)xv[e] / r);
+                nv[e] = bf16_to_f32(nb[e]);
+            }
+            reinterpret_cast<uint2 *>(ns)[tid] =
+                make_uint2((uint32_t)nb[0] | ((uint32_t)nb[1] << 16), (uint32_t)nb[2] | ((uint32_t)nb[3] << 16));
+            uint32_t w[3];
+            const float inv = (NL == 1 && amax_n > 0.0f) ? quant_inv(amax_n) : 0.0f;
+            limb_words<NL>(nv, sh_n, inv, amax_n > 0.0f, w);
+            const int pw = padded_word(tid);
+            xl[pw] = w[0];
+            if (NL > 1) {
+                xl[xlp + pw] = w[1];
+                xl[2 * xlp + pw] = w[2];
             }
         }
-        ss = block_sum_f64(ss, s_red);
-        if (tid == 0) s_r = sqrt(ss / (double)d + p.eps);
-        if (l == 0 && c == 0)
-            for (int i = tid; i < d; i += kStackThreads) p.hist[i] = xs[i];
         __syncthreads();
-        const double r = s_r;
-        float amax = 0.0f;
-        for (int i = tid; i < d; i += kStackThreads) {
-            const uint16_t nb = f64_to_bf16_rne((double)bf16_to_f32(xs[i]) / r);
-            ns[i] = nb;
-            amax = fmaxf(amax, fabsf(bf16_to_f32(nb)));
-        }
-        amax = block_max_nonneg(amax, s_redf);
-        TSTAMP(l, 1)
-        if (tid == 0) {
-            if (NL == 1) s_nscale = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
-            else s_nscale = __int_as_float(fixed_shift(amax));
-        }
+        TSTAMP(l, 2)
         // router rows (prefetched): each row split over kStackWarps / rb_rows warps
         if (nr > 0) {
             const bool okw = mbar_wait(&mb_router, par, lim, p.status);
             alive = __syncthreads_and(okw ? 1 : 0) && alive;
-            const int wpr = kStackWarps / p.rb_rows;  // warps per row (rb_rows <= 16)
+            const int wpr = kStackWarps / p.rb_rows;
             const int rr = warp / wpr, part = warp % wpr;
             double acc = 0.0;
             if (rr < nr) {
@@ -305,110 +362,90 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             if (lane == 0 && rr < nr) s_part[rr][part] = acc;
             __syncthreads();
             if (tid < nr) {
-                double s = 0.0;
-                for (int q = 0; q < wpr; q++) s += s_part[tid][q];
-                p.logits[c + tid * P] = s;
+                double sum = 0.0;
+                for (int q = 0; q < wpr; q++) sum += s_part[tid][q];
+                const unsigned long long b = (unsigned long long)__double_as_longlong(sum);
+                const int e = c + tid * P;
+                ll_store(p.lll + 2 * e, (uint32_t)(b >> 32), tag);
+                ll_store(p.lll + 2 * e + 1, (uint32_t)b, tag);
             }
         }
+        TSTAMP(l, 3)
         __syncthreads();
-        // prefetch the next layer's router rows into the now free buffer
-        if (tid == 0 && nr > 0 && l + 1 < p.n_layers) {
+        if (tid == 0 && nr > 0 && l + 1 < p.n_layers) {  // next layer's router rows
             mbar_expect_tx(&mb_router, (uint32_t)(nr * d * 2));
             n_rt++;
             for (int q = 0; q < nr; q++)
                 bulk_g2s(rbuf + (size_t)q * d, p.layer[l + 1].router + (size_t)(c + q * P) * d, (uint32_t)(d * 2),
                          &mb_router);
         }
-        TSTAMP(l, 2)
-        bar_target += (unsigned)P;
-        if (!stack_grid_sync(p.bar, bar_target, lim, p.status, &s_ok) || !alive) {
-            alive = false;
-            break;
-        }
-        // ---------------------------------------------------------------- B: top-k, issue copies
-        TSTAMP(l, 3)
-        for (int e = tid; e < E; e += kStackThreads) s_logit[e] = __ldcg(p.logits + e);
-        __syncthreads();
-        if (warp == 0) {
-            if (E <= 256) warp_topk<8>(s_logit, E, k, s_idx, s_gate, nullptr);
-            else warp_topk<32>(s_logit, E, k, s_idx, s_gate, nullptr);
-            __syncwarp();
-            if (lane == 0 && c == 0)
-                for (int q = 0; q < k; q++) {
-                    p.idx_hist[l * k + q] = s_idx[q];
-                    p.gate_hist[l * k + q] = s_gate[q];
-                }
-        }
-        __syncthreads();
-        TSTAMP(l, 4)
-        if (tid == 0) {
-            // gate/up rows of this CTA's (slot,row) pairs, then its down rows for every slot
-            const uint32_t rowb = (uint32_t)(d / 4);
-            mbar_expect_tx(&mb_gu, (uint32_t)(2 * (p1 - p0)) * rowb);
-            n_gu++;
-            int q = 0;
-            for (int pp = p0; pp < p1;) {
-                const int s = pp / f, j = pp % f;
-                const int cnt = min(p1 - pp, f - j);
-                const size_t src = ((size_t)s_idx[s] * f + j) * rowb;
-                bulk_g2s(gbuf + (size_t)q * rowb, Ly.gate + src, (uint32_t)cnt * rowb, &mb_gu);
-                bulk_g2s(ubuf + (size_t)q * rowb, Ly.up + src, (uint32_t)cnt * rowb, &mb_gu);
-                q += cnt;
-                pp += cnt;
-            }
-            const uint32_t rowd = (uint32_t)(f / 4);
-            mbar_expect_tx(&mb_dn, (uint32_t)(k * nrows) * rowd);
-            n_dn++;
-            for (int s = 0; s < k; s++)
-                bulk_g2s(dbuf + (size_t)s * p.dn_rows * rowd, Ly.down + ((size_t)s_idx[s] * d + i0) * rowd,
-                         (uint32_t)nrows * rowd, &mb_dn);
-        }
-        TSTAMP(l, 5)
-        // per-row scales of this CTA's rows, fetched while the weight copies are in flight
-        for (int q = tid; q < p1 - p0; q += kStackThreads) {
-            const int pp = p0 + q, s2 = pp / f, j = pp % f;
-            const size_t o = (size_t)s_idx[s2] * f + j;
-            s_sg[q] = __ldg(Ly.sg + o);
-            s_su[q] = __ldg(Ly.su + o);
-        }
-        for (int q = tid; q < k * nrows; q += kStackThreads)
-            s_sd[q] = __ldg(Ly.sd + (size_t)s_idx[q / nrows] * d + i0 + q % nrows);
-        TSTAMP(l, 6)
-        // activation limbs of n: one word (4 elements) per thread into the padded layout,
-        // then every lane loads the limbs of its segment (G = d/64 lanes per row)
-        {
-            const int sh = __float_as_int(s_nscale);
-            const float inv = (NL == 1 && amax > 0.0f) ? quant_inv(amax) : 0.0f;
-            for (int w = tid; w < d / 4; w += kStackThreads) {
-                const uint2 v4 = reinterpret_cast<const uint2 *>(ns)[w];
-                const uint16_t bb[4] = {(uint16_t)(v4.x & 0xFFFFu), (uint16_t)(v4.x >> 16), (uint16_t)(v4.y & 0xFFFFu),
-                                        (uint16_t)(v4.y >> 16)};
-                uint32_t w0 = 0, w1 = 0, w2 = 0;
-#pragma unroll
-                for (int e = 0; e < 4; e++) {
-                    const float v = bf16_to_f32(bb[e]);
-                    if (NL == 1) {
-                        w0 |= ((uint32_t)(amax > 0.0f ? quant_one(v, inv) : 0) & 0xFFu) << (8 * e);
-                    } else {
-                        uint32_t h, m, lo;
-                        fixed_limbs(v, sh, h, m, lo);
-                        w0 |= h << (8 * e);
-                        w1 |= m << (8 * e);
-                        w2 |= lo << (8 * e);
-                    }
-                }
-                const int pw = padded_word(w);
-                xl[pw] = w0;
-                if (NL > 1) {
-                    xl[xlp + pw] = w1;
-                    xl[2 * xlp + pw] = w2;
-                }
-            }
-        }
-        __syncthreads();
+        // activation limbs of this lane's segment, for phase C (G = d/64 = 32 lanes per row)
         SegX<NL> X;
         seg_load_x_padded<NL>(X, xl, xlp, lane % (d / 64));
-        // ---------------------------------------------------------------- C: gate/up -> h
+        // ------------------------------------------------------------ B: logits, top-k, copies
+        {
+            bool ok = true;
+            if (tid < E) {
+                uint32_t lw[2];
+                ok = ll_poll<2>(p.lll + 2 * tid, 2, tag, lw, lim, p.status);
+                s_logit[tid] = __longlong_as_double((long long)(((unsigned long long)lw[0] << 32) | lw[1]));
+            }
+            for (int e = tid + kStackThreads; e < E; e += kStackThreads) {
+                uint32_t lw[2];
+                ok = ll_poll<2>(p.lll + 2 * e, 2, tag, lw, lim, p.status) && ok;
+                s_logit[e] = __longlong_as_double((long long)(((unsigned long long)lw[0] << 32) | lw[1]));
+            }
+            alive = __syncthreads_and(ok ? 1 : 0) && alive;
+        }
+        TSTAMP(l, 4)
+        if (warp == 0) warp_topk<8>(s_logit, E, k, s_idx, s_gate, nullptr);  // E <= 256 on this path
+        __syncthreads();
+        TSTAMP(l, 5)
+        if (warp == 0) {
+            // copies: lanes 0..3 gate/up segments (<= 2 slots x 2 matrices), lanes 4.. down rows
+            const uint32_t rowb = (uint32_t)(d / 4), rowd = (uint32_t)(f / 4);
+            if (lane == 0) {
+                mbar_expect_tx(&mb_gu, (uint32_t)(2 * (p1 - p0)) * rowb);
+                mbar_expect_tx(&mb_dn, (uint32_t)(k * nrows) * rowd);
+                n_gu++;
+                n_dn++;
+                if (c == 0)
+                    for (int q = 0; q < k; q++) {
+                        p.idx_hist[l * k + q] = s_idx[q];
+                        p.gate_hist[l * k + q] = s_gate[q];
+                    }
+            }
+            __syncwarp();
+            if (lane < 4) {
+                const int seg = lane >> 1;
+                const int s0 = p0 / f;
+                const int e0 = min(p1, (s0 + 1) * f);
+                const int a = seg == 0 ? p0 : e0, b = seg == 0 ? e0 : p1;
+                if (b > a) {
+                    const int s = a / f, j = a % f;
+                    const size_t src = ((size_t)s_idx[s] * f + j) * rowb;
+                    const int q0 = a - p0;
+                    if (lane & 1) bulk_g2s(ubuf + (size_t)q0 * rowb, Ly.up + src, (uint32_t)(b - a) * rowb, &mb_gu);
+                    else bulk_g2s(gbuf + (size_t)q0 * rowb, Ly.gate + src, (uint32_t)(b - a) * rowb, &mb_gu);
+                }
+            } else if (lane < 4 + k && nrows > 0) {
+                const int s = lane - 4;
+                bulk_g2s(dbuf + (size_t)s * p.dn_rows * rowd, Ly.down + ((size_t)s_idx[s] * d + i0) * rowd,
+                         (uint32_t)nrows * rowd, &mb_dn);
+            }
+        } else {
+            // per-row scales of this CTA's rows, fetched while the copies are in flight
+            for (int q = tid - 32; q < p1 - p0; q += kStackThreads - 32) {
+                const int pp = p0 + q, s2 = pp / f, j = pp % f;
+                const size_t o = (size_t)s_idx[s2] * f + j;
+                s_sg[q] = __ldg(Ly.sg + o);
+                s_su[q] = __ldg(Ly.su + o);
+            }
+            for (int q = tid - 32; q < k * nrows; q += kStackThreads - 32)
+                s_sd[q] = __ldg(Ly.sd + (size_t)s_idx[q / nrows] * d + i0 + q % nrows);
+        }
+        TSTAMP(l, 6)
+        // ------------------------------------------------------------ C: gate/up -> h
         if (p1 > p0) {
             const bool okw = mbar_wait(&mb_gu, par, lim, p.status);
             alive = __syncthreads_and(okw ? 1 : 0) && alive;
@@ -416,7 +453,6 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             const uint32_t *lut_lane = lut + lane;
             const int rowb = d / 4;
             for (int q = warp; q < p1 - p0; q += kStackWarps) {
-                const int pp = p0 + q, s = pp / f, j = pp % f;
                 const uint4 wg = *reinterpret_cast<const uint4 *>(gbuf + (size_t)q * rowb + lane * 16);
                 const uint4 wu = *reinterpret_cast<const uint4 *>(ubuf + (size_t)q * rowb + lane * 16);
                 int ag[NL], au[NL];
@@ -434,91 +470,80 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                     ub = group_sum<32>(ub);
                 }
                 if (lane == 0) {
-                    const long long Sg = pair_value(NL, ga, gb2), Su = pair_value(NL, ua, ub);
-                    const float sg = s_sg[q], su = s_su[q];
-                    float hv;
-                    if (NL == 1) {
-                        const float gv = __fmul_rn(__fmul_rn(__int2float_rn((int)Sg), sg), s_nscale);
-                        const float uv = __fmul_rn(__fmul_rn(__int2float_rn((int)Su), su), s_nscale);
-                        hv = swiglu_f32((double)gv, (double)uv);
-                    } else {
-                        const int sh = __float_as_int(s_nscale);
-                        hv = swiglu_f32(ldexp((double)Sg, -sh) * (double)sg, ldexp((double)Su, -sh) * (double)su);
-                    }
-                    p.H[(size_t)s * f + j] = hv;
+                    s_S[q][0] = pair_value(NL, ga, gb2);
+                    s_S[q][1] = pair_value(NL, ua, ub);
                 }
             }
+            __syncthreads();
+            TSTAMP(l, 8)
+            // SwiGLU epilogue, one thread per row, fp64
+            if (tid < p1 - p0) {
+                const int q = tid, pp = p0 + q, s = pp / f, j = pp % f;
+                const long long Sg = s_S[q][0], Su = s_S[q][1];
+                float hv;
+                if (NL == 1) {
+                    const float gv = __fmul_rn(__fmul_rn(__int2float_rn((int)Sg), s_sg[q]), s_nq);
+                    const float uv = __fmul_rn(__fmul_rn(__int2float_rn((int)Su), s_su[q]), s_nq);
+                    hv = swiglu_f32((double)gv, (double)uv);
+                } else {
+                    hv = swiglu_f32(ldexp((double)Sg, -sh_n) * (double)s_sg[q], ldexp((double)Su, -sh_n) * (double)s_su[q]);
+                }
+                ll_store(p.hll + (size_t)s * f + j, __float_as_uint(hv), tag);
+            }
         }
-        TSTAMP(l, 8)
-        bar_target += (unsigned)P;
-        if (!stack_grid_sync(p.bar, bar_target, lim, p.status, &s_ok) || !alive) {
-            alive = false;
-            break;
-        }
-        // ---------------------------------------------------------------- D: down + combine + residual
+        TSTAMP(l, 9)
+        // ------------------------------------------------------------ D: down, combine, residual
         {
-            // every slot's h, read once from L2; per-slot absmax via shared atomics
-            TSTAMP(l, 9)
-            const int wpl = f / 4;  // float4 (= limb words) per slot
-            constexpr int kMaxV = 8;
-            float4 hv[kMaxV];
-            if (tid < kSK) s_hmax[tid] = 0u;
+            // thread t owns h words [8t, 8t+8) (k*f = 4096 = 8 * 512): two limb words
+            constexpr int HW = 8;
+            float hv[HW];
+            bool ok = true;
+            const int w0 = HW * tid;
+            if (tid < k) s_hmax[tid] = 0u;
             __syncthreads();
+            if (w0 < k * f) {
+                uint32_t hw[HW];
+                ok = ll_poll<HW>(p.hll + w0, HW, tag, hw, lim, p.status);
+                float m = 0.0f;
 #pragma unroll
-            for (int j = 0; j < kMaxV; j++) {
-                const int w = tid + j * kStackThreads;
-                if (w < k * wpl) {
-                    hv[j] = __ldcg(reinterpret_cast<const float4 *>(p.H) + w);
-                    const float m4 = fmaxf(fmaxf(fabsf(hv[j].x), fabsf(hv[j].y)), fmaxf(fabsf(hv[j].z), fabsf(hv[j].w)));
-                    atomicMax(&s_hmax[w / wpl], __float_as_uint(m4));
+                for (int i = 0; i < HW; i++) {
+                    hv[i] = __uint_as_float(hw[i]);
+                    m = fmaxf(m, fabsf(hv[i]));
                 }
+                atomicMax(&s_hmax[w0 / f], __float_as_uint(m));  // 8 consecutive words share a slot (f % 8 == 0)
             }
-            __syncthreads();
-            if (tid < k) {
-                const float a = __uint_as_float(s_hmax[tid]);
-                if (NL == 1) {
-                    s_hscale[tid] = a > 0.0f ? __fdiv_rn(a, 127.0f) : 0.0f;
-                    s_hshift[tid] = __float_as_int(a);  // keep absmax for the quantiser
-                } else {
-                    s_hshift[tid] = fixed_shift(a);
-                }
-            }
-            __syncthreads();
-#pragma unroll
-            for (int j = 0; j < kMaxV; j++) {
-                const int w = tid + j * kStackThreads;
-                if (w >= k * wpl) continue;
-                const int ss2 = w / wpl, b = w % wpl;
-                const float vv[4] = {hv[j].x, hv[j].y, hv[j].z, hv[j].w};
-                uint32_t w0 = 0, w1 = 0, w2 = 0;
-                if (NL == 1) {
-                    const float a = __int_as_float(s_hshift[ss2]);
-                    const float inv = a > 0.0f ? quant_inv(a) : 0.0f;
-#pragma unroll
-                    for (int e = 0; e < 4; e++) w0 |= ((uint32_t)(a > 0.0f ? quant_one(vv[e], inv) : 0) & 0xFFu) << (8 * e);
-                    hl[(size_t)ss2 * hlp + padded_word(b)] = w0;
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 4; e++) {
-                        uint32_t h, mi, lo;
-                        fixed_limbs(vv[e], s_hshift[ss2], h, mi, lo);
-                        w0 |= h << (8 * e);
-                        w1 |= mi << (8 * e);
-                        w2 |= lo << (8 * e);
-                    }
-                    hl[((size_t)ss2 * NL + 0) * hlp + padded_word(b)] = w0;
-                    hl[((size_t)ss2 * NL + (NL > 1 ? 1 : 0)) * hlp + padded_word(b)] = w1;
-                    hl[((size_t)ss2 * NL + (NL > 2 ? 2 : 0)) * hlp + padded_word(b)] = w2;
-                }
-            }
-            __syncthreads();
+            alive = __syncthreads_and(ok ? 1 : 0) && alive;
             TSTAMP(l, 10)
+            if (w0 < k * f) {
+                const int s = w0 / f;
+                const float a = __uint_as_float(s_hmax[s]);
+                const int sh = (NL == 1) ? 0 : fixed_shift(a);
+                const float inv = (NL == 1 && a > 0.0f) ? quant_inv(a) : 0.0f;
+                if ((w0 % f) == 0) {
+                    s_hshift[s] = sh;
+                    s_hscale[s] = (NL == 1 && a > 0.0f) ? __fdiv_rn(a, 127.0f) : 0.0f;
+                }
+#pragma unroll
+                for (int g = 0; g < 2; g++) {
+                    const float v4[4] = {hv[4 * g], hv[4 * g + 1], hv[4 * g + 2], hv[4 * g + 3]};
+                    uint32_t w[3];
+                    limb_words<NL>(v4, sh, inv, a > 0.0f, w);
+                    const int b = (w0 % f) / 4 + g;  // limb word within the slot
+                    hl[((size_t)s * NL + 0) * hlp + padded_word(b)] = w[0];
+                    if (NL > 1) {
+                        hl[((size_t)s * NL + 1) * hlp + padded_word(b)] = w[1];
+                        hl[((size_t)s * NL + 2) * hlp + padded_word(b)] = w[2];
+                    }
+                }
+            }
+            __syncthreads();
+            TSTAMP(l, 11)
             if (nrows > 0) {
                 const bool okw = mbar_wait(&mb_dn, par, lim, p.status);
                 alive = __syncthreads_and(okw ? 1 : 0) && alive;
             }
-            TSTAMP(l, 11)
-            // (row, slot) pairs, G = f/64 lanes each; 512-wide rows -> 8 lanes, 4 pairs per warp pass
+            TSTAMP(l, 12)
+            // (row, slot) pairs, G = f/64 lanes each (8 for f = 512): 4 pairs per warp pass
             const int G = f / 64;
             const int ppw = 32 / G;
             const int sub = lane / G, gl = lane % G;
@@ -537,7 +562,6 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                 seg_dot<NL>(wd, Hx, lut_lane, acc);
                 int a, b;
                 acc_to_pair<NL>(acc, a, b);
-                // reduce within the G lanes of this pair (G = 8 for f = 512)
                 for (int o = G / 2; o > 0; o >>= 1) {
                     a += __shfl_xor_sync(0xFFFFFFFFu, a, o);
                     if (NL > 1) b += __shfl_xor_sync(0xFFFFFFFFu, b, o);
@@ -552,25 +576,25 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                 }
             }
             __syncthreads();
-            TSTAMP(l, 12)
+            TSTAMP(l, 13)
             const bool last = (l + 1 == p.n_layers);
+            // one output row per thread, fixed top-k order; row pairs leave as one word
+            uint16_t xo = 0;
             if (tid < nrows) {
                 double y = 0.0;
                 for (int q = 0; q < k; q++) y += s_gate[q] * s_ye[tid][q];
                 const uint16_t yb = f64_to_bf16_rne(y);
+                xo = f64_to_bf16_rne((double)bf16_to_f32(xs[i0 + tid]) + (double)bf16_to_f32(yb));
+            }
+            const uint32_t other = __shfl_down_sync(0xFFFFFFFFu, (uint32_t)xo, 1);
+            if (tid < nrows && (tid & 1) == 0) {
+                const uint32_t pr = (uint32_t)xo | (other << 16);
                 const int i = i0 + tid;
-                const uint16_t xo = f64_to_bf16_rne((double)bf16_to_f32(xs[i]) + (double)bf16_to_f32(yb));
-                p.hist[(size_t)(l + 1) * d + i] = xo;
-                if (last) p.x[i] = xo;
+                reinterpret_cast<uint32_t *>(p.hist + (size_t)(l + 1) * d)[i / 2] = pr;
+                if (last) reinterpret_cast<uint32_t *>(p.x)[i / 2] = pr;
+                else ll_store(p.xll + i / 2, pr, (ep << 7) | (uint32_t)(l + 2));
             }
-            TSTAMP(l, 13)
-            if (!last) {
-                bar_target += (unsigned)P;
-                if (!stack_grid_sync(p.bar, bar_target, lim, p.status, &s_ok) || !alive) {
-                    alive = false;
-                    break;
-                }
-            }
+            TSTAMP(l, 14)
         }
     }
 #undef TSTAMP
@@ -580,14 +604,14 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
         if (n_gu) mbar_wait(&mb_gu, (n_gu - 1) & 1u, lim, p.status);
         if (n_dn) mbar_wait(&mb_dn, (n_dn - 1) & 1u, lim, p.status);
     }
-    // leave: the last CTA out resets the barrier counters for the next launch
+    // leave: the last CTA out advances the launch epoch (the next launch's tags differ)
     __syncthreads();
     if (tid == 0) {
         __threadfence();
-        const unsigned int n = atomicAdd(p.bar + 1, 1u);
+        const unsigned int n = atomicAdd(p.ctl, 1u);
         if (n == (unsigned)P - 1) {
-            atomicExch(p.bar + 0, 0u);
-            atomicExch(p.bar + 1, 0u);
+            atomicExch(p.ctl, 0u);
+            atomicAdd(p.ctl + 1, 1u);
         }
     }
 }
@@ -596,7 +620,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
 // Persistent-path workspace: barrier words, logits [E], H [k][f], x history
 // [(kMaxStackLayers+1)][d], routing history [kMaxStackLayers][k] (int32 + fp64).
 struct StackWs {
-    int64_t bar, logits, H, hist, idx_hist, gate_hist, ttrace, total;
+    int64_t ctl, xll, lll, hll, hist, idx_hist, gate_hist, ttrace, total;
 };
 
 static inline int64_t up256_(int64_t v) { return (v + 255) & ~int64_t(255); }
@@ -609,9 +633,10 @@ static StackWs stack_ws_layout(const tern_moe_layer *L0) {
         p = up256_(p + b);
         return r;
     };
-    o.bar = take(256);
-    o.logits = take((int64_t)L0->E * 8);
-    o.H = take((int64_t)L0->k * L0->f * 4);
+    o.ctl = take(256);
+    o.xll = take((int64_t)L0->d / 2 * 8);
+    o.lll = take((int64_t)L0->E * 2 * 8);
+    o.hll = take((int64_t)L0->k * L0->f * 8);
     o.hist = take((int64_t)(kMaxStackLayers + 1) * L0->d * 2);
     o.idx_hist = take((int64_t)kMaxStackLayers * L0->k * 4);
     o.gate_hist = take((int64_t)kMaxStackLayers * L0->k * 8);
@@ -653,8 +678,11 @@ static tern_status stack_plan(const tern_moe_layer &L0, int n_layers, tern_act a
     if (pl.P > kMaxTraceCtas) pl.P = kMaxTraceCtas;
     pl.rb_rows = (L0.E + pl.P - 1) / pl.P;
     pl.gu_pairs = (int)((L0.k * L0.f + pl.P - 1) / pl.P);
-    pl.dn_rows = (int)((L0.d + pl.P - 1) / pl.P);
-    if (pl.rb_rows > kStackWarps || pl.dn_rows > 64 || pl.gu_pairs > 64 || L0.k * L0.f > 8 * 4 * kStackThreads)
+    pl.dn_rows = 2 * (int)((L0.d / 2 + pl.P - 1) / pl.P);
+    // the thread mappings assume d = 4 * threads and k * f = 8 * threads at most, and a CTA's
+    // gate/up pairs spanning at most two slots
+    if (pl.rb_rows > kStackWarps || pl.dn_rows > 64 || pl.gu_pairs > 64 || pl.gu_pairs > L0.f ||
+        L0.k * L0.f > 8 * kStackThreads || (L0.k * L0.f) % 8 || L0.d != 4 * kStackThreads || L0.E > 256)
         return TERN_EUNSUPPORTED;
     const int NL = act == TERN_ACT_INT8 ? 1 : 3;
     pl.sm = smem_map((int)L0.d, (int)L0.f, L0.k, pl.rb_rows, pl.gu_pairs, pl.dn_rows, NL);
@@ -703,13 +731,16 @@ tern_status launch_stack_persistent(const tern_moe_layer *layers, int n_layers, 
     prm.k = L0.k;
     prm.eps = (double)eps;
     prm.x = x;
-    prm.bar = reinterpret_cast<unsigned int *>(b + o.bar);
-    prm.logits = reinterpret_cast<double *>(b + o.logits);
-    prm.H = reinterpret_cast<float *>(b + o.H);
+    prm.ctl = reinterpret_cast<unsigned int *>(b + o.ctl);
+    prm.xll = reinterpret_cast<unsigned long long *>(b + o.xll);
+    prm.lll = reinterpret_cast<unsigned long long *>(b + o.lll);
+    prm.hll = reinterpret_cast<unsigned long long *>(b + o.hll);
     prm.hist = reinterpret_cast<uint16_t *>(b + o.hist);
     prm.idx_hist = reinterpret_cast<int32_t *>(b + o.idx_hist);
     prm.gate_hist = reinterpret_cast<double *>(b + o.gate_hist);
-    prm.ttrace = reinterpret_cast<unsigned long long *>(b + o.ttrace);
+    // phase stamps cost a %globaltimer read and a store each: only when TERNMOE_TRACE=1
+    const char *tenv = getenv("TERNMOE_TRACE");
+    prm.ttrace = (tenv && tenv[0] == '1') ? reinterpret_cast<unsigned long long *>(b + o.ttrace) : nullptr;
     prm.status = status;
     prm.limit_ns = 1000000000ll;  // every in-kernel wait gives up after one second
     prm.P = P;

@@ -35,35 +35,17 @@ __device__ __forceinline__ void set_status(int *st, int code) {
 // ---------------------------------------------------------------------------- bf16 / fp64
 __device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 
-// nearest bf16 (ties to even) of a finite double, directly from the fp64 bits
+// Nearest bf16 (ties to even) of a double.  Two roundings are exact here when the first is
+// round-to-odd and keeps at least two more bits than the second (fp32 keeps 16 more than
+// bf16): truncate to fp32, set the last fp32 bit if anything was cut off (round to odd),
+// then round the fp32 value to nearest-even bf16 with an integer add.  Finite inputs of any
+// magnitude below fp32 overflow (values that would round past bf16 max become inf).
 __device__ __forceinline__ uint16_t f64_to_bf16_rne(double v) {
-    unsigned long long u = (unsigned long long)__double_as_longlong(v);
-    const uint32_t sign = (uint32_t)(u >> 63) << 15;
-    u &= 0x7FFFFFFFFFFFFFFFull;
-    if (u == 0) return (uint16_t)sign;
-    int e = (int)(u >> 52) - 1023;            // unbiased exponent (inputs are normal fp64)
-    unsigned long long m = (u & 0xFFFFFFFFFFFFFull) | (1ull << 52);  // 53-bit significand
-    int keep;                                  // significand bits kept in bf16 at this exponent
-    if (e >= -126) keep = 8;
-    else keep = 8 - (-126 - e);                // bf16 subnormal range
-    if (keep <= 0) {
-        // below half the smallest subnormal (or exactly half: ties to even -> 0)
-        if (keep == 0 && m > (1ull << 52)) return (uint16_t)(sign | 1);
-        return (uint16_t)sign;
-    }
-    const int drop = 53 - keep;
-    unsigned long long q = m >> drop;
-    const unsigned long long rem = m & ((1ull << drop) - 1);
-    const unsigned long long half = 1ull << (drop - 1);
-    if (rem > half || (rem == half && (q & 1))) q++;
-    // q has `keep` (or keep+1 after carry) significant bits; rebuild the bf16 value
-    if (e >= -126) {
-        if (q == (1ull << 8)) { q >>= 1; e++; }
-        if (e > 127) return (uint16_t)(sign | 0x7F80u);
-        return (uint16_t)(sign | ((uint32_t)(e + 127) << 7) | (uint32_t)(q & 0x7F));
-    }
-    // subnormal: value = q * 2^-133 ; if q reached 2^7 it becomes the smallest normal
-    return (uint16_t)(sign | (uint32_t)q);
+    float f = __double2float_rz(v);
+    if ((double)f != v) f = __uint_as_float(__float_as_uint(f) | 1u);
+    uint32_t u = __float_as_uint(f);
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
 }
 
 // ---------------------------------------------------------------------------- dp4a
@@ -270,35 +252,45 @@ __device__ __forceinline__ unsigned long long f64_order_key(double v) {
 template <int J>
 __device__ __forceinline__ void warp_topk(const double *lg, int E, int k, int32_t *idx_out, double *g64, float *g32) {
     const int lane = threadIdx.x & 31;
+    // each lane's J candidates, sorted once by (key desc, index asc) with a bubble network
     unsigned long long key[J];
+    int ix[J];
 #pragma unroll
     for (int j = 0; j < J; j++) {
         const int e = lane + 32 * j;
         key[j] = (e < E) ? f64_order_key(lg[e]) : 0ull;  // 0 = below every finite logit
+        ix[j] = e;
     }
+#pragma unroll
+    for (int a = 0; a < J; a++)
+#pragma unroll
+        for (int b = 0; b < J - 1 - a; b++)
+            if (key[b + 1] > key[b]) {  // strict: equal keys keep the lower index first
+                const unsigned long long tk = key[b];
+                key[b] = key[b + 1];
+                key[b + 1] = tk;
+                const int ti = ix[b];
+                ix[b] = ix[b + 1];
+                ix[b + 1] = ti;
+            }
     int sel_e = 0;
     for (int r = 0; r < k; r++) {
-        // lane-local best (largest key, then lowest index = lowest j)
-        unsigned long long bk = 0ull;
-        int bj = 0;
-#pragma unroll
-        for (int j = 0; j < J; j++)
-            if (key[j] > bk) {
-                bk = key[j];
-                bj = j;
-            }
+        const unsigned long long bk = key[0];
         const unsigned hi = (unsigned)(bk >> 32), lo = (unsigned)bk;
         const unsigned mhi = __reduce_max_sync(0xFFFFFFFFu, hi);
         const unsigned mlo = __reduce_max_sync(0xFFFFFFFFu, hi == mhi ? lo : 0u);
         const bool cand = (hi == mhi) && (lo == mlo);
-        const int e = lane + 32 * bj;
-        const unsigned wi = __reduce_min_sync(0xFFFFFFFFu, cand ? (unsigned)e : 0xFFFFFFFFu);
+        const unsigned wi = __reduce_min_sync(0xFFFFFFFFu, cand ? (unsigned)ix[0] : 0xFFFFFFFFu);
         int win = (int)wi;
         if (win < 0 || win >= E) win = r;  // NaN inputs must still not index out of range
-        if (win == e && cand) {
+        if (cand && ix[0] == win) {        // pop this lane's head
 #pragma unroll
-            for (int j = 0; j < J; j++)
-                if (j == bj) key[j] = 0ull;
+            for (int j = 0; j < J - 1; j++) {
+                key[j] = key[j + 1];
+                ix[j] = ix[j + 1];
+            }
+            key[J - 1] = 0ull;
+            ix[J - 1] = 0x7FFFFFFF;
         }
         if (lane == r) sel_e = win;
     }
