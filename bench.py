@@ -189,10 +189,13 @@ PHASES = [("x_wait", 0, 1), ("norm_limbs", 1, 2), ("router", 2, 3), ("logits_wai
           ("combine", 13, 14)]
 
 
-def phase_summary(tr):
-    """Median over CTAs and layers of each phase (us), the last-arrival -> first-departure
-    latency of the three grid barriers, and the mean layer time."""
-    d = lambda a, b: np.median((tr[:, :, b] - tr[:, :, a]).astype(np.float64)) / 1e3
+def phase_summary(tr, clk=None, mhz=1965.0):
+    """Median over CTAs and layers of each phase (us; from SM clock stamps when given, else
+    from %globaltimer), the exchange latencies, and the layer time."""
+    if clk is not None:
+        d = lambda a, b: np.median((clk[:, :, b] - clk[:, :, a]).astype(np.float64)) / mhz
+    else:
+        d = lambda a, b: np.median((tr[:, :, b] - tr[:, :, a]).astype(np.float64)) / 1e3
     out = {name: round(float(d(a, b)), 3) for name, a, b in PHASES}
     # exchange latency: last producer's publish -> first consumer's receipt
     e_log = np.median(tr[:, :, 4].min(1) - tr[:, :, 3].max(1)) / 1e3
@@ -337,11 +340,12 @@ def main():
     tm.moe_stack_decode(stack, xs[W:W + 1].clone(), act=act, ws=ws)
     torch.cuda.synchronize(dev)
     os.environ["TERNMOE_TRACE"] = "0"
-    tr = ws[lay["trace"]:lay["trace"] + N_LAYERS * P * 16 * 8].view(torch.int64).view(N_LAYERS, P, 16).cpu().numpy()
-    phases = phase_summary(tr) if launches == 1 else None
+    tr2 = ws[lay["trace"]:lay["trace"] + 2 * N_LAYERS * P * 16 * 8].view(torch.int64).view(2, N_LAYERS, P, 16).cpu().numpy()
+    tr = tr2[0]
+    phases = phase_summary(tr, tr2[1]) if launches == 1 else None
     try:
         os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-        np.save(os.path.join(ROOT, "gpurun_out", f"trace_{args.act}_rank{rank}.npy"), tr)
+        np.save(os.path.join(ROOT, "gpurun_out", f"trace_{args.act}_rank{rank}.npy"), tr2)
     except OSError:
         pass
 

@@ -180,9 +180,9 @@ tern_status moe_stack_decode(const tern_moe_layer *layers, int32_t n_layers, uin
  *   hist    uint16 [n_layers+1][d]  bf16 x entering each layer, and the final x;
  *   idx     int32  [n_layers][k]    experts chosen at each layer (descending logit);
  *   gates64 double [n_layers][k]    their renormalised gates;
- *   trace   uint64 [n_layers][P][16] %globaltimer (ns) stamped by each of the P CTAs (one per
- *           SM, P <= 256) at phase boundaries, written only when the environment variable
- *           TERNMOE_TRACE is "1" at the time of the call (the stamps cost time): 0 layer start, 1 x received, 2 n and limbs
+ *   trace   uint64 [2][n_layers][P][16]: %globaltimer (ns), then clock64 (SM cycles), stamped
+ *           by each of the P CTAs (one per SM, P <= 256) at phase boundaries, written only when
+ *           the environment variable TERNMOE_TRACE is "1" at the time of the call: 0 layer start, 1 x received, 2 n and limbs
  *           ready, 3 own logits published, 4 all logits received, 5 top-k done, 6 copies
  *           issued, 7 gate/up rows landed, 8 gate/up dots done, 9 h published, 10 all h
  *           received, 11 h limbs built, 12 down rows landed, 13 down dots done,

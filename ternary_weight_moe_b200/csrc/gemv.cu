@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const uint8_t *__
 
     lut_fill(lut);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const uint32_t *lut_lane = lut + lane;
+    const uint32_t lane4 = (uint32_t)lane << 2;
     const int slice = warp % NS;              // K slice of this warp
     const int rgroup = warp / NS;             // row group inside the CTA
     const int ngroups = kGemvWarps / NS;
@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const uint8_t *__
                 int acc[NL];
 #pragma unroll
                 for (int l = 0; l < NL; l++) acc[l] = 0;
-                seg_dot<NL>(wb, X, lut_lane, acc);
+                seg_dot<NL>(wb, X, lut, lane4, acc);
                 acc_to_pair<NL>(acc, a, b);
             }
             a = group_sum<G>(a);

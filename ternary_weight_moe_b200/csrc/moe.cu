@@ -234,7 +234,7 @@ __global__ void __launch_bounds__(kFfnWarps * 32) gateup_kernel(
     const uint8_t *G0 = gate + (int64_t)e * f * rowb;
     const uint8_t *U0 = up + (int64_t)e * f * rowb;
     const int r0 = blockIdx.y * rows_per_block;
-    const uint32_t *lut_lane = lut + lane;
+    const uint32_t lane4 = (uint32_t)lane << 2;
     for (int q = e0; q < e1; q++) {
         const int entry = ent[q];
         const int t = entry / k;
@@ -250,8 +250,8 @@ __global__ void __launch_bounds__(kFfnWarps * 32) gateup_kernel(
                 int ag[NL], au[NL];
 #pragma unroll
                 for (int l = 0; l < NL; l++) ag[l] = au[l] = 0;
-                seg_dot<NL>(wg, X, lut_lane, ag);
-                seg_dot<NL>(wu, X, lut_lane, au);
+                seg_dot<NL>(wg, X, lut, lane4, ag);
+                seg_dot<NL>(wu, X, lut, lane4, au);
                 acc_to_pair<NL>(ag, ga, gb);
                 acc_to_pair<NL>(au, ua, ub);
             }
@@ -303,7 +303,7 @@ __global__ void __launch_bounds__(kFfnWarps * 32) down_kernel(
     const int64_t rowb = f / 4;
     const uint8_t *D0 = down + (int64_t)e * d * rowb;
     const int r0 = blockIdx.y * rows_per_block;
-    const uint32_t *lut_lane = lut + lane;
+    const uint32_t lane4 = (uint32_t)lane << 2;
     for (int q = e0; q < e1; q++) {
         const int entry = ent[q];
         SegX<NL> X;
@@ -317,7 +317,7 @@ __global__ void __launch_bounds__(kFfnWarps * 32) down_kernel(
                 int acc[NL];
 #pragma unroll
                 for (int l = 0; l < NL; l++) acc[l] = 0;
-                seg_dot<NL>(wd, X, lut_lane, acc);
+                seg_dot<NL>(wd, X, lut, lane4, acc);
                 acc_to_pair<NL>(acc, a, b);
             }
             a = group_sum<G>(a);

@@ -57,7 +57,8 @@ struct StackParams {
     double *gate_hist;            // [n_layers][k]
     int *status;
     long long limit_ns;           // bound on every in-kernel wait
-    unsigned long long *ttrace;   // [n_layers][P][16] %globaltimer stamps of every CTA
+    unsigned long long *ttrace;   // [n_layers][P][16] %globaltimer stamps of every CTA, then
+                                  // [n_layers][P][16] clock64 stamps (SM cycles) at the same points
     int P;                        // CTAs
     int rb_rows;                  // max router rows per CTA
     int gu_pairs;                 // max gate/up pairs per CTA
@@ -119,16 +120,27 @@ __device__ __forceinline__ unsigned long long ll_load(const unsigned long long *
     return w;
 }
 // Poll n words p[0..n) (n <= 8) until every tag equals `tag`; payloads into out[].
-// False on timeout (status set).
-template <int N>
+// After a first direct read, each round issues two reads of every pending word spaced by
+// about half an L2 round trip, so a word that lands is seen after ~1/4 round trip on average
+// instead of ~1/2.  False on timeout (status set).
+template <int N, bool TWO = false>
 __device__ __forceinline__ bool ll_poll(const unsigned long long *p, int n, uint32_t tag, uint32_t (&out)[N],
                                         long long limit_ns, int *status) {
-    unsigned pending = (n >= 32) ? 0xFFFFFFFFu : ((1u << n) - 1u);
-    unsigned long long t0 = 0;
-    bool started = false;
-    while (true) {
+    unsigned pending = (1u << n) - 1u;
 #pragma unroll
-        for (int i = 0; i < N; i++) {
+    for (int i = 0; i < N; i++)
+        if (pending & (1u << i)) {
+            const unsigned long long w = ll_load(p + i);
+            if ((uint32_t)(w >> 32) == tag) {
+                out[i] = (uint32_t)w;
+                pending &= ~(1u << i);
+            }
+        }
+    if (!pending) return true;
+    const unsigned long long t0 = gtimer();
+    while (!TWO) {
+#pragma unroll
+        for (int i = 0; i < N; i++)
             if (pending & (1u << i)) {
                 const unsigned long long w = ll_load(p + i);
                 if ((uint32_t)(w >> 32) == tag) {
@@ -136,12 +148,34 @@ __device__ __forceinline__ bool ll_poll(const unsigned long long *p, int n, uint
                     pending &= ~(1u << i);
                 }
             }
-        }
         if (!pending) return true;
-        if (!started) {
-            t0 = gtimer();
-            started = true;
-        } else if ((long long)(gtimer() - t0) > limit_ns) {
+        if ((long long)(gtimer() - t0) > limit_ns) {
+            set_status(status, TERN_ETIMEOUT);
+            return false;
+        }
+    }
+    while (true) {
+        unsigned long long a[N], b[N];
+#pragma unroll
+        for (int i = 0; i < N; i++)
+            if (pending & (1u << i)) a[i] = ll_load(p + i);
+        __nanosleep(120);
+#pragma unroll
+        for (int i = 0; i < N; i++)
+            if (pending & (1u << i)) b[i] = ll_load(p + i);
+#pragma unroll
+        for (int i = 0; i < N; i++)
+            if (pending & (1u << i)) {
+                if ((uint32_t)(a[i] >> 32) == tag) {
+                    out[i] = (uint32_t)a[i];
+                    pending &= ~(1u << i);
+                } else if ((uint32_t)(b[i] >> 32) == tag) {
+                    out[i] = (uint32_t)b[i];
+                    pending &= ~(1u << i);
+                }
+            }
+        if (!pending) return true;
+        if ((long long)(gtimer() - t0) > limit_ns) {
             set_status(status, TERN_ETIMEOUT);
             return false;
         }
@@ -203,7 +237,7 @@ __device__ __forceinline__ void limb_words(const float (&v)[4], int sh_or_unused
 template <int NL>
 __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_constant__ StackParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
-    __shared__ __align__(8) uint64_t mb_router, mb_gu, mb_dn;
+    __shared__ __align__(8) uint64_t mb_router, mb_gu0, mb_gu1, mb_dn;
     __shared__ double s_red[kStackWarps];
     __shared__ float s_redf[kStackWarps];
     __shared__ double s_part[kStackWarps][kStackWarps];
@@ -243,15 +277,26 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
     const uint32_t ep = ld_acquire_gpu(p.ctl + 1);  // launch epoch, advanced by the previous launch
     bool alive = true;
     unsigned int n_rt = 0, n_gu = 0, n_dn = 0;  // phases issued per mbarrier (thread 0)
+    // gate/up pairs arrive in two halves (first 16 pairs, then the rest) so the dots of the
+    // first half overlap the second half's transfer
+    const int npairs = p1 - p0;
+    const int n0 = npairs < kStackWarps ? npairs : kStackWarps;
+    const int n1 = npairs - n0;
 
     unsigned long long *tt = (tid == 0) ? p.ttrace : nullptr;
-#define TSTAMP(l, ph) \
-    if (tt) tt[((size_t)(l) * P + c) * 16 + (ph)] = gtimer();
+    const size_t ctr_off = (size_t)p.n_layers * P * 16;
+#define TSTAMP(l, ph)                                              \
+    if (tt) {                                                      \
+        const size_t o_ = ((size_t)(l) * P + c) * 16 + (ph);       \
+        tt[o_] = gtimer();                                         \
+        tt[ctr_off + o_] = (unsigned long long)clock64();          \
+    }
 
     lut_fill(lut);
     if (tid == 0) {
         mbar_init(&mb_router, 1);
-        mbar_init(&mb_gu, 1);
+        mbar_init(&mb_gu0, 1);
+        mbar_init(&mb_gu1, 1);
         mbar_init(&mb_dn, 1);
         fence_mbar_init();
     }
@@ -268,6 +313,15 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
         const uint32_t par = (uint32_t)(l & 1);
         const uint32_t tag = (ep << 7) | (uint32_t)(l + 1);  // never 0 (a zeroed workspace holds 0)
         TSTAMP(l, 0)
+        if (tid == 0) {
+            // this layer's transfer sizes depend only on the CTA's share, not on the routing:
+            // register them now so the copies can be issued the moment top-k is known
+            mbar_expect_tx(&mb_gu0, (uint32_t)(2 * n0 * (d / 4)));
+            mbar_expect_tx(&mb_gu1, (uint32_t)(2 * n1 * (d / 4)));
+            mbar_expect_tx(&mb_dn, (uint32_t)(k * nrows * (f / 4)));
+            n_gu++;
+            n_dn++;
+        }
         // ------------------------------------------------------------ A: x_l, norm, limbs
         // thread t owns elements 4t..4t+3 (d = 2048 = 4 * 512)
         float xv[4];
@@ -379,9 +433,6 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                 bulk_g2s(rbuf + (size_t)q * d, p.layer[l + 1].router + (size_t)(c + q * P) * d, (uint32_t)(d * 2),
                          &mb_router);
         }
-        // activation limbs of this lane's segment, for phase C (G = d/64 = 32 lanes per row)
-        SegX<NL> X;
-        seg_load_x_padded<NL>(X, xl, xlp, lane % (d / 64));
         // ------------------------------------------------------------ B: logits, top-k, copies
         {
             bool ok = true;
@@ -402,34 +453,30 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
         __syncthreads();
         TSTAMP(l, 5)
         if (warp == 0) {
-            // copies: lanes 0..3 gate/up segments (<= 2 slots x 2 matrices), lanes 4.. down rows
+            // copies: lanes 0..3 first-half gate/up segments, 4..7 second half (each half spans
+            // at most two slots x two matrices), lanes 8.. down rows of slot lane-8
             const uint32_t rowb = (uint32_t)(d / 4), rowd = (uint32_t)(f / 4);
-            if (lane == 0) {
-                mbar_expect_tx(&mb_gu, (uint32_t)(2 * (p1 - p0)) * rowb);
-                mbar_expect_tx(&mb_dn, (uint32_t)(k * nrows) * rowd);
-                n_gu++;
-                n_dn++;
-                if (c == 0)
-                    for (int q = 0; q < k; q++) {
-                        p.idx_hist[l * k + q] = s_idx[q];
-                        p.gate_hist[l * k + q] = s_gate[q];
-                    }
-            }
-            __syncwarp();
-            if (lane < 4) {
-                const int seg = lane >> 1;
-                const int s0 = p0 / f;
-                const int e0 = min(p1, (s0 + 1) * f);
-                const int a = seg == 0 ? p0 : e0, b = seg == 0 ? e0 : p1;
+            if (lane == 0 && c == 0)
+                for (int q = 0; q < k; q++) {
+                    p.idx_hist[l * k + q] = s_idx[q];
+                    p.gate_hist[l * k + q] = s_gate[q];
+                }
+            if (lane < 8) {
+                const int half = lane >> 2, seg = (lane >> 1) & 1;
+                const int h0 = p0 + (half ? n0 : 0), h1 = half ? p1 : p0 + n0;  // pairs of this half
+                const int s0 = h0 / f;
+                const int e0 = min(h1, (s0 + 1) * f);
+                const int a = seg == 0 ? h0 : e0, b = seg == 0 ? e0 : h1;
                 if (b > a) {
                     const int s = a / f, j = a % f;
                     const size_t src = ((size_t)s_idx[s] * f + j) * rowb;
                     const int q0 = a - p0;
-                    if (lane & 1) bulk_g2s(ubuf + (size_t)q0 * rowb, Ly.up + src, (uint32_t)(b - a) * rowb, &mb_gu);
-                    else bulk_g2s(gbuf + (size_t)q0 * rowb, Ly.gate + src, (uint32_t)(b - a) * rowb, &mb_gu);
+                    uint64_t *mb = half ? &mb_gu1 : &mb_gu0;
+                    if (lane & 1) bulk_g2s(ubuf + (size_t)q0 * rowb, Ly.up + src, (uint32_t)(b - a) * rowb, mb);
+                    else bulk_g2s(gbuf + (size_t)q0 * rowb, Ly.gate + src, (uint32_t)(b - a) * rowb, mb);
                 }
-            } else if (lane < 4 + k && nrows > 0) {
-                const int s = lane - 4;
+            } else if (lane < 8 + k && nrows > 0) {
+                const int s = lane - 8;
                 bulk_g2s(dbuf + (size_t)s * p.dn_rows * rowd, Ly.down + ((size_t)s_idx[s] * d + i0) * rowd,
                          (uint32_t)nrows * rowd, &mb_dn);
             }
@@ -447,31 +494,38 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
         TSTAMP(l, 6)
         // ------------------------------------------------------------ C: gate/up -> h
         if (p1 > p0) {
-            const bool okw = mbar_wait(&mb_gu, par, lim, p.status);
-            alive = __syncthreads_and(okw ? 1 : 0) && alive;
-            TSTAMP(l, 7)
-            const uint32_t *lut_lane = lut + lane;
+            // activation limbs of this lane's segment (G = d/64 = 32 lanes per row)
+            SegX<NL> X;
+            seg_load_x_padded<NL>(X, xl, xlp, lane % (d / 64));
+            const uint32_t lane4 = (uint32_t)lane << 2;
             const int rowb = d / 4;
-            for (int q = warp; q < p1 - p0; q += kStackWarps) {
-                const uint4 wg = *reinterpret_cast<const uint4 *>(gbuf + (size_t)q * rowb + lane * 16);
-                const uint4 wu = *reinterpret_cast<const uint4 *>(ubuf + (size_t)q * rowb + lane * 16);
-                int ag[NL], au[NL];
+            for (int half = 0; half < 2; half++) {
+                const int qa = half ? n0 : 0, qb = half ? npairs : n0;
+                if (qb <= qa) break;
+                const bool okw = mbar_wait(half ? &mb_gu1 : &mb_gu0, par, lim, p.status);
+                alive = __syncthreads_and(okw ? 1 : 0) && alive;
+                if (half == 0) TSTAMP(l, 7)
+                for (int q = qa + warp; q < qb; q += kStackWarps) {
+                    const uint4 wg = *reinterpret_cast<const uint4 *>(gbuf + (size_t)q * rowb + lane * 16);
+                    const uint4 wu = *reinterpret_cast<const uint4 *>(ubuf + (size_t)q * rowb + lane * 16);
+                    int ag[NL], au[NL];
 #pragma unroll
-                for (int z = 0; z < NL; z++) ag[z] = au[z] = 0;
-                seg_dot<NL>(wg, X, lut_lane, ag);
-                seg_dot<NL>(wu, X, lut_lane, au);
-                int ga, gb2, ua, ub;
-                acc_to_pair<NL>(ag, ga, gb2);
-                acc_to_pair<NL>(au, ua, ub);
-                ga = group_sum<32>(ga);
-                ua = group_sum<32>(ua);
-                if (NL > 1) {
-                    gb2 = group_sum<32>(gb2);
-                    ub = group_sum<32>(ub);
-                }
-                if (lane == 0) {
-                    s_S[q][0] = pair_value(NL, ga, gb2);
-                    s_S[q][1] = pair_value(NL, ua, ub);
+                    for (int z = 0; z < NL; z++) ag[z] = au[z] = 0;
+                    seg_dot<NL>(wg, X, lut, lane4, ag);
+                    seg_dot<NL>(wu, X, lut, lane4, au);
+                    int ga, gb2, ua, ub;
+                    acc_to_pair<NL>(ag, ga, gb2);
+                    acc_to_pair<NL>(au, ua, ub);
+                    ga = group_sum<32>(ga);
+                    ua = group_sum<32>(ua);
+                    if (NL > 1) {
+                        gb2 = group_sum<32>(gb2);
+                        ub = group_sum<32>(ub);
+                    }
+                    if (lane == 0) {
+                        s_S[q][0] = pair_value(NL, ga, gb2);
+                        s_S[q][1] = pair_value(NL, ua, ub);
+                    }
                 }
             }
             __syncthreads();
@@ -502,8 +556,14 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             if (tid < k) s_hmax[tid] = 0u;
             __syncthreads();
             if (w0 < k * f) {
-                uint32_t hw[HW];
-                ok = ll_poll<HW>(p.hll + w0, HW, tag, hw, lim, p.status);
+                uint32_t hw[HW], h0[4], h1[4];
+                ok = ll_poll<4, false>(p.hll + w0, 4, tag, h0, lim, p.status);
+                ok = ll_poll<4, false>(p.hll + w0 + 4, 4, tag, h1, lim, p.status) && ok;
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    hw[i] = h0[i];
+                    hw[4 + i] = h1[i];
+                }
                 float m = 0.0f;
 #pragma unroll
                 for (int i = 0; i < HW; i++) {
@@ -543,36 +603,42 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                 alive = __syncthreads_and(okw ? 1 : 0) && alive;
             }
             TSTAMP(l, 12)
-            // (row, slot) pairs, G = f/64 lanes each (8 for f = 512): 4 pairs per warp pass
-            const int G = f / 64;
-            const int ppw = 32 / G;
-            const int sub = lane / G, gl = lane % G;
-            const uint32_t *lut_lane = lut + lane;
-            const int npairs = nrows * k;
-            for (int base = warp * ppw; base < npairs; base += kStackWarps * ppw) {
-                const int pi = base + sub;
-                const bool valid = pi < npairs;
-                const int rrow = valid ? pi / k : 0, sl = valid ? pi % k : 0;
+            // each warp keeps one slot's h limbs in registers and walks that slot's rows:
+            // G = f/64 lanes per row (8 for f = 512), 32/G rows per warp pass
+            {
+                const int G = f / 64;
+                const int rpp = 32 / G;
+                const int wps = kStackWarps / k;  // warps per slot (k divides 16 on this path)
+                const int sl = warp / wps, wi = warp % wps;
+                const int sub = lane / G, gl = lane % G;
+                const uint32_t lane4 = (uint32_t)lane << 2;
                 SegX<NL> Hx;
                 seg_load_x_padded<NL>(Hx, hl + (size_t)sl * NL * hlp, hlp, gl);
-                int acc[NL];
+                const float hsc = s_hscale[sl];
+                const int hsh = s_hshift[sl];
+                for (int r0 = wi * rpp; r0 < nrows; r0 += wps * rpp) {
+                    const int rrow = r0 + sub;
+                    const bool valid = rrow < nrows;
+                    int acc[NL];
 #pragma unroll
-                for (int z = 0; z < NL; z++) acc[z] = 0;
-                const uint4 wd = *reinterpret_cast<const uint4 *>(dbuf + ((size_t)sl * p.dn_rows + rrow) * (f / 4) + gl * 16);
-                seg_dot<NL>(wd, Hx, lut_lane, acc);
-                int a, b;
-                acc_to_pair<NL>(acc, a, b);
-                for (int o = G / 2; o > 0; o >>= 1) {
-                    a += __shfl_xor_sync(0xFFFFFFFFu, a, o);
-                    if (NL > 1) b += __shfl_xor_sync(0xFFFFFFFFu, b, o);
-                }
-                if (valid && gl == 0) {
-                    const long long S = pair_value(NL, a, b);
-                    const float sd = s_sd[sl * nrows + rrow];
-                    double v;
-                    if (NL == 1) v = (double)__fmul_rn(__fmul_rn(__int2float_rn((int)S), sd), s_hscale[sl]);
-                    else v = ldexp((double)S, -s_hshift[sl]) * (double)sd;
-                    s_ye[rrow][sl] = v;
+                    for (int z = 0; z < NL; z++) acc[z] = 0;
+                    const uint4 wd = *reinterpret_cast<const uint4 *>(
+                        dbuf + ((size_t)sl * p.dn_rows + (valid ? rrow : 0)) * (f / 4) + gl * 16);
+                    seg_dot<NL>(wd, Hx, lut, lane4, acc);
+                    int a, b;
+                    acc_to_pair<NL>(acc, a, b);
+                    for (int o = G / 2; o > 0; o >>= 1) {
+                        a += __shfl_xor_sync(0xFFFFFFFFu, a, o);
+                        if (NL > 1) b += __shfl_xor_sync(0xFFFFFFFFu, b, o);
+                    }
+                    if (valid && gl == 0) {
+                        const long long S = pair_value(NL, a, b);
+                        const float sd = s_sd[sl * nrows + rrow];
+                        double v;
+                        if (NL == 1) v = (double)__fmul_rn(__fmul_rn(__int2float_rn((int)S), sd), hsc);
+                        else v = ldexp((double)S, -hsh) * (double)sd;
+                        s_ye[rrow][sl] = v;
+                    }
                 }
             }
             __syncthreads();
@@ -601,7 +667,10 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
     // after a timeout, let this CTA's own copies in flight land (bounded) before leaving
     if (!alive && tid == 0) {
         if (n_rt) mbar_wait(&mb_router, (n_rt - 1) & 1u, lim, p.status);
-        if (n_gu) mbar_wait(&mb_gu, (n_gu - 1) & 1u, lim, p.status);
+        if (n_gu) {
+            mbar_wait(&mb_gu0, (n_gu - 1) & 1u, lim, p.status);
+            mbar_wait(&mb_gu1, (n_gu - 1) & 1u, lim, p.status);
+        }
         if (n_dn) mbar_wait(&mb_dn, (n_dn - 1) & 1u, lim, p.status);
     }
     // leave: the last CTA out advances the launch epoch (the next launch's tags differ)
@@ -640,7 +709,7 @@ static StackWs stack_ws_layout(const tern_moe_layer *L0) {
     o.hist = take((int64_t)(kMaxStackLayers + 1) * L0->d * 2);
     o.idx_hist = take((int64_t)kMaxStackLayers * L0->k * 4);
     o.gate_hist = take((int64_t)kMaxStackLayers * L0->k * 8);
-    o.ttrace = take((int64_t)kMaxStackLayers * kMaxTraceCtas * 16 * 8);
+    o.ttrace = take((int64_t)2 * kMaxStackLayers * kMaxTraceCtas * 16 * 8);
     o.total = p;
     return o;
 }
@@ -682,7 +751,7 @@ static tern_status stack_plan(const tern_moe_layer &L0, int n_layers, tern_act a
     // the thread mappings assume d = 4 * threads and k * f = 8 * threads at most, and a CTA's
     // gate/up pairs spanning at most two slots
     if (pl.rb_rows > kStackWarps || pl.dn_rows > 64 || pl.gu_pairs > 64 || pl.gu_pairs > L0.f ||
-        L0.k * L0.f > 8 * kStackThreads || (L0.k * L0.f) % 8 || L0.d != 4 * kStackThreads || L0.E > 256)
+        L0.k * L0.f > 8 * kStackThreads || (L0.k * L0.f) % 8 || L0.d != 4 * kStackThreads || L0.E > 256 || kStackWarps % L0.k)
         return TERN_EUNSUPPORTED;
     const int NL = act == TERN_ACT_INT8 ? 1 : 3;
     pl.sm = smem_map((int)L0.d, (int)L0.f, L0.k, pl.rb_rows, pl.gu_pairs, pl.dn_rows, NL);

@@ -60,9 +60,13 @@ __device__ __forceinline__ int dp4a_su(uint32_t a, uint32_t b, int c) {
 }
 
 // -------------------------------------------------------------------- decode table
-// lut[b * 32 + lane] = the four weights of byte b as signed int8 lanes (byte j = code j).
-constexpr int kLutWords = 256 * kWarp;
-constexpr int kLutBytes = kLutWords * 4;
+// Entry b (a packed byte) holds the four weights of b as signed int8 lanes (byte j = code j),
+// replicated in 32 lane-private columns: entry stride 256 bytes, lane l reads column l, so
+// lanes never share a bank.  The stride lets ONE byte-permute build the whole shared-memory
+// offset of a lookup: (packed byte << 8) | (lane << 2).
+constexpr int kLutStrideWords = 64;
+constexpr int kLutWords = 256 * kLutStrideWords;
+constexpr int kLutBytes = kLutWords * 4;  // 64 KB (columns 32..63 unused)
 
 __device__ __forceinline__ uint32_t decode_byte(uint32_t b) {
     uint32_t out = 0;
@@ -76,7 +80,11 @@ __device__ __forceinline__ uint32_t decode_byte(uint32_t b) {
 }
 
 __device__ __forceinline__ void lut_fill(uint32_t *lut) {
-    for (int i = threadIdx.x; i < kLutWords; i += blockDim.x) lut[i] = decode_byte((uint32_t)i >> 5);
+    for (int i4 = threadIdx.x; i4 < 256 * 8; i4 += blockDim.x) {
+        const uint32_t b = (uint32_t)i4 >> 3;
+        const uint32_t v = decode_byte(b);
+        reinterpret_cast<uint4 *>(lut + b * kLutStrideWords)[i4 & 7] = make_uint4(v, v, v, v);
+    }
 }
 
 // ------------------------------------------------------------------- segment dot
@@ -87,23 +95,26 @@ struct SegX {
     uint32_t w[NL][16];
 };
 
+// lane4 = lane * 4 (the lane's column offset in bytes)
 template <int NL>
-__device__ __forceinline__ void seg_dot(const uint4 wb, const SegX<NL> &x, const uint32_t *lut_lane,
+__device__ __forceinline__ void seg_dot(const uint4 wb, const SegX<NL> &x, const uint32_t *lut, uint32_t lane4,
                                         int (&acc)[NL]) {
+    const char *lb = reinterpret_cast<const char *>(lut);
     const uint32_t words[4] = {wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
     for (int q = 0; q < 4; q++) {
 #pragma unroll
         for (int i = 0; i < 4; i++) {
-            const uint32_t byte = (words[q] >> (8 * i)) & 0xFFu;
-            const uint32_t wv = lut_lane[byte << 5];
-            const int b = 4 * q + i;
+            // result byte 0 = lane4, byte 1 = packed byte i, bytes 2-3 = 0 (byte 1 of lane4)
+            const uint32_t off = __byte_perm(words[q], lane4, 0x5504u | ((uint32_t)i << 4));
+            const uint32_t wv = *reinterpret_cast<const uint32_t *>(lb + off);
+            const int bb = 4 * q + i;
             if (NL == 1) {
-                acc[0] = dp4a_ss(wv, x.w[0][b], acc[0]);
+                acc[0] = dp4a_ss(wv, x.w[0][bb], acc[0]);
             } else {
-                acc[0] = dp4a_ss(wv, x.w[0][b], acc[0]);   // hi limb: signed
-                acc[1] = dp4a_su(wv, x.w[1][b], acc[1]);   // mid limb: unsigned
-                acc[2] = dp4a_su(wv, x.w[2][b], acc[2]);   // lo limb: unsigned
+                acc[0] = dp4a_ss(wv, x.w[0][bb], acc[0]);   // hi limb: signed
+                acc[1] = dp4a_su(wv, x.w[1][bb], acc[1]);   // mid limb: unsigned
+                acc[2] = dp4a_su(wv, x.w[2][bb], acc[2]);   // lo limb: unsigned
             }
         }
     }
@@ -221,20 +232,24 @@ __device__ __forceinline__ float block_max_f32(float v, float *red) {
 // Shift s such that |x| * 2^s < 2^23 for every element (s = 22 - floor(log2(absmax))).
 __device__ __forceinline__ int fixed_shift(float absmax) {
     if (!(absmax > 0.0f)) return 0;
-    return 22 - ilogbf(absmax);
+    const int be = (__float_as_int(absmax) >> 23) & 0xFF;  // biased exponent
+    if (be == 0) return 22 - ilogbf(absmax);               // subnormal absmax
+    return 22 - (be - 127);
 }
 
-// x_int = rint(x * 2^s) split into three bytes: hi (signed), mid, lo (unsigned)
+// x_int = rint(x * 2^s) split into three bytes: hi (signed), mid, lo (unsigned).  x * 2^s is
+// a power-of-two scale, exact unless it lands below the fp32 normal range, where it rounds
+// to zero either way.
 __device__ __forceinline__ void fixed_limbs(float x, int s, uint32_t &hi, uint32_t &mid, uint32_t &lo) {
-    const int xi = __float2int_rn(scalbnf(x, s));
+    const bool fast = (s >= -126 && s <= 127);
+    const float sx = fast ? __fmul_rn(x, __int_as_float((127 + s) << 23)) : scalbnf(x, s);
+    const int xi = __float2int_rn(sx);
     hi = (uint32_t)(xi >> 16) & 0xFFu;
     mid = (uint32_t)(xi >> 8) & 0xFFu;
     lo = (uint32_t)xi & 0xFFu;
 }
 
 // ---------------------------------------------------------------------------- top-k
-// One warp selects the top k of E fp64 logits: descending value, ties to the lower index.
-// Lane l owns experts l, l+32, ...; selected entries are set to -inf (logits are finite).
 // Order-preserving 64-bit key of a finite double (larger double -> larger unsigned key;
 // -0.0 and +0.0 map to the same key).
 __device__ __forceinline__ unsigned long long f64_order_key(double v) {
@@ -243,47 +258,65 @@ __device__ __forceinline__ unsigned long long f64_order_key(double v) {
     return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
 }
 
+template <int J>
+__device__ __forceinline__ void topk_cas(unsigned long long (&key)[J], int (&ix)[J], int a, int b) {
+    // afterwards (key[a], ix[a]) ranks first: larger key, then lower index
+    const bool sw = (key[b] > key[a]) || (key[b] == key[a] && ix[b] < ix[a]);
+    const unsigned long long ka = key[a], kb = key[b];
+    const int ia = ix[a], ib = ix[b];
+    key[a] = sw ? kb : ka;
+    key[b] = sw ? ka : kb;
+    ix[a] = sw ? ib : ia;
+    ix[b] = sw ? ia : ib;
+}
+
 // One warp selects the top k (k <= 8) of E fp64 logits: descending value, ties to the lower
-// index.  Lane l owns experts l, l+32, ...  Each round reduces the lanes' best 64-bit keys
-// with the single-instruction warp max (__reduce_max_sync) on the high word, then the low
-// word, then the index.  Gates: lanes 0..k-1 each compute one exp(l_i - l_0) in fp64; lane 0
-// sums them in top-k order.  Outputs (written by lanes 0..k-1): idx_out, g64, g32 (either
-// gate pointer may be null).
+// index.  Lane l owns experts l, l+32, ...; each lane sorts its candidates once (Batcher's
+// network for 8), then every round the best lane head wins and that lane pops it.  Heads tie
+// on the high key word only when two logits share sign, exponent and 20 leading mantissa
+// bits; then the low word, then the index decide.  Gates: lanes 0..k-1 each compute one
+// exp(l_i - l_0) in fp64; every lane sums them in top-k order.  Outputs (lanes 0..k-1 write
+// their own entry): idx_out, g64, g32 (either gate pointer may be null).
 template <int J>
 __device__ __forceinline__ void warp_topk(const double *lg, int E, int k, int32_t *idx_out, double *g64, float *g32) {
     const int lane = threadIdx.x & 31;
-    // each lane's J candidates, sorted once by (key desc, index asc) with a bubble network
     unsigned long long key[J];
     int ix[J];
 #pragma unroll
     for (int j = 0; j < J; j++) {
         const int e = lane + 32 * j;
         key[j] = (e < E) ? f64_order_key(lg[e]) : 0ull;  // 0 = below every finite logit
-        ix[j] = e;
+        ix[j] = (e < E) ? e : 0x7FFFFFFF;
     }
+    if (J == 8) {
+        topk_cas<J>(key, ix, 0, 1); topk_cas<J>(key, ix, 2, 3); topk_cas<J>(key, ix, 4, 5); topk_cas<J>(key, ix, 6, 7);
+        topk_cas<J>(key, ix, 0, 2); topk_cas<J>(key, ix, 1, 3); topk_cas<J>(key, ix, 4, 6); topk_cas<J>(key, ix, 5, 7);
+        topk_cas<J>(key, ix, 1, 2); topk_cas<J>(key, ix, 5, 6);
+        topk_cas<J>(key, ix, 0, 4); topk_cas<J>(key, ix, 1, 5); topk_cas<J>(key, ix, 2, 6); topk_cas<J>(key, ix, 3, 7);
+        topk_cas<J>(key, ix, 2, 4); topk_cas<J>(key, ix, 3, 5);
+        topk_cas<J>(key, ix, 1, 2); topk_cas<J>(key, ix, 3, 4); topk_cas<J>(key, ix, 5, 6);
+    } else {
 #pragma unroll
-    for (int a = 0; a < J; a++)
+        for (int a = 0; a < J; a++)
 #pragma unroll
-        for (int b = 0; b < J - 1 - a; b++)
-            if (key[b + 1] > key[b]) {  // strict: equal keys keep the lower index first
-                const unsigned long long tk = key[b];
-                key[b] = key[b + 1];
-                key[b + 1] = tk;
-                const int ti = ix[b];
-                ix[b] = ix[b + 1];
-                ix[b + 1] = ti;
-            }
-    int sel_e = 0;
+            for (int b = 0; b < J - 1 - a; b++) topk_cas<J>(key, ix, b, b + 1);
+    }
+    int my_e = 0;
     for (int r = 0; r < k; r++) {
-        const unsigned long long bk = key[0];
-        const unsigned hi = (unsigned)(bk >> 32), lo = (unsigned)bk;
+        const unsigned hi = (unsigned)(key[0] >> 32);
         const unsigned mhi = __reduce_max_sync(0xFFFFFFFFu, hi);
-        const unsigned mlo = __reduce_max_sync(0xFFFFFFFFu, hi == mhi ? lo : 0u);
-        const bool cand = (hi == mhi) && (lo == mlo);
-        const unsigned wi = __reduce_min_sync(0xFFFFFFFFu, cand ? (unsigned)ix[0] : 0xFFFFFFFFu);
-        int win = (int)wi;
+        unsigned cand = __ballot_sync(0xFFFFFFFFu, hi == mhi);
+        if (__popc(cand) > 1) {
+            const unsigned lo = (unsigned)key[0];
+            const unsigned mlo = __reduce_max_sync(0xFFFFFFFFu, hi == mhi ? lo : 0u);
+            const bool c2 = (hi == mhi) && (lo == mlo);
+            const unsigned mi = __reduce_min_sync(0xFFFFFFFFu, c2 ? (unsigned)ix[0] : 0xFFFFFFFFu);
+            cand = __ballot_sync(0xFFFFFFFFu, c2 && (unsigned)ix[0] == mi);
+        }
+        const int wl = __ffs(cand) - 1;
+        int win = __shfl_sync(0xFFFFFFFFu, ix[0], wl);
         if (win < 0 || win >= E) win = r;  // NaN inputs must still not index out of range
-        if (cand && ix[0] == win) {        // pop this lane's head
+        if (lane == wl) {
 #pragma unroll
             for (int j = 0; j < J - 1; j++) {
                 key[j] = key[j + 1];
@@ -292,16 +325,18 @@ __device__ __forceinline__ void warp_topk(const double *lg, int E, int k, int32_
             key[J - 1] = 0ull;
             ix[J - 1] = 0x7FFFFFFF;
         }
-        if (lane == r) sel_e = win;
+        if (lane == r) my_e = win;
     }
-    // gates: lane r < k holds expert sel_e; logit of the top-1 broadcast from lane 0
-    const double lsel = (lane < k) ? lg[sel_e] : 0.0;
-    const double l0 = __shfl_sync(0xFFFFFFFFu, lsel, 0);
-    const double ev = (lane < k) ? exp(lsel - l0) : 0.0;
+    const double my_l = (lane < k) ? lg[my_e] : 0.0;
+    const double l0 = __shfl_sync(0xFFFFFFFFu, my_l, 0);
+    const double ev = (lane < k) ? exp(my_l - l0) : 0.0;
+    double evs[8];
+#pragma unroll
+    for (int r = 0; r < 8; r++) evs[r] = __shfl_sync(0xFFFFFFFFu, ev, r);
     double z = 0.0;
-    for (int r = 0; r < k; r++) z += __shfl_sync(0xFFFFFFFFu, ev, r);  // top-k order
+    for (int r = 0; r < k; r++) z += evs[r];
     if (lane < k) {
-        idx_out[lane] = sel_e;
+        idx_out[lane] = my_e;
         const double g = ev / z;
         if (g64) g64[lane] = g;
         if (g32) g32[lane] = (float)g;
