@@ -144,6 +144,26 @@ tern_status moe_route_topk(const uint16_t *Wg, const uint16_t *x, int64_t T, int
                            int32_t k, int32_t *topk_idx, float *topk_gate, double *logits,
                            void *workspace, size_t ws_bytes, void *stream);
 
+/* moe_route_topk_static -- the same routing as moe_route_topk, for callers that cannot
+ * allocate device memory (the pages have no counterpart; this is a library convenience).
+ * A caller that only receives device pointers to its inputs and outputs -- a plugin whose
+ * host framework owns every allocation, or a serving loop that forbids allocator calls after
+ * start-up -- has no way to provide a workspace.  This call needs none: its scratch (arrival
+ * counter, fp64 logits, fp64 gates; 135,424 bytes) is a fixed array inside the library,
+ * held on every GPU that loads the library until the process exits.  Inputs and outputs are
+ * the caller's, exactly as for moe_route_topk.
+ *   Limits: 1 <= T <= 64 and T * E <= 16384 (e.g. 64 tokens x 256 experts); larger requests
+ *   return TERN_EINVAL before anything is enqueued.
+ *   The first call on each device looks up the array's device address (once per device, on
+ *   the calling thread's current device); make that first call before any stream capture.
+ *   All calls on a device share the one array: calls that overlap on the GPU (different
+ *   streams, no ordering between them) race and give undefined results.  The call clears
+ *   the part that must start at zero (the arrival counter) itself.
+ *   It allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine. */
+tern_status moe_route_topk_static(const uint16_t *Wg, const uint16_t *x, int64_t T, int64_t d, int32_t E,
+                                  int32_t k, int32_t *topk_idx, float *topk_gate, double *logits,
+                                  void *stream);
+
 /* One MoE FFN layer for T tokens (decode):
  *   route (as moe_route_topk) -> group the (token, slot) pairs by expert so every selected
  *   expert's packed weights stream from memory once per call -> for each pair

@@ -80,6 +80,7 @@ def lib():
             "tern_quant_absmax": (st, [vp, i64, i64, vp, vp, vp]),
             "moe_route_workspace_bytes": (sz, [i64, i32]),
             "moe_route_topk": (st, [vp, vp, i64, i64, i32, i32, vp, vp, vp, vp, sz, vp]),
+            "moe_route_topk_static": (st, [vp, vp, i64, i64, i32, i32, vp, vp, vp, vp]),
             "moe_ffn_workspace_bytes": (sz, [ctypes.POINTER(MoELayerC), i64, st]),
             "moe_ffn_workspace_layout": (st, [ctypes.POINTER(MoELayerC), i64, st, ctypes.POINTER(FfnLayoutC)]),
             "moe_ffn_decode": (st, [ctypes.POINTER(MoELayerC), vp, i64, st, vp, vp, vp, sz, vp]),
@@ -220,6 +221,23 @@ def moe_route_topk(Wg, x, k=8, ws=None, logits=None, idx=None, gates=None, strea
     ws = workspace(need, dev) if ws is None else ws
     _check(lib().moe_route_topk(_ptr(Wg), _ptr(x), T, d, E, k, _ptr(idx), _ptr(gates), _ptr(logits), _ptr(ws),
                                 ws.numel(), _stream(stream)), "moe_route_topk")
+    return idx, gates
+
+
+def moe_route_topk_static(Wg, x, k=8, logits=None, idx=None, gates=None, stream=None):
+    """Routing without a workspace (scratch is a fixed array inside the library; T <= 64,
+    T * E <= 16384).  For callers that cannot allocate device memory."""
+    Wg = _bits16(Wg, "Wg")
+    x = _bits16(x.view(1, -1) if x.dim() == 1 else x, "x")
+    E, d = Wg.shape
+    T = x.shape[0]
+    dev = Wg.device
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev) if idx is None else idx
+    gates = torch.empty((T, k), dtype=torch.float32, device=dev) if gates is None else gates
+    if logits is not None:
+        _dev(logits, torch.float64, "logits")
+    _check(lib().moe_route_topk_static(_ptr(Wg), _ptr(x), T, d, E, k, _ptr(idx), _ptr(gates), _ptr(logits),
+                                       _stream(stream)), "moe_route_topk_static")
     return idx, gates
 
 
