@@ -206,6 +206,26 @@ def phase_summary(tr, clk=None, mhz=1965.0):
     return out
 
 
+def kernel_source_hash():
+    import hashlib
+
+    parts = ["stack.cu", "tern_common.cuh", "kernels.h"]
+    src = "".join(open(os.path.join(ROOT, "ternary_weight_moe_b200", "csrc", p)).read() for p in parts)
+    return hashlib.sha256(src.encode()).hexdigest()[:16]
+
+
+def kernel_traffic(act):
+    """DRAM bytes per launch from the committed ncu record, or None if the kernel changed since."""
+    try:
+        tj = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+        rec = tj.get(f"stack_kernel_{act}")
+        if rec and rec.get("valid") and rec.get("source_hash") == kernel_source_hash():
+            return rec["bytes_per_launch"]
+    except (OSError, ValueError):
+        pass
+    return None
+
+
 def run_reference(args):
     """--impl reference: the CPU oracle as the reference arm (rank 0 only)."""
     world, rank, _ = dist_env()
@@ -384,16 +404,7 @@ def main():
     peak, peak_kind = peaks()
     avg_launch_ms = dev_ms / K / max(launches, 1)
     achieved = BYTES_PER_TOKEN / launches / (avg_launch_ms * 1e-3) / 1e9
-    traffic = None
-    tfile = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tfile):
-        try:
-            tj = json.load(open(tfile))
-            key = f"stack_kernel_{args.act}"
-            if key in tj and tj[key].get("valid", False):
-                traffic = tj[key]["bytes_per_launch"]
-        except Exception:
-            traffic = None
+    traffic = kernel_traffic(args.act) if N_LAYERS == 24 else None
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": dev_ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
