@@ -47,10 +47,11 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(
                 const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w}, xx[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
                 for (int q = 0; q < 4; q++) {
-                    acc = fma((double)bf16_to_f32((uint16_t)(ww[q] & 0xFFFFu)),
-                              (double)bf16_to_f32((uint16_t)(xx[q] & 0xFFFFu)), acc);
-                    acc = fma((double)bf16_to_f32((uint16_t)(ww[q] >> 16)),
-                              (double)bf16_to_f32((uint16_t)(xx[q] >> 16)), acc);
+                    // bf16 x bf16 has at most 16 significant bits: the fp32 product is exact
+                    acc += (double)__fmul_rn(bf16_to_f32((uint16_t)(ww[q] & 0xFFFFu)),
+                                             bf16_to_f32((uint16_t)(xx[q] & 0xFFFFu)));
+                    acc += (double)__fmul_rn(bf16_to_f32((uint16_t)(ww[q] >> 16)),
+                                             bf16_to_f32((uint16_t)(xx[q] >> 16)));
                 }
             }
             acc = warp_sum_f64(acc);

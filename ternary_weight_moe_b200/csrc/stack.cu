@@ -403,8 +403,9 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                 const int per = d / wpr;
                 const uint16_t *wrow = rbuf + (size_t)rr * d + part * per;
                 const uint16_t *nrow = ns + part * per;
+                // bf16 x bf16 has at most 16 significant bits: the fp32 product is exact
                 for (int i = lane; i < per; i += 32)
-                    acc = fma((double)bf16_to_f32(wrow[i]), (double)bf16_to_f32(nrow[i]), acc);
+                    acc += (double)__fmul_rn(bf16_to_f32(wrow[i]), bf16_to_f32(nrow[i]));
             }
             acc = warp_sum_f64(acc);
             if (lane == 0 && rr < nr) s_part[rr][part] = acc;
@@ -437,7 +438,8 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             alive = __syncthreads_and(ok ? 1 : 0) && alive;
         }
         TSTAMP(l, 4)
-        if (warp == 0) warp_topk<8>(s_logit, E, k, s_idx, s_gate, nullptr);  // E <= 256 on this path
+        // only the expert indices are on the critical path; the gates are needed in the combine
+        if (warp == 0) warp_topk_select<8>(s_logit, E, k, s_idx);  // E <= 256 on this path
         __syncthreads();
         TSTAMP(l, 5)
         if (warp == 0) {
@@ -445,11 +447,6 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             // at most two slots x two matrices), lanes 8.. down rows of slot lane-8
             const uint32_t rowb = (uint32_t)(d / 4), rowd = (uint32_t)(f / 4);
             fence_proxy_async();
-            if (lane == 0 && c == 0)
-                for (int q = 0; q < k; q++) {
-                    p.idx_hist[l * k + q] = s_idx[q];
-                    p.gate_hist[l * k + q] = s_gate[q];
-                }
             if (lane < 8) {
                 const int half = lane >> 2, seg = (lane >> 1) & 1;
                 const int h0 = p0 + (half ? n0 : 0), h1 = half ? p1 : p0 + n0;  // pairs of this half
@@ -479,6 +476,14 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             }
             for (int q = tid - 32; q < k * nrows; q += kStackThreads - 32)
                 s_sd[q] = __ldg(Ly.sd + (size_t)s_idx[q / nrows] * d + i0 + q % nrows);
+            if (warp == kStackWarps - 1) {
+                warp_topk_gates(s_logit, k, s_idx, s_gate, nullptr);
+                __syncwarp();
+                if (lane < k && c == 0) {
+                    p.idx_hist[l * k + lane] = s_idx[lane];
+                    p.gate_hist[l * k + lane] = s_gate[lane];
+                }
+            }
         }
         TSTAMP(l, 6)
         // ------------------------------------------------------------ C: gate/up -> h

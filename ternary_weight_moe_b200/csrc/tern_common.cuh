@@ -272,13 +272,12 @@ __device__ __forceinline__ void topk_cas(unsigned long long (&key)[J], int (&ix)
 
 // One warp selects the top k (k <= 8) of E fp64 logits: descending value, ties to the lower
 // index.  Lane l owns experts l, l+32, ...; each lane sorts its candidates once (Batcher's
-// network for 8), then every round the best lane head wins and that lane pops it.  Heads tie
-// on the high key word only when two logits share sign, exponent and 20 leading mantissa
-// bits; then the low word, then the index decide.  Gates: lanes 0..k-1 each compute one
-// exp(l_i - l_0) in fp64; every lane sums them in top-k order.  Outputs (lanes 0..k-1 write
-// their own entry): idx_out, g64, g32 (either gate pointer may be null).
+// network for 8), then every round the best lane head wins; the winning lane writes
+// idx_out[r] and pops its head.  Heads tie on the high key word only when two logits share
+// sign, exponent and 20 leading mantissa bits; then the low word, then the index decide.
+// idx_out must be visible to the whole warp afterwards (shared or global memory).
 template <int J>
-__device__ __forceinline__ void warp_topk(const double *lg, int E, int k, int32_t *idx_out, double *g64, float *g32) {
+__device__ __forceinline__ void warp_topk_select(const double *lg, int E, int k, int32_t *idx_out) {
     const int lane = threadIdx.x & 31;
     unsigned long long key[J];
     int ix[J];
@@ -301,7 +300,6 @@ __device__ __forceinline__ void warp_topk(const double *lg, int E, int k, int32_
 #pragma unroll
             for (int b = 0; b < J - 1 - a; b++) topk_cas<J>(key, ix, b, b + 1);
     }
-    int my_e = 0;
     for (int r = 0; r < k; r++) {
         const unsigned hi = (unsigned)(key[0] >> 32);
         const unsigned mhi = __reduce_max_sync(0xFFFFFFFFu, hi);
@@ -313,10 +311,9 @@ __device__ __forceinline__ void warp_topk(const double *lg, int E, int k, int32_
             const unsigned mi = __reduce_min_sync(0xFFFFFFFFu, c2 ? (unsigned)ix[0] : 0xFFFFFFFFu);
             cand = __ballot_sync(0xFFFFFFFFu, c2 && (unsigned)ix[0] == mi);
         }
-        const int wl = __ffs(cand) - 1;
-        int win = __shfl_sync(0xFFFFFFFFu, ix[0], wl);
-        if (win < 0 || win >= E) win = r;  // NaN inputs must still not index out of range
-        if (lane == wl) {
+        if (lane == __ffs(cand) - 1) {
+            // finite logits always select a valid expert; NaN inputs must still not index out of range
+            idx_out[r] = (ix[0] >= 0 && ix[0] < E) ? ix[0] : r;
 #pragma unroll
             for (int j = 0; j < J - 1; j++) {
                 key[j] = key[j + 1];
@@ -325,9 +322,15 @@ __device__ __forceinline__ void warp_topk(const double *lg, int E, int k, int32_
             key[J - 1] = 0ull;
             ix[J - 1] = 0x7FFFFFFF;
         }
-        if (lane == r) my_e = win;
     }
-    const double my_l = (lane < k) ? lg[my_e] : 0.0;
+    __syncwarp();
+}
+
+// Renormalised gates of the selected experts: g_i = exp(l_i - l_0) / sum_j exp(l_j - l_0),
+// lanes 0..k-1 each one exp in fp64, the sum taken in top-k order.
+__device__ __forceinline__ void warp_topk_gates(const double *lg, int k, const int32_t *idx, double *g64, float *g32) {
+    const int lane = threadIdx.x & 31;
+    const double my_l = (lane < k) ? lg[idx[lane]] : 0.0;
     const double l0 = __shfl_sync(0xFFFFFFFFu, my_l, 0);
     const double ev = (lane < k) ? exp(my_l - l0) : 0.0;
     double evs[8];
@@ -336,11 +339,16 @@ __device__ __forceinline__ void warp_topk(const double *lg, int E, int k, int32_
     double z = 0.0;
     for (int r = 0; r < k; r++) z += evs[r];
     if (lane < k) {
-        idx_out[lane] = my_e;
         const double g = ev / z;
         if (g64) g64[lane] = g;
         if (g32) g32[lane] = (float)g;
     }
+}
+
+template <int J>
+__device__ __forceinline__ void warp_topk(const double *lg, int E, int k, int32_t *idx_out, double *g64, float *g32) {
+    warp_topk_select<J>(lg, E, k, idx_out);
+    warp_topk_gates(lg, k, idx_out, g64, g32);
 }
 
 // ----------------------------------------------------------- absmax int8 quantisation
