@@ -81,9 +81,9 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
-// order this thread's earlier generic-proxy accesses of shared memory before later async-proxy
-// (TMA) writes into the same buffers
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// Shared buffers are rewritten by TMA only after every thread's generic reads of them are
+// ordered before the issuing thread by a CTA (or slot) barrier; write-after-read across the
+// generic and async proxies needs no proxy fence.
 __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -139,7 +139,6 @@ __device__ __forceinline__ bool ll_gather(const unsigned long long *src, int n, 
     const unsigned long long t0 = gtimer();
     while (true) {
         if (threadIdx.x == 0) {
-            fence_proxy_async();
             mbar_expect_tx(mb, (uint32_t)(n * 8));
             bulk_g2s(dst, src, (uint32_t)(n * 8), mb);
         }
@@ -422,7 +421,6 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
         TSTAMP(l, 3)
         __syncthreads();
         if (tid == 0 && nr > 0 && l + 1 < p.n_layers) {  // next layer's router rows
-            fence_proxy_async();
             mbar_expect_tx(&mb_router, (uint32_t)(nr * d * 2));
             n_rt++;
             for (int q = 0; q < nr; q++)
@@ -446,7 +444,6 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             // copies: lanes 0..3 first-half gate/up segments, 4..7 second half (each half spans
             // at most two slots x two matrices), lanes 8.. down rows of slot lane-8
             const uint32_t rowb = (uint32_t)(d / 4), rowd = (uint32_t)(f / 4);
-            fence_proxy_async();
             if (lane < 8) {
                 const int half = lane >> 2, seg = (lane >> 1) & 1;
                 const int h0 = p0 + (half ? n0 : 0), h1 = half ? p1 : p0 + n0;  // pairs of this half
@@ -558,7 +555,6 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                 const unsigned long long t0 = gtimer();
                 while (true) {
                     if (wi == 0 && lane == 0) {
-                        fence_proxy_async();
                         mbar_expect_tx(&mb_h[sl], (uint32_t)(f * 8));
                         bulk_g2s(hb, p.hll + (size_t)sl * f, (uint32_t)(f * 8), &mb_h[sl]);
                         s_hissued[sl]++;
