@@ -209,7 +209,7 @@ def phase_summary(tr, clk=None, mhz=1965.0):
 def kernel_source_hash():
     import hashlib
 
-    parts = ["stack.cu", "tern_common.cuh", "kernels.h"]
+    parts = ["stack.cu", "tern_common.cuh", "tma.cuh", "kernels.h"]
     src = "".join(open(os.path.join(ROOT, "ternary_weight_moe_b200", "csrc", p)).read() for p in parts)
     return hashlib.sha256(src.encode()).hexdigest()[:16]
 
@@ -277,6 +277,62 @@ def run_reference(args):
     return 0
 
 
+def run_gemv_sweep(args):
+    """Extra output: device time of one tern_gemv launch per shape of the GEMV sweep (T = 1,
+    bf16 and int8 activations), L2 flushed before every launch; one JSON line per shape.
+    The last shape (128 MB of packed codes) is a bandwidth check, not one of the sweep's."""
+    import torch
+
+    import synth
+    import ternary_weight_moe_b200 as tm
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peak, peak_kind = peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    shapes = list(synth.GEMV_SWEEP) + [(32768, 16384)]
+    if args.shape:
+        shapes = [tuple(int(v) for v in args.shape.split("x"))]
+    for (M, K) in shapes:
+        base = synth.derive(synth.BASE_SEED + 2, M, K)
+        w = synth.ternary_codes_torch(synth.derive(base, synth.KIND_W), 0, M * K, synth.P0_SPARSE, dev).view(M, K)
+        Wp = tm.tern_pack(w)
+        del w
+        rs = torch.from_numpy(synth.uniform_f32(synth.derive(base, synth.KIND_S), 0, M, 0.01, 0.05)).to(dev)
+        xb = torch.from_numpy(synth.normal_bf16(synth.derive(base, synth.KIND_X), 0, K, 1.0).view(np.int16)).to(dev)
+        xi = torch.from_numpy(synth.int8_uniform(synth.derive(base, synth.KIND_XQ), 0, K)).to(dev)
+        y = torch.empty((1, M), dtype=torch.float32, device=dev)
+        for act_name, act, x in (("bf16", tm.TERN_ACT_BF16, xb), ("int8", tm.TERN_ACT_INT8, xi)):
+            if args.act_only and act_name != args.act:
+                continue
+            for _ in range(max(args.warmup, 3)):
+                tm.tern_gemv(Wp, rs, x, act=act, y=y)
+            # no host wait inside the loop: the flush keeps the device busy while the host
+            # enqueues the next launch, so the events see device time only
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+            torch.cuda.synchronize(dev)
+            for i in range(args.steps):
+                flush.fill_(i & 0xFF)
+                evs[i][0].record(stream)
+                tm.tern_gemv(Wp, rs, x, act=act, y=y)
+                evs[i][1].record(stream)
+            torch.cuda.synchronize(dev)
+            ms = [a.elapsed_time(b) for a, b in evs]
+            if tm.tern_stream_status() != 0:
+                raise RuntimeError("device status set during the sweep")
+            med = statistics.median(ms)
+            nbytes = M * K // 4 + 4 * M + (2 if act_name == "bf16" else 1) * K + 4 * M
+            gbs = nbytes / (med * 1e-3) / 1e9
+            print(json.dumps({"gemv": f"{M}x{K}", "act": act_name, "us_median": med * 1e3,
+                              "us_p10": float(np.percentile(ms, 10)) * 1e3, "bytes": nbytes, "GB/s": gbs,
+                              "frac": gbs / peak, "peak": peak, "peak_kind": peak_kind, "launches": args.steps}),
+                  flush=True)
+        del Wp
+    return 0
+
+
 def main():
     global N_LAYERS, BYTES_PER_TOKEN
     ap = argparse.ArgumentParser()
@@ -288,11 +344,17 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=N_LAYERS,
                     help="profiling only: a shorter stack (the benchmark line is the 24-layer stack)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="extra output: time tern_gemv over the GEMV shape sweep instead of the stack")
+    ap.add_argument("--shape", default=None, help="with --sweep: one shape MxK only")
+    ap.add_argument("--act-only", action="store_true", help="with --sweep: only the --act activations")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.sweep:
+        return run_gemv_sweep(args)
 
     import torch
 

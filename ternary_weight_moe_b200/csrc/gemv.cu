@@ -14,6 +14,7 @@
 
 #include "kernels.h"
 #include "tern_common.cuh"
+#include "tma.cuh"
 
 namespace tern {
 
@@ -100,8 +101,6 @@ cudaError_t launch_quant_absmax(const uint16_t *x, int64_t T, int64_t n, int8_t 
 }
 
 // ------------------------------------------------------------------------ ternary GEMV
-constexpr int kGemvWarps = 8;
-
 // Fill the limb registers of one lane for the segment `seg` (64 codes) of token vector xt.
 //  int8 (NL == 1): the 64 int8 values as 16 words;
 //  bf16 (NL == 3): 24-bit fixed point with per-token shift sh.
@@ -145,32 +144,105 @@ __device__ __forceinline__ void gemv_load_x(SegX<NL> &X, const void *xt, int64_t
     }
 }
 
-// G lanes per row slice; NS row slices of KS = 64*G codes (split-K across warps when NS > 1).
+// ------------------------------------------------------------ the TMA-fed GEMV kernel
+// One CTA per SM.  A producer warp streams chunks of R consecutive rows (R*K/4 contiguous
+// bytes, up to 16 KB) plus their row scales into a ring of kGvStages shared-memory stages
+// with bulk copies; 16 consumer warps decode each stage as it lands and release it through
+// an mbarrier, so about 96 KB of weights per SM stay in flight while the consumers compute.
+//   K <= 2048: G = K/64 lanes per row, 32/G rows per warp pass, no cross-warp combine;
+//   K  > 2048: NS = K/2048 slices of 512 bytes; warp w takes slice w % NS of rows
+//              w / NS, w / NS + 16/NS, ...; the exact integer partial sums of a row meet in
+//              shared memory (order-free 64-bit atomic adds), and the warp that adds the last
+//              one writes the row.
+constexpr int kGvCons = 16;  // consumer warps
+constexpr int kGvThreads = (kGvCons + 1) * 32;
+constexpr int kGvStages = 6;
+constexpr int kGvStageBytes = 16384;
+constexpr int kGvMaxRows = 128;    // rows per chunk (scale ring entries per stage)
+constexpr int kGvMaxSplitRows = 16;  // rows per chunk when K > 2048 (16 KB / 1 KB)
+constexpr long long kGvWaitNs = 1000000000ll;
+
+constexpr size_t gv_smem_bytes() {
+    return (size_t)kLutBytes + (size_t)kGvStages * kGvStageBytes + (size_t)kGvStages * kGvMaxRows * 4 +
+           (size_t)kGvStages * kGvMaxSplitRows * (8 + 4);
+}
+
 template <int NL, int G>
-__global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const uint8_t *__restrict__ Wp,
-                                                                const float *__restrict__ rs, int M, int K,
-                                                                int NS, const void *__restrict__ x,
-                                                                const float *__restrict__ xs, int T,
-                                                                int32_t *__restrict__ acc_out,
-                                                                float *__restrict__ y) {
-    extern __shared__ __align__(16) uint32_t smem[];
-    uint32_t *lut = smem;                                            // kLutWords
-    long long *part = reinterpret_cast<long long *>(smem + kLutWords);  // [kGemvWarps][32/G]
+__global__ void __launch_bounds__(kGvThreads, 1)
+    gemv_kernel(const uint8_t *__restrict__ Wp, const float *__restrict__ rs, int M, int K, int NS, int R,
+                int nchunks, const void *__restrict__ x, const float *__restrict__ xs, int T,
+                int32_t *__restrict__ acc_out, float *__restrict__ y, int *status) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ __align__(8) uint64_t full[kGvStages], empty[kGvStages];
     __shared__ float red[32];
-    __shared__ int sh_shift;
+    uint32_t *lut = reinterpret_cast<uint32_t *>(smem);
+    unsigned char *ring = smem + kLutBytes;
+    float *s_rs = reinterpret_cast<float *>(ring + (size_t)kGvStages * kGvStageBytes);             // [S][kGvMaxRows]
+    unsigned long long *s_acc = reinterpret_cast<unsigned long long *>(s_rs + kGvStages * kGvMaxRows);  // [S][16]
+    int *s_cnt = reinterpret_cast<int *>(s_acc + kGvStages * kGvMaxSplitRows);                    // [S][16]
 
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int RB = K / 4;
+    const int my_n = (nchunks - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;  // chunks per token
+    const int total = my_n * T;
+    const bool rs_bulk = ((uintptr_t)rs % 16u) == 0;
+    // chunk n of this CTA (n counts over tokens too): rows [r0, r0 + nr)
+    auto chunk_rows = [&](int n, int &r0, int &nr) {
+        r0 = ((int)blockIdx.x + (n % my_n) * (int)gridDim.x) * R;
+        nr = min(R, M - r0);
+    };
+    auto issue = [&](int n) {
+        const int st = n % kGvStages;
+        int r0, nr;
+        chunk_rows(n, r0, nr);
+        const uint32_t wbytes = (uint32_t)nr * (uint32_t)RB;
+        const uint32_t sbytes = rs_bulk ? (uint32_t)(nr / 4) * 16u : 0u;
+        mbar_expect_tx(&full[st], wbytes + sbytes);
+        bulk_g2s(ring + (size_t)st * kGvStageBytes, Wp + (size_t)r0 * RB, wbytes, &full[st]);
+        if (sbytes) bulk_g2s(s_rs + st * kGvMaxRows, rs + r0, sbytes, &full[st]);
+    };
+
+    int issued = 0;
+    if (tid == kGvCons * 32) {
+        for (int q = 0; q < kGvStages; q++) {
+            mbar_init(&full[q], 1);
+            mbar_init(&empty[q], kGvCons);
+        }
+        fence_mbar_init();
+        // the first stages need no release: start them before the table is built
+        for (; issued < kGvStages && issued < total; issued++) issue(issued);
+    }
     lut_fill(lut);
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const uint32_t lane4 = (uint32_t)lane << 2;
-    const int slice = warp % NS;              // K slice of this warp
-    const int rgroup = warp / NS;             // row group inside the CTA
-    const int ngroups = kGemvWarps / NS;
-    constexpr int RPW = 32 / G;               // rows per warp pass
-    const int sub = lane / G, gl = lane % G;  // row inside the pass, lane inside the row
-    const int64_t seg = (int64_t)slice * G + gl;  // segment index along K
-    const int64_t row_bytes = K / 4;
-    const int rows_per_cta = ngroups * RPW;
+    for (int q = tid; q < kGvStages * kGvMaxSplitRows; q += blockDim.x) {
+        s_acc[q] = 0ull;
+        s_cnt[q] = 0;
+    }
+    __syncthreads();
 
+    if (warp == kGvCons) {  // ------------------------------------------------ producer
+        if (lane == 0) {
+            for (; issued < total; issued++) {
+                const int st = issued % kGvStages;
+                if (!mbar_wait(&empty[st], (uint32_t)((issued / kGvStages) - 1) & 1u, kGvWaitNs, status)) break;
+                issue(issued);
+            }
+            // leave only after every copy into this CTA's shared memory has landed
+            for (int q = 0; q < kGvStages && q < issued; q++) {
+                const int cnt = (issued - q + kGvStages - 1) / kGvStages;
+                mbar_wait(&full[q], (uint32_t)(cnt - 1) & 1u, kGvWaitNs, status);
+            }
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------------------- consumers
+    constexpr int RPW = 32 / G;  // rows per warp pass (K <= 2048)
+    const int sub = lane / G, gl = lane % G;
+    const int slice = warp % NS, rg = warp / NS, ngroups = kGvCons / NS;
+    const int64_t seg = (NS > 1) ? (int64_t)slice * 32 + lane : (int64_t)gl;
+    const uint32_t lane4 = (uint32_t)lane << 2;
+    bool alive = true;
+    int n = 0;
     for (int t = 0; t < T; t++) {
         int sh = 0;
         const void *xt;
@@ -180,71 +252,114 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const uint8_t *__
             const uint16_t *xb = static_cast<const uint16_t *>(x) + (int64_t)t * K;
             xt = xb;
             float m = 0.0f;
-            for (int i = threadIdx.x; i < K; i += blockDim.x) m = fmaxf(m, fabsf(bf16_to_f32(xb[i])));
-            const float amax = block_max_f32(m, red);
-            if (threadIdx.x == 0) sh_shift = fixed_shift(amax);
-            __syncthreads();
-            sh = sh_shift;
+            for (int i = tid; i < K; i += kGvCons * 32) m = fmaxf(m, fabsf(bf16_to_f32(xb[i])));
+            m = warp_max_f32(m);
+            if (lane == 0) red[warp] = m;
+            named_bar_sync(1, kGvCons * 32);
+            float amax = 0.0f;
+#pragma unroll
+            for (int w = 0; w < kGvCons; w++) amax = fmaxf(amax, red[w]);
+            sh = fixed_shift(amax);
         }
         SegX<NL> X;
         gemv_load_x<NL>(X, xt, seg, sh);
-        __syncthreads();  // lut ready (first iteration) / red reuse
         const float xscale = (NL == 1 && xs != nullptr) ? xs[t] : 1.0f;
+        auto epilogue = [&](int r0, int nr, int st, int row, long long S) {
+            const float sc = (rs_bulk && row < (nr & ~3)) ? s_rs[st * kGvMaxRows + row] : __ldg(rs + r0 + row);
+            const int64_t o = (int64_t)t * M + r0 + row;
+            if (NL == 1) {
+                if (acc_out) acc_out[o] = (int32_t)S;
+                float v = __fmul_rn(__int2float_rn((int)S), sc);
+                if (xs != nullptr) v = __fmul_rn(v, xscale);
+                y[o] = v;
+            } else {
+                y[o] = (float)(ldexp((double)S, -sh) * (double)sc);
+            }
+        };
 
-        for (int base = blockIdx.x * rows_per_cta; base < M; base += gridDim.x * rows_per_cta) {
-            const int row = base + rgroup * RPW + sub;
-            int a = 0, b = 0;
-            if (row < M) {
-                const uint4 wb = __ldg(reinterpret_cast<const uint4 *>(Wp + (int64_t)row * row_bytes) + seg);
-                int acc[NL];
+        for (int j = 0; j < my_n; j++, n++) {
+            const int st = n % kGvStages;
+            if (alive) alive = mbar_wait(&full[st], (uint32_t)(n / kGvStages) & 1u, kGvWaitNs, status);
+            int r0, nr;
+            chunk_rows(n, r0, nr);
+            const unsigned char *stage = ring + (size_t)st * kGvStageBytes;
+            if (alive && NS == 1) {
+                for (int p = warp; p * RPW < nr; p += kGvCons) {
+                    const int row = p * RPW + sub;
+                    const bool valid = row < nr;
+                    const uint4 wv = valid ? *reinterpret_cast<const uint4 *>(stage + (size_t)row * RB + gl * 16)
+                                           : make_uint4(0u, 0u, 0u, 0u);
+                    int acc[NL];
 #pragma unroll
-                for (int l = 0; l < NL; l++) acc[l] = 0;
-                seg_dot<NL>(wb, X, lut, lane4, acc);
-                acc_to_pair<NL>(acc, a, b);
-            }
-            a = group_sum<G>(a);
-            if (NL > 1) b = group_sum<G>(b);
-            long long S = pair_value(NL, a, b);
-            if (NS > 1) {
-                __syncthreads();
-                if (gl == 0) part[warp * RPW + sub] = S;
-                __syncthreads();
-                if (slice != 0) continue;
-                S = 0;
-                for (int sl = 0; sl < NS; sl++) S += part[(rgroup * NS + sl) * RPW + sub];  // fixed order
-            }
-            if (gl == 0 && row < M) {
-                if (NL == 1) {
-                    if (acc_out) acc_out[(int64_t)t * M + row] = (int32_t)S;
-                    float v = __fmul_rn(__int2float_rn((int)S), rs[row]);
-                    if (xs != nullptr) v = __fmul_rn(v, xscale);
-                    y[(int64_t)t * M + row] = v;
-                } else {
-                    y[(int64_t)t * M + row] = (float)(ldexp((double)S, -sh) * (double)rs[row]);
+                    for (int l = 0; l < NL; l++) acc[l] = 0;
+                    seg_dot<NL>(wv, X, lut, lane4, acc);
+                    int a, b;
+                    acc_to_pair<NL>(acc, a, b);
+                    a = group_sum<G>(a);
+                    if (NL > 1) b = group_sum<G>(b);
+                    if (valid && gl == 0) epilogue(r0, nr, st, row, pair_value(NL, a, b));
+                }
+            } else if (alive && rg < ngroups) {
+                for (int row = rg; row < nr; row += ngroups) {
+                    const uint4 wv = *reinterpret_cast<const uint4 *>(stage + (size_t)row * RB + slice * 512 + lane * 16);
+                    int acc[NL];
+#pragma unroll
+                    for (int l = 0; l < NL; l++) acc[l] = 0;
+                    seg_dot<NL>(wv, X, lut, lane4, acc);
+                    int a, b;
+                    acc_to_pair<NL>(acc, a, b);
+                    a = group_sum<32>(a);
+                    if (NL > 1) b = group_sum<32>(b);
+                    if (lane == 0) {
+                        const int q = st * kGvMaxSplitRows + row;
+                        atomicAdd(&s_acc[q], (unsigned long long)pair_value(NL, a, b));
+                        __threadfence_block();
+                        if (atomicAdd(&s_cnt[q], 1) == NS - 1) {  // the last slice of this row
+                            const long long S = (long long)atomicExch(&s_acc[q], 0ull);
+                            s_cnt[q] = 0;
+                            epilogue(r0, nr, st, row, S);
+                        }
+                    }
                 }
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
         }
-        __syncthreads();
+        if (NL > 1) named_bar_sync(1, kGvCons * 32);  // red[] is rewritten by the next token
     }
+}
+
+static int device_sms() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
 }
 
 template <int NL>
 static cudaError_t gemv_dispatch(const uint8_t *Wp, const float *rs, int M, int K, const void *x,
                                  const float *xs, int T, int32_t *acc, float *y, cudaStream_t s) {
-    const int KS = K > 2048 ? 2048 : K;
-    const int NS = K / KS;
-    const int G = KS / 64;
-    const int RPW = 32 / G;
-    const int rows_per_cta = (kGemvWarps / NS) * RPW;
-    int grid = (M + rows_per_cta - 1) / rows_per_cta;
-    if (grid > 148 * 8) grid = 148 * 8;
-    const size_t smem = kLutBytes + sizeof(long long) * kGemvWarps * 32;
-#define TERN_GEMV_CASE(GG)                                                                              \
-    case GG: {                                                                                          \
-        auto kern = gemv_kernel<NL, GG>;                                                                \
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);            \
-        kern<<<grid, kGemvWarps * 32, smem, s>>>(Wp, rs, M, K, NS, x, xs, T, acc, y);                 \
-        break;                                                                                          \
+    const int RB = K / 4;
+    const int NS = K > 2048 ? K / 2048 : 1;
+    const int G = NS > 1 ? 32 : RB / 16;
+    const int sms = device_sms();
+    // rows per chunk: a full stage, fewer when that would leave SMs without a chunk; always a
+    // multiple of 4 so that every chunk's scales start on a 16-byte boundary
+    int R = (kGvStageBytes / RB) & ~3;  // >= 4: RB <= 4096
+    if (R > kGvMaxRows) R = kGvMaxRows;
+    if ((M + R - 1) / R < sms) {
+        int r = (M + sms - 1) / sms;
+        r = (r + 3) & ~3;
+        if (r < R) R = r;
+    }
+    const int nchunks = (M + R - 1) / R;
+    const int grid = nchunks < sms ? nchunks : sms;
+    const size_t smem = gv_smem_bytes();
+#define TERN_GEMV_CASE(GG)                                                                               \
+    case GG: {                                                                                           \
+        auto kern = gemv_kernel<NL, GG>;                                                                 \
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);             \
+        kern<<<grid, kGvThreads, smem, s>>>(Wp, rs, M, K, NS, R, nchunks, x, xs, T, acc, y, status_word()); \
+        break;                                                                                           \
     }
     switch (G) {
         TERN_GEMV_CASE(1)

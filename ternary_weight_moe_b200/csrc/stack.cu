@@ -34,6 +34,7 @@
 
 #include "kernels.h"
 #include "tern_common.cuh"
+#include "tma.cuh"
 
 namespace tern {
 
@@ -65,53 +66,7 @@ struct StackParams {
     int dn_rows;                  // max output rows per CTA (even)
 };
 
-// ------------------------------------------------------------------ PTX helpers
-__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-// Shared buffers are rewritten by TMA only after every thread's generic reads of them are
-// ordered before the issuing thread by a CTA (or slot) barrier; write-after-read across the
-// generic and async proxies needs no proxy fence.
-__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ unsigned long long gtimer() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-// bounded wait on an mbarrier phase; false on timeout (status set)
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, long long limit_ns, int *status) {
-    if (mbar_test(bar, parity)) return true;
-    const unsigned long long t0 = gtimer();
-    while (!mbar_test(bar, parity)) {
-        if ((long long)(gtimer() - t0) > limit_ns) {
-            set_status(status, TERN_ETIMEOUT);
-            return false;
-        }
-    }
-    return true;
-}
-
+// ------------------------------------------------------------------ exchange words
 // ---- flag-carrying words: one 64-bit access carries payload and tag together
 __device__ __forceinline__ void ll_store(unsigned long long *p, uint32_t val, uint32_t tag) {
     const unsigned long long w = ((unsigned long long)tag << 32) | (unsigned long long)val;
@@ -121,10 +76,6 @@ __device__ __forceinline__ unsigned long long ll_load(const unsigned long long *
     unsigned long long w;
     asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
     return w;
-}
-// barrier over `nthreads` threads (multiple of 32) using hardware barrier `id` (1..15)
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // Gather n tagged words (n*8 bytes, 16-byte aligned) from global memory into shared memory
@@ -228,11 +179,17 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
     __shared__ float s_redf[kStackWarps];
     __shared__ double s_part[kStackWarps][kStackWarps];
     __shared__ double s_logit[256];
+    __shared__ __align__(16) uint32_t s_gm[32];  // top-k scratch
+    __shared__ int s_nc;
+    __shared__ ulonglong2 s_cand[256];
     __shared__ int s_idx[kSK];
     __shared__ double s_gate[kSK];
     __shared__ long long s_S[64][2];
     __shared__ double s_ye[64][kSK];
     __shared__ float s_sg[64], s_su[64], s_sd[kSK * 64];
+    // the layers' pointers, copied once: a dynamically indexed kernel parameter is a constant
+    // cache line fetched from L2 on the critical path of every layer
+    __shared__ StackLayerDev s_layer[kMaxStackLayers];
 
     const int d = p.d, f = p.f, E = p.E, k = p.k, P = p.P;
     const int c = blockIdx.x;
@@ -279,6 +236,12 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
     }
 
     lut_fill(lut);
+    {
+        constexpr int kW = (int)(sizeof(StackLayerDev) / sizeof(uint64_t));
+        static_assert(sizeof(StackLayerDev) % sizeof(uint64_t) == 0, "pointer table");
+        for (int q = tid; q < p.n_layers * kW; q += kStackThreads)
+            reinterpret_cast<uint64_t *>(s_layer)[q] = reinterpret_cast<const uint64_t *>(p.layer)[q];
+    }
     if (tid == 0) {
         mbar_init(&mb_router, 1);
         mbar_init(&mb_gu0, 1);
@@ -296,11 +259,11 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
         mbar_expect_tx(&mb_router, (uint32_t)(nr * d * 2));
         n_rt++;
         for (int r = 0; r < nr; r++)
-            bulk_g2s(rbuf + (size_t)r * d, p.layer[0].router + (size_t)(c + r * P) * d, (uint32_t)(d * 2), &mb_router);
+            bulk_g2s(rbuf + (size_t)r * d, s_layer[0].router + (size_t)(c + r * P) * d, (uint32_t)(d * 2), &mb_router);
     }
 
     for (int l = 0; l < p.n_layers && alive; l++) {
-        const StackLayerDev &Ly = p.layer[l];
+        const StackLayerDev &Ly = s_layer[l];
         const uint32_t par = (uint32_t)(l & 1);
         const uint32_t tag = (ep << 7) | (uint32_t)(l + 1);  // never 0 (a zeroed workspace holds 0)
         TSTAMP(l, 0)
@@ -424,21 +387,23 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             mbar_expect_tx(&mb_router, (uint32_t)(nr * d * 2));
             n_rt++;
             for (int q = 0; q < nr; q++)
-                bulk_g2s(rbuf + (size_t)q * d, p.layer[l + 1].router + (size_t)(c + q * P) * d, (uint32_t)(d * 2),
+                bulk_g2s(rbuf + (size_t)q * d, s_layer[l + 1].router + (size_t)(c + q * P) * d, (uint32_t)(d * 2),
                          &mb_router);
         }
         // ------------------------------------------------------------ B: logits, top-k, copies
+        double my_logit = 0.0;  // logit `tid` (E <= 256 on this path)
         {
             const bool ok = ll_gather(p.lll, 2 * E, tag, xch, &mb_x, xph, lim, p.status);
-            for (int e = tid; e < E; e += kStackThreads)
-                s_logit[e] = __longlong_as_double(
-                    (long long)(((unsigned long long)(uint32_t)xch[2 * e] << 32) | (uint32_t)xch[2 * e + 1]));
+            if (tid < E) {
+                my_logit = __longlong_as_double(
+                    (long long)(((unsigned long long)(uint32_t)xch[2 * tid] << 32) | (uint32_t)xch[2 * tid + 1]));
+                s_logit[tid] = my_logit;
+            }
             alive = __syncthreads_and(ok ? 1 : 0) && alive;
         }
         TSTAMP(l, 4)
         // only the expert indices are on the critical path; the gates are needed in the combine
-        if (warp == 0) warp_topk_select<8>(s_logit, E, k, s_idx);  // E <= 256 on this path
-        __syncthreads();
+        block_topk_select(my_logit, E, k, s_idx, s_gm, &s_nc, s_cand);
         TSTAMP(l, 5)
         if (warp == 0) {
             // copies: lanes 0..3 first-half gate/up segments, 4..7 second half (each half spans

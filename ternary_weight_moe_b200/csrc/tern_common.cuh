@@ -326,6 +326,61 @@ __device__ __forceinline__ void warp_topk_select(const double *lg, int E, int k,
     __syncwarp();
 }
 
+// Top-k expert indices of E <= 256 logits by a whole CTA (blockDim.x >= 256), through a
+// filter instead of k rounds of warp-wide maxima.  Order: larger logit first, equal logits
+// by lower index.  Thread t < E holds logit t (`mine`); every thread of the block calls this.
+//  1. h_t = high word of t's order key (sign, exponent, 20 leading mantissa bits); the
+//     32 groups of 8 consecutive logits each take their largest h;
+//  2. tau = the k-th largest group maximum (groups ordered by maximum, then group number);
+//  3. every logit with h_t >= tau is a candidate.  At least k groups hold a logit with
+//     h >= tau, so the k best logits are all candidates -- typically a few more than k pass;
+//  4. each candidate's rank = the number of candidates ordered before it (full 64-bit key,
+//     then index); ranks below k land in idx_out.
+// Shared scratch: s_gm[32] (16-byte aligned), *s_nc, s_cand[256].  Ends with a CTA barrier:
+// idx_out (shared memory) is then visible to every thread.
+__device__ __forceinline__ void block_topk_select(double mine, int E, int k, int32_t *idx_out, uint32_t *s_gm,
+                                                  int *s_nc, ulonglong2 *s_cand) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    const bool has = tid < E;
+    const unsigned long long key = has ? f64_order_key(mine) : 0ull;
+    const uint32_t h = (uint32_t)(key >> 32);
+    uint32_t gm = h;
+    gm = max(gm, __shfl_xor_sync(0xFFFFFFFFu, gm, 1));
+    gm = max(gm, __shfl_xor_sync(0xFFFFFFFFu, gm, 2));
+    gm = max(gm, __shfl_xor_sync(0xFFFFFFFFu, gm, 4));
+    if (tid < 256 && (tid & 7) == 0) s_gm[tid >> 3] = gm;
+    if (tid == 0) *s_nc = 0;
+    __syncthreads();
+    if (tid < 256) {
+        // every warp finds tau itself: lane g ranks group g
+        const uint32_t m = s_gm[lane];
+        int above = 0;
+#pragma unroll
+        for (int q4 = 0; q4 < 8; q4++) {
+            const uint4 v = reinterpret_cast<const uint4 *>(s_gm)[q4];
+            const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int z = 0; z < 4; z++) above += (vv[z] > m || (vv[z] == m && 4 * q4 + z < lane)) ? 1 : 0;
+        }
+        const unsigned who = __ballot_sync(0xFFFFFFFFu, above == k - 1);
+        const uint32_t tau = __shfl_sync(0xFFFFFFFFu, m, __ffs(who) - 1);
+        // slot order is irrelevant: ranks come from comparisons, not positions
+        if (has && h >= tau) s_cand[atomicAdd(s_nc, 1)] = make_ulonglong2(key, (unsigned long long)tid);
+    }
+    __syncthreads();
+    const int nc = *s_nc;
+    for (int i = tid; i < nc; i += blockDim.x) {
+        const ulonglong2 me = s_cand[i];
+        int r = 0;
+        for (int q = 0; q < nc; q++) {
+            const ulonglong2 o = s_cand[q];
+            r += (o.x > me.x || (o.x == me.x && o.y < me.y)) ? 1 : 0;
+        }
+        if (r < k) idx_out[r] = (int)me.y;
+    }
+    __syncthreads();
+}
+
 // Renormalised gates of the selected experts: g_i = exp(l_i - l_0) / sum_j exp(l_j - l_0),
 // lanes 0..k-1 each one exp in fp64, the sum taken in top-k order.
 __device__ __forceinline__ void warp_topk_gates(const double *lg, int k, const int32_t *idx, double *g64, float *g32) {

@@ -59,7 +59,8 @@ def test_gemv_int8_256x512_bit_exact(cuda_dev):
     assert (y.cpu().numpy() == y_ref).all()
 
 
-@pytest.mark.parametrize("M,K,T", [(256, 512, 3), (77, 64, 2), (130, 128, 1), (33, 8192, 2), (1000, 2048, 5)])
+@pytest.mark.parametrize("M,K,T", [(256, 512, 3), (77, 64, 2), (130, 128, 1), (33, 8192, 2), (1000, 2048, 5),
+                                   (5003, 8192, 2), (77, 6144, 2), (301, 14336, 1)])
 def test_gemv_int8_shapes_bit_exact(cuda_dev, M, K, T):
     w = synth.ternary_codes(M + K, 0, M * K, synth.P0_SPARSE).reshape(M, K)
     s = synth.uniform_f32(M + 1, 0, M, 0.01, 0.05)
@@ -88,7 +89,7 @@ def test_gemv_bf16_sweep_tolerance(cuda_dev, M, K):
     assert np.abs(y - y_ref).max() <= 1e-4 * xn
 
 
-@pytest.mark.parametrize("M,K,T", [(100, 64, 3), (333, 1024, 2), (64, 16384, 1)])
+@pytest.mark.parametrize("M,K,T", [(100, 64, 3), (333, 1024, 2), (64, 16384, 1), (4099, 16384, 1), (50, 10240, 2)])
 def test_gemv_bf16_ragged_tolerance(cuda_dev, M, K, T):
     w = synth.ternary_codes(M * 3 + K, 0, M * K, synth.P0_SPARSE).reshape(M, K)
     s = synth.uniform_f32(M + 5, 0, M, 0.01, 0.05)
