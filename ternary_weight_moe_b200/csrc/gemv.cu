@@ -101,46 +101,16 @@ cudaError_t launch_quant_absmax(const uint16_t *x, int64_t T, int64_t n, int8_t 
 }
 
 // ------------------------------------------------------------------------ ternary GEMV
-// Fill the limb registers of one lane for the segment `seg` (64 codes) of token vector xt.
-//  int8 (NL == 1): the 64 int8 values as 16 words;
-//  bf16 (NL == 3): 24-bit fixed point with per-token shift sh.
-template <int NL>
-__device__ __forceinline__ void gemv_load_x(SegX<NL> &X, const void *xt, int64_t seg, int sh) {
-    if (NL == 1) {
-        const uint4 *p = reinterpret_cast<const uint4 *>(static_cast<const int8_t *>(xt) + seg * 64);
+// The 64 int8 activations of segment `seg` (64 codes) of token vector xt as 16 words.
+__device__ __forceinline__ void gemv_load_x(SegX<1> &X, const int8_t *xt, int seg) {
+    const uint4 *p = reinterpret_cast<const uint4 *>(xt + (int64_t)seg * 64);
 #pragma unroll
-        for (int v = 0; v < 4; v++) {
-            const uint4 t = __ldg(p + v);
-            X.w[0][4 * v + 0] = t.x;
-            X.w[0][4 * v + 1] = t.y;
-            X.w[0][4 * v + 2] = t.z;
-            X.w[0][4 * v + 3] = t.w;
-        }
-    } else {
-        const uint4 *p = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(xt) + seg * 64);
-#pragma unroll
-        for (int v = 0; v < 8; v++) {  // 8 bf16 per uint4 -> two limb words per limb
-            const uint4 t = __ldg(p + v);
-            const uint32_t hw[4] = {t.x, t.y, t.z, t.w};
-#pragma unroll
-            for (int half = 0; half < 2; half++) {
-                uint32_t wl[3] = {0, 0, 0};
-#pragma unroll
-                for (int e = 0; e < 4; e++) {
-                    const uint32_t pairw = hw[2 * half + (e >> 1)];
-                    const uint16_t b = (uint16_t)((e & 1) ? (pairw >> 16) : (pairw & 0xFFFFu));
-                    uint32_t h, m, l;
-                    fixed_limbs(bf16_to_f32(b), sh, h, m, l);
-                    wl[0] |= h << (8 * e);
-                    wl[1] |= m << (8 * e);
-                    wl[2] |= l << (8 * e);
-                }
-                const int word = 2 * v + half;
-                X.w[0][word] = wl[0];
-                X.w[NL > 1 ? 1 : 0][word] = wl[1];
-                X.w[NL > 2 ? 2 : 0][word] = wl[2];
-            }
-        }
+    for (int v = 0; v < 4; v++) {
+        const uint4 t = __ldg(p + v);
+        X.w[0][4 * v + 0] = t.x;
+        X.w[0][4 * v + 1] = t.y;
+        X.w[0][4 * v + 2] = t.z;
+        X.w[0][4 * v + 3] = t.w;
     }
 }
 
@@ -148,23 +118,40 @@ __device__ __forceinline__ void gemv_load_x(SegX<NL> &X, const void *xt, int64_t
 // One CTA per SM.  A producer warp streams chunks of R consecutive rows (R*K/4 contiguous
 // bytes, up to 16 KB) plus their row scales into a ring of kGvStages shared-memory stages
 // with bulk copies; 16 consumer warps decode each stage as it lands and release it through
-// an mbarrier, so about 96 KB of weights per SM stay in flight while the consumers compute.
-//   K <= 2048: G = K/64 lanes per row, 32/G rows per warp pass, no cross-warp combine;
+// an mbarrier, so about 80 KB of weights per SM stay in flight while the consumers compute.
+// Waiting warps sleep inside mbarrier.try_wait instead of spinning.
+//   K <= 2048: G = K/64 lanes per row, 32/G rows per warp pass; every warp takes two passes
+//              at a time (two independent dot chains) and reduces both with one shuffle tree;
 //   K  > 2048: NS = K/2048 slices of 512 bytes; warp w takes slice w % NS of rows
-//              w / NS, w / NS + 16/NS, ...; the exact integer partial sums of a row meet in
-//              shared memory (order-free 64-bit atomic adds), and the warp that adds the last
-//              one writes the row.
+//              w / NS, w / NS + 16/NS, ...; each slice's exact integer partial goes to shared
+//              memory and the producer warp sums the NS partials of a row (fixed order) and
+//              writes it before it refills the stage.
+// bf16 activations: the 24-bit fixed-point limbs of the token are built once per CTA in
+// shared memory; each lane then keeps its segment's limbs in registers.
 constexpr int kGvCons = 16;  // consumer warps
-constexpr int kGvThreads = (kGvCons + 1) * 32;
-constexpr int kGvStages = 6;
+constexpr int kGvConsThreads = kGvCons * 32;
+constexpr int kGvThreads = kGvConsThreads + 32;
+constexpr int kGvStages = 5;
 constexpr int kGvStageBytes = 16384;
-constexpr int kGvMaxRows = 128;    // rows per chunk (scale ring entries per stage)
+constexpr int kGvMaxRows = 128;      // rows per chunk (scale ring entries per stage)
 constexpr int kGvMaxSplitRows = 16;  // rows per chunk when K > 2048 (16 KB / 1 KB)
+constexpr int kGvMaxSlices = 8;
+constexpr int kGvMaxK = 16384;
+constexpr int kGvMaxT = 64;
 constexpr long long kGvWaitNs = 1000000000ll;
 
-constexpr size_t gv_smem_bytes() {
-    return (size_t)kLutBytes + (size_t)kGvStages * kGvStageBytes + (size_t)kGvStages * kGvMaxRows * 4 +
-           (size_t)kGvStages * kGvMaxSplitRows * (8 + 4);
+struct GvSmem {
+    uint32_t lut, ring, rs, part, xl, total;
+};
+__host__ __device__ constexpr GvSmem gv_smem() {
+    return GvSmem{0u,
+                  (uint32_t)kLutBytes,
+                  (uint32_t)(kLutBytes + kGvStages * kGvStageBytes),
+                  (uint32_t)(kLutBytes + kGvStages * kGvStageBytes + kGvStages * kGvMaxRows * 4),
+                  (uint32_t)(kLutBytes + kGvStages * kGvStageBytes + kGvStages * kGvMaxRows * 4 +
+                             kGvStages * kGvMaxSplitRows * kGvMaxSlices * 8),
+                  (uint32_t)(kLutBytes + kGvStages * kGvStageBytes + kGvStages * kGvMaxRows * 4 +
+                             kGvStages * kGvMaxSplitRows * kGvMaxSlices * 8 + 3 * (kGvMaxK / 4) * 4)};
 }
 
 template <int NL, int G>
@@ -175,11 +162,13 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t full[kGvStages], empty[kGvStages];
     __shared__ float red[32];
-    uint32_t *lut = reinterpret_cast<uint32_t *>(smem);
-    unsigned char *ring = smem + kLutBytes;
-    float *s_rs = reinterpret_cast<float *>(ring + (size_t)kGvStages * kGvStageBytes);             // [S][kGvMaxRows]
-    unsigned long long *s_acc = reinterpret_cast<unsigned long long *>(s_rs + kGvStages * kGvMaxRows);  // [S][16]
-    int *s_cnt = reinterpret_cast<int *>(s_acc + kGvStages * kGvMaxSplitRows);                    // [S][16]
+    __shared__ int s_shift[kGvMaxT];
+    constexpr GvSmem L = gv_smem();
+    uint32_t *lut = reinterpret_cast<uint32_t *>(smem + L.lut);
+    unsigned char *ring = smem + L.ring;
+    float *s_rs = reinterpret_cast<float *>(smem + L.rs);           // [S][kGvMaxRows]
+    long long *s_part = reinterpret_cast<long long *>(smem + L.part);  // [S][16][8]
+    uint32_t *xl = reinterpret_cast<uint32_t *>(smem + L.xl);       // [NL][K/4] limb words
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int RB = K / 4;
@@ -201,9 +190,22 @@ __global__ void __launch_bounds__(kGvThreads, 1)
         bulk_g2s(ring + (size_t)st * kGvStageBytes, Wp + (size_t)r0 * RB, wbytes, &full[st]);
         if (sbytes) bulk_g2s(s_rs + st * kGvMaxRows, rs + r0, sbytes, &full[st]);
     };
+    // y for row r0 + row of token t from its exact integer sum S
+    auto finish = [&](int t, int r0, int nr, int st, int row, long long S) {
+        const float sc = (rs_bulk && row < (nr & ~3)) ? s_rs[st * kGvMaxRows + row] : __ldg(rs + r0 + row);
+        const int64_t o = (int64_t)t * M + r0 + row;
+        if (NL == 1) {
+            if (acc_out) acc_out[o] = (int32_t)S;
+            float v = __fmul_rn(__int2float_rn((int)S), sc);
+            if (xs != nullptr) v = __fmul_rn(v, xs[t]);
+            y[o] = v;
+        } else {
+            y[o] = (float)(ldexp((double)S, -s_shift[t]) * (double)sc);
+        }
+    };
 
     int issued = 0;
-    if (tid == kGvCons * 32) {
+    if (tid == kGvConsThreads) {
         for (int q = 0; q < kGvStages; q++) {
             mbar_init(&full[q], 1);
             mbar_init(&empty[q], kGvCons);
@@ -213,25 +215,38 @@ __global__ void __launch_bounds__(kGvThreads, 1)
         for (; issued < kGvStages && issued < total; issued++) issue(issued);
     }
     lut_fill(lut);
-    for (int q = tid; q < kGvStages * kGvMaxSplitRows; q += blockDim.x) {
-        s_acc[q] = 0ull;
-        s_cnt[q] = 0;
-    }
     __syncthreads();
 
     if (warp == kGvCons) {  // ------------------------------------------------ producer
-        if (lane == 0) {
-            for (; issued < total; issued++) {
-                const int st = issued % kGvStages;
-                if (!mbar_wait(&empty[st], (uint32_t)((issued / kGvStages) - 1) & 1u, kGvWaitNs, status)) break;
-                issue(issued);
+        bool ok = true;
+        // iteration n: stage n % S is free again once chunk n - S is consumed; for K > 2048
+        // that chunk's rows are summed and written here, then chunk n is issued
+        for (int n = kGvStages; ok && n < total + kGvStages; n++) {
+            const int st = n % kGvStages;
+            ok = mbar_wait_sleep(&empty[st], (uint32_t)((n / kGvStages) - 1) & 1u, kGvWaitNs, status);
+            if (!ok) break;
+            if (NS > 1) {
+                const int m = n - kGvStages;
+                int r0, nr;
+                chunk_rows(m, r0, nr);
+                if (lane < nr) {
+                    long long S = 0;
+                    for (int sl = 0; sl < NS; sl++) S += s_part[(st * kGvMaxSplitRows + lane) * kGvMaxSlices + sl];
+                    finish(m / my_n, r0, nr, st, lane, S);
+                }
+                __syncwarp();
             }
-            // leave only after every copy into this CTA's shared memory has landed
+            if (n < total && lane == 0) {
+                issue(n);
+                issued = n + 1;
+            }
+        }
+        // on a timeout: leave only after every copy into this CTA's shared memory has landed
+        if (!ok && lane == 0)
             for (int q = 0; q < kGvStages && q < issued; q++) {
                 const int cnt = (issued - q + kGvStages - 1) / kGvStages;
                 mbar_wait(&full[q], (uint32_t)(cnt - 1) & 1u, kGvWaitNs, status);
             }
-        }
         return;
     }
 
@@ -239,93 +254,108 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     constexpr int RPW = 32 / G;  // rows per warp pass (K <= 2048)
     const int sub = lane / G, gl = lane % G;
     const int slice = warp % NS, rg = warp / NS, ngroups = kGvCons / NS;
-    const int64_t seg = (NS > 1) ? (int64_t)slice * 32 + lane : (int64_t)gl;
+    const int seg = (NS > 1) ? slice * 32 + lane : gl;
     const uint32_t lane4 = (uint32_t)lane << 2;
     bool alive = true;
     int n = 0;
     for (int t = 0; t < T; t++) {
-        int sh = 0;
-        const void *xt;
-        if (NL == 1) {
-            xt = static_cast<const int8_t *>(x) + (int64_t)t * K;
+        SegX<NL> X;
+        if constexpr (NL == 1) {
+            gemv_load_x(X, static_cast<const int8_t *>(x) + (int64_t)t * K, seg);
         } else {
             const uint16_t *xb = static_cast<const uint16_t *>(x) + (int64_t)t * K;
-            xt = xb;
             float m = 0.0f;
-            for (int i = tid; i < K; i += kGvCons * 32) m = fmaxf(m, fabsf(bf16_to_f32(xb[i])));
+            for (int i = tid; i < K; i += kGvConsThreads) m = fmaxf(m, fabsf(bf16_to_f32(xb[i])));
             m = warp_max_f32(m);
             if (lane == 0) red[warp] = m;
-            named_bar_sync(1, kGvCons * 32);
+            named_bar_sync(1, kGvConsThreads);
             float amax = 0.0f;
 #pragma unroll
             for (int w = 0; w < kGvCons; w++) amax = fmaxf(amax, red[w]);
-            sh = fixed_shift(amax);
-        }
-        SegX<NL> X;
-        gemv_load_x<NL>(X, xt, seg, sh);
-        const float xscale = (NL == 1 && xs != nullptr) ? xs[t] : 1.0f;
-        auto epilogue = [&](int r0, int nr, int st, int row, long long S) {
-            const float sc = (rs_bulk && row < (nr & ~3)) ? s_rs[st * kGvMaxRows + row] : __ldg(rs + r0 + row);
-            const int64_t o = (int64_t)t * M + r0 + row;
-            if (NL == 1) {
-                if (acc_out) acc_out[o] = (int32_t)S;
-                float v = __fmul_rn(__int2float_rn((int)S), sc);
-                if (xs != nullptr) v = __fmul_rn(v, xscale);
-                y[o] = v;
-            } else {
-                y[o] = (float)(ldexp((double)S, -sh) * (double)sc);
+            const int sh = fixed_shift(amax);
+            if (tid == 0) s_shift[t] = sh;
+            // limb words of four consecutive values, one word per limb, built once per CTA
+            for (int wd = tid; wd < K / 4; wd += kGvConsThreads) {
+                const uint2 v = __ldg(reinterpret_cast<const uint2 *>(xb) + wd);
+                const uint32_t hw[2] = {v.x, v.y};
+                uint32_t wl[3] = {0u, 0u, 0u};
+#pragma unroll
+                for (int e = 0; e < 4; e++) {
+                    const uint16_t bb = (uint16_t)((e & 1) ? (hw[e >> 1] >> 16) : (hw[e >> 1] & 0xFFFFu));
+                    uint32_t h, mi, lo;
+                    fixed_limbs(bf16_to_f32(bb), sh, h, mi, lo);
+                    wl[0] |= h << (8 * e);
+                    wl[1] |= mi << (8 * e);
+                    wl[2] |= lo << (8 * e);
+                }
+                xl[wd] = wl[0];
+                xl[K / 4 + wd] = wl[1];
+                xl[2 * (K / 4) + wd] = wl[2];
             }
-        };
+            named_bar_sync(1, kGvConsThreads);
+            seg_load_x_smem<NL>(X, xl, K / 4, seg);
+        }
 
         for (int j = 0; j < my_n; j++, n++) {
             const int st = n % kGvStages;
-            if (alive) alive = mbar_wait(&full[st], (uint32_t)(n / kGvStages) & 1u, kGvWaitNs, status);
+            if (alive) alive = mbar_wait_sleep(&full[st], (uint32_t)(n / kGvStages) & 1u, kGvWaitNs, status);
             int r0, nr;
             chunk_rows(n, r0, nr);
             const unsigned char *stage = ring + (size_t)st * kGvStageBytes;
             if (alive && NS == 1) {
-                for (int p = warp; p * RPW < nr; p += kGvCons) {
-                    const int row = p * RPW + sub;
-                    const bool valid = row < nr;
-                    const uint4 wv = valid ? *reinterpret_cast<const uint4 *>(stage + (size_t)row * RB + gl * 16)
-                                           : make_uint4(0u, 0u, 0u, 0u);
-                    int acc[NL];
+                // passes p and p + 16 of this warp at once
+                for (int p = warp; p * RPW < nr; p += 2 * kGvCons) {
+                    const int rowA = p * RPW + sub, rowB = (p + kGvCons) * RPW + sub;
+                    const bool vA = rowA < nr, vB = rowB < nr;
+                    const uint4 wA = vA ? *reinterpret_cast<const uint4 *>(stage + (size_t)rowA * RB + gl * 16)
+                                        : make_uint4(0u, 0u, 0u, 0u);
+                    const uint4 wB = vB ? *reinterpret_cast<const uint4 *>(stage + (size_t)rowB * RB + gl * 16)
+                                        : make_uint4(0u, 0u, 0u, 0u);
+                    int accA[NL], accB[NL];
 #pragma unroll
-                    for (int l = 0; l < NL; l++) acc[l] = 0;
-                    seg_dot<NL>(wv, X, lut, lane4, acc);
-                    int a, b;
-                    acc_to_pair<NL>(acc, a, b);
-                    a = group_sum<G>(a);
-                    if (NL > 1) b = group_sum<G>(b);
-                    if (valid && gl == 0) epilogue(r0, nr, st, row, pair_value(NL, a, b));
+                    for (int l = 0; l < NL; l++) accA[l] = accB[l] = 0;
+                    seg_dot<NL>(wA, X, lut, lane4, accA);
+                    seg_dot<NL>(wB, X, lut, lane4, accB);
+                    int aA, bA, aB, bB;
+                    acc_to_pair<NL>(accA, aA, bA);
+                    acc_to_pair<NL>(accB, aB, bB);
+                    if (G == 1) {
+                        if (vA) finish(t, r0, nr, st, rowA, pair_value(NL, aA, bA));
+                        if (vB) finish(t, r0, nr, st, rowB, pair_value(NL, aB, bB));
+                    } else {
+                        const int a = group_sum2<(G > 1 ? G : 2)>(aA, aB);
+                        const int b = (NL > 1) ? group_sum2<(G > 1 ? G : 2)>(bA, bB) : 0;
+                        if (gl == 0 && vA) finish(t, r0, nr, st, rowA, pair_value(NL, a, b));
+                        if (gl == G / 2 && vB) finish(t, r0, nr, st, rowB, pair_value(NL, a, b));
+                    }
                 }
             } else if (alive && rg < ngroups) {
-                for (int row = rg; row < nr; row += ngroups) {
-                    const uint4 wv = *reinterpret_cast<const uint4 *>(stage + (size_t)row * RB + slice * 512 + lane * 16);
-                    int acc[NL];
+                for (int rowA = rg; rowA < nr; rowA += 2 * ngroups) {
+                    const int rowB = rowA + ngroups;
+                    const bool vB = rowB < nr;
+                    const uint4 wA = *reinterpret_cast<const uint4 *>(stage + (size_t)rowA * RB + slice * 512 + lane * 16);
+                    const uint4 wB = vB ? *reinterpret_cast<const uint4 *>(stage + (size_t)rowB * RB + slice * 512 +
+                                                                             lane * 16)
+                                        : make_uint4(0u, 0u, 0u, 0u);
+                    int accA[NL], accB[NL];
 #pragma unroll
-                    for (int l = 0; l < NL; l++) acc[l] = 0;
-                    seg_dot<NL>(wv, X, lut, lane4, acc);
-                    int a, b;
-                    acc_to_pair<NL>(acc, a, b);
-                    a = group_sum<32>(a);
-                    if (NL > 1) b = group_sum<32>(b);
-                    if (lane == 0) {
-                        const int q = st * kGvMaxSplitRows + row;
-                        atomicAdd(&s_acc[q], (unsigned long long)pair_value(NL, a, b));
-                        __threadfence_block();
-                        if (atomicAdd(&s_cnt[q], 1) == NS - 1) {  // the last slice of this row
-                            const long long S = (long long)atomicExch(&s_acc[q], 0ull);
-                            s_cnt[q] = 0;
-                            epilogue(r0, nr, st, row, S);
-                        }
-                    }
+                    for (int l = 0; l < NL; l++) accA[l] = accB[l] = 0;
+                    seg_dot<NL>(wA, X, lut, lane4, accA);
+                    seg_dot<NL>(wB, X, lut, lane4, accB);
+                    int aA, bA, aB, bB;
+                    acc_to_pair<NL>(accA, aA, bA);
+                    acc_to_pair<NL>(accB, aB, bB);
+                    const int a = group_sum2<32>(aA, aB);
+                    const int b = (NL > 1) ? group_sum2<32>(bA, bB) : 0;
+                    if (lane == 0) s_part[(st * kGvMaxSplitRows + rowA) * kGvMaxSlices + slice] = pair_value(NL, a, b);
+                    if (lane == 16 && vB)
+                        s_part[(st * kGvMaxSplitRows + rowB) * kGvMaxSlices + slice] = pair_value(NL, a, b);
                 }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);
         }
-        if (NL > 1) named_bar_sync(1, kGvCons * 32);  // red[] is rewritten by the next token
+        if (NL > 1) named_bar_sync(1, kGvConsThreads);  // red[] and xl[] are rewritten by the next token
     }
 }
 
@@ -353,7 +383,7 @@ static cudaError_t gemv_dispatch(const uint8_t *Wp, const float *rs, int M, int 
     }
     const int nchunks = (M + R - 1) / R;
     const int grid = nchunks < sms ? nchunks : sms;
-    const size_t smem = gv_smem_bytes();
+    const size_t smem = gv_smem().total;
 #define TERN_GEMV_CASE(GG)                                                                               \
     case GG: {                                                                                           \
         auto kern = gemv_kernel<NL, GG>;                                                                 \

@@ -267,6 +267,13 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
         const uint32_t par = (uint32_t)(l & 1);
         const uint32_t tag = (ep << 7) | (uint32_t)(l + 1);  // never 0 (a zeroed workspace holds 0)
         TSTAMP(l, 0)
+        if (tid < 3 && c < 32) {
+            // one L2 prefetch per 2 MB page of this layer's gate, up and down arrays: the
+            // address translations are in place before top-k sends the row copies there
+            const uint8_t *base = tid == 0 ? Ly.gate : (tid == 1 ? Ly.up : Ly.down);
+            const size_t off = (size_t)c << 21;
+            if (off < (size_t)E * f * (d / 4)) asm volatile("prefetch.global.L2 [%0];" ::"l"(base + off));
+        }
         if (tid == 0) {
             // this layer's transfer sizes depend only on the CTA's share, not on the routing:
             // register them now so the copies can be issued the moment top-k is known

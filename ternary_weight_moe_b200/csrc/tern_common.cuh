@@ -203,6 +203,20 @@ __device__ __forceinline__ int group_sum(int v) {
     return v;
 }
 
+// Two rows at once: vA, vB are a lane's partials of rows A and B in its aligned group of G
+// lanes (G >= 2).  The first level trades halves (one shuffle serves both rows), the rest
+// reduce within half groups.  Afterwards the group's lane 0 holds row A's sum and its lane
+// G/2 holds row B's.
+template <int G>
+__device__ __forceinline__ int group_sum2(int vA, int vB) {
+    const int lane = threadIdx.x & 31;
+    const bool upper = (lane & (G / 2)) != 0;
+    int v = (upper ? vB : vA) + __shfl_xor_sync(0xFFFFFFFFu, upper ? vA : vB, G / 2);
+#pragma unroll
+    for (int o = G / 4; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    return v;
+}
+
 __device__ __forceinline__ double warp_sum_f64(double v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);

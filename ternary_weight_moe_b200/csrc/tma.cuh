@@ -63,6 +63,29 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, long l
     return true;
 }
 
+// Same wait, but the thread is suspended inside each try_wait until the phase completes or
+// `hint_ns` elapses, so waiting warps take no issue slots from warps that have work.
+__device__ __forceinline__ bool mbar_test_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity, long long limit_ns, int *status) {
+    if (mbar_test_sleep(bar, parity, 20000u)) return true;
+    const unsigned long long t0 = gtimer();
+    while (!mbar_test_sleep(bar, parity, 20000u)) {
+        if ((long long)(gtimer() - t0) > limit_ns) {
+            set_status(status, TERN_ETIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
 // barrier over `nthreads` threads (multiple of 32) using hardware barrier `id` (1..15)
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
