@@ -116,9 +116,9 @@ __device__ __forceinline__ void gemv_load_x(SegX<1> &X, const int8_t *xt, int se
 
 // ------------------------------------------------------------ the TMA-fed GEMV kernel
 // One CTA per SM.  A producer warp streams chunks of R consecutive rows (R*K/4 contiguous
-// bytes, up to 16 KB) plus their row scales into a ring of kGvStages shared-memory stages
+// bytes, up to 32 KB) plus their row scales into a ring of kGvStages shared-memory stages
 // with bulk copies; 16 consumer warps decode each stage as it lands and release it through
-// an mbarrier, so about 80 KB of weights per SM stay in flight while the consumers compute.
+// an mbarrier, so about 96 KB of weights per SM stay in flight while the consumers compute.
 // Waiting warps sleep inside mbarrier.try_wait instead of spinning.
 //   K <= 2048: G = K/64 lanes per row, 32/G rows per warp pass; every warp takes two passes
 //              at a time (two independent dot chains) and reduces both with one shuffle tree;
@@ -131,10 +131,10 @@ __device__ __forceinline__ void gemv_load_x(SegX<1> &X, const int8_t *xt, int se
 constexpr int kGvCons = 16;  // consumer warps
 constexpr int kGvConsThreads = kGvCons * 32;
 constexpr int kGvThreads = kGvConsThreads + 32;
-constexpr int kGvStages = 5;
-constexpr int kGvStageBytes = 16384;
-constexpr int kGvMaxRows = 128;      // rows per chunk (scale ring entries per stage)
-constexpr int kGvMaxSplitRows = 16;  // rows per chunk when K > 2048 (16 KB / 1 KB)
+constexpr int kGvStages = 3;
+constexpr int kGvStageBytes = 32768;
+constexpr int kGvMaxRows = 256;      // rows per chunk (scale ring entries per stage)
+constexpr int kGvMaxSplitRows = 32;  // rows per chunk when K > 2048 (32 KB / 1 KB)
 constexpr int kGvMaxSlices = 8;
 constexpr int kGvMaxK = 16384;
 constexpr int kGvMaxT = 64;
@@ -257,7 +257,8 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     const int seg = (NS > 1) ? slice * 32 + lane : gl;
     const uint32_t lane4 = (uint32_t)lane << 2;
     bool alive = true;
-    int n = 0;
+    int st = 0;        // stage of the next chunk
+    uint32_t ph = 0u;  // its fill phase parity
     for (int t = 0; t < T; t++) {
         SegX<NL> X;
         if constexpr (NL == 1) {
@@ -296,11 +297,10 @@ __global__ void __launch_bounds__(kGvThreads, 1)
             seg_load_x_smem<NL>(X, xl, K / 4, seg);
         }
 
-        for (int j = 0; j < my_n; j++, n++) {
-            const int st = n % kGvStages;
-            if (alive) alive = mbar_wait_sleep(&full[st], (uint32_t)(n / kGvStages) & 1u, kGvWaitNs, status);
-            int r0, nr;
-            chunk_rows(n, r0, nr);
+        for (int j = 0; j < my_n; j++) {
+            if (alive) alive = mbar_wait_sleep(&full[st], ph, kGvWaitNs, status);
+            const int r0 = ((int)blockIdx.x + j * (int)gridDim.x) * R;
+            const int nr = min(R, M - r0);
             const unsigned char *stage = ring + (size_t)st * kGvStageBytes;
             if (alive && NS == 1) {
                 // passes p and p + 16 of this warp at once
@@ -354,6 +354,10 @@ __global__ void __launch_bounds__(kGvThreads, 1)
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);
+            if (++st == kGvStages) {
+                st = 0;
+                ph ^= 1u;
+            }
         }
         if (NL > 1) named_bar_sync(1, kGvConsThreads);  // red[] and xl[] are rewritten by the next token
     }
