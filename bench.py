@@ -333,6 +333,61 @@ def run_gemv_sweep(args):
     return 0
 
 
+def run_batch_sweep(args):
+    """Extra output: one MoE FFN layer (d=2048, 256 experts, top-8) through moe_ffn_decode at
+    T = 1, 4, 16, 64 tokens per step (the kernel-per-stage path), L2 flushed before every step;
+    one JSON line per (T, activations).  Algorithmic bytes per step = U * 798,720 (packed rows
+    and scales of the U distinct experts the step routes to) + 1,048,576 (router)."""
+    import torch
+
+    import synth
+    import ternary_weight_moe_b200 as tm
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peak, peak_kind = peaks()
+    shape = synth.MoEShape()
+    layer = device_layer(0, shape, dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for T in ([int(v) for v in args.batch_T.split(",")] if args.batch_T else (1, 4, 16, 64)):
+        xs_host = synth.tokens_bf16(WID, 90000 + 1000 * T, args.steps + 3, T * shape.d).reshape(-1, T, shape.d)
+        xs = torch.from_numpy(xs_host.view(np.int16)).to(dev)
+        for act_name, act in (("bf16", tm.TERN_ACT_BF16), ("int8", tm.TERN_ACT_INT8)):
+            if args.act_only and act_name != args.act:
+                continue
+            ws = tm.workspace(tm.moe_ffn_workspace_bytes(layer, T, act), dev)
+            lay = tm.moe_ffn_workspace_layout(layer, T, act)
+            y = torch.empty((T, shape.d), dtype=torch.bfloat16, device=dev)
+            for i in range(3):
+                tm.moe_ffn_decode(layer, xs[i], act=act, ws=ws, y=y)
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+            uniq = []
+            torch.cuda.synchronize(dev)
+            for i in range(args.steps):
+                flush.fill_(i & 0xFF)
+                evs[i][0].record(stream)
+                tm.moe_ffn_decode(layer, xs[3 + i], act=act, ws=ws, y=y)
+                evs[i][1].record(stream)
+                if i < 8:  # distinct experts of a few steps (copied after the step's end event)
+                    idx = ws[lay["idx"]:lay["idx"] + 4 * T * shape.k].view(torch.int32).cpu().numpy()
+                    uniq.append(len(np.unique(idx)))
+            torch.cuda.synchronize(dev)
+            if tm.tern_stream_status() != 0:
+                raise RuntimeError("device status set during the batch sweep")
+            ms = [a.elapsed_time(b) for a, b in evs]
+            med = statistics.median(ms)
+            U = float(np.mean(uniq))
+            nbytes = U * 798720 + 1048576
+            gbs = nbytes / (med * 1e-3) / 1e9
+            print(json.dumps({"moe_ffn_decode": f"T={T}", "act": act_name, "us_median": med * 1e3,
+                              "us_p10": float(np.percentile(ms, 10)) * 1e3, "tokens_per_s": T / (med * 1e-3),
+                              "unique_experts": U, "bytes": nbytes, "GB/s": gbs, "frac": gbs / peak,
+                              "peak": peak, "peak_kind": peak_kind, "steps": args.steps}), flush=True)
+    return 0
+
+
 def main():
     global N_LAYERS, BYTES_PER_TOKEN
     ap = argparse.ArgumentParser()
@@ -347,7 +402,10 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="extra output: time tern_gemv over the GEMV shape sweep instead of the stack")
     ap.add_argument("--shape", default=None, help="with --sweep: one shape MxK only")
-    ap.add_argument("--act-only", action="store_true", help="with --sweep: only the --act activations")
+    ap.add_argument("--act-only", action="store_true", help="with --sweep/--batch-sweep: only the --act activations")
+    ap.add_argument("--batch-sweep", action="store_true",
+                    help="extra output: time one MoE FFN layer at T = 1, 4, 16, 64 tokens per step")
+    ap.add_argument("--batch-T", default=None, help="with --batch-sweep: comma-separated T values only")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -355,6 +413,8 @@ def main():
         return run_reference(args)
     if args.sweep:
         return run_gemv_sweep(args)
+    if args.batch_sweep:
+        return run_batch_sweep(args)
 
     import torch
 

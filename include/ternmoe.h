@@ -135,7 +135,7 @@ tern_status tern_quant_absmax(const uint16_t *x, int64_t T, int64_t n, int8_t *q
                               void *stream);
 
 /* Router: logits[t,e] = sum_k Wg[e,k] x[t,k] accumulated in fp64; each bf16 x bf16 product
- * is formed in fp32, exact unless its magnitude is below 2^-126 (fp32 underflow); top-k by
+ * is exact in fp64 and added with one rounding (fused multiply-add); top-k by
  * logit descending, ties to the lower expert index; gates renormalised
  * over the selected experts, g_i = exp(l_i - l_max) / sum_j exp(l_j - l_max), in fp64 and
  * written as fp32.  Wg [E][d] bf16, x [T][d] bf16, topk_idx [T][k], topk_gate [T][k],

@@ -304,7 +304,7 @@ tern_status moe_stack_workspace_layout(const tern_moe_layer *L0, int64_t T_max, 
 int32_t moe_stack_kernel_launches(const tern_moe_layer *L0, int32_t n_layers, int64_t T, tern_act act) {
     if (check_layer(L0) != TERN_OK || n_layers < 1 || n_layers > kMaxLayers || T < 1 || T > kMaxT) return -1;
     if (T == 1 && stack_persistent_supported(L0, n_layers, act)) return 1;
-    return 7 * n_layers;
+    return 8 * n_layers;  // rmsnorm, logits, select, prep, gate/up, prep, down, combine
 }
 
 tern_status tern_stream_status(void *stream) {

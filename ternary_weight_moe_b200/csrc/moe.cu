@@ -1,10 +1,11 @@
 // moe.cu -- one MoE FFN layer for T decode tokens, stage by stage (sm_100a).
 //
-//   route   router GEMV in fp64 + top-k + renormalised gates; the last CTA to finish
-//           also groups the (token, slot) pairs by expert ("iPhone Runs a 20B Model at 120
-//           tok/s", "MoE Is the Other Half of the Story Behind the 20B Figure": tokens routed
-//           to different experts make the runtime fetch scattered weights -- grouping makes
-//           every selected expert stream from HBM once per step);
+//   logits  router GEMV in fp64 (exact products, fused multiply-add), eight tokens per CTA;
+//   select  per token: top-k + renormalised gates; the last CTA to finish also groups the
+//           (token, slot) pairs by expert ("iPhone Runs a 20B Model at 120 tok/s", "MoE Is
+//           the Other Half of the Story Behind the 20B Figure": tokens routed to different
+//           experts make the runtime fetch scattered weights -- grouping makes every selected
+//           expert stream from HBM once per step);
 //   xprep   activation limbs per token (int8 absmax codes, or 24-bit fixed point);
 //   gateup  per (expert, block of rows): G and U rows are read once and applied to every
 //           token routed to that expert; SwiGLU epilogue in fp64, h stored as fp32;
@@ -14,89 +15,157 @@
 #include <cuda_runtime.h>
 #include <math.h>
 
+#include <utility>
+
 #include "kernels.h"
 #include "tern_common.cuh"
 
 namespace tern {
 
-constexpr int kRouteWarps = 8;
+// Launch with arguments converted to the kernel's parameter types; returns the launch error.
+template <typename... K, typename... A>
+static cudaError_t launch_k(void (*kern)(K...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, A &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
+}
+
 constexpr int kMaxE = 1024;
 
-// ------------------------------------------------------------------------- route kernel
-// Warp per expert row, all T tokens; fp64 accumulation of exact bf16 x bf16 products, so
-// the logits do not depend on summation order.  The last CTA (arrival counter) runs
-// top-k for every token and, if asked, groups (token, slot) pairs by expert.
-__global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(
-    const uint16_t *__restrict__ Wg, const uint16_t *__restrict__ x, int T, int d, int E, int k,
-    double *__restrict__ logits, int32_t *__restrict__ idx, float *__restrict__ g32, double *__restrict__ g64,
-    unsigned int *counter, int dispatch, int32_t *n_unique, int32_t *uexp, int32_t *uoff, int32_t *ent) {
+// ------------------------------------------------------------------------- route kernels
+// logits_kernel: one warp per expert row, 16 experts x 8 tokens per CTA.  The tokens' x is
+// converted to fp64 once per CTA, 512 elements at a time, into shared memory.  Each product of
+// two bf16 values is exact in fp64 (at most 16 significant bits), so one fp64 fma per product
+// adds the exact product with one rounding; the sums are exact for the router's magnitudes
+// (checked by the oracle), so the summation order does not change the logits.
+constexpr int kRouteTok = 8;
+constexpr int kLogitWarps = 16;
+constexpr int kLogitChunk = 512;
+
+// bf16 -> fp64 by moving bits (normal values); zero, subnormal, inf and nan go through fp32
+__device__ __forceinline__ double bf16_to_f64(uint16_t b) {
+    const uint32_t e = (b >> 7) & 0xFFu;
+    if (e == 0u || e == 0xFFu) return (double)bf16_to_f32(b);
+    const unsigned long long bits = ((unsigned long long)(b & 0x8000u) << 48) |
+                                    ((unsigned long long)(e + 896u) << 52) | ((unsigned long long)(b & 0x7Fu) << 45);
+    return __longlong_as_double((long long)bits);
+}
+
+__global__ void __launch_bounds__(kLogitWarps * 32) logits_kernel(const uint16_t *__restrict__ Wg,
+                                                                   const uint16_t *__restrict__ x, int T, int d,
+                                                                   int E, double *__restrict__ logits) {
+    __shared__ double s_x[kRouteTok][kLogitChunk];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int e = blockIdx.x * kLogitWarps + warp;
+    const int t0 = blockIdx.y * kRouteTok;
+    const int nt = min(kRouteTok, T - t0);
+    const uint16_t *wr = Wg + (int64_t)(e < E ? e : 0) * d;
+    double acc[kRouteTok];
+#pragma unroll
+    for (int tt = 0; tt < kRouteTok; tt++) acc[tt] = 0.0;
+    constexpr int WPL = kLogitChunk / 32;                             // weights per lane per chunk
+    constexpr int XPT = kRouteTok * kLogitChunk / (kLogitWarps * 32);  // x values per thread per chunk
+    uint16_t wv[WPL], xv[XPT];
+    // loads of chunk c0 into registers (all issued before any is used)
+    auto fetch = [&](int c0) {
+        const int n = min(kLogitChunk, d - c0);
+#pragma unroll
+        for (int i = 0; i < WPL; i++) {
+            const int j = lane + 32 * i;
+            wv[i] = (e < E && j < n) ? __ldg(wr + c0 + j) : (uint16_t)0;
+        }
+#pragma unroll
+        for (int i = 0; i < XPT; i++) {
+            const int q = threadIdx.x + i * kLogitWarps * 32, tt = q / kLogitChunk, j = q % kLogitChunk;
+            xv[i] = (tt < nt && j < n) ? __ldg(x + (int64_t)(t0 + tt) * d + c0 + j) : (uint16_t)0;
+        }
+    };
+    fetch(0);
+    for (int c0 = 0; c0 < d; c0 += kLogitChunk) {
+        __syncthreads();  // previous chunk consumed
+#pragma unroll
+        for (int i = 0; i < XPT; i++) {
+            const int q = threadIdx.x + i * kLogitWarps * 32;
+            s_x[q / kLogitChunk][q % kLogitChunk] = bf16_to_f64(xv[i]);
+        }
+        double w[WPL];
+#pragma unroll
+        for (int i = 0; i < WPL; i++) w[i] = bf16_to_f64(wv[i]);
+        if (c0 + kLogitChunk < d) fetch(c0 + kLogitChunk);  // next chunk's loads fly during this one
+        __syncthreads();
+        if (e < E) {
+#pragma unroll
+            for (int i = 0; i < WPL; i++) {
+                const int j = lane + 32 * i;
+#pragma unroll
+                for (int tt = 0; tt < kRouteTok; tt++) acc[tt] = fma(w[i], s_x[tt][j], acc[tt]);
+            }
+        }
+    }
+    if (e < E) {
+#pragma unroll
+        for (int tt = 0; tt < kRouteTok; tt++) {
+            const double v = warp_sum_f64(acc[tt]);
+            if (lane == 0 && tt < nt) logits[(int64_t)(t0 + tt) * E + e] = v;
+        }
+    }
+}
+
+// select_kernel: one CTA per token -- top-k of its logits, renormalised gates.  The last CTA
+// to finish (arrival counter) groups the (token, slot) pairs by expert when asked.
+constexpr int kSelectThreads = 256;
+
+__global__ void __launch_bounds__(kSelectThreads) select_kernel(
+    const double *__restrict__ logits, int T, int E, int k, int32_t *__restrict__ idx, float *__restrict__ g32,
+    double *__restrict__ g64, unsigned int *counter, int dispatch, int32_t *n_unique, int32_t *uexp, int32_t *uoff,
+    int32_t *ent) {
     __shared__ int s_last;
     __shared__ int s_cnt[kMaxE + 1];
     __shared__ int s_flag[kMaxE + 1];
     __shared__ int s_wsum[32];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int e = blockIdx.x * kRouteWarps + warp;
-    if (e < E) {
-        const uint4 *wr = reinterpret_cast<const uint4 *>(Wg + (int64_t)e * d);
-        const int nchunk = d / 8;
-        for (int t = 0; t < T; t++) {
-            const uint4 *xr = reinterpret_cast<const uint4 *>(x + (int64_t)t * d);
-            double acc = 0.0;
-            for (int c = lane; c < nchunk; c += 32) {
-                const uint4 wv = __ldg(wr + c), xv = __ldg(xr + c);
-                const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w}, xx[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-                for (int q = 0; q < 4; q++) {
-                    // bf16 x bf16 has at most 16 significant bits: the fp32 product is exact
-                    acc += (double)__fmul_rn(bf16_to_f32((uint16_t)(ww[q] & 0xFFFFu)),
-                                             bf16_to_f32((uint16_t)(xx[q] & 0xFFFFu)));
-                    acc += (double)__fmul_rn(bf16_to_f32((uint16_t)(ww[q] >> 16)),
-                                             bf16_to_f32((uint16_t)(xx[q] >> 16)));
-                }
-            }
-            acc = warp_sum_f64(acc);
-            if (lane == 0) logits[(int64_t)t * E + e] = acc;
-        }
+    __shared__ double s_lg[kMaxE];
+    __shared__ int32_t s_idx[8];
+    __shared__ __align__(16) uint32_t s_gm[32];
+    __shared__ int s_nc;
+    __shared__ ulonglong2 s_cand[256];
+    __shared__ int32_t s_all[64 * 8];  // every (token, slot) expert index, T <= 64, k <= 8
+    const int t = blockIdx.x;
+    const double *lg = logits + (int64_t)t * E;
+    double mine = 0.0;
+    for (int e = threadIdx.x; e < E; e += kSelectThreads) {
+        const double v = lg[e];
+        s_lg[e] = v;
+        if (e == (int)threadIdx.x) mine = v;
     }
-    // last block out does the selection
+    __syncthreads();
+    if (E <= 256) {
+        block_topk_select(mine, E, k, s_idx, s_gm, &s_nc, s_cand);
+    } else {
+        if (threadIdx.x < 32) warp_topk_select<32>(s_lg, E, k, s_idx);
+        __syncthreads();
+    }
+    if (threadIdx.x < 32) {
+        warp_topk_gates(s_lg, k, s_idx, g64 + (int64_t)t * k, g32 + (int64_t)t * k);
+        if (threadIdx.x < k) idx[(int64_t)t * k + threadIdx.x] = s_idx[threadIdx.x];
+    }
+    // last CTA out groups the pairs
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) s_last = (atomicAdd(counter, 1u) == gridDim.x - 1);
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    if (E <= 256) {
-        __shared__ double s_lg[kRouteWarps][256];
-        for (int t = warp; t < T; t += kRouteWarps) {
-            const double *lg = logits + (int64_t)t * E;  // written by other blocks: read through L2
-#pragma unroll
-            for (int j = 0; j < 8; j++) {
-                const int ee = lane + 32 * j;
-                s_lg[warp][ee] = (ee < E) ? __ldcg(lg + ee) : 0.0;
-            }
-            __syncwarp();
-            warp_topk<8>(s_lg[warp], E, k, idx + (int64_t)t * k, g64 + (int64_t)t * k, g32 + (int64_t)t * k);
-            __syncwarp();
-        }
-    } else if (warp == 0) {
-        __shared__ double s_big[kMaxE];
-        for (int t = 0; t < T; t++) {
-            const double *lg = logits + (int64_t)t * E;
-            for (int ee = lane; ee < E; ee += 32) s_big[ee] = __ldcg(lg + ee);
-            __syncwarp();
-            warp_topk<32>(s_big, E, k, idx + (int64_t)t * k, g64 + (int64_t)t * k, g32 + (int64_t)t * k);
-            __syncwarp();
-        }
-    }
     if (threadIdx.x == 0) *counter = 0u;  // workspace control word back to zero
     if (!dispatch) return;
-    __syncthreads();
-    __threadfence_block();
     // ---- group (token, slot) pairs by expert: counts, offsets, stable placement
     const int n = T * k;
     for (int i = threadIdx.x; i <= E; i += blockDim.x) s_cnt[i] = 0;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) s_all[i] = __ldcg(idx + i);  // other CTAs' results
     __syncthreads();
-    for (int i = threadIdx.x; i < n; i += blockDim.x) atomicAdd(&s_cnt[idx[i]], 1);
+    for (int i = threadIdx.x; i < n; i += blockDim.x) atomicAdd(&s_cnt[s_all[i]], 1);
     __syncthreads();
     // exclusive scans over experts of counts and of "selected" flags (serial per 32-chunk)
     if (threadIdx.x < 32) {
@@ -145,21 +214,35 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(
         }
     }
     if (threadIdx.x == 0) uoff[s_wsum[0]] = s_wsum[1];
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        const int ex = idx[i];
-        int rank = 0;
-        for (int j = 0; j < i; j++) rank += (idx[j] == ex);
-        ent[s_cnt[ex] + rank] = i;  // entry = t*k + slot, ascending within an expert
+    __syncthreads();  // uoff written from s_cnt; s_cnt now becomes the running placement offset
+    if (threadIdx.x < 32) {
+        // stable placement, 32 entries at a time: entries of one expert keep ascending order
+        const int lane = threadIdx.x;
+        for (int c0 = 0; c0 < n; c0 += 32) {
+            const int i = c0 + lane;
+            const bool v = i < n;
+            const int ex = v ? s_all[i] : -1 - lane;  // distinct values for lanes past the end
+            const unsigned m = __match_any_sync(0xFFFFFFFFu, ex);
+            const int before = __popc(m & ((1u << lane) - 1u));
+            const int base = v ? s_cnt[ex] : 0;
+            __syncwarp();
+            if (v) {
+                ent[base + before] = i;  // entry = t*k + slot
+                if (lane == __ffs(m) - 1) s_cnt[ex] = base + __popc(m);
+            }
+            __syncwarp();
+        }
     }
 }
 
 cudaError_t launch_route(const uint16_t *Wg, const uint16_t *x, int T, int d, int E, int k, double *logits,
                          int32_t *idx, float *g32, double *g64, unsigned int *counter, bool dispatch,
                          int32_t *n_unique, int32_t *uexp, int32_t *uoff, int32_t *ent, cudaStream_t s) {
-    const int grid = (E + kRouteWarps - 1) / kRouteWarps;
-    route_kernel<<<grid, kRouteWarps * 32, 0, s>>>(Wg, x, T, d, E, k, logits, idx, g32, g64, counter,
-                                                   dispatch ? 1 : 0, n_unique, uexp, uoff, ent);
-    return cudaGetLastError();
+    const dim3 g1((E + kLogitWarps - 1) / kLogitWarps, (T + kRouteTok - 1) / kRouteTok);
+    cudaError_t err = launch_k(logits_kernel, g1, dim3(kLogitWarps * 32), 0, s, Wg, x, T, d, E, logits);
+    if (err != cudaSuccess) return err;
+    return launch_k(select_kernel, dim3(T), dim3(kSelectThreads), 0, s, (const double *)logits, T, E, k, idx,
+                    g32, g64, counter, dispatch ? 1 : 0, n_unique, uexp, uoff, ent);
 }
 
 // ------------------------------------------------------------------------ prep kernels
@@ -382,8 +465,7 @@ __global__ void rmsnorm_kernel(const uint16_t *__restrict__ x, int d, double eps
 }
 
 cudaError_t launch_rmsnorm(const uint16_t *x, int T, int d, double eps, uint16_t *n, cudaStream_t s) {
-    rmsnorm_kernel<<<T, 256, 0, s>>>(x, d, eps, n);
-    return cudaGetLastError();
+    return launch_k(rmsnorm_kernel, dim3(T), dim3(256), 0, s, x, d, eps, n);
 }
 
 // ----------------------------------------------------------------- stage launcher
@@ -395,8 +477,9 @@ static cudaError_t ffn_stages_nl(const tern_moe_layer *L, const uint16_t *x, int
     err = launch_route(L->router, x, T, d, E, k, w.logits, w.idx, w.g32, w.g64, w.ctrl, true, w.n_unique, w.uexp,
                        w.uoff, w.ent, s);
     if (err != cudaSuccess) return err;
-    prep_kernel<NL><<<T, 256, 0, s>>>(x, nullptr, d, w.xw, w.xsc, nullptr);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    err = launch_k(prep_kernel<NL>, dim3(T), dim3(256), 0, s, x, (const float *)nullptr, d, w.xw, w.xsc,
+                   (const int32_t *)nullptr);
+    if (err != cudaSuccess) return err;
     const int umax = (E < T * k) ? E : T * k;
     const int Gd = d / 64, Gf = f / 64;
     const int rpb_gu = 32, rpb_dn = 128;
@@ -405,9 +488,10 @@ static cudaError_t ffn_stages_nl(const tern_moe_layer *L, const uint16_t *x, int
     case GG: {                                                                                             \
         auto kern = gateup_kernel<NL, GG>;                                                                 \
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kLutBytes);                \
-        kern<<<g1, kFfnWarps * 32, kLutBytes, s>>>(L->gate, L->up, L->gate_scale, L->up_scale, d, f, k,    \
-                                                   w.n_unique, w.uexp, w.uoff, w.ent, w.xw, w.xsc, w.h,   \
-                                                   w.acc_g, w.acc_u, rpb_gu);                              \
+        err = launch_k(kern, g1, dim3(kFfnWarps * 32), kLutBytes, s, L->gate, L->up, L->gate_scale,  \
+                       L->up_scale, d, f, k, (const int32_t *)w.n_unique, (const int32_t *)w.uexp,          \
+                       (const int32_t *)w.uoff, (const int32_t *)w.ent, (const uint32_t *)w.xw,            \
+                       (const float *)w.xsc, w.h, w.acc_g, w.acc_u, rpb_gu);                               \
         break;                                                                                             \
     }
     switch (Gd) {
@@ -415,15 +499,18 @@ static cudaError_t ffn_stages_nl(const tern_moe_layer *L, const uint16_t *x, int
         default: return cudaErrorInvalidValue;
     }
 #undef TERN_GU_CASE
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    prep_kernel<NL><<<T * k, 128, 0, s>>>(nullptr, w.h, f, w.hw, w.hsc, nullptr);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if (err != cudaSuccess) return err;
+    err = launch_k(prep_kernel<NL>, dim3(T * k), dim3(128), 0, s, (const uint16_t *)nullptr,
+                   (const float *)w.h, f, w.hw, w.hsc, (const int32_t *)nullptr);
+    if (err != cudaSuccess) return err;
 #define TERN_DN_CASE(GG)                                                                                   \
     case GG: {                                                                                             \
         auto kern = down_kernel<NL, GG>;                                                                   \
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kLutBytes);                \
-        kern<<<g2, kFfnWarps * 32, kLutBytes, s>>>(L->down, L->down_scale, d, f, w.n_unique, w.uexp,       \
-                                                   w.uoff, w.ent, w.hw, w.hsc, w.ye, w.acc_d, rpb_dn);     \
+        err = launch_k(kern, g2, dim3(kFfnWarps * 32), kLutBytes, s, L->down, L->down_scale, d, f,   \
+                       (const int32_t *)w.n_unique, (const int32_t *)w.uexp, (const int32_t *)w.uoff,       \
+                       (const int32_t *)w.ent, (const uint32_t *)w.hw, (const float *)w.hsc, w.ye,         \
+                       w.acc_d, rpb_dn);                                                                   \
         break;                                                                                             \
     }
     switch (Gf) {
@@ -431,10 +518,10 @@ static cudaError_t ffn_stages_nl(const tern_moe_layer *L, const uint16_t *x, int
         default: return cudaErrorInvalidValue;
     }
 #undef TERN_DN_CASE
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if (err != cudaSuccess) return err;
     int cg = (T * d + 255) / 256;
-    combine_kernel<<<cg, 256, 0, s>>>(w.g64, w.ye, T, d, k, y, y32, resid, x_out);
-    return cudaGetLastError();
+    return launch_k(combine_kernel, dim3(cg), dim3(256), 0, s, (const double *)w.g64, (const double *)w.ye,
+                    T, d, k, y, y32, resid, x_out);
 }
 
 cudaError_t launch_ffn_stages(const tern_moe_layer *L, const uint16_t *x, int T, tern_act act, const FfnWs &w,

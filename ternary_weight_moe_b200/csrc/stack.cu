@@ -372,9 +372,10 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                 const int per = d / wpr;
                 const uint16_t *wrow = rbuf + (size_t)rr * d + part * per;
                 const uint16_t *nrow = ns + part * per;
-                // bf16 x bf16 has at most 16 significant bits: the fp32 product is exact
+                // bf16 x bf16 has at most 16 significant bits: the product is exact in fp64 and
+                // the fma adds it with one rounding
                 for (int i = lane; i < per; i += 32)
-                    acc += (double)__fmul_rn(bf16_to_f32(wrow[i]), bf16_to_f32(nrow[i]));
+                    acc = fma((double)bf16_to_f32(wrow[i]), (double)bf16_to_f32(nrow[i]), acc);
             }
             acc = warp_sum_f64(acc);
             if (lane == 0 && rr < nr) s_part[rr][part] = acc;
