@@ -421,6 +421,211 @@ __global__ void __launch_bounds__(kFfnWarps * 32) down_kernel(
     }
 }
 
+// ------------------------------------------------- grouped path on int8 tensor cores (T >= 32)
+// At 32 or more tokens a step routes ~2+ tokens to each selected expert and the dp4a kernels
+// above become bound by their decode instructions (one table read and NL dp4a per packed byte
+// PER TOKEN).  Here the decoded weights feed int8 MMAs (mma.sync m16n8k32): a warp owns 16
+// rows; the A fragment register of row r and codes 4c..4c+3 is exactly the table entry of
+// packed byte c of that row, so one table read per packed byte serves up to 8 tokens and
+// every activation limb.  B columns are tokens (expert entries); each limb is its own MMA
+// (hi limb signed x signed, mid and lo signed x unsigned) and the limbs recombine exactly in
+// int64: S = hi * 65536 + mid * 256 + lo.  Same integers as the dp4a kernels, bit for bit.
+constexpr int kMmaGroupedMinT = 32;
+constexpr int kMmaWarps = 8;
+constexpr int kMmaRows = 16 * kMmaWarps;  // rows per CTA
+constexpr int kMmaTok = 8;                // tokens (B columns) per pass
+constexpr int kMmaPad = 4;                // words of padding per staged limb row (bank spread)
+
+template <bool USIGNED>
+__device__ __forceinline__ void mma_s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                       uint32_t b1) {
+    if (USIGNED)
+        asm volatile(
+            "mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+            : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    else
+        asm volatile(
+            "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+            : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Stage the limb words of entries q0..q0+nb-1 (vector v = ent[q] / div, NL*n4 words each) as
+// [kMmaTok][NL][n4 + kMmaPad]; columns nb..kMmaTok-1 are zero.
+template <int NL>
+__device__ __forceinline__ void mma_stage(uint32_t *dst, const uint32_t *__restrict__ src, int n4,
+                                          const int32_t *__restrict__ ent, int q0, int nb, int div) {
+    const int rs = n4 + kMmaPad;
+    for (int i = threadIdx.x; i < kMmaTok * NL * n4; i += blockDim.x) {
+        const int b = i / (NL * n4), r = i % (NL * n4), l = r / n4, w = r % n4;
+        dst[(b * NL + l) * rs + w] = (b < nb) ? __ldg(src + (int64_t)(ent[q0 + b] / div) * NL * n4 + r) : 0u;
+    }
+}
+
+// One 16-row tile x K codes of one matrix against the staged columns: acc[l] += A * B_l.
+// row0 = the tile's first row; rows >= nrows contribute zeros.  K % 64 == 0.
+template <int NL, int NM>
+__device__ __forceinline__ void mma_tile(const uint8_t *const (&mats)[NM], int64_t rowb, int row0, int nrows, int K,
+                                         const uint32_t *xs, int rs, const uint32_t *lut, int (&acc)[NM][NL][4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, tig = lane & 3;
+    const uint32_t lane4 = (uint32_t)lane << 2;
+    const uint32_t sel = 0x5504u | ((uint32_t)tig << 4);  // byte tig of a word -> table offset
+    const char *lb = reinterpret_cast<const char *>(lut);
+    const bool v0 = row0 + g < nrows, v1 = row0 + g + 8 < nrows;
+    for (int m = 0; m < K / 64; m++) {  // 16 packed bytes = two k-blocks of 32 codes
+        uint4 w0[NM], w1[NM];
+#pragma unroll
+        for (int q = 0; q < NM; q++) {
+            w0[q] = v0 ? __ldg(reinterpret_cast<const uint4 *>(mats[q] + (int64_t)(row0 + g) * rowb) + m)
+                       : make_uint4(0u, 0u, 0u, 0u);
+            w1[q] = v1 ? __ldg(reinterpret_cast<const uint4 *>(mats[q] + (int64_t)(row0 + g + 8) * rowb) + m)
+                       : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int jj = 0; jj < 2; jj++) {
+            const int j = 2 * m + jj;  // k-block: codes 32j .. 32j+31, limb words 8j .. 8j+7
+            uint32_t b0[NL], b1[NL];
+#pragma unroll
+            for (int l = 0; l < NL; l++) {
+                b0[l] = xs[(g * NL + l) * rs + 8 * j + tig];
+                b1[l] = xs[(g * NL + l) * rs + 8 * j + 4 + tig];
+            }
+#pragma unroll
+            for (int q = 0; q < NM; q++) {
+                const uint32_t lo0 = jj ? w0[q].z : w0[q].x, hi0 = jj ? w0[q].w : w0[q].y;
+                const uint32_t lo1 = jj ? w1[q].z : w1[q].x, hi1 = jj ? w1[q].w : w1[q].y;
+                const uint32_t a0 = *reinterpret_cast<const uint32_t *>(lb + __byte_perm(lo0, lane4, sel));
+                const uint32_t a1 = *reinterpret_cast<const uint32_t *>(lb + __byte_perm(lo1, lane4, sel));
+                const uint32_t a2 = *reinterpret_cast<const uint32_t *>(lb + __byte_perm(hi0, lane4, sel));
+                const uint32_t a3 = *reinterpret_cast<const uint32_t *>(lb + __byte_perm(hi1, lane4, sel));
+                mma_s8<false>(acc[q][0], a0, a1, a2, a3, b0[0], b1[0]);
+                if (NL > 1) {
+                    mma_s8<true>(acc[q][NL > 1 ? 1 : 0], a0, a1, a2, a3, b0[NL > 1 ? 1 : 0], b1[NL > 1 ? 1 : 0]);
+                    mma_s8<true>(acc[q][NL > 2 ? 2 : 0], a0, a1, a2, a3, b0[NL > 2 ? 2 : 0], b1[NL > 2 ? 2 : 0]);
+                }
+            }
+        }
+    }
+}
+
+// grid: (n_unique_max, ceil(f / 128)); 8 warps x 16 rows of gate and up.
+template <int NL>
+__global__ void __launch_bounds__(kMmaWarps * 32) gateup_mma_kernel(
+    const uint8_t *__restrict__ gate, const uint8_t *__restrict__ up, const float *__restrict__ sg,
+    const float *__restrict__ su, int d, int f, int k, const int32_t *__restrict__ n_unique,
+    const int32_t *__restrict__ uexp, const int32_t *__restrict__ uoff, const int32_t *__restrict__ ent,
+    const uint32_t *__restrict__ xw, const float *__restrict__ xsc, float *__restrict__ h,
+    int32_t *__restrict__ acc_g, int32_t *__restrict__ acc_u) {
+    extern __shared__ __align__(16) uint32_t smem[];
+    uint32_t *lut = smem;
+    uint32_t *xs = smem + kLutWords;  // [kMmaTok][NL][d/4 + pad]
+    const int u = blockIdx.x;
+    if (u >= *n_unique) return;
+    lut_fill(lut);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, tig = lane & 3;
+    const int e = uexp[u], e0 = uoff[u], e1 = uoff[u + 1];
+    const int64_t rowb = d / 4;
+    const int row0 = blockIdx.y * kMmaRows + warp * 16;  // within the expert
+    const uint8_t *const mats[2] = {gate + (int64_t)e * f * rowb, up + (int64_t)e * f * rowb};
+    const int rs = d / 4 + kMmaPad;
+    for (int q0 = e0; q0 < e1; q0 += kMmaTok) {
+        const int nb = min(kMmaTok, e1 - q0);
+        __syncthreads();  // table ready (first pass) / previous columns consumed
+        mma_stage<NL>(xs, xw, d / 4, ent, q0, nb, k);
+        __syncthreads();
+        int acc[2][NL][4];
+#pragma unroll
+        for (int q = 0; q < 2; q++)
+#pragma unroll
+            for (int l = 0; l < NL; l++) acc[q][l][0] = acc[q][l][1] = acc[q][l][2] = acc[q][l][3] = 0;
+        mma_tile<NL, 2>(mats, rowb, row0, f, d, xs, rs, lut, acc);
+        // thread holds rows g, g+8 and columns 2*tig, 2*tig+1
+#pragma unroll
+        for (int c = 0; c < 4; c++) {
+            const int j = row0 + g + ((c & 2) ? 8 : 0), col = 2 * tig + (c & 1);
+            if (j >= f || col >= nb) continue;
+            const int entry = ent[q0 + col];
+            const float xsv = xsc[entry / k];
+            long long Sg, Su;
+            if (NL == 1) {
+                Sg = acc[0][0][c];
+                Su = acc[1][0][c];
+            } else {
+                Sg = (long long)acc[0][0][c] * 65536ll + (long long)acc[0][NL > 1 ? 1 : 0][c] * 256ll +
+                     (long long)acc[0][NL > 2 ? 2 : 0][c];
+                Su = (long long)acc[1][0][c] * 65536ll + (long long)acc[1][NL > 1 ? 1 : 0][c] * 256ll +
+                     (long long)acc[1][NL > 2 ? 2 : 0][c];
+            }
+            const int64_t o = (int64_t)e * f + j;
+            float hv;
+            if (NL == 1) {
+                acc_g[(int64_t)entry * f + j] = (int32_t)Sg;
+                acc_u[(int64_t)entry * f + j] = (int32_t)Su;
+                const float gv = __fmul_rn(__fmul_rn(__int2float_rn((int)Sg), sg[o]), xsv);
+                const float uv = __fmul_rn(__fmul_rn(__int2float_rn((int)Su), su[o]), xsv);
+                hv = swiglu_f32((double)gv, (double)uv);
+            } else {
+                const int sh = __float_as_int(xsv);
+                hv = swiglu_f32(ldexp((double)Sg, -sh) * (double)sg[o], ldexp((double)Su, -sh) * (double)su[o]);
+            }
+            h[(int64_t)entry * f + j] = hv;
+        }
+    }
+}
+
+// grid: (n_unique_max, ceil(d / 128)); 8 warps x 16 output rows.
+template <int NL>
+__global__ void __launch_bounds__(kMmaWarps * 32) down_mma_kernel(
+    const uint8_t *__restrict__ down, const float *__restrict__ sd, int d, int f,
+    const int32_t *__restrict__ n_unique, const int32_t *__restrict__ uexp, const int32_t *__restrict__ uoff,
+    const int32_t *__restrict__ ent, const uint32_t *__restrict__ hw, const float *__restrict__ hsc,
+    double *__restrict__ ye, int32_t *__restrict__ acc_d) {
+    extern __shared__ __align__(16) uint32_t smem[];
+    uint32_t *lut = smem;
+    uint32_t *xs = smem + kLutWords;  // [kMmaTok][NL][f/4 + pad]
+    const int u = blockIdx.x;
+    if (u >= *n_unique) return;
+    lut_fill(lut);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, tig = lane & 3;
+    const int e = uexp[u], e0 = uoff[u], e1 = uoff[u + 1];
+    const int64_t rowb = f / 4;
+    const int row0 = blockIdx.y * kMmaRows + warp * 16;
+    const uint8_t *const mats[1] = {down + (int64_t)e * d * rowb};
+    const int rs = f / 4 + kMmaPad;
+    for (int q0 = e0; q0 < e1; q0 += kMmaTok) {
+        const int nb = min(kMmaTok, e1 - q0);
+        __syncthreads();
+        mma_stage<NL>(xs, hw, f / 4, ent, q0, nb, 1);
+        __syncthreads();
+        int acc[1][NL][4];
+#pragma unroll
+        for (int l = 0; l < NL; l++) acc[0][l][0] = acc[0][l][1] = acc[0][l][2] = acc[0][l][3] = 0;
+        mma_tile<NL, 1>(mats, rowb, row0, d, f, xs, rs, lut, acc);
+#pragma unroll
+        for (int c = 0; c < 4; c++) {
+            const int i = row0 + g + ((c & 2) ? 8 : 0), col = 2 * tig + (c & 1);
+            if (i >= d || col >= nb) continue;
+            const int entry = ent[q0 + col];
+            const float hs = hsc[entry];
+            long long S;
+            if (NL == 1) S = acc[0][0][c];
+            else
+                S = (long long)acc[0][0][c] * 65536ll + (long long)acc[0][NL > 1 ? 1 : 0][c] * 256ll +
+                    (long long)acc[0][NL > 2 ? 2 : 0][c];
+            const float sdv = sd[(int64_t)e * d + i];
+            double v;
+            if (NL == 1) {
+                acc_d[(int64_t)entry * d + i] = (int32_t)S;
+                v = (double)__fmul_rn(__fmul_rn(__int2float_rn((int)S), sdv), hs);
+            } else {
+                v = ldexp((double)S, -__float_as_int(hs)) * (double)sdv;
+            }
+            ye[(int64_t)entry * d + i] = v;
+        }
+    }
+}
+
 // ------------------------------------------------------------------------- combine
 // y[t,i] = sum over slots (top-k order) of g64[t,slot] * ye[t*k+slot, i], fp64.
 __global__ void combine_kernel(const double *__restrict__ g64, const double *__restrict__ ye, int T, int d, int k,
@@ -482,6 +687,28 @@ static cudaError_t ffn_stages_nl(const tern_moe_layer *L, const uint16_t *x, int
     if (err != cudaSuccess) return err;
     const int umax = (E < T * k) ? E : T * k;
     const int Gd = d / 64, Gf = f / 64;
+    if (T >= kMmaGroupedMinT) {  // grouped path on int8 tensor cores
+        const dim3 m1(umax, (f + kMmaRows - 1) / kMmaRows), m2(umax, (d + kMmaRows - 1) / kMmaRows);
+        const size_t sm1 = kLutBytes + (size_t)kMmaTok * NL * (d / 4 + kMmaPad) * 4;
+        const size_t sm2 = kLutBytes + (size_t)kMmaTok * NL * (f / 4 + kMmaPad) * 4;
+        cudaFuncSetAttribute(gateup_mma_kernel<NL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
+        cudaFuncSetAttribute(down_mma_kernel<NL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
+        err = launch_k(gateup_mma_kernel<NL>, m1, dim3(kMmaWarps * 32), sm1, s, L->gate, L->up, L->gate_scale,
+                       L->up_scale, d, f, k, (const int32_t *)w.n_unique, (const int32_t *)w.uexp,
+                       (const int32_t *)w.uoff, (const int32_t *)w.ent, (const uint32_t *)w.xw,
+                       (const float *)w.xsc, w.h, w.acc_g, w.acc_u);
+        if (err != cudaSuccess) return err;
+        err = launch_k(prep_kernel<NL>, dim3(T * k), dim3(128), 0, s, (const uint16_t *)nullptr,
+                       (const float *)w.h, f, w.hw, w.hsc, (const int32_t *)nullptr);
+        if (err != cudaSuccess) return err;
+        err = launch_k(down_mma_kernel<NL>, m2, dim3(kMmaWarps * 32), sm2, s, L->down, L->down_scale, d, f,
+                       (const int32_t *)w.n_unique, (const int32_t *)w.uexp, (const int32_t *)w.uoff,
+                       (const int32_t *)w.ent, (const uint32_t *)w.hw, (const float *)w.hsc, w.ye, w.acc_d);
+        if (err != cudaSuccess) return err;
+        int cg = (T * d + 255) / 256;
+        return launch_k(combine_kernel, dim3(cg), dim3(256), 0, s, (const double *)w.g64, (const double *)w.ye, T,
+                        d, k, y, y32, resid, x_out);
+    }
     const int rpb_gu = 32, rpb_dn = 128;
     dim3 g1(umax, (f + rpb_gu - 1) / rpb_gu), g2(umax, (d + rpb_dn - 1) / rpb_dn);
 #define TERN_GU_CASE(GG)                                                                                   \
