@@ -464,14 +464,14 @@ __device__ __forceinline__ void mma_stage(uint32_t *dst, const uint32_t *__restr
 }
 
 // One 16-row tile x K codes of one matrix against the staged columns: acc[l] += A * B_l.
-// row0 = the tile's first row; rows >= nrows contribute zeros.  K % 64 == 0.
+// row0 = the tile's first row; rows >= nrows contribute zeros.  K % 64 == 0.  lut: the compact
+// 256-word decode table (entry = the four int8 weights of a packed byte); it keeps shared
+// memory small enough for four CTAs per SM, which hide the row loads' latency.
 template <int NL, int NM>
 __device__ __forceinline__ void mma_tile(const uint8_t *const (&mats)[NM], int64_t rowb, int row0, int nrows, int K,
                                          const uint32_t *xs, int rs, const uint32_t *lut, int (&acc)[NM][NL][4]) {
     const int lane = threadIdx.x & 31, g = lane >> 2, tig = lane & 3;
-    const uint32_t lane4 = (uint32_t)lane << 2;
-    const uint32_t sel = 0x5504u | ((uint32_t)tig << 4);  // byte tig of a word -> table offset
-    const char *lb = reinterpret_cast<const char *>(lut);
+    const int sh = 8 * tig;  // byte tig of a word
     const bool v0 = row0 + g < nrows, v1 = row0 + g + 8 < nrows;
     for (int m = 0; m < K / 64; m++) {  // 16 packed bytes = two k-blocks of 32 codes
         uint4 w0[NM], w1[NM];
@@ -495,10 +495,8 @@ __device__ __forceinline__ void mma_tile(const uint8_t *const (&mats)[NM], int64
             for (int q = 0; q < NM; q++) {
                 const uint32_t lo0 = jj ? w0[q].z : w0[q].x, hi0 = jj ? w0[q].w : w0[q].y;
                 const uint32_t lo1 = jj ? w1[q].z : w1[q].x, hi1 = jj ? w1[q].w : w1[q].y;
-                const uint32_t a0 = *reinterpret_cast<const uint32_t *>(lb + __byte_perm(lo0, lane4, sel));
-                const uint32_t a1 = *reinterpret_cast<const uint32_t *>(lb + __byte_perm(lo1, lane4, sel));
-                const uint32_t a2 = *reinterpret_cast<const uint32_t *>(lb + __byte_perm(hi0, lane4, sel));
-                const uint32_t a3 = *reinterpret_cast<const uint32_t *>(lb + __byte_perm(hi1, lane4, sel));
+                const uint32_t a0 = lut[(lo0 >> sh) & 0xFFu], a1 = lut[(lo1 >> sh) & 0xFFu];
+                const uint32_t a2 = lut[(hi0 >> sh) & 0xFFu], a3 = lut[(hi1 >> sh) & 0xFFu];
                 mma_s8<false>(acc[q][0], a0, a1, a2, a3, b0[0], b1[0]);
                 if (NL > 1) {
                     mma_s8<true>(acc[q][NL > 1 ? 1 : 0], a0, a1, a2, a3, b0[NL > 1 ? 1 : 0], b1[NL > 1 ? 1 : 0]);
@@ -518,11 +516,11 @@ __global__ void __launch_bounds__(kMmaWarps * 32) gateup_mma_kernel(
     const uint32_t *__restrict__ xw, const float *__restrict__ xsc, float *__restrict__ h,
     int32_t *__restrict__ acc_g, int32_t *__restrict__ acc_u) {
     extern __shared__ __align__(16) uint32_t smem[];
-    uint32_t *lut = smem;
-    uint32_t *xs = smem + kLutWords;  // [kMmaTok][NL][d/4 + pad]
+    uint32_t *lut = smem;        // [256] compact decode table
+    uint32_t *xs = smem + 256;  // [kMmaTok][NL][d/4 + pad]
     const int u = blockIdx.x;
     if (u >= *n_unique) return;
-    lut_fill(lut);
+    for (int b = threadIdx.x; b < 256; b += blockDim.x) lut[b] = decode_byte((uint32_t)b);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, tig = lane & 3;
     const int e = uexp[u], e0 = uoff[u], e1 = uoff[u + 1];
     const int64_t rowb = d / 4;
@@ -582,11 +580,11 @@ __global__ void __launch_bounds__(kMmaWarps * 32) down_mma_kernel(
     const int32_t *__restrict__ ent, const uint32_t *__restrict__ hw, const float *__restrict__ hsc,
     double *__restrict__ ye, int32_t *__restrict__ acc_d) {
     extern __shared__ __align__(16) uint32_t smem[];
-    uint32_t *lut = smem;
-    uint32_t *xs = smem + kLutWords;  // [kMmaTok][NL][f/4 + pad]
+    uint32_t *lut = smem;        // [256] compact decode table
+    uint32_t *xs = smem + 256;  // [kMmaTok][NL][f/4 + pad]
     const int u = blockIdx.x;
     if (u >= *n_unique) return;
-    lut_fill(lut);
+    for (int b = threadIdx.x; b < 256; b += blockDim.x) lut[b] = decode_byte((uint32_t)b);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, tig = lane & 3;
     const int e = uexp[u], e0 = uoff[u], e1 = uoff[u + 1];
     const int64_t rowb = f / 4;
@@ -689,8 +687,8 @@ static cudaError_t ffn_stages_nl(const tern_moe_layer *L, const uint16_t *x, int
     const int Gd = d / 64, Gf = f / 64;
     if (T >= kMmaGroupedMinT) {  // grouped path on int8 tensor cores
         const dim3 m1(umax, (f + kMmaRows - 1) / kMmaRows), m2(umax, (d + kMmaRows - 1) / kMmaRows);
-        const size_t sm1 = kLutBytes + (size_t)kMmaTok * NL * (d / 4 + kMmaPad) * 4;
-        const size_t sm2 = kLutBytes + (size_t)kMmaTok * NL * (f / 4 + kMmaPad) * 4;
+        const size_t sm1 = 1024 + (size_t)kMmaTok * NL * (d / 4 + kMmaPad) * 4;
+        const size_t sm2 = 1024 + (size_t)kMmaTok * NL * (f / 4 + kMmaPad) * 4;
         cudaFuncSetAttribute(gateup_mma_kernel<NL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
         cudaFuncSetAttribute(down_mma_kernel<NL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
         err = launch_k(gateup_mma_kernel<NL>, m1, dim3(kMmaWarps * 32), sm1, s, L->gate, L->up, L->gate_scale,
