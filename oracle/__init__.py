@@ -65,6 +65,12 @@ def lib():
             L.or_pack.argtypes = [vp, i64, i64, vp]
             L.or_unpack.restype = i64
             L.or_unpack.argtypes = [vp, i64, i64, vp]
+            L.or_tern5_row_bytes.restype = i64
+            L.or_tern5_row_bytes.argtypes = [i64]
+            L.or_pack5.restype = i64
+            L.or_pack5.argtypes = [vp, i64, i64, vp]
+            L.or_unpack5.restype = i64
+            L.or_unpack5.argtypes = [vp, i64, i64, vp]
             L.or_gemv_i8.restype = ctypes.c_int
             L.or_gemv_i8.argtypes = [vp, vp, i64, i64, i64, vp, vp, vp, vp]
             L.or_gemv_bf16.restype = i64
@@ -112,6 +118,40 @@ def unpack(p, K):
     w = np.empty((M, K), dtype=np.int8)
     bad = lib().or_unpack(_p(p), M, K, _p(w))
     return w, int(bad)
+
+
+def tern5_row_bytes(K):
+    """Bytes per row of the base-3 format (five weights per byte, rows padded to 16 bytes)."""
+    return int(lib().or_tern5_row_bytes(int(K)))
+
+
+def pack5(w):
+    w = _c(w, np.int8)
+    M, K = w.shape
+    out = np.empty((M, tern5_row_bytes(K)), dtype=np.uint8)
+    bad = lib().or_pack5(_p(w), M, K, _p(out))
+    return out, int(bad)
+
+
+def unpack5(p, K):
+    p = _c(p, np.uint8)
+    M = p.shape[0]
+    w = np.empty((M, K), dtype=np.int8)
+    bad = lib().or_unpack5(_p(p), M, K, _p(w))
+    return w, int(bad)
+
+
+def gemv5_i8(W5, s, q, x_scale=None):
+    """The int8 GEMV of base-3 packed weights: the weights it decodes to, through gemv_i8."""
+    q = np.atleast_2d(q)
+    w, _ = unpack5(W5, q.shape[1])
+    return gemv_i8(pack(w)[0], s, q, x_scale)
+
+
+def gemv5_bf16(W5, s, x):
+    x = np.atleast_2d(x)
+    w, _ = unpack5(W5, x.shape[1])
+    return gemv_bf16(pack(w)[0], s, x)
 
 
 def gemv_i8(Wp, s, q, x_scale=None):

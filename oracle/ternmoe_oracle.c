@@ -153,6 +153,63 @@ int64_t or_unpack(const uint8_t *p, int64_t M, int64_t K, int8_t *w) {
     return bad;
 }
 
+/* ------------------------------------------------ base-3 packing: five weights per byte
+ * The pages give the information content of a ternary weight, log2(3) ~ 1.585 bits ("How a
+ * 20B Model Hits 120 tok/s on an iPhone", "Why the number is plausible"; "A 20B AI Model
+ * Trained in Ternary...", "What Ternary Actually Means").  3^5 = 243 <= 256, so five weights
+ * fit one byte: 1.6 bits per weight.  Reading taken here: weight w[5b+i] contributes the digit
+ * t_i in {0,1,2} -- the same code as the 2-bit format (0 -> 0, 1 -> +1, 2 -> -1) -- and byte b
+ * of a row holds t_0 + 3 t_1 + 9 t_2 + 27 t_3 + 81 t_4 (little-endian along K).  Positions past
+ * K hold digit 0; each row is padded with zero bytes to a multiple of 16 bytes.  Bytes 243..255
+ * are never produced and decode to five zeros (reported). */
+int64_t or_tern5_row_bytes(int64_t K) {
+    const int64_t b = (K + 4) / 5;
+    return (b + 15) / 16 * 16;
+}
+
+int64_t or_pack5(const int8_t *w, int64_t M, int64_t K, uint8_t *out) {
+    const int64_t rb = or_tern5_row_bytes(K);
+    int64_t bad = 0;
+    for (int64_t m = 0; m < M; m++)
+        for (int64_t b = 0; b < rb; b++) {
+            unsigned value = 0, place = 1;
+            for (int i = 0; i < 5; i++) {
+                const int64_t k = 5 * b + i;
+                unsigned digit = 0;
+                if (k < K) {
+                    const int v = w[m * K + k];
+                    if (v == 1) digit = 1;
+                    else if (v == -1) digit = 2;
+                    else if (v != 0) bad++;
+                }
+                value += digit * place;
+                place *= 3;
+            }
+            out[m * rb + b] = (uint8_t)value;
+        }
+    return bad;
+}
+
+/* Returns the number of bytes >= 243 among the bytes that hold weights of [0, K). */
+int64_t or_unpack5(const uint8_t *p, int64_t M, int64_t K, int8_t *w) {
+    const int64_t rb = or_tern5_row_bytes(K);
+    int64_t bad = 0;
+    for (int64_t m = 0; m < M; m++)
+        for (int64_t b = 0; b * 5 < K; b++) {
+            unsigned value = p[m * rb + b];
+            if (value >= 243) {
+                bad++;
+                value = 0;
+            }
+            for (int i = 0; i < 5; i++) {
+                const int64_t k = 5 * b + i;
+                if (k < K) w[m * K + k] = (int8_t)code_to_weight(value % 3);
+                value /= 3;
+            }
+        }
+    return bad;
+}
+
 static int weight_at(const uint8_t *row, int64_t k) {
     return code_to_weight((row[k / 4] >> (2 * (k % 4))) & 3u);
 }

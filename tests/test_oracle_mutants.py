@@ -23,6 +23,10 @@ MUTANTS = {
     "residual_dropped": ("f64_to_bf16(bf16_to_f64(x[i]) + bf16_to_f64(y[i]))", "y[i]"),
     "gate_up_swapped": ("h[j] = (float)silu_times(g, u);", "h[j] = (float)silu_times(u, g);"),
     "int8_scale_order": ("g = g * sg;\n                    g = g * sx;", "g = g * sx;\n                    g = g * sx;"),
+    "base3_big_endian": ("value += digit * place;\n                place *= 3;",
+                         "value = value * 3 + digit;\n                place *= 3;"),
+    "base3_digits_swapped": ("if (v == 1) digit = 1;\n                    else if (v == -1) digit = 2;",
+                             "if (v == 1) digit = 2;\n                    else if (v == -1) digit = 1;"),
 }
 
 

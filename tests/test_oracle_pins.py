@@ -443,3 +443,53 @@ def test_synthetic_model_byte_count():
     assert per_layer_token == 7438336
     assert 24 * per_layer_token == 178520064
     assert 24 * (256 * (packed + scales) + router) == 4932501504
+
+
+# ------------------------------------------------ base-3 packing (five weights per byte)
+
+def test_pack5_is_a_bijection_on_all_243_quintuples():
+    """Every ternary 5-tuple packs to its own byte below 243, and unpacks back."""
+    tuples = np.array(list(itertools.product((-1, 0, 1), repeat=5)), dtype=np.int8)  # [243, 5]
+    p, bad = oracle.pack5(tuples)
+    assert bad == 0 and p.shape == (243, 16)
+    assert (p[:, 1:] == 0).all()                     # row padding to 16 bytes
+    assert len(set(p[:, 0].tolist())) == 243 and p[:, 0].max() <= 242
+    w, bad = oracle.unpack5(p, 5)
+    assert bad == 0 and (w == tuples).all()
+
+
+def test_pack5_place_values():
+    """Little-endian base 3 along K with the 2-bit format's digits (0, +1 -> 1, -1 -> 2)."""
+    rows = np.array([[1, 0, 0, 0, 0], [0, 0, 0, 0, -1], [1, 1, 1, 1, 1], [-1] * 5, [0] * 5,
+                     [0, -1, 1, 0, 0]], dtype=np.int8)
+    p, _ = oracle.pack5(rows)
+    assert p[:, 0].tolist() == [1, 162, 121, 242, 0, 2 * 3 + 1 * 9]
+
+
+def test_pack5_tail_density_and_bad_bytes():
+    # K = 7: the second byte holds two weights, its other three digits are zero
+    w = np.array([[1, -1, 0, 1, -1, -1, 1]], dtype=np.int8)
+    p, _ = oracle.pack5(w)
+    assert p[0, 1] == 2 + 3 * 1 and (p[0, 2:] == 0).all()
+    assert (oracle.unpack5(p, 7)[0] == w).all()
+    # bytes per row: ceil(K/5) rounded up to 16; 2048 weights take 416 bytes instead of 512
+    assert [oracle.tern5_row_bytes(k) for k in (1, 5, 80, 81, 2048, 16384)] == [16, 16, 16, 32, 416, 3280]
+    assert oracle.tern5_row_bytes(2048) / 512 == 0.8125
+    # a byte that no 5-tuple produces is reported and read as five zeros
+    q = np.zeros((1, 16), np.uint8)
+    q[0, 0] = 250
+    wq, bad = oracle.unpack5(q, 5)
+    assert bad == 1 and (wq == 0).all()
+    # values that are not ternary are counted
+    assert oracle.pack5(np.array([[2, 0, 0, 0, 0]], np.int8))[1] == 1
+
+
+def test_gemv5_equals_two_bit_gemv():
+    """The base-3 GEMV computes the same dot products as the 2-bit one on the same weights."""
+    w = synth.ternary_codes(41, 0, 33 * 128, synth.P0_UNIFORM).reshape(33, 128)
+    s = synth.uniform_f32(42, 0, 33, 0.5, 1.5)
+    q = synth.int8_uniform(43, 0, 3 * 128).reshape(3, 128)
+    a5, y5 = oracle.gemv5_i8(oracle.pack5(w)[0], s, q)
+    a2, y2 = oracle.gemv_i8(oracle.pack(w)[0], s, q)
+    assert (a5 == a2).all() and (y5 == y2).all()
+    assert (a2 == q.astype(np.int64) @ w.T.astype(np.int64)).all()
