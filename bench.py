@@ -278,9 +278,10 @@ def run_reference(args):
 
 
 def run_gemv_sweep(args):
-    """Extra output: device time of one tern_gemv launch per shape of the GEMV sweep (T = 1,
-    bf16 and int8 activations), L2 flushed before every launch; one JSON line per shape.
-    The last shape (128 MB of packed codes) is a bandwidth check, not one of the sweep's."""
+    """Extra output: device time of one tern_gemv launch (four codes per byte) and one
+    tern5_gemv launch (five weights per byte, base 3) per shape of the GEMV sweep (T = 1, bf16
+    and int8 activations), L2 flushed before every launch; one JSON line per case.  The last
+    shape (128 MB of packed codes) is a bandwidth check, not one of the sweep's."""
     import torch
 
     import synth
@@ -298,16 +299,26 @@ def run_gemv_sweep(args):
         base = synth.derive(synth.BASE_SEED + 2, M, K)
         w = synth.ternary_codes_torch(synth.derive(base, synth.KIND_W), 0, M * K, synth.P0_SPARSE, dev).view(M, K)
         Wp = tm.tern_pack(w)
+        W5 = tm.tern5_pack(w)  # five weights per byte, for the base-3 lines
         del w
         rs = torch.from_numpy(synth.uniform_f32(synth.derive(base, synth.KIND_S), 0, M, 0.01, 0.05)).to(dev)
         xb = torch.from_numpy(synth.normal_bf16(synth.derive(base, synth.KIND_X), 0, K, 1.0).view(np.int16)).to(dev)
         xi = torch.from_numpy(synth.int8_uniform(synth.derive(base, synth.KIND_XQ), 0, K)).to(dev)
         y = torch.empty((1, M), dtype=torch.float32, device=dev)
-        for act_name, act, x in (("bf16", tm.TERN_ACT_BF16, xb), ("int8", tm.TERN_ACT_INT8, xi)):
+        cases = [("2bit", act_name, act, x) for act_name, act, x in
+                 (("bf16", tm.TERN_ACT_BF16, xb), ("int8", tm.TERN_ACT_INT8, xi))]
+        cases += [("base3", c[1], c[2], c[3]) for c in cases]
+        for fmt, act_name, act, x in cases:
             if args.act_only and act_name != args.act:
                 continue
+            if fmt == "2bit":
+                call = lambda: tm.tern_gemv(Wp, rs, x, act=act, y=y)  # noqa: E731
+                wbytes = M * K // 4
+            else:
+                call = lambda: tm.tern5_gemv(W5, rs, x, K, act=act, y=y)  # noqa: E731
+                wbytes = M * tm.tern5_row_bytes(K)
             for _ in range(max(args.warmup, 3)):
-                tm.tern_gemv(Wp, rs, x, act=act, y=y)
+                call()
             # no host wait inside the loop: the flush keeps the device busy while the host
             # enqueues the next launch, so the events see device time only
             evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -316,20 +327,20 @@ def run_gemv_sweep(args):
             for i in range(args.steps):
                 flush.fill_(i & 0xFF)
                 evs[i][0].record(stream)
-                tm.tern_gemv(Wp, rs, x, act=act, y=y)
+                call()
                 evs[i][1].record(stream)
             torch.cuda.synchronize(dev)
             ms = [a.elapsed_time(b) for a, b in evs]
             if tm.tern_stream_status() != 0:
                 raise RuntimeError("device status set during the sweep")
             med = statistics.median(ms)
-            nbytes = M * K // 4 + 4 * M + (2 if act_name == "bf16" else 1) * K + 4 * M
+            nbytes = wbytes + 4 * M + (2 if act_name == "bf16" else 1) * K + 4 * M
             gbs = nbytes / (med * 1e-3) / 1e9
-            print(json.dumps({"gemv": f"{M}x{K}", "act": act_name, "us_median": med * 1e3,
+            print(json.dumps({"gemv": f"{M}x{K}", "format": fmt, "act": act_name, "us_median": med * 1e3,
                               "us_p10": float(np.percentile(ms, 10)) * 1e3, "bytes": nbytes, "GB/s": gbs,
                               "frac": gbs / peak, "peak": peak, "peak_kind": peak_kind, "launches": args.steps}),
                   flush=True)
-        del Wp
+        del Wp, W5
     return 0
 
 

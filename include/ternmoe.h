@@ -128,6 +128,30 @@ tern_status tern_gemv(const uint8_t *Wp, const float *row_scale, int64_t M, int6
                       const void *x, const float *x_scale, int64_t T, int32_t *acc, float *y,
                       void *stream);
 
+/* Base-3 packed format: five ternary weights per byte, 1.6 bits per weight (a ternary weight
+ * carries log2(3) ~ 1.585 bits: "How a 20B Model Hits 120 tok/s on an iPhone", "Why the
+ * number is plausible").  Byte b of a row holds t0 + 3 t1 + 9 t2 + 27 t3 + 81 t4, where t_i is
+ * the 2-bit code of weight 5b+i (0 -> 0, 1 -> +1, 2 -> -1); positions past K and the row's
+ * padding bytes are 0.  A row takes tern5_row_bytes(K) bytes: ceil(K/5) rounded up to a
+ * multiple of 16 (416 bytes for K = 2048, against 512 for four codes per byte).
+ * Returns 0 for K < 1. */
+int64_t tern5_row_bytes(int64_t K);
+
+/* Pack int8 w [M][K] (values in {-1,0,1}) into packed [M][tern5_row_bytes(K)].  Waits for its
+ * kernel; returns TERN_ECODE if any weight is outside {-1,0,1} (packed as 0).  Any K >= 1. */
+tern_status tern5_pack(const int8_t *w, int64_t M, int64_t K, uint8_t *packed, void *stream);
+
+/* Unpack into int8 w [M][K].  Waits; returns TERN_ECODE if a byte holding weights is >= 243
+ * (its five weights are written as 0). */
+tern_status tern5_unpack(const uint8_t *packed, int64_t M, int64_t K, int8_t *w, void *stream);
+
+/* The ternary GEMV of tern_gemv on base-3 packed rows W5 [M][tern5_row_bytes(K)]: same
+ * arguments, same arithmetic and results (exact integer sums).  1 <= K <= 16384; W5 16-byte
+ * aligned, x 2-byte aligned. */
+tern_status tern5_gemv(const uint8_t *W5, const float *row_scale, int64_t M, int64_t K, tern_act act,
+                       const void *x, const float *x_scale, int64_t T, int32_t *acc, float *y,
+                       void *stream);
+
 /* Per-vector absmax int8 quantisation of bf16 rows x [T][n]:  s[t] = absmax/127,
  * q = clamp(rint(x * (127/absmax)), -127, 127) in fp32, ties to even; a zero row gives
  * q = 0, s = 0.  (The pages are silent on activation precision; this is the int8 reading.) */

@@ -78,6 +78,10 @@ def lib():
             "tern_unpack": (st, [vp, i64, i64, vp, vp]),
             "tern_gemv": (st, [vp, vp, i64, i64, st, vp, vp, i64, vp, vp, vp]),
             "tern_quant_absmax": (st, [vp, i64, i64, vp, vp, vp]),
+            "tern5_row_bytes": (i64, [i64]),
+            "tern5_pack": (st, [vp, i64, i64, vp, vp]),
+            "tern5_unpack": (st, [vp, i64, i64, vp, vp]),
+            "tern5_gemv": (st, [vp, vp, i64, i64, st, vp, vp, i64, vp, vp, vp]),
             "moe_route_workspace_bytes": (sz, [i64, i32]),
             "moe_route_topk": (st, [vp, vp, i64, i64, i32, i32, vp, vp, vp, vp, sz, vp]),
             "moe_route_topk_static": (st, [vp, vp, i64, i64, i32, i32, vp, vp, vp, vp]),
@@ -189,6 +193,55 @@ def tern_gemv(Wp, row_scale, x, act=TERN_ACT_BF16, x_scale=None, acc=None, y=Non
         _dev(acc, torch.int32, "acc")
     _check(lib().tern_gemv(_ptr(Wp), _ptr(row_scale), M, K, act, _ptr(x), _ptr(x_scale), T, _ptr(acc),
                            _ptr(y), _stream(stream)), "tern_gemv")
+    return y
+
+
+def tern5_row_bytes(K: int) -> int:
+    return int(lib().tern5_row_bytes(int(K)))
+
+
+def tern5_pack(w: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Five weights per byte (base 3): [M, K] int8 -> [M, tern5_row_bytes(K)] uint8."""
+    _dev(w, torch.int8, "w")
+    M, K = w.shape
+    if out is None:
+        out = torch.empty((M, tern5_row_bytes(K)), dtype=torch.uint8, device=w.device)
+    _dev(out, torch.uint8, "packed")
+    _check(lib().tern5_pack(_ptr(w), M, K, _ptr(out), _stream(stream)), "tern5_pack")
+    return out
+
+
+def tern5_unpack(p: torch.Tensor, K: int, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    _dev(p, torch.uint8, "packed")
+    M = p.shape[0]
+    if out is None:
+        out = torch.empty((M, K), dtype=torch.int8, device=p.device)
+    _dev(out, torch.int8, "w")
+    _check(lib().tern5_unpack(_ptr(p), M, K, _ptr(out), _stream(stream)), "tern5_unpack")
+    return out
+
+
+def tern5_gemv(W5, row_scale, x, K, act=TERN_ACT_BF16, x_scale=None, acc=None, y=None, stream=None):
+    """tern_gemv on base-3 packed rows; K is the number of weights per row."""
+    _dev(W5, torch.uint8, "W5")
+    _dev(row_scale, torch.float32, "row_scale")
+    M = W5.shape[0]
+    if x.dim() == 1:
+        x = x.view(1, -1)
+    T = x.shape[0]
+    if act == TERN_ACT_INT8:
+        _dev(x, torch.int8, "x")
+        if x_scale is not None:
+            _dev(x_scale, torch.float32, "x_scale")
+    else:
+        x = _bits16(x, "x")
+    if y is None:
+        y = torch.empty((T, M), dtype=torch.float32, device=W5.device)
+    _dev(y, torch.float32, "y")
+    if acc is not None:
+        _dev(acc, torch.int32, "acc")
+    _check(lib().tern5_gemv(_ptr(W5), _ptr(row_scale), M, K, act, _ptr(x), _ptr(x_scale), T, _ptr(acc), _ptr(y),
+                            _stream(stream)), "tern5_gemv")
     return y
 
 

@@ -81,3 +81,18 @@ def test_argument_checks_before_any_launch():
     assert L.moe_stack_decode(arr, 0, p, 1, 1e-6, 0, p, 1 << 30, None) == 1
     assert L.moe_stack_decode(arr, 1, p, 1, -1.0, 0, p, 1 << 30, None) == 1
     assert L.tern_test_bounded_wait(None, 10, None) == 1
+
+
+def test_base3_format_host_checks():
+    """The five-weights-per-byte calls: row size arithmetic and argument checks, no GPU."""
+    L = tm.lib()
+    assert [L.tern5_row_bytes(k) for k in (0, 1, 5, 80, 81, 2048, 16384)] == [0, 16, 16, 16, 32, 416, 3280]
+    p = ctypes.c_void_p(1 << 40)
+    assert L.tern5_gemv(p, p, 16, 0, 0, p, None, 1, None, p, None) == 1          # K < 1
+    assert L.tern5_gemv(p, p, 16, 16385, 0, p, None, 1, None, p, None) == 1      # K too large
+    assert L.tern5_gemv(p, p, 16, 2048, 0, p, None, 65, None, p, None) == 1      # T out of range
+    assert L.tern5_gemv(p, p, 16, 2048, 0, p, None, 1, p, p, None) == 1          # bf16 with acc
+    q = ctypes.c_void_p((1 << 40) + 8)
+    assert L.tern5_gemv(q, p, 16, 2048, 1, p, None, 1, None, p, None) == 2       # misaligned rows
+    assert L.tern5_pack(None, 4, 10, p, None) == 1
+    assert L.tern5_unpack(p, 0, 10, p, None) == 1
