@@ -399,6 +399,50 @@ def run_batch_sweep(args):
     return 0
 
 
+def run_head(args):
+    """Extra output: the approximate output head (151,936 tokens in 4,748 clusters of 32,
+    d = 2048, top 512 clusters) against the full head (every cluster kept), one token per
+    call, L2 flushed before every call; one JSON line each."""
+    import torch
+
+    import synth
+    import ternary_weight_moe_b200 as tm
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peak, peak_kind = peaks()
+    hs = synth.head_shape()
+    V, d, nc, cs = hs["V"], hs["d"], hs["n_clusters"], hs["cluster_size"]
+    W = synth.normal_bf16_torch(synth.derive(synth.BASE_SEED + 6, 1), 0, V * d, 0.02, dev).view(V, d)
+    C4, sc = tm.flash_head_centroids(W, cs)
+    xs = torch.from_numpy(synth.normal_bf16(synth.derive(synth.BASE_SEED + 6, 3), 0, (args.steps + 3) * d, 1.0)
+                          .view(np.int16)).to(dev).view(-1, d)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for name, top_c in (("flash_head top-512", hs["top_c"]), ("full head", nc)):
+        out = tm.flash_head(C4, sc, W, xs[0], cs, top_c)
+        for i in range(3):
+            tm.flash_head(C4, sc, W, xs[i], cs, top_c, out=out)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        torch.cuda.synchronize(dev)
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            evs[i][0].record(stream)
+            tm.flash_head(C4, sc, W, xs[3 + i], cs, top_c, out=out)
+            evs[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        ms = [a.elapsed_time(b) for a, b in evs]
+        med = statistics.median(ms)
+        nbytes = nc * (d // 2 + 8) + top_c * cs * (2 * d + 12) + 2 * d + 8 * nc
+        gbs = nbytes / (med * 1e-3) / 1e9
+        print(json.dumps({"head": name, "top_clusters": top_c, "us_median": med * 1e3,
+                          "us_p10": float(np.percentile(ms, 10)) * 1e3, "tokens_per_s": 1.0 / (med * 1e-3),
+                          "bytes": nbytes, "GB/s": gbs, "frac": gbs / peak, "peak": peak, "peak_kind": peak_kind,
+                          "vocab": V, "d": d, "steps": args.steps}), flush=True)
+    return 0
+
+
 def main():
     global N_LAYERS, BYTES_PER_TOKEN
     ap = argparse.ArgumentParser()
@@ -417,6 +461,8 @@ def main():
     ap.add_argument("--batch-sweep", action="store_true",
                     help="extra output: time one MoE FFN layer at T = 1, 4, 16, 64 tokens per step")
     ap.add_argument("--batch-T", default=None, help="with --batch-sweep: comma-separated T values only")
+    ap.add_argument("--head", action="store_true",
+                    help="extra output: time the approximate output head against the full head")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -426,6 +472,8 @@ def main():
         return run_gemv_sweep(args)
     if args.batch_sweep:
         return run_batch_sweep(args)
+    if args.head:
+        return run_head(args)
 
     import torch
 

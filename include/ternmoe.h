@@ -220,6 +220,33 @@ tern_status moe_stack_decode(const tern_moe_layer *layers, int32_t n_layers, uin
                              float rms_eps, tern_act act, void *workspace, size_t ws_bytes,
                              void *stream);
 
+/* Approximate output head ("A 20B AI Model Trained in Ternary Just Hit 218 Tokens/Second on
+ * a $599 Mac Mini", "The Architecture: Designed for the Hardware": cluster the vocabulary,
+ * score 4-bit cluster centroids, project only the tokens of the best clusters).
+ * The unembedding W [V][d] (bf16, V = n_clusters * cluster_size) is stored cluster-major:
+ * cluster c holds tokens c*cluster_size .. (c+1)*cluster_size - 1.
+ *
+ * flash_head_centroids (preparation, once per W): centroid c = exact mean of its cluster's
+ * rows; stored as symmetric int4 codes C4 [n_clusters][d/2] (values in [-7, 7], element 2j in
+ * the low nibble of byte j, two's complement) and one fp64 scale c_scale[c] = absmax / 7
+ * (codes = clamp(rint(centroid / scale)), ties to even; a zero centroid has scale 0).
+ *
+ * flash_head, one token x [d] (bf16):
+ *   scores[c] = c_scale[c] * sum_k code_ck x_k           (fp64, exact sum) [n_clusters];
+ *   sel_clusters = the top_c clusters by score, larger first, ties to the lower index [top_c];
+ *   cand_ids / cand_logits = the tokens of the selected clusters in selection order, then row
+ *     order, and sum_k W_vk x_k (fp64, exact products)   [top_c * cluster_size];
+ *   best_id[0] = the candidate with the largest logit, ties to the lower token id.
+ * top_c = n_clusters gives the full head.  64 <= d <= 8192, d % 64 == 0,
+ * 1 <= n_clusters <= 8192, 1 <= cluster_size <= 1024, 1 <= top_c <= n_clusters.  W 16-byte
+ * aligned.  All outputs are caller-owned device arrays; nothing else is allocated. */
+tern_status flash_head_centroids(const uint16_t *W, int64_t d, int32_t n_clusters, int32_t cluster_size,
+                                 uint8_t *C4, double *c_scale, void *stream);
+tern_status flash_head(const uint8_t *C4, const double *c_scale, const uint16_t *W, const uint16_t *x,
+                       int64_t d, int32_t n_clusters, int32_t cluster_size, int32_t top_c,
+                       double *scores, int32_t *sel_clusters, int32_t *cand_ids, double *cand_logits,
+                       int32_t *best_id, void *stream);
+
 /* Where, inside a moe_stack_decode workspace, a T == 1 call (the persistent kernel) leaves
  * its per-layer record, for inspection and parity checks (byte offsets):
  *   hist    uint16 [n_layers+1][d]  bf16 x entering each layer, and the final x;

@@ -30,6 +30,8 @@ from __future__ import annotations
 
 from fractions import Fraction
 
+import math
+
 import numpy as np
 
 GAMMA = 0x9E3779B97F4A7C15
@@ -186,6 +188,48 @@ def ternary_codes_torch(seed: int, offset: int, n: int, p0, device, chunk: int =
         o[v < t0] = 0
         out[start:start + m] = o
     return out
+
+
+def normal_bf16_torch(seed: int, offset: int, n: int, sigma: float, device, chunk: int = 1 << 25):
+    """N(0, sigma^2) as bf16 bits (int16 tensor of length n) on `device`: the draws of
+    normal_bf16() (same SplitMix64 stream, same Box-Muller pairing) with the transcendental
+    functions evaluated by torch on the device, rounded fp64 -> fp32 -> bf16 (nearest, ties to
+    even each time).  The values follow the same distribution as normal_bf16() but need not
+    match it bit for bit: tests hand the device values themselves to the oracle."""
+    import torch
+
+    out = torch.empty(n, dtype=torch.int16, device=device)
+    g = _signed(GAMMA)
+    c1 = _signed(C1)
+    c2 = _signed(C2)
+    s = _signed(seed & M64)
+
+    def lsr(z, k):
+        return (z >> k) & ((1 << (64 - k)) - 1)
+
+    def draws(first, m):
+        i = torch.arange(first + 1, first + m + 1, dtype=torch.int64, device=device)
+        z = i * g + s
+        z = z ^ lsr(z, 30)
+        z = z * c1
+        z = z ^ lsr(z, 27)
+        z = z * c2
+        z = z ^ lsr(z, 31)
+        return lsr(z, 11).to(torch.float64) * (2.0 ** -53)
+
+    for start in range(0, n, chunk):
+        m = min(chunk, n - start)
+        u = draws(2 * (offset + start), 2 * m)
+        u1, u2 = u[0::2], u[1::2]
+        z = torch.sqrt(-2.0 * torch.log1p(-u1)) * torch.cos(2.0 * math.pi * u2) * sigma
+        out[start:start + m] = z.to(torch.float32).to(torch.bfloat16).view(torch.int16)
+    return out
+
+
+def head_shape():
+    """The approximate head's workload: a 151,936-token vocabulary in 4,748 clusters of 32
+    tokens, hidden size 2,048, the top 512 clusters kept."""
+    return {"V": 151936, "d": 2048, "n_clusters": 4748, "cluster_size": 32, "top_c": 512}
 
 
 # ---------------------------------------------------------------------------

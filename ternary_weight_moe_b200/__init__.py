@@ -78,6 +78,8 @@ def lib():
             "tern_unpack": (st, [vp, i64, i64, vp, vp]),
             "tern_gemv": (st, [vp, vp, i64, i64, st, vp, vp, i64, vp, vp, vp]),
             "tern_quant_absmax": (st, [vp, i64, i64, vp, vp, vp]),
+            "flash_head_centroids": (st, [vp, i64, i32, i32, vp, vp, vp]),
+            "flash_head": (st, [vp, vp, vp, vp, i64, i32, i32, i32, vp, vp, vp, vp, vp, vp]),
             "tern5_row_bytes": (i64, [i64]),
             "tern5_pack": (st, [vp, i64, i64, vp, vp]),
             "tern5_unpack": (st, [vp, i64, i64, vp, vp]),
@@ -243,6 +245,37 @@ def tern5_gemv(W5, row_scale, x, K, act=TERN_ACT_BF16, x_scale=None, acc=None, y
     _check(lib().tern5_gemv(_ptr(W5), _ptr(row_scale), M, K, act, _ptr(x), _ptr(x_scale), T, _ptr(acc), _ptr(y),
                             _stream(stream)), "tern5_gemv")
     return y
+
+
+def flash_head_centroids(W, cluster_size: int, stream=None):
+    """4-bit cluster centroids of a cluster-major bf16 unembedding W [V, d]: (C4, c_scale)."""
+    W = _bits16(W, "W")
+    V, d = W.shape
+    nc = V // cluster_size
+    C4 = torch.empty((nc, d // 2), dtype=torch.uint8, device=W.device)
+    sc = torch.empty(nc, dtype=torch.float64, device=W.device)
+    _check(lib().flash_head_centroids(_ptr(W), d, nc, cluster_size, _ptr(C4), _ptr(sc), _stream(stream)),
+           "flash_head_centroids")
+    return C4, sc
+
+
+def flash_head(C4, c_scale, W, x, cluster_size: int, top_c: int, out=None, stream=None) -> dict:
+    """One token through the approximate head; returns the device arrays of every output."""
+    W = _bits16(W, "W")
+    x = _bits16(x.view(-1), "x")
+    V, d = W.shape
+    nc = C4.shape[0]
+    dev = W.device
+    if out is None:
+        out = {"scores": torch.empty(nc, dtype=torch.float64, device=dev),
+               "sel": torch.empty(top_c, dtype=torch.int32, device=dev),
+               "ids": torch.empty(top_c * cluster_size, dtype=torch.int32, device=dev),
+               "logits": torch.empty(top_c * cluster_size, dtype=torch.float64, device=dev),
+               "best": torch.empty(1, dtype=torch.int32, device=dev)}
+    _check(lib().flash_head(_ptr(C4), _ptr(c_scale), _ptr(W), _ptr(x), d, nc, cluster_size, top_c,
+                            _ptr(out["scores"]), _ptr(out["sel"]), _ptr(out["ids"]), _ptr(out["logits"]),
+                            _ptr(out["best"]), _stream(stream)), "flash_head")
+    return out
 
 
 def tern_quant_absmax(x, q=None, s=None, stream=None):
