@@ -27,6 +27,9 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+# side files (clock samples, per-phase traces) go here
+OUT_DIR = os.environ.get("TERNMOE_BENCH_OUT", os.path.join(ROOT, "bench_out"))
+
 METRIC = "ternary MoE FFN decode tokens/s @batch1; achieved HBM GB/s vs B200 peak"
 UNIT = "tokens/s"
 N_LAYERS = 24
@@ -83,7 +86,7 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        self.path = os.path.join(OUT_DIR, f"clocks_rank{gpu_index}.csv")
 
     def __enter__(self):
         try:
@@ -545,8 +548,8 @@ def main():
     tr = tr2[0]
     phases = phase_summary(tr, tr2[1]) if launches == 1 else None
     try:
-        os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-        np.save(os.path.join(ROOT, "gpurun_out", f"trace_{args.act}_rank{rank}.npy"), tr2)
+        os.makedirs(OUT_DIR, exist_ok=True)
+        np.save(os.path.join(OUT_DIR, f"trace_{args.act}_rank{rank}.npy"), tr2)
     except OSError:
         pass
 
