@@ -96,3 +96,24 @@ def test_base3_format_host_checks():
     assert L.tern5_gemv(q, p, 16, 2048, 1, p, None, 1, None, p, None) == 2       # misaligned rows
     assert L.tern5_pack(None, 4, 10, p, None) == 1
     assert L.tern5_unpack(p, 0, 10, p, None) == 1
+
+
+def test_flash_head_host_checks():
+    """Argument checks of the approximate head, before any launch (no GPU needed)."""
+    L = tm.lib()
+    p = ctypes.c_void_p(1 << 40)
+    args = dict(d=2048, nc=4748, cs=32, top=512)
+
+    def call(d=2048, nc=4748, cs=32, top=512, W=p):
+        return L.flash_head(p, p, W, p, d, nc, cs, top, p, p, p, p, p, None)
+
+    assert call(d=100) == 1               # d not a multiple of 64
+    assert call(d=16384) == 1             # d too large for the staged activations
+    assert call(nc=8193) == 1             # too many clusters for the one-CTA selection
+    assert call(top=0) == 1 and call(top=4749) == 1
+    assert call(cs=0) == 1
+    assert call(W=ctypes.c_void_p((1 << 40) + 2)) == 2   # rows not 16-byte aligned
+    assert L.flash_head(None, p, p, p, 2048, 4748, 32, 512, p, p, p, p, p, None) == 1
+    assert L.flash_head_centroids(p, 2048, 0, 32, p, p, None) == 1
+    assert L.flash_head_centroids(p, 2048, 4748, 32, p, ctypes.c_void_p((1 << 40) + 4), None) == 2
+    assert args["nc"] * args["cs"] == 151936
