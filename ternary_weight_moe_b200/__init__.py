@@ -60,7 +60,7 @@ def header_functions():
     """Names of the functions declared in include/ternmoe.h."""
     txt = open(HEADER).read()
     txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
-    return sorted(set(re.findall(r"\b(tern_\w+|moe_\w+)\s*\(", txt)))
+    return sorted(set(re.findall(r"\b(tern_\w+|tern5_\w+|moe_\w+|flash_head\w*)\s*\(", txt)))
 
 
 def lib():

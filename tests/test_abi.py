@@ -117,3 +117,20 @@ def test_flash_head_host_checks():
     assert L.flash_head_centroids(p, 2048, 0, 32, p, p, None) == 1
     assert L.flash_head_centroids(p, 2048, 4748, 32, p, ctypes.c_void_p((1 << 40) + 4), None) == 2
     assert args["nc"] * args["cs"] == 151936
+
+
+def test_binding_signatures_match_the_header():
+    """Every declared function has a binding whose argument count matches its declaration."""
+    import re
+
+    txt = open(tm.HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    L = tm.lib()
+    names = tm.header_functions()
+    assert {"flash_head", "flash_head_centroids", "tern5_gemv", "moe_stack_decode"} <= set(names)
+    for name in names:
+        m = re.search(r"\b" + name + r"\s*\(([^)]*)\)\s*;", txt)
+        assert m, name
+        params = [p for p in m.group(1).split(",") if p.strip() and p.strip() != "void"]
+        assert getattr(L, name).argtypes is not None, name
+        assert len(getattr(L, name).argtypes) == len(params), name
