@@ -25,13 +25,15 @@
  *   - All array pointers are DEVICE pointers owned by the caller; the library never frees
  *     them.  bf16 values travel as uint16_t bit patterns.  Row-major layouts.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Calls
- *     enqueue work and return without waiting, except tern_pack / tern_unpack (they wait
- *     for their own kernel to report invalid codes) and tern_stream_status.
+ *     enqueue work and return without waiting, except tern_pack / tern_unpack and
+ *     tern5_pack / tern5_unpack (they wait for their own kernel to report invalid codes) and
+ *     tern_stream_status.
  *   - Arguments are checked on the host before anything is enqueued; a failed check returns
  *     TERN_EINVAL / TERN_EALIGN / TERN_EWORKSPACE and enqueues nothing.  A CUDA launch
  *     error returns TERN_ECUDA.  No C++ exception crosses the ABI.
  *   - K (the reduction length of a ternary matrix) must be a multiple of 64 so packed rows
- *     are whole 16-byte vectors; K <= 2048, or a multiple of 2048 up to 16384.  Packed
+ *     are whole 16-byte vectors; K <= 2048, or a multiple of 2048 up to 16384 (the base-3
+ *     calls take any K up to 16384: their rows are padded to 16 bytes).  Packed
  *     arrays and activations must be 16-byte aligned, scales 4-byte aligned.
  *   - The library allocates no device memory on these paths: scratch space is the
  *     caller's `workspace`.  A workspace must be zero-filled once before its first use
