@@ -43,3 +43,15 @@ def test_normal_bf16_and_rounding():
     v32 = v.astype(np.float32)
     ref = torch.from_numpy(v32).to(torch.bfloat16).view(torch.int16).numpy().astype(np.uint16)
     assert (synth.f64_to_bf16_bits(v32.astype(np.float64)) == ref).all()
+
+
+def test_device_normal_generator_matches_host_on_cpu():
+    """The torch variant draws the same SplitMix64 stream with the same Box-Muller pairing;
+    evaluated on the CPU it reproduces the host generator bit for bit (the device may differ
+    in the last ulp of its transcendental functions, so GPU tests hand its values on)."""
+    import torch
+
+    t = synth.normal_bf16_torch(77, 5, 4099, 0.02, "cpu", chunk=1000)
+    h = synth.normal_bf16(77, 5, 4099, 0.02)
+    assert (t.numpy().view(np.uint16) == h).all()
+    assert t.dtype == torch.int16
