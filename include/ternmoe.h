@@ -181,8 +181,10 @@ tern_status moe_route_topk(const uint16_t *Wg, const uint16_t *x, int64_t T, int
  * the caller's, exactly as for moe_route_topk.
  *   Limits: 1 <= T <= 64 and T * E <= 16384 (e.g. 64 tokens x 256 experts); larger requests
  *   return TERN_EINVAL before anything is enqueued.
- *   The first call on each device looks up the array's device address (once per device, on
- *   the calling thread's current device); make that first call before any stream capture.
+ *   Each call outside stream capture looks up the array's device address on the calling
+ *   thread's current device (so a context rebuilt by cudaDeviceReset is handled); a call made
+ *   while `stream` is capturing reuses the address of the last non-capturing call on that
+ *   device, so make the first call on each device before any stream capture.
  *   All calls on a device share the one array: calls that overlap on the GPU (different
  *   streams, no ordering between them) race and give undefined results.  The call clears
  *   the part that must start at zero (the arrival counter) itself.

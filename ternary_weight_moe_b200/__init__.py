@@ -293,16 +293,32 @@ def moe_route_workspace_bytes(T: int, E: int) -> int:
     return int(lib().moe_route_workspace_bytes(T, E))
 
 
-def moe_route_topk(Wg, x, k=8, ws=None, logits=None, idx=None, gates=None, stream=None):
-    Wg = _bits16(Wg, "Wg")
-    x = _bits16(x.view(1, -1) if x.dim() == 1 else x, "x")
+def _route_args(Wg, x, k, logits, idx, gates):
+    """Shape checks of the routing calls (before anything touches the device): Wg [E][d],
+    x [T][d] (or [d]), logits [T][E], idx and gates [T][k]; then dtype/device checks."""
+    if Wg.dim() != 2:
+        raise ValueError(f"Wg must be [E, d], got {tuple(Wg.shape)}")
     E, d = Wg.shape
+    x = x.view(1, -1) if x.dim() == 1 else x
+    if x.dim() != 2 or x.shape[1] != d:
+        raise ValueError(f"x must be [T, {d}], got {tuple(x.shape)}")
     T = x.shape[0]
+    for name, t, shp in (("logits", logits, (T, E)), ("idx", idx, (T, k)), ("gates", gates, (T, k))):
+        if t is not None and tuple(t.shape) != shp:
+            raise ValueError(f"{name} must be {list(shp)}, got {tuple(t.shape)}")
+    Wg = _bits16(Wg, "Wg")
+    x = _bits16(x, "x")
     dev = Wg.device
-    idx = torch.empty((T, k), dtype=torch.int32, device=dev) if idx is None else idx
-    gates = torch.empty((T, k), dtype=torch.float32, device=dev) if gates is None else gates
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev) if idx is None else _dev(idx, torch.int32, "idx")
+    gates = torch.empty((T, k), dtype=torch.float32, device=dev) if gates is None else _dev(gates, torch.float32,
+                                                                                              "gates")
     if logits is not None:
         _dev(logits, torch.float64, "logits")
+    return Wg, x, E, d, T, dev, idx, gates
+
+
+def moe_route_topk(Wg, x, k=8, ws=None, logits=None, idx=None, gates=None, stream=None):
+    Wg, x, E, d, T, dev, idx, gates = _route_args(Wg, x, k, logits, idx, gates)
     need = moe_route_workspace_bytes(T, E)
     ws = workspace(need, dev) if ws is None else ws
     _check(lib().moe_route_topk(_ptr(Wg), _ptr(x), T, d, E, k, _ptr(idx), _ptr(gates), _ptr(logits), _ptr(ws),
@@ -313,15 +329,7 @@ def moe_route_topk(Wg, x, k=8, ws=None, logits=None, idx=None, gates=None, strea
 def moe_route_topk_static(Wg, x, k=8, logits=None, idx=None, gates=None, stream=None):
     """Routing without a workspace (scratch is a fixed array inside the library; T <= 64,
     T * E <= 16384).  For callers that cannot allocate device memory."""
-    Wg = _bits16(Wg, "Wg")
-    x = _bits16(x.view(1, -1) if x.dim() == 1 else x, "x")
-    E, d = Wg.shape
-    T = x.shape[0]
-    dev = Wg.device
-    idx = torch.empty((T, k), dtype=torch.int32, device=dev) if idx is None else idx
-    gates = torch.empty((T, k), dtype=torch.float32, device=dev) if gates is None else gates
-    if logits is not None:
-        _dev(logits, torch.float64, "logits")
+    Wg, x, E, d, T, dev, idx, gates = _route_args(Wg, x, k, logits, idx, gates)
     _check(lib().moe_route_topk_static(_ptr(Wg), _ptr(x), T, d, E, k, _ptr(idx), _ptr(gates), _ptr(logits),
                                        _stream(stream)), "moe_route_topk_static")
     return idx, gates

@@ -21,11 +21,6 @@ using namespace tern;
 
 namespace {
 
-constexpr int64_t kMaxT = 64;
-constexpr int32_t kMaxE = 1024;
-constexpr int32_t kMaxKsel = 8;
-constexpr int32_t kMaxLayers = 64;
-
 inline bool aligned(const void *p, uintptr_t a) { return ((uintptr_t)p % a) == 0; }
 inline cudaStream_t S(void *s) { return reinterpret_cast<cudaStream_t>(s); }
 inline int64_t up256(int64_t v) { return (v + 255) & ~int64_t(255); }

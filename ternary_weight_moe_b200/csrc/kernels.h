@@ -9,6 +9,22 @@
 
 namespace tern {
 
+// ---- limits shared by the host checks and the kernels' fixed-size shared arrays
+constexpr int64_t kMaxT = 64;      // tokens per call
+constexpr int32_t kMaxE = 1024;    // experts per layer
+constexpr int32_t kMaxKsel = 8;    // experts selected per token
+constexpr int32_t kMaxLayers = 64; // layers per stack call
+
+// ---- fixed scratch of the allocation-free routing call (moe_route_topk_static)
+constexpr int64_t kStaticRouteMaxT = 64;      // tokens
+constexpr int64_t kStaticRouteMaxTE = 16384;  // tokens x experts, e.g. 64 x 256
+constexpr size_t kStaticCtrlBytes = 256;
+constexpr size_t kStaticLogitsBytes = (size_t)kStaticRouteMaxTE * 8;             // fp64 logits
+constexpr size_t kStaticGatesBytes = (size_t)kStaticRouteMaxT * kMaxKsel * 8;    // fp64 gates
+constexpr size_t kStaticRouteBytes = kStaticCtrlBytes + kStaticLogitsBytes + kStaticGatesBytes;  // 135,424 B
+static_assert(kStaticRouteMaxT <= kMaxT, "the static route serves at most the tokens the kernels handle");
+static_assert(kStaticRouteBytes == 135424, "documented size of the fixed routing scratch");
+
 // ---- format
 cudaError_t launch_pack(const int8_t *w, int64_t M, int64_t K, uint8_t *packed, unsigned long long *bad,
                         cudaStream_t s);

@@ -33,7 +33,6 @@ static cudaError_t launch_k(void (*kern)(K...), dim3 grid, dim3 block, size_t sm
     return cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
 }
 
-constexpr int kMaxE = 1024;
 
 // ------------------------------------------------------------------------- route kernels
 // logits_kernel: one warp per expert row, 16 experts x 8 tokens per CTA.  The tokens' x is
@@ -131,7 +130,7 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(
     __shared__ __align__(16) uint32_t s_gm[32];
     __shared__ int s_nc;
     __shared__ ulonglong2 s_cand[256];
-    __shared__ int32_t s_all[64 * 8];  // every (token, slot) expert index, T <= 64, k <= 8
+    __shared__ int32_t s_all[kMaxT * kMaxKsel];  // every (token, slot) expert index
     const int t = blockIdx.x;
     const double *lg = logits + (int64_t)t * E;
     double mine = 0.0;

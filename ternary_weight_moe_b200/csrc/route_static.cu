@@ -18,30 +18,39 @@
 
 namespace {
 
-constexpr int64_t kStaticRouteMaxT = 64;
-constexpr int64_t kStaticRouteMaxTE = 16384;  // tokens x experts, e.g. 64 x 256
-constexpr size_t kStaticCtrlBytes = 256;
-constexpr size_t kStaticLogitsBytes = (size_t)kStaticRouteMaxTE * 8;
-constexpr size_t kStaticGatesBytes = (size_t)kStaticRouteMaxT * 8 * 8;
-constexpr size_t kStaticRouteBytes = kStaticCtrlBytes + kStaticLogitsBytes + kStaticGatesBytes;  // 135,424 B
+using tern::kMaxE;
+using tern::kMaxKsel;
+using tern::kStaticCtrlBytes;
+using tern::kStaticLogitsBytes;
+using tern::kStaticRouteBytes;
+using tern::kStaticRouteMaxT;
+using tern::kStaticRouteMaxTE;
 
 // The scratch itself.  In host code this name is only a stand-in for the symbol, never a
-// device address: the address is looked up once per device with cudaGetSymbolAddress.
+// device address: the address comes from cudaGetSymbolAddress on the device that runs.
 static __device__ __align__(256) unsigned char g_route_scratch[kStaticRouteBytes];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mu;
 unsigned char *g_scratch_ptr[kMaxDevices] = {nullptr};
 
-// Device address of the scratch on the current device (looked up on first use).
-tern_status scratch_on_current_device(unsigned char **out) {
+// Device address of the scratch on the current device.  Outside stream capture it is looked
+// up again on every call, so a context torn down and rebuilt (cudaDeviceReset) cannot leave a
+// stale address behind; while `stream` is capturing, the address cached by the last
+// non-capturing call on this device is used (a lookup may not be legal then), so the first
+// call on a device must come before any capture.
+tern_status scratch_on_current_device(cudaStream_t stream, unsigned char **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TERN_ECUDA;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return TERN_ECUDA;
     std::lock_guard<std::mutex> lock(g_setup_mu);
-    if (g_scratch_ptr[dev] == nullptr) {
+    if (cap == cudaStreamCaptureStatusNone) {
         unsigned char *p = nullptr;
         if (cudaGetSymbolAddress((void **)&p, g_route_scratch) != cudaSuccess || p == nullptr) return TERN_ECUDA;
         g_scratch_ptr[dev] = p;
+    } else if (g_scratch_ptr[dev] == nullptr) {
+        return TERN_ECUDA;  // never set up on this device outside a capture
     }
     *out = g_scratch_ptr[dev];
     return TERN_OK;
@@ -54,17 +63,17 @@ inline bool aligned(const void *p, uintptr_t a) { return ((uintptr_t)p % a) == 0
 extern "C" tern_status moe_route_topk_static(const uint16_t *Wg, const uint16_t *x, int64_t T, int64_t d, int32_t E,
                                              int32_t k, int32_t *topk_idx, float *topk_gate, double *logits,
                                              void *stream) {
-    if (!Wg || !x || !topk_idx || !topk_gate || T < 1 || d < 8 || d % 8 || E < 1 || E > 1024 || k < 1 || k > 8 ||
-        k > E)
+    if (!Wg || !x || !topk_idx || !topk_gate || T < 1 || d < 8 || d % 8 || E < 1 || E > kMaxE || k < 1 ||
+        k > kMaxKsel || k > E)
         return TERN_EINVAL;
     if (T > kStaticRouteMaxT || T * (int64_t)E > kStaticRouteMaxTE) return TERN_EINVAL;  // beyond the fixed scratch
     if (!aligned(Wg, 16) || !aligned(x, 16) || !aligned(topk_idx, 4) || !aligned(topk_gate, 4) ||
         (logits && !aligned(logits, 8)))
         return TERN_EALIGN;
-    unsigned char *base = nullptr;
-    const tern_status st = scratch_on_current_device(&base);
-    if (st != TERN_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    unsigned char *base = nullptr;
+    const tern_status st = scratch_on_current_device(s, &base);
+    if (st != TERN_OK) return st;
     unsigned int *ctrl = reinterpret_cast<unsigned int *>(base);
     double *lg = logits ? logits : reinterpret_cast<double *>(base + kStaticCtrlBytes);
     double *g64 = reinterpret_cast<double *>(base + kStaticCtrlBytes + kStaticLogitsBytes);

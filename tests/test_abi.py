@@ -134,3 +134,36 @@ def test_binding_signatures_match_the_header():
         params = [p for p in m.group(1).split(",") if p.strip() and p.strip() != "void"]
         assert getattr(L, name).argtypes is not None, name
         assert len(getattr(L, name).argtypes) == len(params), name
+
+
+def test_static_route_limits_before_any_launch():
+    """The allocation-free routing call refuses, on the host, every request its fixed
+    scratch cannot hold or that is malformed: more than 64 tokens even with few experts,
+    more than 16,384 token-expert logits, k > E, d not a multiple of 8."""
+    L = tm.lib()
+    p = ctypes.c_void_p(1 << 40)
+    assert L.moe_route_topk_static(p, p, 65, 64, 8, 8, p, p, None, None) == 1      # T > 64, small E
+    assert L.moe_route_topk_static(p, p, 64, 64, 512, 8, p, p, None, None) == 1     # T*E = 32768
+    assert L.moe_route_topk_static(p, p, 4, 64, 4, 8, p, p, None, None) == 1        # k > E
+    assert L.moe_route_topk_static(p, p, 4, 60, 256, 8, p, p, None, None) == 1      # d % 8 != 0
+    assert L.moe_route_topk_static(p, p, 4, 64, 256, 9, p, p, None, None) == 1      # k > 8
+    q = ctypes.c_void_p((1 << 40) + 4)
+    assert L.moe_route_topk_static(q, p, 4, 64, 256, 8, p, p, None, None) == 2      # misaligned router
+
+
+def test_route_binding_rejects_wrong_shapes():
+    """The Python routing calls check x, logits, idx and gates against Wg's shape before
+    they touch the device (so a short buffer is a ValueError, not an out-of-bounds write)."""
+    import torch
+
+    Wg = torch.zeros((256, 2048), dtype=torch.int16)
+    for fn in (tm.moe_route_topk, tm.moe_route_topk_static):
+        with pytest.raises(ValueError):
+            fn(Wg, torch.zeros((2, 1024), dtype=torch.int16))                     # x width != d
+        x = torch.zeros((2, 2048), dtype=torch.int16)
+        with pytest.raises(ValueError):
+            fn(Wg, x, 8, logits=torch.zeros((2, 128), dtype=torch.float64))        # logits [T][E]
+        with pytest.raises(ValueError):
+            fn(Wg, x, 8, idx=torch.zeros((2, 4), dtype=torch.int32))               # idx [T][k]
+        with pytest.raises(ValueError):
+            fn(Wg, x, 8, gates=torch.zeros((1, 8), dtype=torch.float32))           # gates [T][k]
