@@ -160,30 +160,60 @@ def build_stack(dev):
     return shape, layers, tm.Stack(layers)
 
 
-def cpu_baseline(act_oracle, budget_s=12.0, max_tokens=4):
-    """The oracle (single-threaded C, fp64/exact) decoding whole tokens through the same
-    24-layer stack; experts are regenerated on the host outside the timed region."""
+def cpu_model():
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def host_cores():
+    return len(os.sched_getaffinity(0))
+
+
+def _oracle_tokens(act_oracle, omp, n_tokens, seed0, hosts=None):
+    """Decode n_tokens whole tokens through the 24-layer stack with the CPU oracle; returns
+    (seconds inside the oracle, tokens).  Experts are regenerated on the host (from the same
+    seeds as the device stack) outside the timed region."""
     import oracle
     import synth
     from tests.gpu_cases import HostLayer
 
     shape = synth.MoEShape()
-    hosts = [HostLayer(WID, l, shape) for l in range(N_LAYERS)]
-    spent, tokens = 0.0, 0
-    while tokens < max_tokens and (spent < budget_s or tokens == 0):
-        x = synth.tokens_bf16(WID, 50000 + tokens, 1, shape.d)
+    hosts = hosts if hosts is not None else [HostLayer(WID, l, shape) for l in range(N_LAYERS)]
+    spent = 0.0
+    for t in range(n_tokens):
+        x = synth.tokens_bf16(WID, seed0 + t, 1, shape.d)
         for l in range(N_LAYERS):
             n, _ = oracle.rmsnorm(x, 1e-6)
             _, idx, _, _ = hosts[l].route(n)
             hosts[l].fill(idx)
             L = hosts[l].oracle_layer()
             t0 = time.perf_counter()
-            x = oracle.stack_layer(L, x, eps=1e-6, act=act_oracle)["x_out"]
+            x = oracle.stack_layer(L, x, eps=1e-6, act=act_oracle, omp=omp)["x_out"]
             spent += time.perf_counter() - t0
-        tokens += 1
-    return {"value": tokens / spent, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{tokens} tokens x {N_LAYERS} layers through the CPU oracle (C, fp64/exact, one thread); "
-                      "host expert regeneration excluded"}
+    return spent, n_tokens
+
+
+def cpu_baseline(act_oracle, n_tokens=4):
+    """The oracle (C, fp64/exact) decoding whole tokens through the same 24-layer stack, on
+    all host cores (the OpenMP build: rows split across threads, identical results) and on
+    one core (the single-threaded build)."""
+    import oracle
+
+    oracle.build(omp=True)
+    spent_all, tok = _oracle_tokens(act_oracle, True, n_tokens, 50000)
+    spent_one, tok1 = _oracle_tokens(act_oracle, False, n_tokens, 50000)
+    cores = host_cores()
+    return {"value": tok / spent_all, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "cpu_model": cpu_model(),
+            "single_thread": {"value": tok1 / spent_one, "unit": UNIT, "cores": 1},
+            "sample": f"{tok} whole tokens x {N_LAYERS} layers through the CPU oracle (C, fp64/exact): the OpenMP "
+                      f"build on all {cores} cores (value) and the single-threaded build (single_thread); host "
+                      "expert regeneration excluded"}
 
 
 PHASES = [("x_wait", 0, 1), ("norm_limbs", 1, 2), ("router", 2, 3), ("logits_wait", 3, 4), ("topk", 4, 5),
@@ -230,7 +260,8 @@ def kernel_traffic(act):
 
 
 def run_reference(args):
-    """--impl reference: the CPU oracle as the reference arm (rank 0 only)."""
+    """--impl reference: the CPU oracle as the reference arm (rank 0 only).  One step = one
+    whole token through the 24 layers, on all host cores (the oracle's OpenMP build)."""
     world, rank, _ = dist_env()
     if rank != 0:
         return 0
@@ -239,42 +270,24 @@ def run_reference(args):
     from tests.gpu_cases import HostLayer
 
     act = oracle.ACT_INT8 if args.act == "int8" else oracle.ACT_BF16
+    oracle.build(omp=True)
     shape = synth.MoEShape()
     hosts = [HostLayer(WID, l, shape) for l in range(N_LAYERS)]
-    # one step = one layer of one token (1/24 of a token); tokens cycle over a small set so
-    # the host copies of the experts stay bounded
-    ntok = 2
-    chain = {}
-
-    def step(i):
-        t = (i // N_LAYERS) % ntok
-        l = i % N_LAYERS
-        x = chain.get((t, l))
-        if x is None:
-            x = synth.tokens_bf16(WID, 60000 + t, 1, shape.d) if l == 0 else chain[(t, l - 1, "out")]
-            chain[(t, l)] = x
-        n, _ = oracle.rmsnorm(x, 1e-6)
-        _, idx, _, _ = hosts[l].route(n)
-        hosts[l].fill(idx)
-        L = hosts[l].oracle_layer()
-        t0 = time.perf_counter()
-        out = oracle.stack_layer(L, x, eps=1e-6, act=act)["x_out"]
-        dt = time.perf_counter() - t0
-        chain[(t, l, "out")] = out
-        return dt
-
+    # tokens cycle over a small set so the host copies of the experts stay bounded
+    ntok = 4
     for i in range(args.warmup):
-        step(i)
-    spent = sum(step(args.warmup + i) for i in range(args.steps))
-    tokens = args.steps / N_LAYERS
-    value = tokens / spent
+        _oracle_tokens(act, True, 1, 60000 + i % ntok, hosts)
+    spent = sum(_oracle_tokens(act, True, 1, 60000 + (args.warmup + i) % ntok, hosts)[0] for i in range(args.steps))
+    value = args.steps / spent
+    cores = host_cores()
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": spent / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": _config(args.act, world, "n/a (CPU)"), "impl": "reference",
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                             "sample": f"{args.steps} layer-token steps (one layer of one token each) through "
-                                       "the CPU oracle (C, fp64/exact, one thread)"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "cpu_model": cpu_model(),
+                             "sample": f"{args.steps} whole tokens (24 layers each) through the CPU oracle "
+                                       f"(C, fp64/exact, OpenMP build on all {cores} cores)"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0

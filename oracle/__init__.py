@@ -21,22 +21,26 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "ternmoe_oracle.c")
 _LIB = os.path.join(_HERE, "libternmoe_oracle.so")
+_LIB_OMP = os.path.join(_HERE, "libternmoe_oracle_omp.so")
 _lock = threading.Lock()
 _lib = None
+_lib_omp = None
 
 ACT_BF16 = 0
 ACT_INT8 = 1
 
 
-def build(force: bool = False) -> str:
-    """Compile the oracle with gcc (no fast-math, no FMA contraction)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        tmp = _LIB + ".tmp%d" % os.getpid()
+def build(force: bool = False, omp: bool = False) -> str:
+    """Compile the oracle with gcc (no fast-math, no FMA contraction).  omp=True builds the
+    same source with -fopenmp (rows split across cores, identical results; timing only)."""
+    out = _LIB_OMP if omp else _LIB
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(_SRC):
+        tmp = out + ".tmp%d" % os.getpid()
         subprocess.check_call([
             "gcc", "-O2", "-std=gnu11", "-fPIC", "-shared", "-ffp-contract=off",
-            "-fno-fast-math", "-o", tmp, _SRC, "-lm"])
-        os.replace(tmp, _LIB)
-    return _LIB
+            "-fno-fast-math", *(["-fopenmp"] if omp else []), "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, out)
+    return out
 
 
 class _Layer(ctypes.Structure):
@@ -54,45 +58,58 @@ class _Trace(ctypes.Structure):
 
 
 def lib():
+    """The single-threaded oracle (the one every test uses)."""
     global _lib
     with _lock:
         if _lib is None:
             # a test may point the wrapper at a deliberately broken copy of the oracle
-            path = os.environ.get("TERNMOE_ORACLE_LIB") or build()
-            L = ctypes.CDLL(path)
-            i64, i32, vp, dbl = ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p, ctypes.c_double
-            L.or_pack.restype = i64
-            L.or_pack.argtypes = [vp, i64, i64, vp]
-            L.or_unpack.restype = i64
-            L.or_unpack.argtypes = [vp, i64, i64, vp]
-            L.or_tern5_row_bytes.restype = i64
-            L.or_tern5_row_bytes.argtypes = [i64]
-            L.or_pack5.restype = i64
-            L.or_pack5.argtypes = [vp, i64, i64, vp]
-            L.or_unpack5.restype = i64
-            L.or_unpack5.argtypes = [vp, i64, i64, vp]
-            L.or_gemv_i8.restype = ctypes.c_int
-            L.or_gemv_i8.argtypes = [vp, vp, i64, i64, i64, vp, vp, vp, vp]
-            L.or_gemv_bf16.restype = i64
-            L.or_gemv_bf16.argtypes = [vp, vp, i64, i64, i64, vp, vp]
-            L.or_quant_absmax.restype = None
-            L.or_quant_absmax.argtypes = [vp, i64, vp, vp]
-            L.or_rmsnorm.restype = i64
-            L.or_rmsnorm.argtypes = [vp, i64, dbl, vp]
-            L.or_route.restype = i64
-            L.or_route.argtypes = [vp, vp, i64, i64, i32, i32, vp, vp, vp]
-            L.or_moe_ffn.restype = i64
-            L.or_moe_ffn.argtypes = [ctypes.POINTER(_Layer), vp, i64, ctypes.c_int, vp, vp,
-                                     ctypes.POINTER(_Trace), vp, vp, vp]
-            L.or_stack_layer.restype = i64
-            L.or_stack_layer.argtypes = [ctypes.POINTER(_Layer), vp, i64, dbl, ctypes.c_int, vp,
-                                         vp, vp, vp, ctypes.POINTER(_Trace)]
-            L.or_f64_to_bf16.restype = ctypes.c_uint16
-            L.or_f64_to_bf16.argtypes = [dbl]
-            L.or_bf16_to_f64.restype = dbl
-            L.or_bf16_to_f64.argtypes = [ctypes.c_uint16]
-            _lib = L
+            _lib = _load(os.environ.get("TERNMOE_ORACLE_LIB") or build())
     return _lib
+
+
+def lib_omp():
+    """The same oracle built with OpenMP (for the benchmark's all-cores CPU timing)."""
+    global _lib_omp
+    with _lock:
+        if _lib_omp is None:
+            _lib_omp = _load(build(omp=True))
+    return _lib_omp
+
+
+def _load(path):
+    L = ctypes.CDLL(path)
+    i64, i32, vp, dbl = ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p, ctypes.c_double
+    L.or_pack.restype = i64
+    L.or_pack.argtypes = [vp, i64, i64, vp]
+    L.or_unpack.restype = i64
+    L.or_unpack.argtypes = [vp, i64, i64, vp]
+    L.or_tern5_row_bytes.restype = i64
+    L.or_tern5_row_bytes.argtypes = [i64]
+    L.or_pack5.restype = i64
+    L.or_pack5.argtypes = [vp, i64, i64, vp]
+    L.or_unpack5.restype = i64
+    L.or_unpack5.argtypes = [vp, i64, i64, vp]
+    L.or_gemv_i8.restype = ctypes.c_int
+    L.or_gemv_i8.argtypes = [vp, vp, i64, i64, i64, vp, vp, vp, vp]
+    L.or_gemv_bf16.restype = i64
+    L.or_gemv_bf16.argtypes = [vp, vp, i64, i64, i64, vp, vp]
+    L.or_quant_absmax.restype = None
+    L.or_quant_absmax.argtypes = [vp, i64, vp, vp]
+    L.or_rmsnorm.restype = i64
+    L.or_rmsnorm.argtypes = [vp, i64, dbl, vp]
+    L.or_route.restype = i64
+    L.or_route.argtypes = [vp, vp, i64, i64, i32, i32, vp, vp, vp]
+    L.or_moe_ffn.restype = i64
+    L.or_moe_ffn.argtypes = [ctypes.POINTER(_Layer), vp, i64, ctypes.c_int, vp, vp,
+                             ctypes.POINTER(_Trace), vp, vp, vp]
+    L.or_stack_layer.restype = i64
+    L.or_stack_layer.argtypes = [ctypes.POINTER(_Layer), vp, i64, dbl, ctypes.c_int, vp,
+                                 vp, vp, vp, ctypes.POINTER(_Trace)]
+    L.or_f64_to_bf16.restype = ctypes.c_uint16
+    L.or_f64_to_bf16.argtypes = [dbl]
+    L.or_bf16_to_f64.restype = dbl
+    L.or_bf16_to_f64.argtypes = [ctypes.c_uint16]
+    return L
 
 
 def _p(a):
@@ -266,8 +283,9 @@ def moe_ffn(layer: Layer, x, act=ACT_BF16, qh_in=None, sh_in=None, h_in=None):
     return out
 
 
-def stack_layer(layer: Layer, x, eps=1e-6, act=ACT_BF16):
-    """One residual layer: returns x_out, n, y (bf16 bits), y64 and the FFN trace."""
+def stack_layer(layer: Layer, x, eps=1e-6, act=ACT_BF16, omp=False):
+    """One residual layer: returns x_out, n, y (bf16 bits), y64 and the FFN trace.
+    omp=True runs the OpenMP build (same results, rows split across cores)."""
     x = _c(np.atleast_2d(x), np.uint16)
     T = x.shape[0]
     d, f, E, k = layer.d, layer.f, layer.E, layer.k
@@ -281,7 +299,7 @@ def stack_layer(layer: Layer, x, eps=1e-6, act=ACT_BF16):
                   ("idx", "gates", "logits", "h", "acc_g", "acc_u", "qx", "sx", "qh", "sh",
                    "acc_d", "ye")])
     L = layer._struct()
-    bad = lib().or_stack_layer(ctypes.byref(L), _p(x), T, float(eps), act, _p(x_out), _p(n),
+    bad = (lib_omp() if omp else lib()).or_stack_layer(ctypes.byref(L), _p(x), T, float(eps), act, _p(x_out), _p(n),
                                _p(y), _p(y64), ctypes.byref(tr))
     return {"x_out": x_out, "n": n, "y": y, "y64": y64, "inexact": int(bad), **tr_arrays}
 

@@ -5,7 +5,11 @@
  * TEST INFRASTRUCTURE ONLY.  Only the test suite, the package's smoke check and the
  * CPU-baseline leg of the benchmark may load this code.  It shares no code, header,
  * table or constant with the CUDA library; it is compiled by gcc with
- * -O2 -ffp-contract=off (no fused multiply-adds, no fast-math), single-threaded.
+ * -O2 -ffp-contract=off (no fused multiply-adds, no fast-math), single-threaded.  The
+ * benchmark also times a second build of this same file with -fopenmp: the `omp` pragmas
+ * below then split independent rows (router rows, gate/up rows, down rows) across the
+ * host's cores.  Every value is still computed by one thread in the same order, so both
+ * builds return identical results; the pragmas change the timing only.
  *
  * What it computes (sources are the five web pages on the Maple-Preview model):
  *  - ternary weights w in {-1,0,+1}, four 2-bit codes per byte ("How a 20B Model
@@ -355,6 +359,7 @@ int64_t or_route(const uint16_t *Wg, const uint16_t *x, int64_t T, int64_t d, in
     double *l = (double *)malloc(sizeof(double) * (size_t)E);
     char *taken = (char *)malloc((size_t)E);
     for (int64_t t = 0; t < T; t++) {
+#pragma omp parallel for reduction(+ : bad) schedule(static)
         for (int32_t e = 0; e < E; e++) {
             double plain = 0.0;
             xsum ex;
@@ -476,6 +481,7 @@ int64_t or_moe_ffn(const or_layer *L, const uint16_t *x, int64_t T, int act, uin
             const int32_t e = idx[t * k + i];
             const int64_t slot = t * k + i;
             /* gate / up rows, SwiGLU */
+#pragma omp parallel for reduction(+ : bad, unchecked) schedule(static)
             for (int64_t j = 0; j < f; j++) {
                 const uint8_t *grow = L->gate + ((int64_t)e * f + j) * (d / 4);
                 const uint8_t *urow = L->up + ((int64_t)e * f + j) * (d / 4);
@@ -515,6 +521,7 @@ int64_t or_moe_ffn(const or_layer *L, const uint16_t *x, int64_t T, int act, uin
                 const float *hs = h_in ? h_in + slot * f : h;
                 for (int64_t j = 0; j < f; j++) hd[j] = (double)hs[j];
             }
+#pragma omp parallel for reduction(+ : bad, unchecked) schedule(static)
             for (int64_t c = 0; c < d; c++) {
                 const uint8_t *drow = L->down + ((int64_t)e * d + c) * (f / 4);
                 float sd = L->down_scale[(int64_t)e * d + c];

@@ -493,3 +493,22 @@ def test_gemv5_equals_two_bit_gemv():
     a2, y2 = oracle.gemv_i8(oracle.pack(w)[0], s, q)
     assert (a5 == a2).all() and (y5 == y2).all()
     assert (a2 == q.astype(np.int64) @ w.T.astype(np.int64)).all()
+
+
+def test_openmp_build_returns_identical_results():
+    """The all-cores build (same source, -fopenmp) only splits independent rows across
+    threads: a full-size layer gives the same bits as the single-threaded build."""
+    from gpu_cases import HostLayer
+
+    shape = synth.MoEShape()
+    H = HostLayer(5, 0, shape)
+    x = synth.tokens_bf16(5, 77, 1, shape.d)
+    n, _ = oracle.rmsnorm(x, 1e-6)
+    _, idx, _, _ = H.route(n)
+    H.fill(idx)
+    for act in (oracle.ACT_BF16, oracle.ACT_INT8):
+        a = oracle.stack_layer(H.oracle_layer(), x, act=act)
+        b = oracle.stack_layer(H.oracle_layer(), x, act=act, omp=True)
+        assert (a["x_out"] == b["x_out"]).all() and (a["y64"] == b["y64"]).all()
+        assert (a["idx"] == b["idx"]).all() and (a["gates"] == b["gates"]).all()
+        assert a["inexact"] == b["inexact"] == 0
