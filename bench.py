@@ -216,10 +216,10 @@ def cpu_baseline(act_oracle, n_tokens=4):
                       "expert regeneration excluded"}
 
 
-PHASES = [("x_wait", 0, 1), ("norm_limbs", 1, 2), ("router", 2, 3), ("logits_wait", 3, 4), ("topk", 4, 5),
-          ("issue", 5, 6), ("gate_up_rows_wait", 6, 7), ("gate_up_dots", 7, 8), ("swiglu", 8, 9),
-          ("h_wait", 9, 10), ("h_limbs", 10, 11), ("down_rows_wait", 11, 12), ("down_dots", 12, 13),
-          ("combine", 13, 14)]
+PHASES = [("x_wait", 0, 1), ("norm_router", 1, 2), ("predict_next", 2, 3), ("logits_wait", 3, 4),
+          ("topk_issue", 4, 5), ("gate_up_rows_wait", 5, 6), ("gate_up_dots", 6, 7), ("swiglu", 7, 8),
+          ("h_wait", 8, 9), ("h_limbs", 9, 10), ("down_rows_wait", 10, 11), ("down_dots", 11, 12),
+          ("y_wait", 12, 13), ("combine", 13, 14)]
 
 
 def phase_summary(tr, clk=None, mhz=1965.0):
@@ -231,10 +231,12 @@ def phase_summary(tr, clk=None, mhz=1965.0):
         d = lambda a, b: np.median((tr[:, :, b] - tr[:, :, a]).astype(np.float64)) / 1e3
     out = {name: round(float(d(a, b)), 3) for name, a, b in PHASES}
     # exchange latency: last producer's publish -> first consumer's receipt
-    e_log = np.median(tr[:, :, 4].min(1) - tr[:, :, 3].max(1)) / 1e3
-    e_h = np.median(tr[:, :, 10].min(1) - tr[:, :, 9].max(1)) / 1e3
+    e_log = np.median(tr[:, :, 4].min(1) - tr[:, :, 2].max(1)) / 1e3
+    e_h = np.median(tr[:, :, 9].min(1) - tr[:, :, 8].max(1)) / 1e3
+    e_y = np.median(tr[:, :, 13].min(1) - tr[:, :, 12].max(1)) / 1e3
     e_x = np.median(tr[1:, :, 1].min(1) - tr[:-1, :, 14].max(1)) / 1e3
-    out["exchange_latency"] = {"logits": round(float(e_log), 3), "h": round(float(e_h), 3), "x": round(float(e_x), 3)}
+    out["exchange_latency"] = {"logits": round(float(e_log), 3), "h": round(float(e_h), 3),
+                               "y": round(float(e_y), 3), "x": round(float(e_x), 3)}
     out["layer_total"] = round(float(np.median(np.diff(tr[:, :, 0].min(1)))) / 1e3, 3)
     return out
 
@@ -242,7 +244,7 @@ def phase_summary(tr, clk=None, mhz=1965.0):
 def kernel_source_hash():
     import hashlib
 
-    parts = ["stack.cu", "tern_common.cuh", "tma.cuh", "kernels.h"]
+    parts = ["stack.cu", "tern_common.cuh", "tma.cuh", "kernels.h", "decode.cuh", "cluster.cuh"]
     src = "".join(open(os.path.join(ROOT, "ternary_weight_moe_b200", "csrc", p)).read() for p in parts)
     return hashlib.sha256(src.encode()).hexdigest()[:16]
 
@@ -551,7 +553,7 @@ def main():
     step_ms = [a.elapsed_time(b) for a, b in ev]
     dev_ms = sum(step_ms)
     # one extra, traced step (outside the timed region): every CTA stamps every phase
-    P = torch.cuda.get_device_properties(dev).multi_processor_count
+    P = max(tm.moe_stack_persistent_ctas(layers[0], N_LAYERS, act), 1)
     os.environ["TERNMOE_TRACE"] = "1"
     flush.fill_(1)
     tm.moe_stack_decode(stack, xs[W:W + 1].clone(), act=act, ws=ws)

@@ -50,7 +50,7 @@
 extern "C" {
 #endif
 
-#define TERNMOE_ABI_VERSION 1
+#define TERNMOE_ABI_VERSION 2
 
 typedef enum {
     TERN_OK = 0,
@@ -197,7 +197,9 @@ tern_status moe_route_topk_static(const uint16_t *Wg, const uint16_t *x, int64_t
  *   route (as moe_route_topk) -> group the (token, slot) pairs by expert so every selected
  *   expert's packed weights stream from memory once per call -> for each pair
  *   h = silu(s_g * (G x)) * (s_u * (U x)) -> y_e = s_d * (D h) -> y[t] = sum over the k
- *   slots in top-k order of gate * y_e, in fp64, written as bf16 (nearest even) and, if
+ *   slots in top-k order of gate * fp32(y_e) (each expert output rounded once to fp32, the
+ *   precision in which the persistent kernel passes it between SMs), accumulated in fp64,
+ *   written as bf16 (nearest even) and, if
  *   y_f32 != NULL, as fp32.
  *   act = TERN_ACT_BF16: x and h enter the dots on a 24-bit fixed-point grid (see tern_gemv).
  *   act = TERN_ACT_INT8: x is absmax-quantised per token and h per (token, slot); the dots
@@ -215,10 +217,11 @@ tern_status moe_ffn_decode(const tern_moe_layer *L, const uint16_t *x, int64_t T
  *   n = bf16(x / sqrt(mean(x^2) + rms_eps))   (fp64, no learned gain)
  *   x = bf16(x + moe_ffn_decode(n))            (exact sum, one rounding)
  * All layers must share d, f, E, k.  1 <= n_layers <= 64.  For T == 1 the whole stack runs
- * as ONE persistent kernel (one CTA per SM, in-kernel grid barriers with bounded waits);
+ * as ONE persistent kernel (one CTA per SM, cooperative launch; the CTAs exchange data
+ * through tagged words in the workspace and every in-kernel wait is bounded);
  * otherwise layer by layer.  A timed-out in-kernel wait sets the device status word to
- * TERN_ETIMEOUT (read it with tern_stream_status) and the workspace must be zero-filled
- * again before reuse. */
+ * TERN_ETIMEOUT (read it with tern_stream_status); x is then unspecified, and the workspace
+ * can be used again as it is. */
 size_t moe_stack_workspace_bytes(const tern_moe_layer *L0, int64_t T_max, tern_act act);
 tern_status moe_stack_decode(const tern_moe_layer *layers, int32_t n_layers, uint16_t *x, int64_t T,
                              float rms_eps, tern_act act, void *workspace, size_t ws_bytes,
@@ -256,18 +259,30 @@ tern_status flash_head(const uint8_t *C4, const double *c_scale, const uint16_t 
  *   hist    uint16 [n_layers+1][d]  bf16 x entering each layer, and the final x;
  *   idx     int32  [n_layers][k]    experts chosen at each layer (descending logit);
  *   gates64 double [n_layers][k]    their renormalised gates;
+ *   y32     float  [n_layers][d]    each layer's FFN output y before its bf16 cast (the value
+ *                                   the residual adds), for parity checks of every layer;
+ *   h32     float  [n_layers][k][f] each layer's SwiGLU output h of every slot (the down
+ *                                   projection's input, before its limbs or int8 codes);
  *   trace   uint64 [2][n_layers][P][16]: %globaltimer (ns), then clock64 (SM cycles), stamped
- *           by each of the P CTAs (one per SM, P <= 256) at phase boundaries, written only when
- *           the environment variable TERNMOE_TRACE is "1" at the time of the call: 0 layer start, 1 x received, 2 n and limbs
- *           ready, 3 own logits published, 4 all logits received, 5 top-k done, 6 copies
- *           issued, 7 gate/up rows landed, 8 gate/up dots done, 9 h published, 10 all h
- *           received, 11 h limbs built, 12 down rows landed, 13 down dots done,
- *           14 x' published. */
+ *           by each of the P CTAs (one per SM, P = moe_stack_persistent_ctas(), P <= 256) at
+ *           phase boundaries, written only when
+ *           the environment variable TERNMOE_TRACE is "1" at the time of the call: 0 layer
+ *           start, 1 x received, 2 router logits published, 3 predicted next-layer logits
+ *           published, 4 all logits received, 5 top-k done and row copies issued, 6 first
+ *           gate/up rows landed, 7 gate/up dots done, 8 h published, 9 slot's h received,
+ *           10 h limbs built, 11 down rows landed, 12 down dots done and published, 13 the
+ *           slots' outputs of this CTA's rows received, 14 x' published.
+ * The persistent kernel prefetches the experts it predicts for the next layer into L2 (a hint
+ * that changes no value); TERNMOE_PREDICT=0 in the environment turns that off. */
 typedef struct {
-    int64_t hist, idx, gates64, trace, total;
+    int64_t hist, idx, gates64, y32, h32, trace, total;
 } tern_stack_layout;
 tern_status moe_stack_workspace_layout(const tern_moe_layer *L0, int64_t T_max, tern_act act,
                                        tern_stack_layout *out);
+
+/* CTAs of the persistent T == 1 kernel for these layers on the current device (k groups of
+ * G CTAs, at most one per SM), or 0 when a T == 1 call would run layer by layer instead. */
+int32_t moe_stack_persistent_ctas(const tern_moe_layer *L0, int32_t n_layers, tern_act act);
 
 /* Number of kernel launches one moe_stack_decode call with these arguments makes on the
  * current device (1 on the persistent T == 1 path), or -1 if the arguments are invalid. */
@@ -277,6 +292,18 @@ int32_t moe_stack_kernel_launches(const tern_moe_layer *L0, int32_t n_layers, in
  * (TERN_OK, or TERN_ETIMEOUT if an in-kernel bounded wait gave up since the last read), or
  * TERN_ECUDA if the wait itself failed. */
 tern_status tern_stream_status(void *stream);
+
+/* Test hook for the persistent stack kernel's own bounded waits: the same launch as
+ * moe_stack_decode at T = 1, except that at layer `stall_layer` CTA 0 waits for a slot's h
+ * with a tag no CTA ever writes, and every in-kernel wait gives up after limit_ns (1 us ..
+ * 1 s) instead of one second.  CTA 0 gives up first; the others then miss its outputs and give
+ * up too; each lets its own bulk copies land before it leaves.  The kernel returns by itself:
+ * tern_stream_status then reports TERN_ETIMEOUT, and the next moe_stack_decode call on the
+ * same workspace runs normally (its tags carry a new launch epoch).  x is left unspecified.
+ * Returns TERN_EUNSUPPORTED when the arguments would not take the persistent path. */
+tern_status tern_test_stack_stall(const tern_moe_layer *layers, int32_t n_layers, uint16_t *x, float rms_eps,
+                                  tern_act act, int32_t stall_layer, int64_t limit_ns, void *workspace,
+                                  size_t ws_bytes, void *stream);
 
 /* Test hook for the bounded waits: launches one block that waits on a flag nobody sets,
  * for at most `spin_limit` polls, then sets TERN_ETIMEOUT in the device status word and

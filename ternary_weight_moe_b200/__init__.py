@@ -50,7 +50,7 @@ class FfnLayoutC(ctypes.Structure):
 
 
 class StackLayoutC(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int64) for n in ("hist", "idx", "gates64", "trace", "total")]
+    _fields_ = [(n, ctypes.c_int64) for n in ("hist", "idx", "gates64", "y32", "h32", "trace", "total")]
 
 
 _lib = None
@@ -96,6 +96,9 @@ def lib():
             "moe_stack_kernel_launches": (i32, [ctypes.POINTER(MoELayerC), i32, i64, st]),
             "tern_stream_status": (st, [vp]),
             "tern_test_bounded_wait": (st, [vp, i64, vp]),
+            "moe_stack_persistent_ctas": (i32, [ctypes.POINTER(MoELayerC), i32, st]),
+            "tern_test_stack_stall": (st, [ctypes.POINTER(MoELayerC), i32, vp, ctypes.c_float, st, i32, i64, vp, sz,
+                                           vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -413,7 +416,11 @@ def moe_stack_workspace_layout(layer0: MoELayer, T_max: int = 1, act=TERN_ACT_BF
     out = StackLayoutC()
     _check(lib().moe_stack_workspace_layout(ctypes.byref(layer0.c), T_max, act, ctypes.byref(out)),
            "moe_stack_workspace_layout")
-    return {n: int(getattr(out, n)) for n in ("hist", "idx", "gates64", "trace", "total")}
+    return {n: int(getattr(out, n)) for n in ("hist", "idx", "gates64", "y32", "h32", "trace", "total")}
+
+
+def moe_stack_persistent_ctas(layer0: MoELayer, n_layers: int, act=TERN_ACT_BF16) -> int:
+    return int(lib().moe_stack_persistent_ctas(ctypes.byref(layer0.c), n_layers, act))
 
 
 def moe_stack_kernel_launches(layer0: MoELayer, n_layers: int, T: int, act=TERN_ACT_BF16) -> int:
@@ -422,6 +429,19 @@ def moe_stack_kernel_launches(layer0: MoELayer, n_layers: int, T: int, act=TERN_
 
 def tern_stream_status(stream=None) -> int:
     return int(lib().tern_stream_status(_stream(stream)))
+
+
+def tern_test_stack_stall(stack: Stack, x, stall_layer: int, limit_ns: int, eps=1e-6, act=TERN_ACT_BF16, ws=None,
+                          stream=None):
+    """The T = 1 stack launch with one exchange that never completes (CTA 0, layer
+    stall_layer) and every in-kernel wait bounded by limit_ns; the kernel must give up by
+    itself and leave TERN_ETIMEOUT in the device status word."""
+    xb = _bits16(x.view(1, -1) if x.dim() == 1 else x, "x")
+    if ws is None:
+        ws = workspace(moe_stack_workspace_bytes(stack.layers[0], 1, act), xb.device)
+    _check(lib().tern_test_stack_stall(stack.c, len(stack.layers), _ptr(xb), float(eps), act, int(stall_layer),
+                                       int(limit_ns), _ptr(ws), ws.numel(), _stream(stream)), "tern_test_stack_stall")
+    return ws
 
 
 def tern_test_bounded_wait(flag: torch.Tensor, spin_limit: int, stream=None):

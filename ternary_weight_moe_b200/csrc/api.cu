@@ -24,6 +24,7 @@ namespace {
 inline bool aligned(const void *p, uintptr_t a) { return ((uintptr_t)p % a) == 0; }
 inline cudaStream_t S(void *s) { return reinterpret_cast<cudaStream_t>(s); }
 inline int64_t up256(int64_t v) { return (v + 255) & ~int64_t(255); }
+constexpr long long kStackWaitLimitNs = 1000000000ll;  // every wait of the persistent kernel: 1 s
 
 // K <= 2048 must give a power-of-two lane count (K/64 in {1,2,4,...,32})
 bool lanes_ok(int64_t K) {
@@ -266,7 +267,7 @@ tern_status moe_stack_decode(const tern_moe_layer *layers, int32_t n_layers, uin
         tern_status st = launch_stack_persistent(layers, n_layers, x, rms_eps, act,
                                                  b + o.total + up256(T * layers[0].d * 2),
                                                  (size_t)up256((int64_t)stack_persistent_ws_bytes(&layers[0])),
-                                                 status_word(), S(stream));
+                                                 status_word(), -1, kStackWaitLimitNs, S(stream));
         if (st != TERN_EUNSUPPORTED) return st;
     }
     const FfnWs w = carve(workspace, o, act);
@@ -286,11 +287,13 @@ tern_status moe_stack_workspace_layout(const tern_moe_layer *L0, int64_t T_max, 
     if (!out || T_max < 1 || T_max > kMaxT) return TERN_EINVAL;
     const Layout o = make_layout(L0->d, L0->f, L0->E, L0->k, T_max, act);
     const int64_t base = o.total + up256(T_max * L0->d * 2);
-    int64_t hist, idx, g, tr;
-    stack_persistent_offsets(L0, &hist, &idx, &g, &tr);
+    int64_t hist, idx, g, y32, h32, tr;
+    stack_persistent_offsets(L0, &hist, &idx, &g, &y32, &h32, &tr);
     out->hist = base + hist;
     out->idx = base + idx;
     out->gates64 = base + g;
+    out->y32 = base + y32;
+    out->h32 = base + h32;
     out->trace = base + tr;
     out->total = (int64_t)moe_stack_workspace_bytes(L0, T_max, act);
     return TERN_OK;
@@ -302,6 +305,11 @@ int32_t moe_stack_kernel_launches(const tern_moe_layer *L0, int32_t n_layers, in
     return 8 * n_layers;  // rmsnorm, logits, select, prep, gate/up, prep, down, combine
 }
 
+int32_t moe_stack_persistent_ctas(const tern_moe_layer *L0, int32_t n_layers, tern_act act) {
+    if (check_layer(L0) != TERN_OK || n_layers < 1 || n_layers > kMaxLayers) return 0;
+    return stack_persistent_ctas(L0, n_layers, act);
+}
+
 tern_status tern_stream_status(void *stream) {
     if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return TERN_ECUDA;
     int h = 0;
@@ -309,6 +317,33 @@ tern_status tern_stream_status(void *stream) {
     const int z = 0;
     if (cudaMemcpyToSymbol(g_status, &z, sizeof(int)) != cudaSuccess) return TERN_ECUDA;
     return (tern_status)h;
+}
+
+tern_status tern_test_stack_stall(const tern_moe_layer *layers, int32_t n_layers, uint16_t *x, float rms_eps,
+                                  tern_act act, int32_t stall_layer, int64_t limit_ns, void *workspace,
+                                  size_t ws_bytes, void *stream) {
+    if (!layers || n_layers < 1 || n_layers > kMaxLayers || !x || stall_layer < 0 || stall_layer >= n_layers ||
+        limit_ns < 1000 || limit_ns > kStackWaitLimitNs)
+        return TERN_EINVAL;
+    if (act != TERN_ACT_INT8 && act != TERN_ACT_BF16) return TERN_EINVAL;
+    for (int i = 0; i < n_layers; i++) {
+        tern_status st = check_layer(&layers[i]);
+        if (st != TERN_OK) return st;
+        if (layers[i].d != layers[0].d || layers[i].f != layers[0].f || layers[i].E != layers[0].E ||
+            layers[i].k != layers[0].k)
+            return TERN_EINVAL;
+    }
+    if (!aligned(x, 16)) return TERN_EALIGN;
+    const size_t need = moe_stack_workspace_bytes(&layers[0], 1, act);
+    if (!workspace || ws_bytes < need) return TERN_EWORKSPACE;
+    if (!aligned(workspace, 256)) return TERN_EALIGN;
+    const Layout o = make_layout(layers[0].d, layers[0].f, layers[0].E, layers[0].k, 1, act);
+    char *b = static_cast<char *>(workspace);
+    int *st = status_word();
+    if (!st) return TERN_ECUDA;
+    return launch_stack_persistent(layers, n_layers, x, rms_eps, act, b + o.total + up256(layers[0].d * 2),
+                                   (size_t)up256((int64_t)stack_persistent_ws_bytes(&layers[0])), st, stall_layer,
+                                   (long long)limit_ns, S(stream));
 }
 
 tern_status tern_test_bounded_wait(int32_t *flag, int64_t spin_limit, void *stream) {

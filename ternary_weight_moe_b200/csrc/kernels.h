@@ -75,10 +75,14 @@ struct StackLayerDev {
 };
 size_t stack_persistent_ws_bytes(const tern_moe_layer *L0);
 bool stack_persistent_supported(const tern_moe_layer *L0, int n_layers, tern_act act);
+int stack_persistent_ctas(const tern_moe_layer *L0, int n_layers, tern_act act);
 void stack_persistent_offsets(const tern_moe_layer *L0, int64_t *hist, int64_t *idx_hist, int64_t *gate_hist,
-                              int64_t *ttrace);
+                              int64_t *y_hist, int64_t *h_hist, int64_t *ttrace);
+// stall_layer: -1, or a layer at which CTA 0 waits for data nobody sends (timeout test);
+// limit_ns: bound on every in-kernel wait
 tern_status launch_stack_persistent(const tern_moe_layer *layers, int n_layers, uint16_t *x, float eps,
-                                    tern_act act, void *ws, size_t ws_bytes, int *status, cudaStream_t s);
+                                    tern_act act, void *ws, size_t ws_bytes, int *status, int stall_layer,
+                                    long long limit_ns, cudaStream_t s);
 
 // ---- bounded-wait test hook
 cudaError_t launch_test_wait(int32_t *flag, long long limit, int *status, cudaStream_t s);

@@ -44,15 +44,6 @@ constexpr int kRouteTok = 8;
 constexpr int kLogitWarps = 16;
 constexpr int kLogitChunk = 512;
 
-// bf16 -> fp64 by moving bits (normal values); zero, subnormal, inf and nan go through fp32
-__device__ __forceinline__ double bf16_to_f64(uint16_t b) {
-    const uint32_t e = (b >> 7) & 0xFFu;
-    if (e == 0u || e == 0xFFu) return (double)bf16_to_f32(b);
-    const unsigned long long bits = ((unsigned long long)(b & 0x8000u) << 48) |
-                                    ((unsigned long long)(e + 896u) << 52) | ((unsigned long long)(b & 0x7Fu) << 45);
-    return __longlong_as_double((long long)bits);
-}
-
 __global__ void __launch_bounds__(kLogitWarps * 32) logits_kernel(const uint16_t *__restrict__ Wg,
                                                                    const uint16_t *__restrict__ x, int T, int d,
                                                                    int E, double *__restrict__ logits) {
@@ -624,7 +615,10 @@ __global__ void __launch_bounds__(kMmaWarps * 32) down_mma_kernel(
 }
 
 // ------------------------------------------------------------------------- combine
-// y[t,i] = sum over slots (top-k order) of g64[t,slot] * ye[t*k+slot, i], fp64.
+// y[t,i] = sum over slots (top-k order) of g64[t,slot] * fp32(ye[t*k+slot, i]), in fp64.  The
+// expert outputs enter the sum rounded to fp32 (one rounding, 2^-24 relative): that is the
+// precision in which the persistent stack kernel passes them between SMs, and both paths give
+// the same bits.  On the int8 path ye is an fp32 value already.
 __global__ void combine_kernel(const double *__restrict__ g64, const double *__restrict__ ye, int T, int d, int k,
                                uint16_t *__restrict__ y, float *__restrict__ y32, const uint16_t *__restrict__ resid,
                                uint16_t *__restrict__ x_out) {
@@ -632,7 +626,7 @@ __global__ void combine_kernel(const double *__restrict__ g64, const double *__r
     for (int64_t p = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; p < n; p += (int64_t)gridDim.x * blockDim.x) {
         const int t = (int)(p / d), i = (int)(p % d);
         double acc = 0.0;
-        for (int s = 0; s < k; s++) acc += g64[t * k + s] * ye[((int64_t)t * k + s) * d + i];
+        for (int s = 0; s < k; s++) acc += g64[t * k + s] * (double)(float)ye[((int64_t)t * k + s) * d + i];
         const uint16_t yb = f64_to_bf16_rne(acc);
         if (y) y[p] = yb;
         if (y32) y32[p] = (float)acc;

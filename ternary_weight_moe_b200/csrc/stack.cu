@@ -3,35 +3,57 @@
 // Batch-1 decode streams the active weights layer after layer and is bound by memory
 // bandwidth ("How a 20B Model Hits 120 tok/s on an iPhone", "Why the number is plausible";
 // "A 20B AI Model Trained in Ternary Just Hit 218 Tokens/Second on a $599 Mac Mini", "What
-// Ternary Actually Means").  At d = 2048 one layer moves only 7.4 MB, about a microsecond of
-// HBM time on a B200, so the chain router -> top-k -> expert rows -> h -> down -> residual
-// is bound by latency, not by bytes.  This kernel therefore:
-//   * runs the whole stack in ONE launch: one CTA per SM, all co-resident (cooperative
-//     launch), no kernel boundary between layers;
-//   * exchanges data between CTAs with flag-carrying 64-bit words: {32-bit payload, 32-bit
-//     tag}, written and read as single 64-bit accesses (single-copy atomic), where the tag
-//     names the launch and the layer.  A consumer polls the data itself, so each exchange
-//     costs one L2 round trip instead of a barrier plus a read, and no arrival counter has
-//     to be reset between launches;
-//   * gives every CTA a fixed share of each layer's bytes and moves it with TMA bulk copies
-//     (cp.async.bulk global -> shared, mbarrier completion) as early as the dependencies
-//     allow: the next layer's router rows during the current layer; a CTA's gate/up AND down
-//     rows together as soon as top-k is known (the down rows do not depend on h);
-//   * decodes the packed bytes in registers (one table read + one dp4a per limb per byte).
+// Ternary Actually Means").  At d = 2048 a layer moves only 7.4 MB, about a microsecond of
+// HBM time on a B200, so the chain x -> norm -> router -> top-k -> expert rows -> h -> down
+// -> residual is bound by the latency of its steps, not by bytes.  This kernel:
+//   * runs the whole stack in ONE launch: P = k * G CTAs, one per SM, co-resident
+//     (cooperative launch); no kernel boundary between layers;
+//   * is slot-major: CTA (s, c) -- group s, part c of G -- works only on the expert chosen at
+//     rank s of the top-k: a contiguous block of its gate/up rows and of its down rows, moved
+//     by three bulk copies (TMA, mbarrier completion) the moment top-k is known;
+//   * exchanges data between CTAs through flag-carrying 64-bit words {32-bit payload, 32-bit
+//     tag} in global memory, stored and polled with single 64-bit relaxed accesses at GPU
+//     scope (each word is single-copy atomic, so a reader sees the payload that belongs to
+//     the tag it reads; no fence is needed because nothing else is read).  The tag names the
+//     launch and the layer.  Four exchanges per layer, three of them inside small groups:
+//       logits  every CTA computes <= 2 router rows and publishes them; all CTAs read all;
+//       h       the G CTAs of a group publish their h; the group reads the slot's f values;
+//       y       the k CTAs with the same part c (one per slot) publish their slot's output
+//               rows, rounded to fp32; each reads the k outputs of its rows and sums them;
+//       x       the G CTAs of a group publish x' for their rows (+ the sum of squares and
+//               the absmax of those rows); the group reads the whole vector;
+//     every exchange buffer has two copies (layer parity), see "buffer reuse" below;
+//   * prefetches the next layer's experts to L2: with its own n it also computes its router
+//     rows of the NEXT layer (fp32, a prediction only), the CTAs exchange these, and group s
+//     prefetches its rows of predicted experts s and s + 8 (kPredTop = 12 in all) while the
+//     current layer runs.  A prefetch changes no value; it only moves the HBM reads of
+//     correctly predicted experts off the critical path;
+//   * decodes the packed bytes in registers by integer logic (decode.cuh): no lookup table.
 //
-// Per layer l, in every CTA (P = #SMs CTAs):
-//   A  x_l (exchange) -> sum of squares and absmax in one block reduction -> n = bf16(x/r),
-//      activation limbs; its router rows (prefetched) -> logits -> exchange
-//   B  all logits -> top-k + gates -> TMA copies of its gate/up pairs and down rows
-//   C  its (slot,row) gate/up pairs -> h = silu(g) * u (fp64 epilogue, one thread per row)
-//      -> exchange
-//   D  all h -> limbs; its output rows: down for every slot, gate-weighted sum in top-k order
-//      (fp64), bf16, residual add -> x_{l+1} -> exchange
+// Per layer l, in CTA (s, c):
+//   A  x_l (exchange x, or the input at l = 0) -> r = sqrt(sum x^2 / d + eps) from the parts'
+//      sums, n = bf16(x / r), activation limbs; router rows -> logits -> publish; the next
+//      layer's router rows -> predicted logits -> publish
+//   B  all logits -> top-k (one warp) -> bulk copies of this CTA's gate/up and down rows of
+//      expert idx[s]; meanwhile other warps load the rows' scales, compute the gates and
+//      issue the L2 prefetches of the predicted next-layer experts
+//   C  gate/up dots -> h = silu(g) * u (fp64, one thread per row) -> exchange h
+//   D  h limbs -> down dots -> y_s rows (fp32) -> exchange y -> y = sum_q g_q y_q in top-k
+//      order (fp64) -> x' = bf16(x + bf16(y)) -> exchange x
+//
+// Buffer reuse.  Each exchange buffer is written at layer l and again at layer l + 2 (same
+// parity).  A CTA writes its layer-(l+2) words only after it has read the layer-(l+1) words
+// of every other producer of the same exchange, and each of those producers wrote them only
+// after reading the layer-l words: so no word is overwritten before every consumer has read
+// it.  The tag carries the launch epoch (advanced by the last CTA to leave), so a fresh launch
+// never matches words left by an earlier one and the workspace needs no clearing between
+// calls.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdlib.h>
 #include <string.h>
 
+#include "cluster.cuh"
 #include "kernels.h"
 #include "tern_common.cuh"
 #include "tma.cuh"
@@ -40,128 +62,109 @@ namespace tern {
 
 constexpr int kStackWarps = 16;
 constexpr int kStackThreads = kStackWarps * 32;
-constexpr int kMaxStackLayers = 64;
-constexpr int kSK = 8;  // max experts per token on this path
+constexpr int kSK = 8;              // max experts per token on this path
 constexpr int kMaxTraceCtas = 256;
+constexpr int kMaxGroup = 32;       // CTAs per slot group
+constexpr int kMaxGU = 32;          // gate/up rows per CTA (two chunks of 16)
+constexpr int kMaxDN = 128;         // down rows per CTA
+constexpr int kMaxRouterRows = 8;   // router rows per CTA
+constexpr int kPredTop = 12;        // predicted next-layer experts prefetched to L2
+constexpr int kTracePoints = 16;
 
 struct StackParams {
-    StackLayerDev layer[kMaxStackLayers];
+    StackLayerDev layer[kMaxLayers];
     int n_layers, d, f, E, k;
     double eps;
     uint16_t *x;                  // [d] in/out
     unsigned int *ctl;            // [0] CTAs that left this launch, [1] launch epoch
-    unsigned long long *xll;      // [d/2]  {two bf16 of x_{l}, tag}
-    unsigned long long *lll;      // [2E]   {high / low word of the fp64 logit, tag}
-    unsigned long long *hll;      // [k*f]  {fp32 h, tag}
+    unsigned long long *xb;       // [2][k][d/2]        {two bf16 of x, tag}
+    unsigned long long *xst;      // [2][k][G][4]       {sum x^2 hi, lo, absmax, 0} of each part, tagged
+    unsigned long long *lb;       // [2][E][2]          {fp64 logit hi, lo}, tagged
+    unsigned long long *pb;       // [2][E]             {fp32 predicted next-layer logit}, tagged
+    unsigned long long *hb;       // [2][k][f]          {fp32 h}, tagged
+    unsigned long long *yb;       // [2][G][k][kMaxDN]  {fp32 expert output row}, tagged
     uint16_t *hist;               // [n_layers+1][d]  x before each layer and after the last
     int32_t *idx_hist;            // [n_layers][k]
     double *gate_hist;            // [n_layers][k]
+    float *y_hist;                // [n_layers][d]    FFN output before the bf16 cast
+    float *h_hist;                // [n_layers][k][f] SwiGLU output of each slot
     int *status;
     long long limit_ns;           // bound on every in-kernel wait
-    unsigned long long *ttrace;   // [n_layers][P][16] %globaltimer stamps of every CTA, then
-                                  // [n_layers][P][16] clock64 stamps (SM cycles) at the same points
-    int P;                        // CTAs
-    int rb_rows;                  // max router rows per CTA
-    int gu_pairs;                 // max gate/up pairs per CTA
-    int dn_rows;                  // max output rows per CTA (even)
+    unsigned long long *ttrace;   // [n_layers][P][16] %globaltimer stamps, then the same for clock64
+    int P, G;
+    int stall_layer;              // test hook: at this layer CTA 0 waits for an h tag nobody writes
+    int predict;                  // 1: prefetch predicted next-layer experts to L2
 };
 
-// ------------------------------------------------------------------ exchange words
-// ---- flag-carrying words: one 64-bit access carries payload and tag together
-__device__ __forceinline__ void ll_store(unsigned long long *p, uint32_t val, uint32_t tag) {
-    const unsigned long long w = ((unsigned long long)tag << 32) | (unsigned long long)val;
-    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+// ------------------------------------------------------------------ tagged words
+__device__ __forceinline__ unsigned long long tagged(uint32_t payload, uint32_t tag) {
+    return ((unsigned long long)tag << 32) | (unsigned long long)payload;
 }
-__device__ __forceinline__ unsigned long long ll_load(const unsigned long long *p) {
-    unsigned long long w;
-    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
-    return w;
+__device__ __forceinline__ void st_word(unsigned long long *p, uint32_t payload, uint32_t tag) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(tagged(payload, tag)) : "memory");
 }
 
-// Gather n tagged words (n*8 bytes, 16-byte aligned) from global memory into shared memory
-// with one TMA bulk copy, then check every tag in shared memory; re-fetch until all carry
-// `tag`.  One bulk copy per CTA replaces thousands of per-thread polls of the same hot L2
-// lines (measured on B200: 1.3-1.6 us per 148-CTA exchange instead of 1.5-2.9 us).  Called
-// by every thread of the CTA; `phase` is the mbarrier phase counter (same in every thread).
-// Returns false (uniformly) on timeout, status set.
-__device__ __forceinline__ bool ll_gather(const unsigned long long *src, int n, uint32_t tag,
-                                          unsigned long long *dst, uint64_t *mb, uint32_t &phase, long long limit_ns,
-                                          int *status) {
-    const unsigned long long t0 = gtimer();
+// Poll the pair of tagged words at src until both carry `tag`; false once `t0 + limit` passes.
+__device__ __forceinline__ bool poll_pair(const unsigned long long *src, uint32_t tag, unsigned long long t0,
+                                          long long limit, ulonglong2 &out) {
     while (true) {
-        if (threadIdx.x == 0) {
-            mbar_expect_tx(mb, (uint32_t)(n * 8));
-            bulk_g2s(dst, src, (uint32_t)(n * 8), mb);
-        }
-        const bool landed = mbar_wait(mb, phase & 1u, limit_ns, status);
-        phase++;
-        int mine = landed ? 1 : 0;
-        for (int w = threadIdx.x; w < n; w += blockDim.x)
-            if ((uint32_t)(dst[w] >> 32) != tag) mine = 0;
-        if (__syncthreads_and(mine)) return true;
-        // uniform timeout decision: thread 0's clock, broadcast by the barrier below
-        const int late = (threadIdx.x == 0) && ((long long)(gtimer() - t0) > limit_ns);
-        if (__syncthreads_or(late)) {
-            set_status(status, TERN_ETIMEOUT);
-            return false;
-        }
+        out = ld_relaxed_v2(src);
+        if ((uint32_t)(out.x >> 32) == tag && (uint32_t)(out.y >> 32) == tag) return true;
+        if ((long long)(gtimer() - t0) > limit) return false;
     }
 }
 
 // ------------------------------------------------------------------ shared memory map
 struct SmemMap {
-    uint32_t lut, rbuf, gbuf, ubuf, dbuf, xs, ns, xl, hl, xch, total;
+    uint32_t gbuf, ubuf, dbuf, rbuf0, rbuf1, xs, xl, hl, lg, plg, hv, yv, cand, total;
 };
 
 __host__ __device__ inline uint32_t align128(uint32_t v) { return (v + 127u) & ~127u; }
 
-__host__ __device__ inline SmemMap smem_map(int d, int f, int k, int rb_rows, int gu_pairs, int dn_rows, int NL) {
+__host__ __device__ inline SmemMap smem_map(int d, int f, int k, int gu_max, int dn_max, int rb_max, int NL) {
     SmemMap m;
     uint32_t p = 0;
-    m.lut = p;
-    p = align128(p + kLutBytes);
-    m.rbuf = p;
-    p = align128(p + (uint32_t)rb_rows * d * 2);
-    m.gbuf = p;
-    p = align128(p + (uint32_t)gu_pairs * (d / 4));
-    m.ubuf = p;
-    p = align128(p + (uint32_t)gu_pairs * (d / 4));
-    m.dbuf = p;
-    p = align128(p + (uint32_t)k * dn_rows * (f / 4));
-    m.xs = p;
-    p = align128(p + (uint32_t)d * 2);
-    m.ns = p;
-    p = align128(p + (uint32_t)d * 2);
-    m.xl = p;
-    p = align128(p + (uint32_t)NL * (d / 64) * kSegPad * 4);
-    m.hl = p;
-    p = align128(p + (uint32_t)k * NL * (f / 64) * kSegPad * 4);
-    m.xch = p;  // exchange landing buffer: max(d/2, 2E, k*f) words
-    {
-        uint32_t nw = (uint32_t)(d / 2);
-        if ((uint32_t)(2 * 256) > nw) nw = 2 * 256;
-        if ((uint32_t)(k * f) > nw) nw = (uint32_t)(k * f);
-        p = align128(p + nw * 8);
-    }
+    auto take = [&](uint32_t bytes) {
+        const uint32_t r = p;
+        p = align128(p + bytes);
+        return r;
+    };
+    m.gbuf = take((uint32_t)gu_max * (d / 4));
+    m.ubuf = take((uint32_t)gu_max * (d / 4));
+    m.dbuf = take((uint32_t)dn_max * (f / 4));
+    m.rbuf0 = take((uint32_t)rb_max * d * 2);
+    m.rbuf1 = take((uint32_t)rb_max * d * 2);
+    m.xs = take((uint32_t)d * 2);
+    m.xl = take((uint32_t)NL * (d / 64) * kSegPad * 4);
+    m.hl = take((uint32_t)NL * (f / 64) * kSegPad * 4);
+    m.lg = take(256 * 8);
+    m.plg = take(256 * 8);
+    m.hv = take((uint32_t)f * 4);
+    m.yv = take((uint32_t)k * kMaxDN * 4);
+    m.cand = take(256 * 16);
     m.total = p;
     return m;
 }
 
-// limb words of four consecutive values v[0..3] (one word per limb)
+// Limb bytes of four consecutive values v[0..3] (elements 4t..4t+3 of a vector whose limbs go
+// to `limbs`, laid out [NL][segments][kSegPad words], position-major inside each segment):
+// element 4t+e lands in byte (t & 3) of word 4 * ((t >> 2) & 3) + e of segment t >> 4.
 template <int NL>
-__device__ __forceinline__ void limb_words(const float (&v)[4], int sh_or_unused, float inv, bool nonzero,
-                                           uint32_t (&w)[3]) {
-    w[0] = w[1] = w[2] = 0;
+__device__ __forceinline__ void store_limbs4(uint32_t *limbs, int seg_words_per_limb, int t, const float (&v)[4], int sh,
+                                             float inv, bool nonzero) {
+    uint8_t *lb = reinterpret_cast<uint8_t *>(limbs);
+    const int g = t >> 4, q = (t >> 2) & 3, b = t & 3;
 #pragma unroll
     for (int e = 0; e < 4; e++) {
+        const int w = g * kSegPad + 4 * q + e;
         if (NL == 1) {
-            w[0] |= ((uint32_t)(nonzero ? quant_one(v[e], inv) : 0) & 0xFFu) << (8 * e);
+            lb[4 * w + b] = (uint8_t)((nonzero ? quant_one(v[e], inv) : 0) & 0xFF);
         } else {
-            uint32_t h, m, lo;
-            fixed_limbs(v[e], sh_or_unused, h, m, lo);
-            w[0] |= h << (8 * e);
-            w[1] |= m << (8 * e);
-            w[2] |= lo << (8 * e);
+            uint32_t hi, mid, lo;
+            fixed_limbs(v[e], sh, hi, mid, lo);
+            lb[4 * w + b] = (uint8_t)hi;
+            lb[4 * (seg_words_per_limb + w) + b] = (uint8_t)mid;
+            lb[4 * (2 * seg_words_per_limb + w) + b] = (uint8_t)lo;
         }
     }
 }
@@ -170,72 +173,63 @@ __device__ __forceinline__ void limb_words(const float (&v)[4], int sh_or_unused
 template <int NL>
 __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_constant__ StackParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
-    __shared__ __align__(8) uint64_t mb_router, mb_gu0, mb_gu1, mb_dn, mb_x;
-    __shared__ __align__(8) uint64_t mb_h[kSK];        // per-slot h fetch
-    __shared__ int s_hok[kSK][kStackWarps], s_hlate[kSK];
-    __shared__ float s_hpart[kSK][kStackWarps];
-    __shared__ unsigned int s_hissued[kSK];
+    __shared__ __align__(8) uint64_t mb_r[2], mb_gu0, mb_gu1, mb_dn;
     __shared__ double s_red[kStackWarps];
     __shared__ float s_redf[kStackWarps];
-    __shared__ double s_part[kStackWarps][kStackWarps];
-    __shared__ double s_logit[256];
-    __shared__ __align__(16) uint32_t s_gm[32];  // top-k scratch
-    __shared__ int s_nc;
-    __shared__ ulonglong2 s_cand[256];
-    __shared__ int s_idx[kSK];
+    __shared__ double s_rp[kStackWarps][kMaxRouterRows];
+    __shared__ float s_pp[kStackWarps][kMaxRouterRows];
+    __shared__ double s_xss[kMaxGroup];
+    __shared__ float s_xam[kMaxGroup];
+    __shared__ int32_t s_idx[kSK];
+    __shared__ int32_t s_pidx[kPredTop];
     __shared__ double s_gate[kSK];
-    __shared__ long long s_S[64][2];
-    __shared__ double s_ye[64][kSK];
-    __shared__ float s_sg[64], s_su[64], s_sd[kSK * 64];
+    __shared__ long long s_S[kMaxGU][2];
+    __shared__ float s_sg[kMaxGU], s_su[kMaxGU], s_sd[kMaxDN];
+    __shared__ float s_hmax[kStackWarps];
     // the layers' pointers, copied once: a dynamically indexed kernel parameter is a constant
     // cache line fetched from L2 on the critical path of every layer
-    __shared__ StackLayerDev s_layer[kMaxStackLayers];
+    __shared__ StackLayerDev s_layer[kMaxLayers];
 
-    const int d = p.d, f = p.f, E = p.E, k = p.k, P = p.P;
-    const int c = blockIdx.x;
+    const int d = p.d, f = p.f, E = p.E, k = p.k, P = p.P, G = p.G;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const SmemMap sm = smem_map(d, f, k, p.rb_rows, p.gu_pairs, p.dn_rows, NL);
-    uint32_t *lut = reinterpret_cast<uint32_t *>(smem + sm.lut);
-    uint16_t *rbuf = reinterpret_cast<uint16_t *>(smem + sm.rbuf);
+    const int pid = blockIdx.x, s = pid / G, c = pid % G;
+    // this CTA's shares: gate/up rows [j0, j1), down rows [i0, i1) (even bounds), router rows [e0, e1)
+    const int j0 = (c * f) / G, j1 = ((c + 1) * f) / G, ngu = j1 - j0;
+    const int i0 = 2 * ((c * (d / 2)) / G), i1 = 2 * (((c + 1) * (d / 2)) / G), ndn = i1 - i0;
+    const int e0 = (E * pid) / P, e1 = (E * (pid + 1)) / P, nr = e1 - e0;
+    const int n0 = ngu < 16 ? ngu : 16, n1 = ngu - n0;  // gate/up rows in the first / second copy
+    const int gu_max = (f + G - 1) / G, dn_max = 2 * ((d / 2 + G - 1) / G), rb_max = (E + P - 1) / P;
+    const SmemMap sm = smem_map(d, f, k, gu_max, dn_max, rb_max, NL);
     uint8_t *gbuf = smem + sm.gbuf;
     uint8_t *ubuf = smem + sm.ubuf;
     uint8_t *dbuf = smem + sm.dbuf;
+    uint16_t *const rbuf0 = reinterpret_cast<uint16_t *>(smem + sm.rbuf0);
+    uint16_t *const rbuf1 = reinterpret_cast<uint16_t *>(smem + sm.rbuf1);
     uint16_t *xs = reinterpret_cast<uint16_t *>(smem + sm.xs);
-    uint16_t *ns = reinterpret_cast<uint16_t *>(smem + sm.ns);
     uint32_t *xl = reinterpret_cast<uint32_t *>(smem + sm.xl);
     uint32_t *hl = reinterpret_cast<uint32_t *>(smem + sm.hl);
-    unsigned long long *xch = reinterpret_cast<unsigned long long *>(smem + sm.xch);
+    double *lg = reinterpret_cast<double *>(smem + sm.lg);
+    double *plg = reinterpret_cast<double *>(smem + sm.plg);
+    float *hv = reinterpret_cast<float *>(smem + sm.hv);
+    float *yv = reinterpret_cast<float *>(smem + sm.yv);
+    ulonglong2 *cand = reinterpret_cast<ulonglong2 *>(smem + sm.cand);
     const int xlp = (d / 64) * kSegPad;  // padded words per limb of n
-    const int hlp = (f / 64) * kSegPad;  // padded words per limb of one slot's h
+    const int hlp = (f / 64) * kSegPad;  // padded words per limb of h
 
-    // static shares of this CTA
-    const int nr = (E - c + P - 1) / P;  // router rows: c, c+P, ...
-    const int NPt = k * f;
-    const int p0 = (int)((long long)c * NPt / P), p1 = (int)((long long)(c + 1) * NPt / P);
-    const int i0 = 2 * (int)((long long)c * (d / 2) / P), i1 = 2 * (int)((long long)(c + 1) * (d / 2) / P);
-    const int nrows = i1 - i0;
     const long long lim = p.limit_ns;
     const uint32_t ep = ld_acquire_gpu(p.ctl + 1);  // launch epoch, advanced by the previous launch
     bool alive = true;
-    unsigned int n_rt = 0, n_gu = 0, n_dn = 0;  // phases issued per mbarrier (thread 0)
-    uint32_t xph = 0;                            // phase counter of the exchange mbarrier
-    uint32_t hph = 0;                            // phase counter of this warp's slot mbarrier
-    // gate/up pairs arrive in two halves (first 16 pairs, then the rest) so the dots of the
-    // first half overlap the second half's transfer
-    const int npairs = p1 - p0;
-    const int n0 = npairs < kStackWarps ? npairs : kStackWarps;
-    const int n1 = npairs - n0;
+    unsigned int n_rt0 = 0, n_rt1 = 0, n_gu = 0, n_dn = 0;  // phases armed per mbarrier (thread 0)
 
     unsigned long long *tt = (tid == 0) ? p.ttrace : nullptr;
-    const size_t ctr_off = (size_t)p.n_layers * P * 16;
-#define TSTAMP(l, ph)                                              \
-    if (tt) {                                                      \
-        const size_t o_ = ((size_t)(l) * P + c) * 16 + (ph);       \
-        tt[o_] = gtimer();                                         \
-        tt[ctr_off + o_] = (unsigned long long)clock64();          \
+    const size_t ctr_off = (size_t)p.n_layers * P * kTracePoints;
+#define TSTAMP(l, ph)                                                  \
+    if (tt) {                                                          \
+        const size_t o_ = ((size_t)(l) * P + pid) * kTracePoints + (ph); \
+        tt[o_] = gtimer();                                             \
+        tt[ctr_off + o_] = (unsigned long long)clock64();              \
     }
 
-    lut_fill(lut);
     {
         constexpr int kW = (int)(sizeof(StackLayerDev) / sizeof(uint64_t));
         static_assert(sizeof(StackLayerDev) % sizeof(uint64_t) == 0, "pointer table");
@@ -243,243 +237,300 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             reinterpret_cast<uint64_t *>(s_layer)[q] = reinterpret_cast<const uint64_t *>(p.layer)[q];
     }
     if (tid == 0) {
-        mbar_init(&mb_router, 1);
+        mbar_init(&mb_r[0], 1);
+        mbar_init(&mb_r[1], 1);
         mbar_init(&mb_gu0, 1);
         mbar_init(&mb_gu1, 1);
         mbar_init(&mb_dn, 1);
-        mbar_init(&mb_x, 1);
-        for (int q = 0; q < kSK; q++) {
-            mbar_init(&mb_h[q], 1);
-            s_hissued[q] = 0u;
-        }
         fence_mbar_init();
     }
     __syncthreads();
-    if (tid == 0 && nr > 0) {  // router rows of layer 0
-        mbar_expect_tx(&mb_router, (uint32_t)(nr * d * 2));
-        n_rt++;
-        for (int r = 0; r < nr; r++)
-            bulk_g2s(rbuf + (size_t)r * d, s_layer[0].router + (size_t)(c + r * P) * d, (uint32_t)(d * 2), &mb_router);
+    // router rows of layers 0 and 1 (buffer l & 1 holds layer l's rows)
+    if (tid == 0 && nr > 0) {
+        mbar_expect_tx(&mb_r[0], (uint32_t)(nr * d * 2));
+        n_rt0++;
+        bulk_g2s(rbuf0, s_layer[0].router + (size_t)e0 * d, (uint32_t)(nr * d * 2), &mb_r[0]);
+        if (p.n_layers > 1) {
+            mbar_expect_tx(&mb_r[1], (uint32_t)(nr * d * 2));
+            n_rt1++;
+            bulk_g2s(rbuf1, s_layer[1].router + (size_t)e0 * d, (uint32_t)(nr * d * 2), &mb_r[1]);
+        }
     }
 
     for (int l = 0; l < p.n_layers && alive; l++) {
         const StackLayerDev &Ly = s_layer[l];
         const uint32_t par = (uint32_t)(l & 1);
         const uint32_t tag = (ep << 7) | (uint32_t)(l + 1);  // never 0 (a zeroed workspace holds 0)
+        const bool has_next = l + 1 < p.n_layers;
         TSTAMP(l, 0)
-        if (tid < 3 && c < 32) {
-            // one L2 prefetch per 2 MB page of this layer's gate, up and down arrays: the
-            // address translations are in place before top-k sends the row copies there
-            const uint8_t *base = tid == 0 ? Ly.gate : (tid == 1 ? Ly.up : Ly.down);
-            const size_t off = (size_t)c << 21;
-            if (off < (size_t)E * f * (d / 4)) asm volatile("prefetch.global.L2 [%0];" ::"l"(base + off));
-        }
-        if (tid == 0) {
-            // this layer's transfer sizes depend only on the CTA's share, not on the routing:
-            // register them now so the copies can be issued the moment top-k is known
-            mbar_expect_tx(&mb_gu0, (uint32_t)(2 * n0 * (d / 4)));
-            mbar_expect_tx(&mb_gu1, (uint32_t)(2 * n1 * (d / 4)));
-            mbar_expect_tx(&mb_dn, (uint32_t)(k * nrows * (f / 4)));
-            n_gu++;
-            n_dn++;
-        }
         // ------------------------------------------------------------ A: x_l, norm, limbs
-        // thread t owns elements 4t..4t+3 (d = 2048 = 4 * 512)
+        // thread t owns elements 4t..4t+3 (d = 4 * threads)
         float xv[4];
+        double r;
+        float amax;
         {
             bool ok = true;
-            uint32_t pr[2] = {0, 0};
+            uint2 pr;
             if (l == 0) {
-                const uint2 v4 = __ldcg(reinterpret_cast<const uint2 *>(p.x) + tid);
-                pr[0] = v4.x;
-                pr[1] = v4.y;
+                pr = __ldcg(reinterpret_cast<const uint2 *>(p.x) + tid);
             } else {
-                ok = ll_gather(p.xll, d / 2, tag, xch, &mb_x, xph, lim, p.status);
-                pr[0] = (uint32_t)xch[2 * tid];
-                pr[1] = (uint32_t)xch[2 * tid + 1];
+                const unsigned long long t0 = gtimer();
+                ulonglong2 w;
+                ok = poll_pair(p.xb + ((size_t)par * k + s) * (d / 2) + 2 * tid, tag, t0, lim, w);
+                pr = make_uint2((uint32_t)w.x, (uint32_t)w.y);
+                if (tid < 2 * G) {
+                    ulonglong2 st;
+                    const bool ok2 = poll_pair(p.xst + (((size_t)par * k + s) * G + (tid >> 1)) * 4 + 2 * (tid & 1), tag,
+                                               t0, lim, st);
+                    ok = ok && ok2;
+                    if (tid & 1) s_xam[tid >> 1] = __uint_as_float((uint32_t)st.x);
+                    else s_xss[tid >> 1] = __longlong_as_double((long long)(((unsigned long long)(uint32_t)st.x << 32) |
+                                                                            (uint32_t)st.y));
+                }
             }
-            alive = __syncthreads_and(ok ? 1 : 0) && alive;
-            reinterpret_cast<uint2 *>(xs)[tid] = make_uint2(pr[0], pr[1]);
-            xv[0] = bf16_to_f32((uint16_t)(pr[0] & 0xFFFFu));
-            xv[1] = bf16_to_f32((uint16_t)(pr[0] >> 16));
-            xv[2] = bf16_to_f32((uint16_t)(pr[1] & 0xFFFFu));
-            xv[3] = bf16_to_f32((uint16_t)(pr[1] >> 16));
-        }
-        TSTAMP(l, 1)
-        if (l == 0 && c == 0) reinterpret_cast<uint2 *>(p.hist)[tid] = reinterpret_cast<const uint2 *>(xs)[tid];
-        double r;
-        float amax_n;
-        {
-            double ss = 0.0;
-            float am = 0.0f;
+            reinterpret_cast<uint2 *>(xs)[tid] = pr;
+            xv[0] = bf16_to_f32((uint16_t)(pr.x & 0xFFFFu));
+            xv[1] = bf16_to_f32((uint16_t)(pr.x >> 16));
+            xv[2] = bf16_to_f32((uint16_t)(pr.y & 0xFFFFu));
+            xv[3] = bf16_to_f32((uint16_t)(pr.y >> 16));
+            if (l == 0) {
+                double ss = 0.0;
+                float am = 0.0f;
 #pragma unroll
-            for (int e = 0; e < 4; e++) {
-                const double v = (double)xv[e];
-                ss = fma(v, v, ss);
-                am = fmaxf(am, fabsf(xv[e]));
+                for (int e = 0; e < 4; e++) {
+                    ss = fma((double)xv[e], (double)xv[e], ss);
+                    am = fmaxf(am, fabsf(xv[e]));
+                }
+                ss = warp_sum_f64(ss);
+                am = warp_max_f32(am);
+                if (lane == 0) {
+                    s_red[warp] = ss;
+                    s_redf[warp] = am;
+                }
             }
-            ss = warp_sum_f64(ss);
-            am = warp_max_f32(am);
-            if (lane == 0) {
-                s_red[warp] = ss;
-                s_redf[warp] = am;
+            if (!__syncthreads_and(ok ? 1 : 0)) {
+                set_status(p.status, TERN_ETIMEOUT);
+                alive = false;
+                break;
             }
-            __syncthreads();
-            // every thread folds the 16 warp partials in the same order: same r everywhere
+            // every thread folds the partial sums in the same order: the same r in every CTA
             double ts = 0.0;
             float ta = 0.0f;
+            if (l == 0) {
 #pragma unroll
-            for (int w = 0; w < kStackWarps; w++) {
-                ts += s_red[w];
-                ta = fmaxf(ta, s_redf[w]);
+                for (int w = 0; w < kStackWarps; w++) {
+                    ts += s_red[w];
+                    ta = fmaxf(ta, s_redf[w]);
+                }
+            } else {
+                for (int q = 0; q < G; q++) {
+                    ts += s_xss[q];
+                    ta = fmaxf(ta, s_xam[q]);
+                }
             }
             r = sqrt(ts / (double)d + p.eps);
-            // rounding is monotone, so max |bf16(x_k / r)| = bf16(max |x_k| / r)
-            amax_n = bf16_to_f32(f64_to_bf16_rne((double)ta / r));
+            amax = ta;
         }
+        TSTAMP(l, 1)
+        if (l == 0 && pid == 0) reinterpret_cast<uint2 *>(p.hist)[tid] = reinterpret_cast<const uint2 *>(xs)[tid];
+        // rounding is monotone, so max |bf16(x_k / r)| = bf16(max |x_k| / r)
+        const float amax_n = bf16_to_f32(f64_to_bf16_rne((double)amax / r));
         const float s_nq = (NL == 1) ? (amax_n > 0.0f ? __fdiv_rn(amax_n, 127.0f) : 0.0f) : 0.0f;
         const int sh_n = (NL == 1) ? 0 : fixed_shift(amax_n);
+        double nd[4];
+        float nf[4];
         {
-            float nv[4];
-            uint16_t nb[4];
 #pragma unroll
             for (int e = 0; e < 4; e++) {
-                nb[e] = f64_to_bf16_rne((double)xv[e] / r);
-                nv[e] = bf16_to_f32(nb[e]);
+                const uint16_t nb = f64_to_bf16_rne((double)xv[e] / r);
+                nf[e] = bf16_to_f32(nb);
+                nd[e] = (double)nf[e];
             }
-            reinterpret_cast<uint2 *>(ns)[tid] =
-                make_uint2((uint32_t)nb[0] | ((uint32_t)nb[1] << 16), (uint32_t)nb[2] | ((uint32_t)nb[3] << 16));
-            uint32_t w[3];
             const float inv = (NL == 1 && amax_n > 0.0f) ? quant_inv(amax_n) : 0.0f;
-            limb_words<NL>(nv, sh_n, inv, amax_n > 0.0f, w);
-            const int pw = padded_word(tid);
-            xl[pw] = w[0];
-            if (NL > 1) {
-                xl[xlp + pw] = w[1];
-                xl[2 * xlp + pw] = w[2];
+            store_limbs4<NL>(xl, xlp, tid, nf, sh_n, inv, amax_n > 0.0f);
+        }
+        // router rows of this layer: thread t multiplies columns 4t..4t+3; bf16 x bf16 has at
+        // most 16 significant bits, so each product is exact in fp64 and the fma adds it with
+        // one rounding (the sums are exact at these magnitudes: the order does not matter)
+        if (nr > 0) {
+            if (!mbar_wait(&mb_r[par], (uint32_t)((l >> 1) & 1), lim, p.status)) alive = false;
+#pragma unroll
+            for (int q = 0; q < kMaxRouterRows; q++) {
+                if (q < nr) {
+                    const uint2 w = reinterpret_cast<const uint2 *>((par ? rbuf1 : rbuf0) + (size_t)q * d)[tid];
+                    double a = 0.0;
+                    a = fma(bf16_to_f64((uint16_t)(w.x & 0xFFFFu)), nd[0], a);
+                    a = fma(bf16_to_f64((uint16_t)(w.x >> 16)), nd[1], a);
+                    a = fma(bf16_to_f64((uint16_t)(w.y & 0xFFFFu)), nd[2], a);
+                    a = fma(bf16_to_f64((uint16_t)(w.y >> 16)), nd[3], a);
+                    a = warp_sum_f64(a);
+                    if (lane == 0) s_rp[warp][q] = a;
+                }
             }
         }
-        __syncthreads();
+        if (!__syncthreads_and(alive ? 1 : 0)) break;  // also: limbs and router partials visible
+        if (tid < nr) {
+            double sum = 0.0;
+            for (int w = 0; w < kStackWarps; w++) sum += s_rp[w][tid];
+            const unsigned long long b = (unsigned long long)__double_as_longlong(sum);
+            st_relaxed_v2(p.lb + ((size_t)par * E + e0 + tid) * 2, tagged((uint32_t)(b >> 32), tag),
+                          tagged((uint32_t)b, tag));
+        }
         TSTAMP(l, 2)
-        // router rows (prefetched): each row split over kStackWarps / rb_rows warps
-        if (nr > 0) {
-            const bool okw = mbar_wait(&mb_router, par, lim, p.status);
-            alive = __syncthreads_and(okw ? 1 : 0) && alive;
-            const int wpr = kStackWarps / p.rb_rows;
-            const int rr = warp / wpr, part = warp % wpr;
-            double acc = 0.0;
-            if (rr < nr) {
-                const int per = d / wpr;
-                const uint16_t *wrow = rbuf + (size_t)rr * d + part * per;
-                const uint16_t *nrow = ns + part * per;
-                // bf16 x bf16 has at most 16 significant bits: the product is exact in fp64 and
-                // the fma adds it with one rounding
-                for (int i = lane; i < per; i += 32)
-                    acc = fma((double)bf16_to_f32(wrow[i]), (double)bf16_to_f32(nrow[i]), acc);
+        // predicted logits of the next layer (fp32; used only to choose L2 prefetches)
+        if (p.predict && has_next && nr > 0) {
+            const uint32_t npar = (uint32_t)((l + 1) & 1);
+            const bool okr = mbar_wait(&mb_r[npar], (uint32_t)(((l + 1) >> 1) & 1), lim, p.status);
+            if (!okr) alive = false;
+            const bool okw = __all_sync(0xFFFFFFFFu, okr);  // the shuffles below need the whole warp
+#pragma unroll
+            for (int q = 0; q < kMaxRouterRows; q++) {
+                if (q < nr && okw) {
+                    const uint2 w = reinterpret_cast<const uint2 *>((npar ? rbuf1 : rbuf0) + (size_t)q * d)[tid];
+                    float a = 0.0f;
+                    a = fmaf(__uint_as_float(w.x << 16), nf[0], a);
+                    a = fmaf(__uint_as_float(w.x & 0xFFFF0000u), nf[1], a);
+                    a = fmaf(__uint_as_float(w.y << 16), nf[2], a);
+                    a = fmaf(__uint_as_float(w.y & 0xFFFF0000u), nf[3], a);
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xFFFFFFFFu, a, o);
+                    if (lane == 0) s_pp[warp][q] = a;
+                }
             }
-            acc = warp_sum_f64(acc);
-            if (lane == 0 && rr < nr) s_part[rr][part] = acc;
-            __syncthreads();
-            if (tid < nr) {
-                double sum = 0.0;
-                for (int q = 0; q < wpr; q++) sum += s_part[tid][q];
-                const unsigned long long b = (unsigned long long)__double_as_longlong(sum);
-                const int e = c + tid * P;
-                ll_store(p.lll + 2 * e, (uint32_t)(b >> 32), tag);
-                ll_store(p.lll + 2 * e + 1, (uint32_t)b, tag);
-            }
+        }
+        if (!__syncthreads_and(alive ? 1 : 0)) break;
+        if (p.predict && has_next && tid < nr) {
+            float sum = 0.0f;
+            for (int w = 0; w < kStackWarps; w++) sum += s_pp[w][tid];
+            st_word(p.pb + (size_t)par * E + e0 + tid, __float_as_uint(sum), tag);
+        }
+        // rbuf[par] is free (this layer's rows are used): fetch the rows of layer l + 2 into it
+        if (tid == 0 && nr > 0 && l + 2 < p.n_layers) {
+            mbar_expect_tx(&mb_r[par], (uint32_t)(nr * d * 2));
+            if (par) n_rt1++;
+            else n_rt0++;
+            bulk_g2s(par ? rbuf1 : rbuf0, s_layer[l + 2].router + (size_t)e0 * d, (uint32_t)(nr * d * 2), &mb_r[par]);
         }
         TSTAMP(l, 3)
-        __syncthreads();
-        if (tid == 0 && nr > 0 && l + 1 < p.n_layers) {  // next layer's router rows
-            mbar_expect_tx(&mb_router, (uint32_t)(nr * d * 2));
-            n_rt++;
-            for (int q = 0; q < nr; q++)
-                bulk_g2s(rbuf + (size_t)q * d, s_layer[l + 1].router + (size_t)(c + q * P) * d, (uint32_t)(d * 2),
-                         &mb_router);
-        }
         // ------------------------------------------------------------ B: logits, top-k, copies
-        double my_logit = 0.0;  // logit `tid` (E <= 256 on this path)
         {
-            const bool ok = ll_gather(p.lll, 2 * E, tag, xch, &mb_x, xph, lim, p.status);
+            bool ok = true;
             if (tid < E) {
-                my_logit = __longlong_as_double(
-                    (long long)(((unsigned long long)(uint32_t)xch[2 * tid] << 32) | (uint32_t)xch[2 * tid + 1]));
-                s_logit[tid] = my_logit;
+                ulonglong2 w;
+                ok = poll_pair(p.lb + ((size_t)par * E + tid) * 2, tag, gtimer(), lim, w);
+                lg[tid] = __longlong_as_double((long long)(((unsigned long long)(uint32_t)w.x << 32) | (uint32_t)w.y));
             }
-            alive = __syncthreads_and(ok ? 1 : 0) && alive;
+            if (!__syncthreads_and(ok ? 1 : 0)) {
+                set_status(p.status, TERN_ETIMEOUT);
+                alive = false;
+                break;
+            }
         }
         TSTAMP(l, 4)
-        // only the expert indices are on the critical path; the gates are needed in the combine
-        block_topk_select(my_logit, E, k, s_idx, s_gm, &s_nc, s_cand);
-        TSTAMP(l, 5)
         if (warp == 0) {
-            // copies: lanes 0..3 first-half gate/up segments, 4..7 second half (each half spans
-            // at most two slots x two matrices), lanes 8.. down rows of slot lane-8
-            const uint32_t rowb = (uint32_t)(d / 4), rowd = (uint32_t)(f / 4);
-            if (lane < 8) {
-                const int half = lane >> 2, seg = (lane >> 1) & 1;
-                const int h0 = p0 + (half ? n0 : 0), h1 = half ? p1 : p0 + n0;  // pairs of this half
-                const int s0 = h0 / f;
-                const int e0 = min(h1, (s0 + 1) * f);
-                const int a = seg == 0 ? h0 : e0, b = seg == 0 ? e0 : h1;
-                if (b > a) {
-                    const int s = a / f, j = a % f;
-                    const size_t src = ((size_t)s_idx[s] * f + j) * rowb;
-                    const int q0 = a - p0;
-                    uint64_t *mb = half ? &mb_gu1 : &mb_gu0;
-                    if (lane & 1) bulk_g2s(ubuf + (size_t)q0 * rowb, Ly.up + src, (uint32_t)(b - a) * rowb, mb);
-                    else bulk_g2s(gbuf + (size_t)q0 * rowb, Ly.gate + src, (uint32_t)(b - a) * rowb, mb);
+            warp_topk_filter(lg, E, k, s_idx, cand);
+            // copies of expert idx[s]: first gate/up chunk, second chunk, down rows; thread 0
+            // registers the byte counts first (counted here, so only issued phases are drained)
+            if (lane == 0) {
+                mbar_expect_tx(&mb_gu0, (uint32_t)(2 * n0 * (d / 4)));
+                mbar_expect_tx(&mb_gu1, (uint32_t)(2 * n1 * (d / 4)));
+                mbar_expect_tx(&mb_dn, (uint32_t)(ndn * (f / 4)));
+                n_gu++;
+                n_dn++;
+            }
+            __syncwarp();
+            if (lane < 5) {
+                const size_t e = (size_t)s_idx[s];
+                const uint32_t rowg = (uint32_t)(d / 4), rowd = (uint32_t)(f / 4);
+                if (lane == 0 && n0 > 0) bulk_g2s(gbuf, Ly.gate + (e * f + j0) * rowg, (uint32_t)n0 * rowg, &mb_gu0);
+                if (lane == 1 && n0 > 0) bulk_g2s(ubuf, Ly.up + (e * f + j0) * rowg, (uint32_t)n0 * rowg, &mb_gu0);
+                if (lane == 2 && n1 > 0)
+                    bulk_g2s(gbuf + (size_t)n0 * rowg, Ly.gate + (e * f + j0 + n0) * rowg, (uint32_t)n1 * rowg, &mb_gu1);
+                if (lane == 3 && n1 > 0)
+                    bulk_g2s(ubuf + (size_t)n0 * rowg, Ly.up + (e * f + j0 + n0) * rowg, (uint32_t)n1 * rowg, &mb_gu1);
+                if (lane == 4 && ndn > 0) bulk_g2s(dbuf, Ly.down + (e * d + i0) * rowd, (uint32_t)ndn * rowd, &mb_dn);
+            }
+        }
+        __syncthreads();
+        TSTAMP(l, 5)
+        if (warp == 1) {
+            // the scales of this CTA's rows (read while the rows travel)
+            const size_t e = (size_t)s_idx[s];
+            for (int q = lane; q < ngu; q += 32) {
+                s_sg[q] = __ldg(Ly.sg + e * f + j0 + q);
+                s_su[q] = __ldg(Ly.su + e * f + j0 + q);
+            }
+            for (int q = lane; q < ndn; q += 32) s_sd[q] = __ldg(Ly.sd + e * d + i0 + q);
+        } else if (warp == 2) {
+            warp_topk_gates(lg, k, s_idx, s_gate, nullptr);
+            __syncwarp();
+            if (lane < k && pid == 0) {
+                p.idx_hist[l * k + lane] = s_idx[lane];
+                p.gate_hist[l * k + lane] = s_gate[lane];
+            }
+        } else if (warp == 3 && p.predict && has_next) {
+            // predicted experts of the next layer -> L2 prefetch of this CTA's rows of
+            // predictions s and s + 8 (what it would copy if one of them lands in its slot)
+            bool ok = true;
+            const unsigned long long t0 = gtimer();
+            for (int e = lane; e < E; e += 32) {
+                unsigned long long w;
+                while (true) {
+                    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(p.pb + (size_t)par * E + e) : "memory");
+                    if ((uint32_t)(w >> 32) == tag) break;
+                    if ((long long)(gtimer() - t0) > lim) {
+                        ok = false;
+                        break;
+                    }
                 }
-            } else if (lane < 8 + k && nrows > 0) {
-                const int s = lane - 8;
-                bulk_g2s(dbuf + (size_t)s * p.dn_rows * rowd, Ly.down + ((size_t)s_idx[s] * d + i0) * rowd,
-                         (uint32_t)nrows * rowd, &mb_dn);
+                plg[e] = (double)__uint_as_float((uint32_t)w);
+                if (!ok) break;
             }
-        } else {
-            // per-row scales of this CTA's rows, fetched while the copies are in flight
-            for (int q = tid - 32; q < p1 - p0; q += kStackThreads - 32) {
-                const int pp = p0 + q, s2 = pp / f, j = pp % f;
-                const size_t o = (size_t)s_idx[s2] * f + j;
-                s_sg[q] = __ldg(Ly.sg + o);
-                s_su[q] = __ldg(Ly.su + o);
-            }
-            for (int q = tid - 32; q < k * nrows; q += kStackThreads - 32)
-                s_sd[q] = __ldg(Ly.sd + (size_t)s_idx[q / nrows] * d + i0 + q % nrows);
-            if (warp == kStackWarps - 1) {
-                warp_topk_gates(s_logit, k, s_idx, s_gate, nullptr);
-                __syncwarp();
-                if (lane < k && c == 0) {
-                    p.idx_hist[l * k + lane] = s_idx[lane];
-                    p.gate_hist[l * k + lane] = s_gate[lane];
+            // a missing prediction only skips the prefetch (the real exchanges decide timeouts)
+            if (__all_sync(0xFFFFFFFFu, ok)) {
+                const int np = E < kPredTop ? E : kPredTop;
+                warp_topk_filter(plg, E, np, s_pidx, cand);
+                const StackLayerDev &Ln = s_layer[l + 1];
+                const uint32_t rowg = (uint32_t)(d / 4), rowd = (uint32_t)(f / 4);
+                for (int q = s; q < np; q += kSK) {
+                    const size_t e = (size_t)s_pidx[q];
+                    if (lane == 0 && ngu > 0) prefetch_l2_bulk(Ln.gate + (e * f + j0) * rowg, (uint32_t)ngu * rowg);
+                    if (lane == 1 && ngu > 0) prefetch_l2_bulk(Ln.up + (e * f + j0) * rowg, (uint32_t)ngu * rowg);
+                    if (lane == 2 && ndn > 0) prefetch_l2_bulk(Ln.down + (e * d + i0) * rowd, (uint32_t)ndn * rowd);
+                    if (lane == 3) asm volatile("prefetch.global.L2 [%0];" ::"l"(Ln.sg + e * f + j0));
+                    if (lane == 4) asm volatile("prefetch.global.L2 [%0];" ::"l"(Ln.su + e * f + j0));
+                    if (lane >= 5 && lane < 9 && 32 * (lane - 5) < ndn)
+                        asm volatile("prefetch.global.L2 [%0];" ::"l"(Ln.sd + e * d + i0 + 32 * (lane - 5)));
                 }
             }
         }
-        TSTAMP(l, 6)
         // ------------------------------------------------------------ C: gate/up -> h
-        if (p1 > p0) {
-            // activation limbs of this lane's segment (G = d/64 = 32 lanes per row)
+        {
+            // activation limbs of this lane's segment (d / 64 = 32 segments: lane = segment)
             SegX<NL> X;
-            seg_load_x_padded<NL>(X, xl, xlp, lane % (d / 64));
-            const uint32_t lane4 = (uint32_t)lane << 2;
+            seg_load_x_padded<NL>(X, xl, xlp, lane);
             const int rowb = d / 4;
             for (int half = 0; half < 2; half++) {
-                const int qa = half ? n0 : 0, qb = half ? npairs : n0;
-                if (qb <= qa) break;
+                const int qa = half ? n0 : 0, qb = half ? ngu : n0;
+                if (qb <= qa) continue;
                 const bool okw = mbar_wait(half ? &mb_gu1 : &mb_gu0, par, lim, p.status);
-                alive = __syncthreads_and(okw ? 1 : 0) && alive;
-                if (half == 0) TSTAMP(l, 7)
-                for (int q = qa + warp; q < qb; q += kStackWarps) {
+                if (!__syncthreads_and(okw ? 1 : 0)) {
+                    alive = false;
+                    break;
+                }
+                if (half == 0) TSTAMP(l, 6)
+                const int q = qa + warp;
+                if (q < qb) {
                     const uint4 wg = *reinterpret_cast<const uint4 *>(gbuf + (size_t)q * rowb + lane * 16);
                     const uint4 wu = *reinterpret_cast<const uint4 *>(ubuf + (size_t)q * rowb + lane * 16);
                     int ag[NL], au[NL];
 #pragma unroll
                     for (int z = 0; z < NL; z++) ag[z] = au[z] = 0;
-                    seg_dot<NL>(wg, X, lut, lane4, ag);
-                    seg_dot<NL>(wu, X, lut, lane4, au);
+                    seg_dot_alu<NL>(wg, X, ag);
+                    seg_dot_alu<NL>(wu, X, au);
                     int ga, gb2, ua, ub;
-                    acc_to_pair<NL>(ag, ga, gb2);
-                    acc_to_pair<NL>(au, ua, ub);
+                    acc_to_pair_x64<NL>(ag, ga, gb2);
+                    acc_to_pair_x64<NL>(au, ua, ub);
                     ga = group_sum<32>(ga);
                     ua = group_sum<32>(ua);
                     if (NL > 1) {
@@ -492,160 +543,179 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                     }
                 }
             }
-            __syncthreads();
-            TSTAMP(l, 8)
-            // SwiGLU epilogue, one thread per row, fp64
-            if (tid < p1 - p0) {
-                const int q = tid, pp = p0 + q, s = pp / f, j = pp % f;
-                const long long Sg = s_S[q][0], Su = s_S[q][1];
-                float hv;
-                if (NL == 1) {
-                    const float gv = __fmul_rn(__fmul_rn(__int2float_rn((int)Sg), s_sg[q]), s_nq);
-                    const float uv = __fmul_rn(__fmul_rn(__int2float_rn((int)Su), s_su[q]), s_nq);
-                    hv = swiglu_f32((double)gv, (double)uv);
-                } else {
-                    hv = swiglu_f32(ldexp((double)Sg, -sh_n) * (double)s_sg[q], ldexp((double)Su, -sh_n) * (double)s_su[q]);
-                }
-                ll_store(p.hll + (size_t)s * f + j, __float_as_uint(hv), tag);
+            if (!alive) break;
+        }
+        __syncthreads();
+        TSTAMP(l, 7)
+        // SwiGLU epilogue, one thread per row, fp64
+        if (tid < ngu) {
+            const int q = tid;
+            const long long Sg = s_S[q][0], Su = s_S[q][1];
+            float h;
+            if (NL == 1) {
+                const float gv = __fmul_rn(__fmul_rn(__int2float_rn((int)Sg), s_sg[q]), s_nq);
+                const float uv = __fmul_rn(__fmul_rn(__int2float_rn((int)Su), s_su[q]), s_nq);
+                h = swiglu_f32((double)gv, (double)uv);
+            } else {
+                h = swiglu_f32(ldexp((double)Sg, -sh_n) * (double)s_sg[q], ldexp((double)Su, -sh_n) * (double)s_su[q]);
+            }
+            st_word(p.hb + ((size_t)par * k + s) * f + j0 + q, __float_as_uint(h), tag);
+            p.h_hist[((size_t)l * k + s) * f + j0 + q] = h;
+        }
+        TSTAMP(l, 8)
+        // ------------------------------------------------------------ D: down, combine, residual
+        {
+            bool ok = true;
+            float m = 0.0f;
+            // the test hook makes CTA 0 wait for a tag no producer writes (bounded wait)
+            const uint32_t htag = (l == p.stall_layer && pid == 0) ? (tag ^ 0x40000000u) : tag;
+            if (2 * tid < f) {
+                ulonglong2 w;
+                ok = poll_pair(p.hb + ((size_t)par * k + s) * f + 2 * tid, htag, gtimer(), lim, w);
+                const float h0 = __uint_as_float((uint32_t)w.x), h1 = __uint_as_float((uint32_t)w.y);
+                hv[2 * tid] = h0;
+                hv[2 * tid + 1] = h1;
+                m = fmaxf(fabsf(h0), fabsf(h1));
+            }
+            m = warp_max_f32(m);
+            if (lane == 0) s_hmax[warp] = m;
+            if (!__syncthreads_and(ok ? 1 : 0)) {
+                set_status(p.status, TERN_ETIMEOUT);
+                alive = false;
+                break;
             }
         }
         TSTAMP(l, 9)
-        // ------------------------------------------------------------ D: down, combine, residual
-        {
-            // Each slot is owned by wps = 16/k warps.  They fetch that slot's h (f tagged words)
-            // with one TMA copy, agree on its tags over a per-slot hardware barrier, build its
-            // limbs and run their down rows -- without waiting for the other slots.
-            const int G = f / 64;
-            const int rpp = 32 / G;
-            const int wps = kStackWarps / k;
-            const int sl = warp / wps, wi = warp % wps;
-            const int nthr = wps * 32;
-            const int bar_id = 1 + sl;
-            unsigned long long *hb = xch + (size_t)sl * f;
-            const int share = f / wps;  // words of the slot this warp checks and converts
-            bool okg = true;
-            {
-                const unsigned long long t0 = gtimer();
-                while (true) {
-                    if (wi == 0 && lane == 0) {
-                        mbar_expect_tx(&mb_h[sl], (uint32_t)(f * 8));
-                        bulk_g2s(hb, p.hll + (size_t)sl * f, (uint32_t)(f * 8), &mb_h[sl]);
-                        s_hissued[sl]++;
-                    }
-                    const bool landed = mbar_wait(&mb_h[sl], hph & 1u, lim, p.status);
-                    hph++;
-                    int mine = landed ? 1 : 0;
-                    for (int w = wi * share + lane; w < (wi + 1) * share; w += 32)
-                        if ((uint32_t)(hb[w] >> 32) != tag) mine = 0;
-                    mine = __all_sync(0xFFFFFFFFu, mine);
-                    if (lane == 0) s_hok[sl][wi] = mine;
-                    named_bar_sync(bar_id, nthr);
-                    int all = 1;
-                    for (int q = 0; q < wps; q++) all &= s_hok[sl][q];
-                    if (wi == 0 && lane == 0) s_hlate[sl] = (!all) && ((long long)(gtimer() - t0) > lim);
-                    named_bar_sync(bar_id, nthr);
-                    if (all) break;
-                    if (s_hlate[sl]) {
-                        set_status(p.status, TERN_ETIMEOUT);
-                        okg = false;
-                        break;
-                    }
-                }
-            }
-            // slot absmax -> shift (bf16 path) or scale (int8 path); identical in the slot's warps
-            float m = 0.0f;
-            for (int w = wi * share + lane; w < (wi + 1) * share; w += 32)
-                m = fmaxf(m, fabsf(__uint_as_float((uint32_t)hb[w])));
-            m = warp_max_f32(m);
-            if (lane == 0) s_hpart[sl][wi] = m;
-            named_bar_sync(bar_id, nthr);
-            float a = 0.0f;
-            for (int q = 0; q < wps; q++) a = fmaxf(a, s_hpart[sl][q]);
-            const int hsh = (NL == 1) ? 0 : fixed_shift(a);
-            const float hinv = (NL == 1 && a > 0.0f) ? quant_inv(a) : 0.0f;
-            const float hsc = (NL == 1 && a > 0.0f) ? __fdiv_rn(a, 127.0f) : 0.0f;
-            // limb words of this warp's share of the slot (4 values per word)
-            for (int bw = wi * (share / 4) + lane; bw < (wi + 1) * (share / 4); bw += 32) {
-                const float v4[4] = {__uint_as_float((uint32_t)hb[4 * bw]), __uint_as_float((uint32_t)hb[4 * bw + 1]),
-                                     __uint_as_float((uint32_t)hb[4 * bw + 2]), __uint_as_float((uint32_t)hb[4 * bw + 3])};
-                uint32_t wd[3];
-                limb_words<NL>(v4, hsh, hinv, a > 0.0f, wd);
-                hl[((size_t)sl * NL + 0) * hlp + padded_word(bw)] = wd[0];
-                if (NL > 1) {
-                    hl[((size_t)sl * NL + 1) * hlp + padded_word(bw)] = wd[1];
-                    hl[((size_t)sl * NL + 2) * hlp + padded_word(bw)] = wd[2];
-                }
-            }
-            named_bar_sync(bar_id, nthr);
-            if (warp == 0) TSTAMP(l, 10)
-            if (nrows > 0 && !mbar_wait(&mb_dn, par, lim, p.status)) okg = false;
-            if (warp == 0) TSTAMP(l, 11)
-            if (warp == 0) TSTAMP(l, 12)
-            // down rows of this slot: G lanes per row, rpp rows per warp pass
-            {
-                const int sub = lane / G, gl = lane % G;
-                const uint32_t lane4 = (uint32_t)lane << 2;
-                SegX<NL> Hx;
-                seg_load_x_padded<NL>(Hx, hl + (size_t)sl * NL * hlp, hlp, gl);
-                for (int r0 = wi * rpp; r0 < nrows; r0 += wps * rpp) {
-                    const int rrow = r0 + sub;
-                    const bool valid = rrow < nrows;
-                    int acc[NL];
+        float ha = 0.0f;
 #pragma unroll
-                    for (int z = 0; z < NL; z++) acc[z] = 0;
-                    const uint4 wd = *reinterpret_cast<const uint4 *>(
-                        dbuf + ((size_t)sl * p.dn_rows + (valid ? rrow : 0)) * (f / 4) + gl * 16);
-                    seg_dot<NL>(wd, Hx, lut, lane4, acc);
-                    int aa, bb;
-                    acc_to_pair<NL>(acc, aa, bb);
-                    for (int o = G / 2; o > 0; o >>= 1) {
-                        aa += __shfl_xor_sync(0xFFFFFFFFu, aa, o);
-                        if (NL > 1) bb += __shfl_xor_sync(0xFFFFFFFFu, bb, o);
-                    }
-                    if (valid && gl == 0) {
-                        const long long S = pair_value(NL, aa, bb);
-                        const float sd = s_sd[sl * nrows + rrow];
-                        double v;
-                        if (NL == 1) v = (double)__fmul_rn(__fmul_rn(__int2float_rn((int)S), sd), hsc);
-                        else v = ldexp((double)S, -hsh) * (double)sd;
-                        s_ye[rrow][sl] = v;
-                    }
+        for (int w = 0; w < kStackWarps; w++) ha = fmaxf(ha, s_hmax[w]);
+        const int hsh = (NL == 1) ? 0 : fixed_shift(ha);
+        const float hsc = (NL == 1 && ha > 0.0f) ? __fdiv_rn(ha, 127.0f) : 0.0f;
+        if (4 * tid < f) {
+            const float v4[4] = {hv[4 * tid], hv[4 * tid + 1], hv[4 * tid + 2], hv[4 * tid + 3]};
+            const float hinv = (NL == 1 && ha > 0.0f) ? quant_inv(ha) : 0.0f;
+            store_limbs4<NL>(hl, hlp, tid, v4, hsh, hinv, ha > 0.0f);
+        }
+        __syncthreads();
+        TSTAMP(l, 10)
+        if (ndn > 0 && !mbar_wait(&mb_dn, par, lim, p.status)) alive = false;
+        if (!__syncthreads_and(alive ? 1 : 0)) break;
+        TSTAMP(l, 11)
+        // down rows: Gf = f / 64 lanes per row, 32 / Gf rows per warp pass
+        {
+            const int Gf = f / 64;
+            const int rpp = 32 / Gf;
+            const int sub = lane / Gf, gl = lane % Gf;
+            SegX<NL> Hx;
+            seg_load_x_padded<NL>(Hx, hl, hlp, gl);
+            const uint32_t ytag = tag;
+            for (int r0 = warp * rpp; r0 < ndn; r0 += kStackWarps * rpp) {
+                const int rr = r0 + sub;
+                const bool valid = rr < ndn;
+                int acc[NL];
+#pragma unroll
+                for (int z = 0; z < NL; z++) acc[z] = 0;
+                const uint4 wd = *reinterpret_cast<const uint4 *>(dbuf + (size_t)(valid ? rr : 0) * (f / 4) + gl * 16);
+                seg_dot_alu<NL>(wd, Hx, acc);
+                int aa, bb;
+                acc_to_pair_x64<NL>(acc, aa, bb);
+                for (int o = Gf / 2; o > 0; o >>= 1) {
+                    aa += __shfl_xor_sync(0xFFFFFFFFu, aa, o);
+                    if (NL > 1) bb += __shfl_xor_sync(0xFFFFFFFFu, bb, o);
+                }
+                if (valid && gl == 0) {
+                    const long long S = pair_value(NL, aa, bb);
+                    const float sd = s_sd[rr];
+                    float v;
+                    if (NL == 1) v = __fmul_rn(__fmul_rn(__int2float_rn((int)S), sd), hsc);
+                    else v = (float)(ldexp((double)S, -hsh) * (double)sd);
+                    st_word(p.yb + (((size_t)par * G + c) * k + s) * kMaxDN + rr, __float_as_uint(v), ytag);
                 }
             }
-            alive = __syncthreads_and(okg ? 1 : 0) && alive;
-            TSTAMP(l, 13)
-            const bool last = (l + 1 == p.n_layers);
+        }
+        TSTAMP(l, 12)
+        {
+            // the k slots' outputs of rows [i0, i1)
+            bool ok = true;
+            const int half_rows = ndn / 2;
+            const unsigned long long t0 = gtimer();
+            for (int t = tid; t < k * half_rows; t += kStackThreads) {
+                const int q = t / half_rows, w2 = 2 * (t % half_rows);
+                ulonglong2 w;
+                if (!poll_pair(p.yb + (((size_t)par * G + c) * k + q) * kMaxDN + w2, tag, t0, lim, w)) {
+                    ok = false;
+                    break;
+                }
+                yv[q * kMaxDN + w2] = __uint_as_float((uint32_t)w.x);
+                yv[q * kMaxDN + w2 + 1] = __uint_as_float((uint32_t)w.y);
+            }
+            if (!__syncthreads_and(ok ? 1 : 0)) {
+                set_status(p.status, TERN_ETIMEOUT);
+                alive = false;
+                break;
+            }
+        }
+        TSTAMP(l, 13)
+        {
+            const bool last = !has_next;
+            const uint32_t ntag = (ep << 7) | (uint32_t)(l + 2);
+            const uint32_t npar = (uint32_t)((l + 1) & 1);
             // one output row per thread, fixed top-k order; row pairs leave as one word
             uint16_t xo = 0;
-            if (tid < nrows) {
+            double sq = 0.0;
+            float am = 0.0f;
+            if (tid < ndn) {
                 double y = 0.0;
-                for (int q = 0; q < k; q++) y += s_gate[q] * s_ye[tid][q];
+                for (int q = 0; q < k; q++) y += s_gate[q] * (double)yv[q * kMaxDN + tid];
                 const uint16_t yb = f64_to_bf16_rne(y);
                 xo = f64_to_bf16_rne((double)bf16_to_f32(xs[i0 + tid]) + (double)bf16_to_f32(yb));
+                const double xv2 = (double)bf16_to_f32(xo);
+                sq = xv2 * xv2;
+                am = fabsf((float)xv2);
+                if (s == 0) {
+                    p.hist[(size_t)(l + 1) * d + i0 + tid] = xo;
+                    p.y_hist[(size_t)l * d + i0 + tid] = (float)y;
+                    if (last) p.x[i0 + tid] = xo;
+                }
             }
             const uint32_t other = __shfl_down_sync(0xFFFFFFFFu, (uint32_t)xo, 1);
-            if (tid < nrows && (tid & 1) == 0) {
-                const uint32_t pr = (uint32_t)xo | (other << 16);
-                const int i = i0 + tid;
-                reinterpret_cast<uint32_t *>(p.hist + (size_t)(l + 1) * d)[i / 2] = pr;
-                if (last) reinterpret_cast<uint32_t *>(p.x)[i / 2] = pr;
-                else ll_store(p.xll + i / 2, pr, (ep << 7) | (uint32_t)(l + 2));
+            if (!last && tid < ndn && (tid & 1) == 0)
+                st_word(p.xb + ((size_t)npar * k + s) * (d / 2) + (i0 + tid) / 2, (uint32_t)xo | (other << 16), ntag);
+            if (!last) {
+                // sum of squares and absmax of this part (threads < ndn <= kMaxDN = 128: warps 0..3)
+                sq = warp_sum_f64(sq);
+                am = warp_max_f32(am);
+                if (lane == 0) {
+                    s_red[warp] = sq;
+                    s_redf[warp] = am;
+                }
+                __syncthreads();
+                if (tid == 0) {
+                    double ts = 0.0;
+                    float ta = 0.0f;
+                    for (int w = 0; w < (ndn + 31) / 32; w++) {
+                        ts += s_red[w];
+                        ta = fmaxf(ta, s_redf[w]);
+                    }
+                    const unsigned long long b = (unsigned long long)__double_as_longlong(ts);
+                    unsigned long long *dst = p.xst + (((size_t)npar * k + s) * G + c) * 4;
+                    st_relaxed_v2(dst, tagged((uint32_t)(b >> 32), ntag), tagged((uint32_t)b, ntag));
+                    st_relaxed_v2(dst + 2, tagged(__float_as_uint(ta), ntag), tagged(0u, ntag));
+                }
             }
-            TSTAMP(l, 14)
         }
+        TSTAMP(l, 14)
     }
 #undef TSTAMP
     // after a timeout, let this CTA's own copies in flight land (bounded) before leaving
     if (!alive && tid == 0) {
-        if (n_rt) mbar_wait(&mb_router, (n_rt - 1) & 1u, lim, p.status);
+        if (n_rt0) mbar_wait(&mb_r[0], (n_rt0 - 1) & 1u, lim, p.status);
+        if (n_rt1) mbar_wait(&mb_r[1], (n_rt1 - 1) & 1u, lim, p.status);
         if (n_gu) {
             mbar_wait(&mb_gu0, (n_gu - 1) & 1u, lim, p.status);
             mbar_wait(&mb_gu1, (n_gu - 1) & 1u, lim, p.status);
         }
         if (n_dn) mbar_wait(&mb_dn, (n_dn - 1) & 1u, lim, p.status);
-        if (xph) mbar_wait(&mb_x, (xph - 1) & 1u, lim, p.status);
-        for (int q = 0; q < kSK; q++)
-            if (s_hissued[q]) mbar_wait(&mb_h[q], (s_hissued[q] - 1) & 1u, lim, p.status);
     }
     // leave: the last CTA out advances the launch epoch (the next launch's tags differ)
     __syncthreads();
@@ -660,10 +730,9 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
 }
 
 // ------------------------------------------------------------------ host side
-// Persistent-path workspace: barrier words, logits [E], H [k][f], x history
-// [(kMaxStackLayers+1)][d], routing history [kMaxStackLayers][k] (int32 + fp64).
+// Persistent-path workspace: control words, exchange buffers, per-layer record, trace.
 struct StackWs {
-    int64_t ctl, xll, lll, hll, hist, idx_hist, gate_hist, ttrace, total;
+    int64_t ctl, xb, xst, lb, pb, hb, yb, hist, idx_hist, gate_hist, y_hist, h_hist, ttrace, total;
 };
 
 static inline int64_t up256_(int64_t v) { return (v + 255) & ~int64_t(255); }
@@ -676,14 +745,20 @@ static StackWs stack_ws_layout(const tern_moe_layer *L0) {
         p = up256_(p + b);
         return r;
     };
+    const int64_t d = L0->d, f = L0->f, E = L0->E, k = L0->k;
     o.ctl = take(256);
-    o.xll = take((int64_t)L0->d / 2 * 8);
-    o.lll = take((int64_t)L0->E * 2 * 8);
-    o.hll = take((int64_t)L0->k * L0->f * 8);
-    o.hist = take((int64_t)(kMaxStackLayers + 1) * L0->d * 2);
-    o.idx_hist = take((int64_t)kMaxStackLayers * L0->k * 4);
-    o.gate_hist = take((int64_t)kMaxStackLayers * L0->k * 8);
-    o.ttrace = take((int64_t)2 * kMaxStackLayers * kMaxTraceCtas * 16 * 8);
+    o.xb = take(2 * k * (d / 2) * 8);
+    o.xst = take(2 * k * kMaxGroup * 4 * 8);
+    o.lb = take(2 * E * 2 * 8);
+    o.pb = take(2 * E * 8);
+    o.hb = take(2 * k * f * 8);
+    o.yb = take(2 * kMaxGroup * k * kMaxDN * 8);
+    o.hist = take((int64_t)(kMaxLayers + 1) * d * 2);
+    o.idx_hist = take((int64_t)kMaxLayers * k * 4);
+    o.gate_hist = take((int64_t)kMaxLayers * k * 8);
+    o.y_hist = take((int64_t)kMaxLayers * d * 4);
+    o.h_hist = take((int64_t)kMaxLayers * k * f * 4);
+    o.ttrace = take((int64_t)2 * kMaxLayers * kMaxTraceCtas * kTracePoints * 8);
     o.total = p;
     return o;
 }
@@ -691,11 +766,13 @@ static StackWs stack_ws_layout(const tern_moe_layer *L0) {
 size_t stack_persistent_ws_bytes(const tern_moe_layer *L0) { return (size_t)stack_ws_layout(L0).total; }
 
 void stack_persistent_offsets(const tern_moe_layer *L0, int64_t *hist, int64_t *idx_hist, int64_t *gate_hist,
-                              int64_t *ttrace) {
+                              int64_t *y_hist, int64_t *h_hist, int64_t *ttrace) {
     const StackWs o = stack_ws_layout(L0);
     *hist = o.hist;
     *idx_hist = o.idx_hist;
     *gate_hist = o.gate_hist;
+    *y_hist = o.y_hist;
+    *h_hist = o.h_hist;
     *ttrace = o.ttrace;
 }
 
@@ -707,35 +784,38 @@ static int sm_count() {
 }
 
 struct StackPlan {
-    int P, rb_rows, gu_pairs, dn_rows;
+    int P, G;
     SmemMap sm;
     const void *fn;
 };
 
 static tern_status stack_plan(const tern_moe_layer &L0, int n_layers, tern_act act, StackPlan &pl) {
-    if (n_layers > kMaxStackLayers || L0.d != 2048 || L0.k > kSK || L0.f % 64 || L0.f > 2048) return TERN_EUNSUPPORTED;
-    const int64_t g = L0.f / 64;
-    if ((g & (g - 1)) != 0) return TERN_EUNSUPPORTED;
-    pl.P = sm_count();
-    if (pl.P <= 0) return TERN_ECUDA;
-    if (pl.P > kMaxTraceCtas) pl.P = kMaxTraceCtas;
-    pl.rb_rows = (L0.E + pl.P - 1) / pl.P;
-    pl.gu_pairs = (int)((L0.k * L0.f + pl.P - 1) / pl.P);
-    pl.dn_rows = 2 * (int)((L0.d / 2 + pl.P - 1) / pl.P);
-    // the thread mappings assume d = 4 * threads and k * f = 8 * threads at most, and a CTA's
-    // gate/up pairs spanning at most two slots
-    if (pl.rb_rows > kStackWarps || pl.dn_rows > 64 || pl.gu_pairs > 64 || pl.gu_pairs > L0.f ||
-        L0.k * L0.f > 8 * kStackThreads || (L0.k * L0.f) % 8 || L0.d != 4 * kStackThreads || L0.E > 256 || kStackWarps % L0.k)
+    const int d = (int)L0.d, f = (int)L0.f, E = L0.E, k = L0.k;
+    // thread mappings: d = 4 * threads; f / 64 segments per down row, a power of two <= 32;
+    // f <= 2 * threads (h gather), E <= 256 (top-k); k <= 8 slot groups
+    if (n_layers > kMaxLayers || d != 4 * kStackThreads || k > kSK || f % 64 || f > 2 * kStackThreads || E > 256)
         return TERN_EUNSUPPORTED;
+    const int gf = f / 64;
+    if (gf < 1 || gf > 32 || (gf & (gf - 1)) != 0) return TERN_EUNSUPPORTED;
+    const int sms = sm_count();
+    if (sms <= 0) return TERN_ECUDA;
+    int G = sms / k;
+    if (G > kMaxGroup) G = kMaxGroup;
+    // shares: <= 32 gate/up rows (two copies of 16), <= 128 down rows, <= 8 router rows per CTA
+    if (G < 1 || (f + G - 1) / G > kMaxGU || 2 * ((d / 2 + G - 1) / G) > kMaxDN) return TERN_EUNSUPPORTED;
+    const int P = k * G;
+    if (P > kMaxTraceCtas || (E + P - 1) / P > kMaxRouterRows) return TERN_EUNSUPPORTED;
+    pl.P = P;
+    pl.G = G;
     const int NL = act == TERN_ACT_INT8 ? 1 : 3;
-    pl.sm = smem_map((int)L0.d, (int)L0.f, L0.k, pl.rb_rows, pl.gu_pairs, pl.dn_rows, NL);
+    pl.sm = smem_map(d, f, k, (f + G - 1) / G, 2 * ((d / 2 + G - 1) / G), (E + P - 1) / P, NL);
     pl.fn = act == TERN_ACT_INT8 ? (const void *)stack_kernel<1> : (const void *)stack_kernel<3>;
     if (cudaFuncSetAttribute(pl.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.sm.total) != cudaSuccess)
         return TERN_ECUDA;
     int nb = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, pl.fn, kStackThreads, pl.sm.total) != cudaSuccess)
         return TERN_ECUDA;
-    if (nb < 1) return TERN_EUNSUPPORTED;
+    if (nb < 1 || nb * sms < P) return TERN_EUNSUPPORTED;
     return TERN_OK;
 }
 
@@ -744,13 +824,18 @@ bool stack_persistent_supported(const tern_moe_layer *L0, int n_layers, tern_act
     return stack_plan(*L0, n_layers, act, pl) == TERN_OK;
 }
 
+int stack_persistent_ctas(const tern_moe_layer *L0, int n_layers, tern_act act) {
+    StackPlan pl;
+    return stack_plan(*L0, n_layers, act, pl) == TERN_OK ? pl.P : 0;
+}
+
 tern_status launch_stack_persistent(const tern_moe_layer *layers, int n_layers, uint16_t *x, float eps, tern_act act,
-                                    void *ws, size_t ws_bytes, int *status, cudaStream_t s) {
+                                    void *ws, size_t ws_bytes, int *status, int stall_layer, long long limit_ns,
+                                    cudaStream_t s) {
     const tern_moe_layer &L0 = layers[0];
     StackPlan pl;
     const tern_status pst = stack_plan(L0, n_layers, act, pl);
     if (pst != TERN_OK) return pst;
-    const int P = pl.P, rb_rows = pl.rb_rows, gu_pairs = pl.gu_pairs, dn_rows = pl.dn_rows;
     const StackWs o = stack_ws_layout(&L0);
     if (ws_bytes < (size_t)o.total) return TERN_EWORKSPACE;
     if (!status) return TERN_ECUDA;
@@ -775,26 +860,31 @@ tern_status launch_stack_persistent(const tern_moe_layer *layers, int n_layers, 
     prm.eps = (double)eps;
     prm.x = x;
     prm.ctl = reinterpret_cast<unsigned int *>(b + o.ctl);
-    prm.xll = reinterpret_cast<unsigned long long *>(b + o.xll);
-    prm.lll = reinterpret_cast<unsigned long long *>(b + o.lll);
-    prm.hll = reinterpret_cast<unsigned long long *>(b + o.hll);
+    prm.xb = reinterpret_cast<unsigned long long *>(b + o.xb);
+    prm.xst = reinterpret_cast<unsigned long long *>(b + o.xst);
+    prm.lb = reinterpret_cast<unsigned long long *>(b + o.lb);
+    prm.pb = reinterpret_cast<unsigned long long *>(b + o.pb);
+    prm.hb = reinterpret_cast<unsigned long long *>(b + o.hb);
+    prm.yb = reinterpret_cast<unsigned long long *>(b + o.yb);
     prm.hist = reinterpret_cast<uint16_t *>(b + o.hist);
     prm.idx_hist = reinterpret_cast<int32_t *>(b + o.idx_hist);
     prm.gate_hist = reinterpret_cast<double *>(b + o.gate_hist);
+    prm.y_hist = reinterpret_cast<float *>(b + o.y_hist);
+    prm.h_hist = reinterpret_cast<float *>(b + o.h_hist);
     // phase stamps cost a %globaltimer read and a store each: only when TERNMOE_TRACE=1
     const char *tenv = getenv("TERNMOE_TRACE");
     prm.ttrace = (tenv && tenv[0] == '1') ? reinterpret_cast<unsigned long long *>(b + o.ttrace) : nullptr;
+    // L2 prefetch of predicted next-layer experts: on unless TERNMOE_PREDICT=0
+    const char *penv = getenv("TERNMOE_PREDICT");
+    prm.predict = (penv && penv[0] == '0') ? 0 : 1;
     prm.status = status;
-    prm.limit_ns = 1000000000ll;  // every in-kernel wait gives up after one second
-    prm.P = P;
-    prm.rb_rows = rb_rows;
-    prm.gu_pairs = gu_pairs;
-    prm.dn_rows = dn_rows;
+    prm.limit_ns = limit_ns;
+    prm.P = pl.P;
+    prm.G = pl.G;
+    prm.stall_layer = stall_layer;
 
-    const SmemMap sm = pl.sm;
-    const void *fn = pl.fn;
     void *args[] = {&prm};
-    const cudaError_t e = cudaLaunchCooperativeKernel(fn, dim3(P), dim3(kStackThreads), args, sm.total, s);
+    const cudaError_t e = cudaLaunchCooperativeKernel(pl.fn, dim3(pl.P), dim3(kStackThreads), args, pl.sm.total, s);
     return e == cudaSuccess ? TERN_OK : TERN_ECUDA;
 }
 

@@ -20,6 +20,7 @@
 #include <stdint.h>
 
 #include "../../include/ternmoe.h"
+#include "decode.cuh"
 
 namespace tern {
 
@@ -46,6 +47,15 @@ __device__ __forceinline__ uint16_t f64_to_bf16_rne(double v) {
     uint32_t u = __float_as_uint(f);
     u += 0x7FFFu + ((u >> 16) & 1u);
     return (uint16_t)(u >> 16);
+}
+
+// bf16 -> fp64 by moving bits (normal values); zero, subnormal, inf and nan go through fp32
+__device__ __forceinline__ double bf16_to_f64(uint16_t b) {
+    const uint32_t e = (b >> 7) & 0xFFu;
+    if (e == 0u || e == 0xFFu) return (double)bf16_to_f32(b);
+    const unsigned long long bits = ((unsigned long long)(b & 0x8000u) << 48) |
+                                    ((unsigned long long)(e + 896u) << 52) | ((unsigned long long)(b & 0x7Fu) << 45);
+    return __longlong_as_double((long long)bits);
 }
 
 // ---------------------------------------------------------------------------- dp4a
@@ -120,6 +130,29 @@ __device__ __forceinline__ void seg_dot(const uint4 wb, const SegX<NL> &x, const
     }
 }
 
+// The same segment dot without a table (decode.cuh): x holds the limbs in position-major
+// order (word 4q+j of limb l = the four activations of position j of packed word q).  Every
+// dp4a term is 64 times a weight-activation product, so acc is 64 times the limb dot; use
+// acc_to_pair_x64 to reduce it.
+template <int NL>
+__device__ __forceinline__ void seg_dot_alu(const uint4 wb, const SegX<NL> &x, int (&acc)[NL]) {
+    const uint32_t words[4] = {wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+    for (int q = 0; q < 4; q++) {
+        const uint32_t sgn = tern_signed_fields(words[q]);
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const uint32_t m = tern_position_lanes(sgn, j);
+            const int bb = 4 * q + j;
+            acc[0] = dp4a_ss(m, x.w[0][bb], acc[0]);
+            if (NL > 1) {
+                acc[1] = dp4a_su(m, x.w[1][bb], acc[1]);
+                acc[2] = dp4a_su(m, x.w[2][bb], acc[2]);
+            }
+        }
+    }
+}
+
 // load the limbs of one segment from a limb-word array laid out [NL][n/4] (u32 words)
 template <int NL>
 __device__ __forceinline__ void seg_load_x(SegX<NL> &x, const uint32_t *limbw, int64_t words_per_limb,
@@ -188,6 +221,18 @@ __device__ __forceinline__ void acc_to_pair(const int (&acc)[NL], int &a, int &b
     } else {
         a = acc[0];
         b = acc[1] * 256 + acc[2];
+    }
+}
+
+// acc_to_pair for accumulators of seg_dot_alu (64 times the limb dot; exact shift)
+template <int NL>
+__device__ __forceinline__ void acc_to_pair_x64(const int (&acc)[NL], int &a, int &b) {
+    if (NL == 1) {
+        a = acc[0] >> 6;
+        b = 0;
+    } else {
+        a = acc[0] >> 6;
+        b = (acc[1] >> 6) * 256 + (acc[2] >> 6);
     }
 }
 
@@ -395,6 +440,59 @@ __device__ __forceinline__ void block_topk_select(double mine, int E, int k, int
     __syncthreads();
 }
 
+// One warp selects the top k (k <= 8) of E <= 256 fp64 logits held in shared memory `lg`:
+// larger logit first, equal logits by lower index.  Lane l owns experts l, l+32, ..., l+224.
+//  1. h = high word of each order key (sign, exponent, 20 leading mantissa bits); each lane
+//     takes the largest h of its eight;
+//  2. tau = the k-th largest lane maximum (lanes ordered by maximum, then lane number).  At
+//     least k logits have h >= tau, and a logit with h < tau is below at least k others, so the
+//     k best logits all have h >= tau;
+//  3. the logits with h >= tau (typically a few more than k) are compacted into `cand`;
+//  4. each candidate's rank = the number of candidates ordered before it (full 64-bit key, then
+//     index); ranks below k land in idx_out.
+// cand: shared scratch of 256 entries; idx_out: shared memory.  No CTA barrier: only the
+// calling warp takes part, and it ends with __syncwarp.
+__device__ __forceinline__ void warp_topk_filter(const double *lg, int E, int k, int32_t *idx_out,
+                                                 ulonglong2 *cand) {
+    const int lane = threadIdx.x & 31;
+    unsigned long long key[8];
+    uint32_t m = 0;
+#pragma unroll
+    for (int j = 0; j < 8; j++) {
+        const int e = lane + 32 * j;
+        key[j] = e < E ? f64_order_key(lg[e]) : 0ull;  // 0 = below every finite logit
+        m = max(m, (uint32_t)(key[j] >> 32));
+    }
+    int above = 0;
+#pragma unroll
+    for (int i = 0; i < 32; i++) {
+        const uint32_t v = __shfl_sync(0xFFFFFFFFu, m, i);
+        above += (v > m || (v == m && i < lane)) ? 1 : 0;
+    }
+    const unsigned who = __ballot_sync(0xFFFFFFFFu, above == k - 1);
+    const uint32_t tau = __shfl_sync(0xFFFFFFFFu, m, __ffs(who) - 1);
+    int nc = 0;
+#pragma unroll
+    for (int j = 0; j < 8; j++) {
+        const int e = lane + 32 * j;
+        const bool take = e < E && (uint32_t)(key[j] >> 32) >= tau;
+        const unsigned mask = __ballot_sync(0xFFFFFFFFu, take);
+        if (take) cand[nc + __popc(mask & ((1u << lane) - 1u))] = make_ulonglong2(key[j], (unsigned long long)e);
+        nc += __popc(mask);
+    }
+    __syncwarp();
+    for (int i = lane; i < nc; i += 32) {
+        const ulonglong2 me = cand[i];
+        int r = 0;
+        for (int q = 0; q < nc; q++) {
+            const ulonglong2 o = cand[q];
+            r += (o.x > me.x || (o.x == me.x && o.y < me.y)) ? 1 : 0;
+        }
+        if (r < k) idx_out[r] = (int)me.y;
+    }
+    __syncwarp();
+}
+
 // Renormalised gates of the selected experts: g_i = exp(l_i - l_0) / sum_j exp(l_j - l_0),
 // lanes 0..k-1 each one exp in fp64, the sum taken in top-k order.
 __device__ __forceinline__ void warp_topk_gates(const double *lg, int k, const int32_t *idx, double *g64, float *g32) {
@@ -402,11 +500,8 @@ __device__ __forceinline__ void warp_topk_gates(const double *lg, int k, const i
     const double my_l = (lane < k) ? lg[idx[lane]] : 0.0;
     const double l0 = __shfl_sync(0xFFFFFFFFu, my_l, 0);
     const double ev = (lane < k) ? exp(my_l - l0) : 0.0;
-    double evs[8];
-#pragma unroll
-    for (int r = 0; r < 8; r++) evs[r] = __shfl_sync(0xFFFFFFFFu, ev, r);
     double z = 0.0;
-    for (int r = 0; r < k; r++) z += evs[r];
+    for (int r = 0; r < k; r++) z += __shfl_sync(0xFFFFFFFFu, ev, r);  // top-k order
     if (lane < k) {
         const double g = ev / z;
         if (g64) g64[lane] = g;

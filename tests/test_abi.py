@@ -1,6 +1,7 @@
 """The C-ABI library: it loads without a GPU, exports every function the header declares,
 and rejects bad arguments on the host before touching CUDA."""
 import ctypes
+import os
 
 import pytest
 
@@ -13,7 +14,7 @@ def test_library_exports_every_header_function():
     L = tm.lib()
     for n in names:
         assert hasattr(L, n), n
-    assert tm.abi_version() == 1
+    assert tm.abi_version() == 2
 
 
 def test_status_strings():
@@ -167,3 +168,16 @@ def test_route_binding_rejects_wrong_shapes():
             fn(Wg, x, 8, idx=torch.zeros((2, 4), dtype=torch.int32))               # idx [T][k]
         with pytest.raises(ValueError):
             fn(Wg, x, 8, gates=torch.zeros((1, 8), dtype=torch.float32))           # gates [T][k]
+
+
+def test_table_free_decode_matches_the_code_table(tmp_path):
+    """The integer-logic decode of the fused kernels (csrc/decode.cuh), compiled for the host:
+    every byte value, byte position and code position gives 64 * w with w the code's weight
+    (11 reads as 0), and the position-major segment dot equals the plain sum."""
+    import subprocess
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    exe = str(tmp_path / "decode_check")
+    subprocess.check_call(["g++", "-O2", "-std=c++17", "-o", exe, os.path.join(root, "tests", "decode_check.cpp")])
+    out = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0 and "decode ok" in out.stdout, out.stdout + out.stderr
