@@ -222,19 +222,25 @@ PHASES = [("x_wait", 0, 1), ("norm_router", 1, 2), ("predict_next", 2, 3), ("log
           ("y_wait", 12, 13), ("combine", 13, 14)]
 
 
-def phase_summary(tr, clk=None, mhz=1965.0):
+def phase_summary(tr, clk=None, mhz=1965.0, k=8):
     """Median over CTAs and layers of each phase (us; from SM clock stamps when given, else
-    from %globaltimer), the exchange latencies, and the layer time."""
+    from %globaltimer), the exchange latencies, and the layer time.  CTA p is part p % G of
+    slot group p // G (G = P / k)."""
     if clk is not None:
         d = lambda a, b: np.median((clk[:, :, b] - clk[:, :, a]).astype(np.float64)) / mhz
     else:
         d = lambda a, b: np.median((tr[:, :, b] - tr[:, :, a]).astype(np.float64)) / 1e3
     out = {name: round(float(d(a, b)), 3) for name, a, b in PHASES}
-    # exchange latency: last producer's publish -> first consumer's receipt
+    L, P, _ = tr.shape
+    G = P // k
+    by_slot = tr.reshape(L, k, G, -1)            # [layer, slot group, part, stamp]
+    by_part = by_slot.transpose(0, 2, 1, 3)      # [layer, part, slot, stamp]
+    # exchange latency: last producer's publish -> first consumer's receipt, within the group
+    # that exchanges (all CTAs for the logits, a slot group for h and x, a part for y)
     e_log = np.median(tr[:, :, 4].min(1) - tr[:, :, 2].max(1)) / 1e3
-    e_h = np.median(tr[:, :, 9].min(1) - tr[:, :, 8].max(1)) / 1e3
-    e_y = np.median(tr[:, :, 13].min(1) - tr[:, :, 12].max(1)) / 1e3
-    e_x = np.median(tr[1:, :, 1].min(1) - tr[:-1, :, 14].max(1)) / 1e3
+    e_h = np.median(by_slot[:, :, :, 9].min(2) - by_slot[:, :, :, 8].max(2)) / 1e3
+    e_y = np.median(by_part[:, :, :, 13].min(2) - by_part[:, :, :, 12].max(2)) / 1e3
+    e_x = np.median(by_slot[1:, :, :, 1].min(2) - by_slot[:-1, :, :, 14].max(2)) / 1e3
     out["exchange_latency"] = {"logits": round(float(e_log), 3), "h": round(float(e_h), 3),
                                "y": round(float(e_y), 3), "x": round(float(e_x), 3)}
     out["layer_total"] = round(float(np.median(np.diff(tr[:, :, 0].min(1)))) / 1e3, 3)

@@ -70,6 +70,7 @@ constexpr int kMaxDN = 128;         // down rows per CTA
 constexpr int kMaxRouterRows = 8;   // router rows per CTA
 constexpr int kPredTop = 12;        // predicted next-layer experts prefetched to L2
 constexpr int kTracePoints = 16;
+constexpr long long kPredictWaitNs = 5000;  // the prediction exchange is a hint: give up after 5 us
 
 struct StackParams {
     StackLayerDev layer[kMaxLayers];
@@ -116,7 +117,7 @@ __device__ __forceinline__ bool poll_pair(const unsigned long long *src, uint32_
 
 // ------------------------------------------------------------------ shared memory map
 struct SmemMap {
-    uint32_t gbuf, ubuf, dbuf, rbuf0, rbuf1, xs, xl, hl, lg, plg, hv, yv, cand, total;
+    uint32_t gbuf, ubuf, dbuf, rbuf0, rbuf1, xs, ns, xl, hl, lg, plg, hv, yv, cand, total;
 };
 
 __host__ __device__ inline uint32_t align128(uint32_t v) { return (v + 127u) & ~127u; }
@@ -135,6 +136,7 @@ __host__ __device__ inline SmemMap smem_map(int d, int f, int k, int gu_max, int
     m.rbuf0 = take((uint32_t)rb_max * d * 2);
     m.rbuf1 = take((uint32_t)rb_max * d * 2);
     m.xs = take((uint32_t)d * 2);
+    m.ns = take((uint32_t)d * 2);
     m.xl = take((uint32_t)NL * (d / 64) * kSegPad * 4);
     m.hl = take((uint32_t)NL * (f / 64) * kSegPad * 4);
     m.lg = take(256 * 8);
@@ -184,7 +186,9 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
     __shared__ int32_t s_pidx[kPredTop];
     __shared__ double s_gate[kSK];
     __shared__ long long s_S[kMaxGU][2];
-    __shared__ float s_sg[kMaxGU], s_su[kMaxGU], s_sd[kMaxDN];
+    // scales of this CTA's rows, bulk-copied with the rows: a 16-byte aligned superset of the
+    // range, so entry q is at [q + offset], offset < 4
+    __shared__ __align__(16) float s_sgb[kMaxGU + 8], s_sub[kMaxGU + 8], s_sdb[kMaxDN + 8];
     __shared__ float s_hmax[kStackWarps];
     // the layers' pointers, copied once: a dynamically indexed kernel parameter is a constant
     // cache line fetched from L2 on the critical path of every layer
@@ -206,6 +210,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
     uint16_t *const rbuf0 = reinterpret_cast<uint16_t *>(smem + sm.rbuf0);
     uint16_t *const rbuf1 = reinterpret_cast<uint16_t *>(smem + sm.rbuf1);
     uint16_t *xs = reinterpret_cast<uint16_t *>(smem + sm.xs);
+    uint16_t *ns = reinterpret_cast<uint16_t *>(smem + sm.ns);
     uint32_t *xl = reinterpret_cast<uint32_t *>(smem + sm.xl);
     uint32_t *hl = reinterpret_cast<uint32_t *>(smem + sm.hl);
     double *lg = reinterpret_cast<double *>(smem + sm.lg);
@@ -340,14 +345,15 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
         double nd[4];
         float nf[4];
         {
+            uint16_t nb[4];
 #pragma unroll
             for (int e = 0; e < 4; e++) {
-                const uint16_t nb = f64_to_bf16_rne((double)xv[e] / r);
-                nf[e] = bf16_to_f32(nb);
+                nb[e] = f64_to_bf16_rne((double)xv[e] / r);
+                nf[e] = bf16_to_f32(nb[e]);
                 nd[e] = (double)nf[e];
             }
-            const float inv = (NL == 1 && amax_n > 0.0f) ? quant_inv(amax_n) : 0.0f;
-            store_limbs4<NL>(xl, xlp, tid, nf, sh_n, inv, amax_n > 0.0f);
+            reinterpret_cast<uint2 *>(ns)[tid] =
+                make_uint2((uint32_t)nb[0] | ((uint32_t)nb[1] << 16), (uint32_t)nb[2] | ((uint32_t)nb[3] << 16));
         }
         // router rows of this layer: thread t multiplies columns 4t..4t+3; bf16 x bf16 has at
         // most 16 significant bits, so each product is exact in fp64 and the fma adds it with
@@ -368,7 +374,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                 }
             }
         }
-        if (!__syncthreads_and(alive ? 1 : 0)) break;  // also: limbs and router partials visible
+        if (!__syncthreads_and(alive ? 1 : 0)) break;  // router partials (and n) visible
         if (tid < nr) {
             double sum = 0.0;
             for (int w = 0; w < kStackWarps; w++) sum += s_rp[w][tid];
@@ -377,32 +383,10 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                           tagged((uint32_t)b, tag));
         }
         TSTAMP(l, 2)
-        // predicted logits of the next layer (fp32; used only to choose L2 prefetches)
-        if (p.predict && has_next && nr > 0) {
-            const uint32_t npar = (uint32_t)((l + 1) & 1);
-            const bool okr = mbar_wait(&mb_r[npar], (uint32_t)(((l + 1) >> 1) & 1), lim, p.status);
-            if (!okr) alive = false;
-            const bool okw = __all_sync(0xFFFFFFFFu, okr);  // the shuffles below need the whole warp
-#pragma unroll
-            for (int q = 0; q < kMaxRouterRows; q++) {
-                if (q < nr && okw) {
-                    const uint2 w = reinterpret_cast<const uint2 *>((npar ? rbuf1 : rbuf0) + (size_t)q * d)[tid];
-                    float a = 0.0f;
-                    a = fmaf(__uint_as_float(w.x << 16), nf[0], a);
-                    a = fmaf(__uint_as_float(w.x & 0xFFFF0000u), nf[1], a);
-                    a = fmaf(__uint_as_float(w.y << 16), nf[2], a);
-                    a = fmaf(__uint_as_float(w.y & 0xFFFF0000u), nf[3], a);
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xFFFFFFFFu, a, o);
-                    if (lane == 0) s_pp[warp][q] = a;
-                }
-            }
-        }
-        if (!__syncthreads_and(alive ? 1 : 0)) break;
-        if (p.predict && has_next && tid < nr) {
-            float sum = 0.0f;
-            for (int w = 0; w < kStackWarps; w++) sum += s_pp[w][tid];
-            st_word(p.pb + (size_t)par * E + e0 + tid, __float_as_uint(sum), tag);
+        // activation limbs for the gate/up dots (needed only after top-k and the row copies)
+        {
+            const float inv = (NL == 1 && amax_n > 0.0f) ? quant_inv(amax_n) : 0.0f;
+            store_limbs4<NL>(xl, xlp, tid, nf, sh_n, inv, amax_n > 0.0f);
         }
         // rbuf[par] is free (this layer's rows are used): fetch the rows of layer l + 2 into it
         if (tid == 0 && nr > 0 && l + 2 < p.n_layers) {
@@ -431,16 +415,20 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             warp_topk_filter(lg, E, k, s_idx, cand);
             // copies of expert idx[s]: first gate/up chunk, second chunk, down rows; thread 0
             // registers the byte counts first (counted here, so only issued phases are drained)
+            const size_t e = (size_t)s_idx[s];
+            // scales: aligned supersets [ga, ga + gn) of rows j0..j1 and [da, da + dn) of i0..i1
+            const size_t ga = (e * f + j0) & ~(size_t)3, da = (e * d + i0) & ~(size_t)3;
+            const uint32_t gn = (uint32_t)((((e * f + j1) + 3) & ~(size_t)3) - ga);
+            const uint32_t dn = ndn > 0 ? (uint32_t)((((e * d + i1) + 3) & ~(size_t)3) - da) : 0u;
             if (lane == 0) {
-                mbar_expect_tx(&mb_gu0, (uint32_t)(2 * n0 * (d / 4)));
+                mbar_expect_tx(&mb_gu0, (uint32_t)(2 * n0 * (d / 4)) + 8u * gn);
                 mbar_expect_tx(&mb_gu1, (uint32_t)(2 * n1 * (d / 4)));
-                mbar_expect_tx(&mb_dn, (uint32_t)(ndn * (f / 4)));
+                mbar_expect_tx(&mb_dn, (uint32_t)(ndn * (f / 4)) + 4u * dn);
                 n_gu++;
                 n_dn++;
             }
             __syncwarp();
-            if (lane < 5) {
-                const size_t e = (size_t)s_idx[s];
+            if (lane < 8) {
                 const uint32_t rowg = (uint32_t)(d / 4), rowd = (uint32_t)(f / 4);
                 if (lane == 0 && n0 > 0) bulk_g2s(gbuf, Ly.gate + (e * f + j0) * rowg, (uint32_t)n0 * rowg, &mb_gu0);
                 if (lane == 1 && n0 > 0) bulk_g2s(ubuf, Ly.up + (e * f + j0) * rowg, (uint32_t)n0 * rowg, &mb_gu0);
@@ -449,60 +437,11 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                 if (lane == 3 && n1 > 0)
                     bulk_g2s(ubuf + (size_t)n0 * rowg, Ly.up + (e * f + j0 + n0) * rowg, (uint32_t)n1 * rowg, &mb_gu1);
                 if (lane == 4 && ndn > 0) bulk_g2s(dbuf, Ly.down + (e * d + i0) * rowd, (uint32_t)ndn * rowd, &mb_dn);
+                if (lane == 5) bulk_g2s(s_sgb, Ly.sg + ga, 4u * gn, &mb_gu0);
+                if (lane == 6) bulk_g2s(s_sub, Ly.su + ga, 4u * gn, &mb_gu0);
+                if (lane == 7 && dn > 0) bulk_g2s(s_sdb, Ly.sd + da, 4u * dn, &mb_dn);
             }
-        }
-        __syncthreads();
-        TSTAMP(l, 5)
-        if (warp == 1) {
-            // the scales of this CTA's rows (read while the rows travel)
-            const size_t e = (size_t)s_idx[s];
-            for (int q = lane; q < ngu; q += 32) {
-                s_sg[q] = __ldg(Ly.sg + e * f + j0 + q);
-                s_su[q] = __ldg(Ly.su + e * f + j0 + q);
-            }
-            for (int q = lane; q < ndn; q += 32) s_sd[q] = __ldg(Ly.sd + e * d + i0 + q);
-        } else if (warp == 2) {
-            warp_topk_gates(lg, k, s_idx, s_gate, nullptr);
-            __syncwarp();
-            if (lane < k && pid == 0) {
-                p.idx_hist[l * k + lane] = s_idx[lane];
-                p.gate_hist[l * k + lane] = s_gate[lane];
-            }
-        } else if (warp == 3 && p.predict && has_next) {
-            // predicted experts of the next layer -> L2 prefetch of this CTA's rows of
-            // predictions s and s + 8 (what it would copy if one of them lands in its slot)
-            bool ok = true;
-            const unsigned long long t0 = gtimer();
-            for (int e = lane; e < E; e += 32) {
-                unsigned long long w;
-                while (true) {
-                    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(p.pb + (size_t)par * E + e) : "memory");
-                    if ((uint32_t)(w >> 32) == tag) break;
-                    if ((long long)(gtimer() - t0) > lim) {
-                        ok = false;
-                        break;
-                    }
-                }
-                plg[e] = (double)__uint_as_float((uint32_t)w);
-                if (!ok) break;
-            }
-            // a missing prediction only skips the prefetch (the real exchanges decide timeouts)
-            if (__all_sync(0xFFFFFFFFu, ok)) {
-                const int np = E < kPredTop ? E : kPredTop;
-                warp_topk_filter(plg, E, np, s_pidx, cand);
-                const StackLayerDev &Ln = s_layer[l + 1];
-                const uint32_t rowg = (uint32_t)(d / 4), rowd = (uint32_t)(f / 4);
-                for (int q = s; q < np; q += kSK) {
-                    const size_t e = (size_t)s_pidx[q];
-                    if (lane == 0 && ngu > 0) prefetch_l2_bulk(Ln.gate + (e * f + j0) * rowg, (uint32_t)ngu * rowg);
-                    if (lane == 1 && ngu > 0) prefetch_l2_bulk(Ln.up + (e * f + j0) * rowg, (uint32_t)ngu * rowg);
-                    if (lane == 2 && ndn > 0) prefetch_l2_bulk(Ln.down + (e * d + i0) * rowd, (uint32_t)ndn * rowd);
-                    if (lane == 3) asm volatile("prefetch.global.L2 [%0];" ::"l"(Ln.sg + e * f + j0));
-                    if (lane == 4) asm volatile("prefetch.global.L2 [%0];" ::"l"(Ln.su + e * f + j0));
-                    if (lane >= 5 && lane < 9 && 32 * (lane - 5) < ndn)
-                        asm volatile("prefetch.global.L2 [%0];" ::"l"(Ln.sd + e * d + i0 + 32 * (lane - 5)));
-                }
-            }
+            TSTAMP(l, 5)
         }
         // ------------------------------------------------------------ C: gate/up -> h
         {
@@ -510,17 +449,15 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             SegX<NL> X;
             seg_load_x_padded<NL>(X, xl, xlp, lane);
             const int rowb = d / 4;
+            bool okc = true;
             for (int half = 0; half < 2; half++) {
                 const int qa = half ? n0 : 0, qb = half ? ngu : n0;
-                if (qb <= qa) continue;
-                const bool okw = mbar_wait(half ? &mb_gu1 : &mb_gu0, par, lim, p.status);
-                if (!__syncthreads_and(okw ? 1 : 0)) {
-                    alive = false;
-                    break;
-                }
-                if (half == 0) TSTAMP(l, 6)
                 const int q = qa + warp;
-                if (q < qb) {
+                if (q >= qb) continue;  // no row of this copy for this warp
+                // each warp waits for the copy itself: no CTA barrier between the copies and the dots
+                if (!mbar_wait(half ? &mb_gu1 : &mb_gu0, par, lim, p.status)) okc = false;
+                if (half == 0) TSTAMP(l, 6)
+                {
                     const uint4 wg = *reinterpret_cast<const uint4 *>(gbuf + (size_t)q * rowb + lane * 16);
                     const uint4 wu = *reinterpret_cast<const uint4 *>(ubuf + (size_t)q * rowb + lane * 16);
                     int ag[NL], au[NL];
@@ -543,27 +480,73 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                     }
                 }
             }
-            if (!alive) break;
+            // warps without rows also take mb_gu0 (the scales the SwiGLU threads read)
+            if (warp >= n0 && !mbar_wait(&mb_gu0, par, lim, p.status)) okc = false;
+            if (!__syncthreads_and(okc ? 1 : 0)) {
+                alive = false;
+                break;
+            }
         }
-        __syncthreads();
         TSTAMP(l, 7)
         // SwiGLU epilogue, one thread per row, fp64
+        const int sgo = (int)(((size_t)s_idx[s] * f + j0) & 3);  // offset of row j0's scale in s_sgb / s_sub
         if (tid < ngu) {
             const int q = tid;
             const long long Sg = s_S[q][0], Su = s_S[q][1];
             float h;
             if (NL == 1) {
-                const float gv = __fmul_rn(__fmul_rn(__int2float_rn((int)Sg), s_sg[q]), s_nq);
-                const float uv = __fmul_rn(__fmul_rn(__int2float_rn((int)Su), s_su[q]), s_nq);
+                const float gv = __fmul_rn(__fmul_rn(__int2float_rn((int)Sg), s_sgb[q + sgo]), s_nq);
+                const float uv = __fmul_rn(__fmul_rn(__int2float_rn((int)Su), s_sub[q + sgo]), s_nq);
                 h = swiglu_f32((double)gv, (double)uv);
             } else {
-                h = swiglu_f32(ldexp((double)Sg, -sh_n) * (double)s_sg[q], ldexp((double)Su, -sh_n) * (double)s_su[q]);
+                h = swiglu_f32(ldexp((double)Sg, -sh_n) * (double)s_sgb[q + sgo],
+                               ldexp((double)Su, -sh_n) * (double)s_sub[q + sgo]);
             }
             st_word(p.hb + ((size_t)par * k + s) * f + j0 + q, __float_as_uint(h), tag);
             p.h_hist[((size_t)l * k + s) * f + j0 + q] = h;
         }
         TSTAMP(l, 8)
         // ------------------------------------------------------------ D: down, combine, residual
+        // While warps 0..7 wait for the slot's h: warp 8 computes the gates (needed at the
+        // combine); warps 8..15 compute this CTA's router rows of the NEXT layer against n
+        // (fp32, a prediction) and publish them.
+        if (warp == kStackWarps / 2) {
+            warp_topk_gates(lg, k, s_idx, s_gate, nullptr);
+            __syncwarp();
+            if (lane < k && pid == 0) {
+                p.idx_hist[l * k + lane] = s_idx[lane];
+                p.gate_hist[l * k + lane] = s_gate[lane];
+            }
+        }
+        const bool predict = p.predict && has_next && nr > 0;
+        if (predict && warp >= kStackWarps / 2) {
+            const uint32_t npar = (uint32_t)((l + 1) & 1);
+            const bool okr = __all_sync(0xFFFFFFFFu, mbar_wait(&mb_r[npar], (uint32_t)(((l + 1) >> 1) & 1), lim, p.status));
+            const int t2 = tid - kStackThreads / 2;  // 256 threads x 8 columns
+            const uint4 nv = reinterpret_cast<const uint4 *>(ns)[t2];
+#pragma unroll
+            for (int q = 0; q < kMaxRouterRows; q++) {
+                if (q < nr && okr) {
+                    const uint4 w = reinterpret_cast<const uint4 *>((npar ? rbuf1 : rbuf0) + (size_t)q * d)[t2];
+                    float a = 0.0f;
+                    const uint32_t wv[4] = {w.x, w.y, w.z, w.w}, nn[4] = {nv.x, nv.y, nv.z, nv.w};
+#pragma unroll
+                    for (int z = 0; z < 4; z++) {
+                        a = fmaf(__uint_as_float(wv[z] << 16), __uint_as_float(nn[z] << 16), a);
+                        a = fmaf(__uint_as_float(wv[z] & 0xFFFF0000u), __uint_as_float(nn[z] & 0xFFFF0000u), a);
+                    }
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xFFFFFFFFu, a, o);
+                    if (lane == 0) s_pp[warp - kStackWarps / 2][q] = a;
+                }
+            }
+            named_bar_sync(1, kStackThreads / 2);
+            if (t2 < nr && okr) {
+                float sum = 0.0f;
+                for (int w = 0; w < kStackWarps / 2; w++) sum += s_pp[w][t2];
+                st_word(p.pb + (size_t)par * E + e0 + t2, __float_as_uint(sum), tag);
+            }
+        }
         {
             bool ok = true;
             float m = 0.0f;
@@ -608,6 +591,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             const int sub = lane / Gf, gl = lane % Gf;
             SegX<NL> Hx;
             seg_load_x_padded<NL>(Hx, hl, hlp, gl);
+            const int sdo = (int)(((size_t)s_idx[s] * d + i0) & 3);  // offset of row i0's scale in s_sdb
             const uint32_t ytag = tag;
             for (int r0 = warp * rpp; r0 < ndn; r0 += kStackWarps * rpp) {
                 const int rr = r0 + sub;
@@ -625,7 +609,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                 }
                 if (valid && gl == 0) {
                     const long long S = pair_value(NL, aa, bb);
-                    const float sd = s_sd[rr];
+                    const float sd = s_sdb[rr + sdo];
                     float v;
                     if (NL == 1) v = __fmul_rn(__fmul_rn(__int2float_rn((int)S), sd), hsc);
                     else v = (float)(ldexp((double)S, -hsh) * (double)sd);
@@ -634,12 +618,47 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             }
         }
         TSTAMP(l, 12)
+        if (warp == kStackWarps - 1 && p.predict && has_next) {
+            // predicted experts of the next layer -> L2 prefetch of this CTA's rows of
+            // predictions s and s + 8 (what it would copy if one of them lands in its slot).
+            // Only a hint: if the predictions are not all there within a few microseconds, skip.
+            bool ok = true;
+            const unsigned long long t0 = gtimer();
+            for (int e = lane; e < E && ok; e += 32) {
+                unsigned long long w;
+                while (true) {
+                    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(p.pb + (size_t)par * E + e) : "memory");
+                    if ((uint32_t)(w >> 32) == tag) break;
+                    if ((long long)(gtimer() - t0) > kPredictWaitNs) {
+                        ok = false;
+                        break;
+                    }
+                }
+                plg[e] = (double)__uint_as_float((uint32_t)w);
+            }
+            if (__all_sync(0xFFFFFFFFu, ok)) {
+                const int np = E < kPredTop ? E : kPredTop;
+                warp_topk_filter(plg, E, np, s_pidx, cand);
+                const StackLayerDev &Ln = s_layer[l + 1];
+                const uint32_t rowg = (uint32_t)(d / 4), rowd = (uint32_t)(f / 4);
+                for (int q = s; q < np; q += kSK) {
+                    const size_t e = (size_t)s_pidx[q];
+                    if (lane == 0 && ngu > 0) prefetch_l2_bulk(Ln.gate + (e * f + j0) * rowg, (uint32_t)ngu * rowg);
+                    if (lane == 1 && ngu > 0) prefetch_l2_bulk(Ln.up + (e * f + j0) * rowg, (uint32_t)ngu * rowg);
+                    if (lane == 2 && ndn > 0) prefetch_l2_bulk(Ln.down + (e * d + i0) * rowd, (uint32_t)ndn * rowd);
+                    if (lane == 3) asm volatile("prefetch.global.L2 [%0];" ::"l"(Ln.sg + e * f + j0));
+                    if (lane == 4) asm volatile("prefetch.global.L2 [%0];" ::"l"(Ln.su + e * f + j0));
+                    if (lane >= 5 && lane < 9 && 32 * (lane - 5) < ndn)
+                        asm volatile("prefetch.global.L2 [%0];" ::"l"(Ln.sd + e * d + i0 + 32 * (lane - 5)));
+                }
+            }
+        }
         {
             // the k slots' outputs of rows [i0, i1)
             bool ok = true;
             const int half_rows = ndn / 2;
             const unsigned long long t0 = gtimer();
-            for (int t = tid; t < k * half_rows; t += kStackThreads) {
+            for (int t = tid; t < k * half_rows && warp < kStackWarps - 1; t += kStackThreads - 32) {
                 const int q = t / half_rows, w2 = 2 * (t % half_rows);
                 ulonglong2 w;
                 if (!poll_pair(p.yb + (((size_t)par * G + c) * k + q) * kMaxDN + w2, tag, t0, lim, w)) {
@@ -797,6 +816,8 @@ static tern_status stack_plan(const tern_moe_layer &L0, int n_layers, tern_act a
         return TERN_EUNSUPPORTED;
     const int gf = f / 64;
     if (gf < 1 || gf > 32 || (gf & (gf - 1)) != 0) return TERN_EUNSUPPORTED;
+    // the scales are bulk-copied in 16-byte aligned blocks (every layer is checked at launch)
+    if (((uintptr_t)L0.gate_scale | (uintptr_t)L0.up_scale | (uintptr_t)L0.down_scale) & 15u) return TERN_EUNSUPPORTED;
     const int sms = sm_count();
     if (sms <= 0) return TERN_ECUDA;
     int G = sms / k;
@@ -839,6 +860,10 @@ tern_status launch_stack_persistent(const tern_moe_layer *layers, int n_layers, 
     const StackWs o = stack_ws_layout(&L0);
     if (ws_bytes < (size_t)o.total) return TERN_EWORKSPACE;
     if (!status) return TERN_ECUDA;
+    // the scales are bulk-copied in 16-byte aligned blocks: the arrays must start 16-byte aligned
+    for (int l = 0; l < n_layers; l++)
+        if (((uintptr_t)layers[l].gate_scale | (uintptr_t)layers[l].up_scale | (uintptr_t)layers[l].down_scale) & 15u)
+            return TERN_EUNSUPPORTED;
 
     StackParams prm;
     memset(&prm, 0, sizeof(prm));
