@@ -360,9 +360,9 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
         // one rounding (the sums are exact at these magnitudes: the order does not matter)
         if (nr > 0) {
             if (!mbar_wait(&mb_r[par], (uint32_t)((l >> 1) & 1), lim, p.status)) alive = false;
-#pragma unroll
-            for (int q = 0; q < kMaxRouterRows; q++) {
-                if (q < nr) {
+#pragma unroll 1
+            for (int q = 0; q < nr; q++) {
+                {
                     const uint2 w = reinterpret_cast<const uint2 *>((par ? rbuf1 : rbuf0) + (size_t)q * d)[tid];
                     double a = 0.0;
                     a = fma(bf16_to_f64((uint16_t)(w.x & 0xFFFFu)), nd[0], a);
@@ -450,6 +450,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             seg_load_x_padded<NL>(X, xl, xlp, lane);
             const int rowb = d / 4;
             bool okc = true;
+#pragma unroll 1
             for (int half = 0; half < 2; half++) {
                 const int qa = half ? n0 : 0, qb = half ? ngu : n0;
                 const int q = qa + warp;
@@ -499,8 +500,8 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                 const float uv = __fmul_rn(__fmul_rn(__int2float_rn((int)Su), s_sub[q + sgo]), s_nq);
                 h = swiglu_f32((double)gv, (double)uv);
             } else {
-                h = swiglu_f32(ldexp((double)Sg, -sh_n) * (double)s_sgb[q + sgo],
-                               ldexp((double)Su, -sh_n) * (double)s_sub[q + sgo]);
+                const double p2 = pow2_f64(-sh_n);
+                h = swiglu_f32((double)Sg * p2 * (double)s_sgb[q + sgo], (double)Su * p2 * (double)s_sub[q + sgo]);
             }
             st_word(p.hb + ((size_t)par * k + s) * f + j0 + q, __float_as_uint(h), tag);
             p.h_hist[((size_t)l * k + s) * f + j0 + q] = h;
@@ -524,9 +525,9 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             const bool okr = __all_sync(0xFFFFFFFFu, mbar_wait(&mb_r[npar], (uint32_t)(((l + 1) >> 1) & 1), lim, p.status));
             const int t2 = tid - kStackThreads / 2;  // 256 threads x 8 columns
             const uint4 nv = reinterpret_cast<const uint4 *>(ns)[t2];
-#pragma unroll
-            for (int q = 0; q < kMaxRouterRows; q++) {
-                if (q < nr && okr) {
+#pragma unroll 1
+            for (int q = 0; q < nr; q++) {
+                if (okr) {
                     const uint4 w = reinterpret_cast<const uint4 *>((npar ? rbuf1 : rbuf0) + (size_t)q * d)[t2];
                     float a = 0.0f;
                     const uint32_t wv[4] = {w.x, w.y, w.z, w.w}, nn[4] = {nv.x, nv.y, nv.z, nv.w};
@@ -612,7 +613,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                     const float sd = s_sdb[rr + sdo];
                     float v;
                     if (NL == 1) v = __fmul_rn(__fmul_rn(__int2float_rn((int)S), sd), hsc);
-                    else v = (float)(ldexp((double)S, -hsh) * (double)sd);
+                    else v = (float)((double)S * pow2_f64(-hsh) * (double)sd);
                     st_word(p.yb + (((size_t)par * G + c) * k + s) * kMaxDN + rr, __float_as_uint(v), ytag);
                 }
             }
