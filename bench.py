@@ -565,7 +565,7 @@ def main():
     tm.moe_stack_decode(stack, xs[W:W + 1].clone(), act=act, ws=ws)
     torch.cuda.synchronize(dev)
     os.environ["TERNMOE_TRACE"] = "0"
-    tr2 = ws[lay["trace"]:lay["trace"] + 2 * N_LAYERS * P * 16 * 8].view(torch.int64).view(2, N_LAYERS, P, 16).cpu().numpy()
+    tr2 = ws[lay["trace"]:lay["trace"] + 2 * N_LAYERS * P * 24 * 8].view(torch.int64).view(2, N_LAYERS, P, 24).cpu().numpy()
     tr = tr2[0]
     phases = phase_summary(tr, tr2[1]) if launches == 1 else None
     try:

@@ -263,7 +263,7 @@ tern_status flash_head(const uint8_t *C4, const double *c_scale, const uint16_t 
  *                                   the residual adds), for parity checks of every layer;
  *   h32     float  [n_layers][k][f] each layer's SwiGLU output h of every slot (the down
  *                                   projection's input, before its limbs or int8 codes);
- *   trace   uint64 [2][n_layers][P][16]: %globaltimer (ns), then clock64 (SM cycles), stamped
+ *   trace   uint64 [2][n_layers][P][24]: %globaltimer (ns), then clock64 (SM cycles), stamped
  *           by each of the P CTAs (one per SM, P = moe_stack_persistent_ctas(), P <= 256) at
  *           phase boundaries, written only when
  *           the environment variable TERNMOE_TRACE is "1" at the time of the call: 0 layer
@@ -271,7 +271,9 @@ tern_status flash_head(const uint8_t *C4, const double *c_scale, const uint16_t 
  *           published, 4 all logits received, 5 top-k done and row copies issued, 6 first
  *           gate/up rows landed, 7 gate/up dots done, 8 h published, 9 slot's h received,
  *           10 h limbs built, 11 down rows landed, 12 down dots done and published, 13 the
- *           slots' outputs of this CTA's rows received, 14 x' published.
+ *           slots' outputs of this CTA's rows received, 14 x' published; inside the phases
+ *           (CTA thread 0): 15 r known, 16 n known, 17 own router partials written, 18 top-k
+ *           known (before the copies are issued); 19..23 unused.
  * The persistent kernel prefetches the experts it predicts for the next layer into L2 (a hint
  * that changes no value); TERNMOE_PREDICT=0 in the environment turns that off. */
 typedef struct {

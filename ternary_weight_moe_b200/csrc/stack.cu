@@ -69,8 +69,10 @@ constexpr int kMaxGU = 32;          // gate/up rows per CTA (two chunks of 16)
 constexpr int kMaxDN = 128;         // down rows per CTA
 constexpr int kMaxRouterRows = 8;   // router rows per CTA
 constexpr int kPredTop = 12;        // predicted next-layer experts prefetched to L2
-constexpr int kTracePoints = 16;
-constexpr long long kPredictWaitNs = 5000;  // the prediction exchange is a hint: give up after 5 us
+constexpr int kTracePoints = 24;
+constexpr long long kPredictWaitCycles = 10000;  // the prediction exchange is a hint: give up after ~5 us
+constexpr unsigned kPollSleepNs = 32;           // sleep between two polls of a tagged word
+constexpr int kTraceExtra = 8;                  // stamps inside the layer's phases (15 .. 22)
 
 struct StackParams {
     StackLayerDev layer[kMaxLayers];
@@ -105,14 +107,28 @@ __device__ __forceinline__ void st_word(unsigned long long *p, uint32_t payload,
     asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(tagged(payload, tag)) : "memory");
 }
 
-// Poll the pair of tagged words at src until both carry `tag`; false once `t0 + limit` passes.
-__device__ __forceinline__ bool poll_pair(const unsigned long long *src, uint32_t tag, unsigned long long t0,
-                                          long long limit, ulonglong2 &out) {
+// Poll the pair of tagged words at src until both carry `tag`; false once `limit` SM cycles
+// have passed since t0 (clock64).  Between polls the thread sleeps briefly, so polling warps
+// leave the issue slots to the warps that compute.
+__device__ __forceinline__ bool poll_pair(const unsigned long long *src, uint32_t tag, long long t0, long long limit,
+                                          ulonglong2 &out) {
     while (true) {
         out = ld_relaxed_v2(src);
         if ((uint32_t)(out.x >> 32) == tag && (uint32_t)(out.y >> 32) == tag) return true;
-        if ((long long)(gtimer() - t0) > limit) return false;
+        if (clock64() - t0 > limit) return false;
+        __nanosleep(kPollSleepNs);
     }
+}
+
+// CTA-wide AND over the threads of hardware barrier `id` (nthreads, a multiple of 32)
+__device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n barrier.red.and.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
 }
 
 // ------------------------------------------------------------------ shared memory map
@@ -222,6 +238,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
     const int hlp = (f / 64) * kSegPad;  // padded words per limb of h
 
     const long long lim = p.limit_ns;
+    const long long limc = 2 * p.limit_ns;  // the same bound in SM cycles (clocks <= 2 GHz)
     const uint32_t ep = ld_acquire_gpu(p.ctl + 1);  // launch epoch, advanced by the previous launch
     bool alive = true;
     unsigned int n_rt0 = 0, n_rt1 = 0, n_gu = 0, n_dn = 0;  // phases armed per mbarrier (thread 0)
@@ -279,14 +296,14 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             if (l == 0) {
                 pr = __ldcg(reinterpret_cast<const uint2 *>(p.x) + tid);
             } else {
-                const unsigned long long t0 = gtimer();
+                const long long t0 = clock64();
                 ulonglong2 w;
-                ok = poll_pair(p.xb + ((size_t)par * k + s) * (d / 2) + 2 * tid, tag, t0, lim, w);
+                ok = poll_pair(p.xb + ((size_t)par * k + s) * (d / 2) + 2 * tid, tag, t0, limc, w);
                 pr = make_uint2((uint32_t)w.x, (uint32_t)w.y);
                 if (tid < 2 * G) {
                     ulonglong2 st;
                     const bool ok2 = poll_pair(p.xst + (((size_t)par * k + s) * G + (tid >> 1)) * 4 + 2 * (tid & 1), tag,
-                                               t0, lim, st);
+                                               t0, limc, st);
                     ok = ok && ok2;
                     if (tid & 1) s_xam[tid >> 1] = __uint_as_float((uint32_t)st.x);
                     else s_xss[tid >> 1] = __longlong_as_double((long long)(((unsigned long long)(uint32_t)st.x << 32) |
@@ -337,6 +354,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             amax = ta;
         }
         TSTAMP(l, 1)
+        TSTAMP(l, 15)  // r known
         if (l == 0 && pid == 0) reinterpret_cast<uint2 *>(p.hist)[tid] = reinterpret_cast<const uint2 *>(xs)[tid];
         // rounding is monotone, so max |bf16(x_k / r)| = bf16(max |x_k| / r)
         const float amax_n = bf16_to_f32(f64_to_bf16_rne((double)amax / r));
@@ -355,11 +373,12 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             reinterpret_cast<uint2 *>(ns)[tid] =
                 make_uint2((uint32_t)nb[0] | ((uint32_t)nb[1] << 16), (uint32_t)nb[2] | ((uint32_t)nb[3] << 16));
         }
+        TSTAMP(l, 16)  // n known
         // router rows of this layer: thread t multiplies columns 4t..4t+3; bf16 x bf16 has at
         // most 16 significant bits, so each product is exact in fp64 and the fma adds it with
         // one rounding (the sums are exact at these magnitudes: the order does not matter)
         if (nr > 0) {
-            if (!mbar_wait(&mb_r[par], (uint32_t)((l >> 1) & 1), lim, p.status)) alive = false;
+            if (!mbar_wait_sleep(&mb_r[par], (uint32_t)((l >> 1) & 1), lim, p.status)) alive = false;
 #pragma unroll 1
             for (int q = 0; q < nr; q++) {
                 {
@@ -374,6 +393,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                 }
             }
         }
+        TSTAMP(l, 17)  // this warp's router partials written
         if (!__syncthreads_and(alive ? 1 : 0)) break;  // router partials (and n) visible
         if (tid < nr) {
             double sum = 0.0;
@@ -401,7 +421,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             bool ok = true;
             if (tid < E) {
                 ulonglong2 w;
-                ok = poll_pair(p.lb + ((size_t)par * E + tid) * 2, tag, gtimer(), lim, w);
+                ok = poll_pair(p.lb + ((size_t)par * E + tid) * 2, tag, clock64(), limc, w);
                 lg[tid] = __longlong_as_double((long long)(((unsigned long long)(uint32_t)w.x << 32) | (uint32_t)w.y));
             }
             if (!__syncthreads_and(ok ? 1 : 0)) {
@@ -413,6 +433,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
         TSTAMP(l, 4)
         if (warp == 0) {
             warp_topk_filter(lg, E, k, s_idx, cand);
+            TSTAMP(l, 18)  // top-k known
             // copies of expert idx[s]: first gate/up chunk, second chunk, down rows; thread 0
             // registers the byte counts first (counted here, so only issued phases are drained)
             const size_t e = (size_t)s_idx[s];
@@ -456,7 +477,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                 const int q = qa + warp;
                 if (q >= qb) continue;  // no row of this copy for this warp
                 // each warp waits for the copy itself: no CTA barrier between the copies and the dots
-                if (!mbar_wait(half ? &mb_gu1 : &mb_gu0, par, lim, p.status)) okc = false;
+                if (!mbar_wait_sleep(half ? &mb_gu1 : &mb_gu0, par, lim, p.status)) okc = false;
                 if (half == 0) TSTAMP(l, 6)
                 {
                     const uint4 wg = *reinterpret_cast<const uint4 *>(gbuf + (size_t)q * rowb + lane * 16);
@@ -482,7 +503,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                 }
             }
             // warps without rows also take mb_gu0 (the scales the SwiGLU threads read)
-            if (warp >= n0 && !mbar_wait(&mb_gu0, par, lim, p.status)) okc = false;
+            if (warp >= n0 && !mbar_wait_sleep(&mb_gu0, par, lim, p.status)) okc = false;
             if (!__syncthreads_and(okc ? 1 : 0)) {
                 alive = false;
                 break;
@@ -522,7 +543,8 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
         const bool predict = p.predict && has_next && nr > 0;
         if (predict && warp >= kStackWarps / 2) {
             const uint32_t npar = (uint32_t)((l + 1) & 1);
-            const bool okr = __all_sync(0xFFFFFFFFu, mbar_wait(&mb_r[npar], (uint32_t)(((l + 1) >> 1) & 1), lim, p.status));
+            const bool okr =
+                __all_sync(0xFFFFFFFFu, mbar_wait_sleep(&mb_r[npar], (uint32_t)(((l + 1) >> 1) & 1), lim, p.status));
             const int t2 = tid - kStackThreads / 2;  // 256 threads x 8 columns
             const uint4 nv = reinterpret_cast<const uint4 *>(ns)[t2];
 #pragma unroll 1
@@ -555,7 +577,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             const uint32_t htag = (l == p.stall_layer && pid == 0) ? (tag ^ 0x40000000u) : tag;
             if (2 * tid < f) {
                 ulonglong2 w;
-                ok = poll_pair(p.hb + ((size_t)par * k + s) * f + 2 * tid, htag, gtimer(), lim, w);
+                ok = poll_pair(p.hb + ((size_t)par * k + s) * f + 2 * tid, htag, clock64(), limc, w);
                 const float h0 = __uint_as_float((uint32_t)w.x), h1 = __uint_as_float((uint32_t)w.y);
                 hv[2 * tid] = h0;
                 hv[2 * tid + 1] = h1;
@@ -582,7 +604,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
         }
         __syncthreads();
         TSTAMP(l, 10)
-        if (ndn > 0 && !mbar_wait(&mb_dn, par, lim, p.status)) alive = false;
+        if (ndn > 0 && !mbar_wait_sleep(&mb_dn, par, lim, p.status)) alive = false;
         if (!__syncthreads_and(alive ? 1 : 0)) break;
         TSTAMP(l, 11)
         // down rows: Gf = f / 64 lanes per row, 32 / Gf rows per warp pass
@@ -619,21 +641,46 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             }
         }
         TSTAMP(l, 12)
+        {
+            // the k slots' outputs of rows [i0, i1)
+            bool ok = true;
+            const int half_rows = ndn / 2;
+            const long long t0 = clock64();
+            for (int t = tid; t < k * half_rows; t += kStackThreads) {
+                const int q = t / half_rows, w2 = 2 * (t % half_rows);
+                ulonglong2 w;
+                if (!poll_pair(p.yb + (((size_t)par * G + c) * k + q) * kMaxDN + w2, tag, t0, limc, w)) {
+                    ok = false;
+                    break;
+                }
+                yv[q * kMaxDN + w2] = __uint_as_float((uint32_t)w.x);
+                yv[q * kMaxDN + w2 + 1] = __uint_as_float((uint32_t)w.y);
+            }
+            if (!__syncthreads_and(ok ? 1 : 0)) {
+                set_status(p.status, TERN_ETIMEOUT);
+                alive = false;
+                break;
+            }
+        }
+        TSTAMP(l, 13)
         if (warp == kStackWarps - 1 && p.predict && has_next) {
             // predicted experts of the next layer -> L2 prefetch of this CTA's rows of
             // predictions s and s + 8 (what it would copy if one of them lands in its slot).
             // Only a hint: if the predictions are not all there within a few microseconds, skip.
+            // This warp runs it while warps 0..3 combine; it joins the CTA again at the next
+            // layer's first barrier.
             bool ok = true;
-            const unsigned long long t0 = gtimer();
+            const long long t0 = clock64();
             for (int e = lane; e < E && ok; e += 32) {
                 unsigned long long w;
                 while (true) {
                     asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(p.pb + (size_t)par * E + e) : "memory");
                     if ((uint32_t)(w >> 32) == tag) break;
-                    if ((long long)(gtimer() - t0) > kPredictWaitNs) {
+                    if (clock64() - t0 > kPredictWaitCycles) {
                         ok = false;
                         break;
                     }
+                    __nanosleep(kPollSleepNs);
                 }
                 plg[e] = (double)__uint_as_float((uint32_t)w);
             }
@@ -654,28 +701,6 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                 }
             }
         }
-        {
-            // the k slots' outputs of rows [i0, i1)
-            bool ok = true;
-            const int half_rows = ndn / 2;
-            const unsigned long long t0 = gtimer();
-            for (int t = tid; t < k * half_rows && warp < kStackWarps - 1; t += kStackThreads - 32) {
-                const int q = t / half_rows, w2 = 2 * (t % half_rows);
-                ulonglong2 w;
-                if (!poll_pair(p.yb + (((size_t)par * G + c) * k + q) * kMaxDN + w2, tag, t0, lim, w)) {
-                    ok = false;
-                    break;
-                }
-                yv[q * kMaxDN + w2] = __uint_as_float((uint32_t)w.x);
-                yv[q * kMaxDN + w2 + 1] = __uint_as_float((uint32_t)w.y);
-            }
-            if (!__syncthreads_and(ok ? 1 : 0)) {
-                set_status(p.status, TERN_ETIMEOUT);
-                alive = false;
-                break;
-            }
-        }
-        TSTAMP(l, 13)
         {
             const bool last = !has_next;
             const uint32_t ntag = (ep << 7) | (uint32_t)(l + 2);
@@ -701,15 +726,16 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             const uint32_t other = __shfl_down_sync(0xFFFFFFFFu, (uint32_t)xo, 1);
             if (!last && tid < ndn && (tid & 1) == 0)
                 st_word(p.xb + ((size_t)npar * k + s) * (d / 2) + (i0 + tid) / 2, (uint32_t)xo | (other << 16), ntag);
-            if (!last) {
-                // sum of squares and absmax of this part (threads < ndn <= kMaxDN = 128: warps 0..3)
+            if (!last && warp < kMaxDN / 32) {
+                // sum of squares and absmax of this part (threads < ndn <= kMaxDN = 128: warps
+                // 0..3, synchronised by hardware barrier 2 alone)
                 sq = warp_sum_f64(sq);
                 am = warp_max_f32(am);
                 if (lane == 0) {
                     s_red[warp] = sq;
                     s_redf[warp] = am;
                 }
-                __syncthreads();
+                named_bar_sync(2, kMaxDN);
                 if (tid == 0) {
                     double ts = 0.0;
                     float ta = 0.0f;

@@ -458,7 +458,7 @@ __device__ __forceinline__ void block_topk_select(double mine, int E, int k, int
 //     index); ranks below k land in idx_out.
 // cand: shared scratch of 256 entries; idx_out: shared memory.  No CTA barrier: only the
 // calling warp takes part, and it ends with __syncwarp.
-__device__ __noinline__ void warp_topk_filter(const double *lg, int E, int k, int32_t *idx_out,
+static __device__ __noinline__ void warp_topk_filter(const double *lg, int E, int k, int32_t *idx_out,
                                               ulonglong2 *cand) {
     const int lane = threadIdx.x & 31;
     unsigned long long key[8];
@@ -501,7 +501,7 @@ __device__ __noinline__ void warp_topk_filter(const double *lg, int E, int k, in
 
 // Renormalised gates of the selected experts: g_i = exp(l_i - l_0) / sum_j exp(l_j - l_0),
 // lanes 0..k-1 each one exp in fp64, the sum taken in top-k order.
-__device__ __noinline__ void warp_topk_gates(const double *lg, int k, const int32_t *idx, double *g64, float *g32) {
+static __device__ __noinline__ void warp_topk_gates(const double *lg, int k, const int32_t *idx, double *g64, float *g32) {
     const int lane = threadIdx.x & 31;
     const double my_l = (lane < k) ? lg[idx[lane]] : 0.0;
     const double l0 = __shfl_sync(0xFFFFFFFFu, my_l, 0);
