@@ -301,6 +301,21 @@ def run_reference(args):
     return 0
 
 
+def run_latency_probe(args):
+    """--latency-probe: compile and run ternary_weight_moe_b200/probes/latency_probe.cu (dependent
+    operation chains, barriers, two top-k formulations, bulk-copy issue; cycles) and print its
+    JSON line."""
+    here = os.path.join(ROOT, "ternary_weight_moe_b200")
+    src = os.path.join(here, "probes", "latency_probe.cu")
+    exe = os.path.join(here, "_build", "latency_probe")
+    os.makedirs(os.path.dirname(exe), exist_ok=True)
+    subprocess.check_call(["/usr/local/cuda/bin/nvcc", "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a",
+                           "-fmad=false", "--expt-relaxed-constexpr", "-o", exe, src])
+    out = subprocess.run([exe], capture_output=True, text=True, timeout=300)
+    print(out.stdout.strip(), flush=True)
+    return out.returncode
+
+
 def run_gemv_sweep(args):
     """Extra output: device time of one tern_gemv launch (four codes per byte) and one
     tern5_gemv launch (five weights per byte, base 3) per shape of the GEMV sweep (T = 1, bf16
@@ -485,6 +500,8 @@ def main():
     ap.add_argument("--batch-sweep", action="store_true",
                     help="extra output: time one MoE FFN layer at T = 1, 4, 16, 64 tokens per step")
     ap.add_argument("--batch-T", default=None, help="with --batch-sweep: comma-separated T values only")
+    ap.add_argument("--latency-probe", action="store_true",
+                    help="compile and run the on-chip latency probe (probes/latency_probe.cu) and print its JSON")
     ap.add_argument("--head", action="store_true",
                     help="extra output: time the approximate output head against the full head")
     args = ap.parse_args()
@@ -492,6 +509,8 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.latency_probe:
+        return run_latency_probe(args)
     if args.sweep:
         return run_gemv_sweep(args)
     if args.batch_sweep:

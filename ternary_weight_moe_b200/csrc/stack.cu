@@ -364,9 +364,10 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
         float nf[4];
         {
             uint16_t nb[4];
+            const double rinv = 1.0 / r;
 #pragma unroll
             for (int e = 0; e < 4; e++) {
-                nb[e] = f64_to_bf16_rne((double)xv[e] / r);
+                nb[e] = bf16_of_quotient((double)xv[e], r, rinv);
                 nf[e] = bf16_to_f32(nb[e]);
                 nd[e] = (double)nf[e];
             }
@@ -379,17 +380,30 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
         // one rounding (the sums are exact at these magnitudes: the order does not matter)
         if (nr > 0) {
             if (!mbar_wait_sleep(&mb_r[par], (uint32_t)((l >> 1) & 1), lim, p.status)) alive = false;
+            const uint16_t *rb = par ? rbuf1 : rbuf0;
 #pragma unroll 1
-            for (int q = 0; q < nr; q++) {
-                {
-                    const uint2 w = reinterpret_cast<const uint2 *>((par ? rbuf1 : rbuf0) + (size_t)q * d)[tid];
-                    double a = 0.0;
-                    a = fma(bf16_to_f64((uint16_t)(w.x & 0xFFFFu)), nd[0], a);
-                    a = fma(bf16_to_f64((uint16_t)(w.x >> 16)), nd[1], a);
-                    a = fma(bf16_to_f64((uint16_t)(w.y & 0xFFFFu)), nd[2], a);
-                    a = fma(bf16_to_f64((uint16_t)(w.y >> 16)), nd[3], a);
-                    a = warp_sum_f64(a);
-                    if (lane == 0) s_rp[warp][q] = a;
+            for (int q = 0; q < nr; q += 2) {
+                // rows q and q + 1 together (two independent chains); a missing second row is 0
+                const uint2 w0 = reinterpret_cast<const uint2 *>(rb + (size_t)q * d)[tid];
+                const uint2 w1 = q + 1 < nr ? reinterpret_cast<const uint2 *>(rb + (size_t)(q + 1) * d)[tid]
+                                            : make_uint2(0u, 0u);
+                double a0 = 0.0, a1 = 0.0;
+                a0 = fma(bf16_to_f64((uint16_t)(w0.x & 0xFFFFu)), nd[0], a0);
+                a1 = fma(bf16_to_f64((uint16_t)(w1.x & 0xFFFFu)), nd[0], a1);
+                a0 = fma(bf16_to_f64((uint16_t)(w0.x >> 16)), nd[1], a0);
+                a1 = fma(bf16_to_f64((uint16_t)(w1.x >> 16)), nd[1], a1);
+                a0 = fma(bf16_to_f64((uint16_t)(w0.y & 0xFFFFu)), nd[2], a0);
+                a1 = fma(bf16_to_f64((uint16_t)(w1.y & 0xFFFFu)), nd[2], a1);
+                a0 = fma(bf16_to_f64((uint16_t)(w0.y >> 16)), nd[3], a0);
+                a1 = fma(bf16_to_f64((uint16_t)(w1.y >> 16)), nd[3], a1);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    a0 += __shfl_xor_sync(0xFFFFFFFFu, a0, o);
+                    a1 += __shfl_xor_sync(0xFFFFFFFFu, a1, o);
+                }
+                if (lane == 0) {
+                    s_rp[warp][q] = a0;
+                    if (q + 1 < nr) s_rp[warp][q + 1] = a1;
                 }
             }
         }
@@ -616,27 +630,43 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             seg_load_x_padded<NL>(Hx, hl, hlp, gl);
             const int sdo = (int)(((size_t)s_idx[s] * d + i0) & 3);  // offset of row i0's scale in s_sdb
             const uint32_t ytag = tag;
-            for (int r0 = warp * rpp; r0 < ndn; r0 += kStackWarps * rpp) {
-                const int rr = r0 + sub;
-                const bool valid = rr < ndn;
-                int acc[NL];
+            const int step = kStackWarps * rpp;
+            // two rows per lane group at a time (independent chains), then both reductions
+#pragma unroll 1
+            for (int r0 = warp * rpp; r0 < ndn; r0 += 2 * step) {
+                const int ra = r0 + sub, rb2 = r0 + step + sub;
+                const bool va = ra < ndn, vb = rb2 < ndn;
+                int acca[NL], accb[NL];
 #pragma unroll
-                for (int z = 0; z < NL; z++) acc[z] = 0;
-                const uint4 wd = *reinterpret_cast<const uint4 *>(dbuf + (size_t)(valid ? rr : 0) * (f / 4) + gl * 16);
-                seg_dot_alu<NL>(wd, Hx, acc);
-                int aa, bb;
-                acc_to_pair_x64<NL>(acc, aa, bb);
+                for (int z = 0; z < NL; z++) acca[z] = accb[z] = 0;
+                const uint4 wa = *reinterpret_cast<const uint4 *>(dbuf + (size_t)(va ? ra : 0) * (f / 4) + gl * 16);
+                const uint4 wb = *reinterpret_cast<const uint4 *>(dbuf + (size_t)(vb ? rb2 : 0) * (f / 4) + gl * 16);
+                seg_dot_alu<NL>(wa, Hx, acca);
+                seg_dot_alu<NL>(wb, Hx, accb);
+                int aa, ab, ba, bb;
+                acc_to_pair_x64<NL>(acca, aa, ab);
+                acc_to_pair_x64<NL>(accb, ba, bb);
                 for (int o = Gf / 2; o > 0; o >>= 1) {
                     aa += __shfl_xor_sync(0xFFFFFFFFu, aa, o);
-                    if (NL > 1) bb += __shfl_xor_sync(0xFFFFFFFFu, bb, o);
+                    ba += __shfl_xor_sync(0xFFFFFFFFu, ba, o);
+                    if (NL > 1) {
+                        ab += __shfl_xor_sync(0xFFFFFFFFu, ab, o);
+                        bb += __shfl_xor_sync(0xFFFFFFFFu, bb, o);
+                    }
                 }
-                if (valid && gl == 0) {
-                    const long long S = pair_value(NL, aa, bb);
-                    const float sd = s_sdb[rr + sdo];
-                    float v;
-                    if (NL == 1) v = __fmul_rn(__fmul_rn(__int2float_rn((int)S), sd), hsc);
-                    else v = (float)((double)S * pow2_f64(-hsh) * (double)sd);
-                    st_word(p.yb + (((size_t)par * G + c) * k + s) * kMaxDN + rr, __float_as_uint(v), ytag);
+                if (gl == 0) {
+                    const double p2 = pow2_f64(-hsh);
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; h2++) {
+                        const int rr = h2 ? rb2 : ra;
+                        if (!(h2 ? vb : va)) continue;
+                        const long long S = pair_value(NL, h2 ? ba : aa, h2 ? bb : ab);
+                        const float sd = s_sdb[rr + sdo];
+                        float v;
+                        if (NL == 1) v = __fmul_rn(__fmul_rn(__int2float_rn((int)S), sd), hsc);
+                        else v = (float)((double)S * p2 * (double)sd);
+                        st_word(p.yb + (((size_t)par * G + c) * k + s) * kMaxDN + rr, __float_as_uint(v), ytag);
+                    }
                 }
             }
         }

@@ -64,6 +64,26 @@ __device__ __forceinline__ double pow2_f64(int e) {
     return __longlong_as_double((long long)(unsigned long long)(1023 + e) << 52);
 }
 
+// bf16(x / r), nearest even, as f64_to_bf16_rne(x / r), from q = x * rinv (rinv = 1 / r rounded):
+// q is within a few units in the last place of the exact quotient, so its bf16 rounding is the
+// quotient's unless q lies within 8 units of a point halfway between two bf16 values (or outside
+// the normal bf16 range); those take the exact division.  The rounding itself is integer
+// arithmetic on q's bits: the top 19 bits (sign, exponent, 7 mantissa bits) plus one when the
+// 45 bits below exceed the halfway point or equal it with an odd last kept bit.
+__device__ __forceinline__ uint16_t bf16_of_quotient(double x, double r, double rinv) {
+    const double q = x * rinv;
+    const unsigned long long b = (unsigned long long)__double_as_longlong(q);
+    const unsigned long long low = b & ((1ull << 45) - 1), half = 1ull << 44;
+    const long long dist = (long long)low - (long long)half;
+    const uint32_t e11 = (uint32_t)(b >> 52) & 0x7FFu;
+    if (dist >= -8 && dist <= 8) return f64_to_bf16_rne(x / r);        // near a tie: exact path
+    if (e11 < 1023 - 126 + 1 || e11 > 1023 + 127 - 1) return f64_to_bf16_rne(x / r);  // not a normal bf16
+    uint32_t t = (uint32_t)(b >> 45);                                   // sign | e11 | 7 mantissa bits
+    t += (dist > 0) ? 1u : 0u;                                          // no ties here (|dist| > 8)
+    const uint32_t sign = (t >> 18) & 1u, e = (t >> 7) & 0x7FFu, m = t & 0x7Fu;
+    return (uint16_t)((sign << 15) | ((e - 896u) << 7) | m);
+}
+
 // ---------------------------------------------------------------------------- dp4a
 __device__ __forceinline__ int dp4a_ss(uint32_t a, uint32_t b, int c) {
     return __dp4a((int)a, (int)b, c);

@@ -1,0 +1,309 @@
+// latency_probe.cu -- measurements of the on-chip latencies the persistent decode kernel is
+// built around, on the current GPU (a standalone program, not part of libternmoe; run with
+// `python bench.py --latency-probe`, which compiles it with nvcc and prints its JSON).
+//
+// Every figure is a median over repetitions of clock64 differences read by one thread, in SM
+// cycles:
+//   chain_*      one warp, one dependent chain of 256 operations: cycles per operation
+//   bar_*        a CTA barrier (512 threads) / a named barrier (256 threads): cycles per barrier
+//   topk_*       top-8 of 256 fp64 logits (ties to the lower index): the one-warp filter of the
+//                library (tern_common.cuh) and a CTA-wide filter, cycles per selection
+//   bulk_*       issuing bulk copies (cp.async.bulk global -> shared): n copies from one lane,
+//                or one copy from each of n warps; cycles until the issuing returns / until all
+//                copies have landed
+// Every wait is bounded; nothing here waits on another CTA.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdio.h>
+
+#include <algorithm>
+#include <vector>
+
+#include "../csrc/tern_common.cuh"
+#include "../csrc/tma.cuh"
+
+using namespace tern;
+
+constexpr int kReps = 64;
+
+__global__ void chains(unsigned long long *out, const double *dsrc, const int *isrc) {
+    __shared__ int s_i[1024];
+    __shared__ double s_d[256];
+    const int lane = threadIdx.x & 31;
+    for (int i = threadIdx.x; i < 1024; i += blockDim.x) s_i[i] = (i * 7 + 3) & 1023;
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) s_d[i] = dsrc[i];
+    __syncthreads();
+    if (threadIdx.x >= 32) return;
+    unsigned long long t0, t1;
+    // SHFL chain
+    int v = lane;
+    t0 = clock64();
+#pragma unroll 1
+    for (int i = 0; i < 256; i++) v = __shfl_xor_sync(0xFFFFFFFFu, v, 1) + 1;
+    t1 = clock64();
+    if (lane == 0) out[0] = (t1 - t0);
+    // LDS chain (pointer chasing)
+    int ix = lane;
+    t0 = clock64();
+#pragma unroll 1
+    for (int i = 0; i < 256; i++) ix = s_i[ix];
+    t1 = clock64();
+    if (lane == 0) out[1] = (t1 - t0);
+    // DFMA chain
+    double a = dsrc[lane], b = dsrc[lane + 1];
+    t0 = clock64();
+#pragma unroll 1
+    for (int i = 0; i < 256; i++) a = fma(a, b, 1.0);
+    t1 = clock64();
+    if (lane == 0) out[2] = (t1 - t0);
+    // fp64 division chain
+    double q = dsrc[lane] + 2.0;
+    t0 = clock64();
+#pragma unroll 1
+    for (int i = 0; i < 256; i++) q = 3.0 / q;
+    t1 = clock64();
+    if (lane == 0) out[3] = (t1 - t0);
+    // redux.sync max chain
+    unsigned m = (unsigned)lane;
+    t0 = clock64();
+#pragma unroll 1
+    for (int i = 0; i < 256; i++) m = __reduce_max_sync(0xFFFFFFFFu, m + (unsigned)lane) & 0xFFFFu;
+    t1 = clock64();
+    if (lane == 0) out[4] = (t1 - t0);
+    // fp32 -> fp64 -> fp32 conversion chain
+    float fl = (float)dsrc[lane];
+    t0 = clock64();
+#pragma unroll 1
+    for (int i = 0; i < 256; i++) fl = (float)((double)fl * 1.0000001);
+    t1 = clock64();
+    if (lane == 0) out[5] = (t1 - t0);
+    // integer ALU chain
+    unsigned u = (unsigned)lane;
+    t0 = clock64();
+#pragma unroll 1
+    for (int i = 0; i < 256; i++) u = (u ^ (u >> 3)) + 0x9E37u;
+    t1 = clock64();
+    if (lane == 0) out[6] = (t1 - t0);
+    // keep results alive
+    if (v == -1 || ix == -1 || a == -1.0 || q == -1.0 || m == 0xFFFFFFFFu || fl == -1.0f || u == 1u) out[7] = 1;
+}
+
+__global__ void barriers(unsigned long long *out) {
+    unsigned long long t0 = clock64();
+#pragma unroll 1
+    for (int i = 0; i < 256; i++) __syncthreads();
+    unsigned long long t1 = clock64();
+    if (threadIdx.x == 0) out[0] = t1 - t0;
+    if (threadIdx.x < 256) {
+        t0 = clock64();
+#pragma unroll 1
+        for (int i = 0; i < 256; i++) named_bar_sync(1, 256);
+        t1 = clock64();
+        if (threadIdx.x == 0) out[1] = t1 - t0;
+    }
+}
+
+// CTA-wide filter: thread t < E holds logit t; result in idx_out (shared); all threads call.
+__device__ void block_filter(const double *lg, int E, int k, int32_t *idx_out, uint32_t *s_gm, int *s_nc,
+                             ulonglong2 *s_cand) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    const bool has = tid < E;
+    const unsigned long long key = has ? f64_order_key(lg[tid]) : 0ull;
+    const uint32_t h = (uint32_t)(key >> 32);
+    uint32_t gm = h;
+    gm = max(gm, __shfl_xor_sync(0xFFFFFFFFu, gm, 1));
+    gm = max(gm, __shfl_xor_sync(0xFFFFFFFFu, gm, 2));
+    gm = max(gm, __shfl_xor_sync(0xFFFFFFFFu, gm, 4));
+    if (tid < 256 && (tid & 7) == 0) s_gm[tid >> 3] = gm;
+    if (tid == 0) *s_nc = 0;
+    __syncthreads();
+    if (tid < 256) {
+        const uint32_t mm = s_gm[lane];
+        int above = 0;
+#pragma unroll
+        for (int q4 = 0; q4 < 8; q4++) {
+            const uint4 v = reinterpret_cast<const uint4 *>(s_gm)[q4];
+            const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int z = 0; z < 4; z++) above += (vv[z] > mm || (vv[z] == mm && 4 * q4 + z < lane)) ? 1 : 0;
+        }
+        const unsigned who = __ballot_sync(0xFFFFFFFFu, above == k - 1);
+        const uint32_t tau = __shfl_sync(0xFFFFFFFFu, mm, __ffs(who) - 1);
+        const bool take = has && h >= tau;
+        const unsigned msk = __ballot_sync(0xFFFFFFFFu, take);
+        int base = 0;
+        if (lane == 0 && msk) base = atomicAdd(s_nc, __popc(msk));
+        base = __shfl_sync(0xFFFFFFFFu, base, 0);
+        if (take) s_cand[base + __popc(msk & ((1u << lane) - 1u))] = make_ulonglong2(key, (unsigned long long)tid);
+    }
+    __syncthreads();
+    const int nc = *s_nc;
+    if (tid < nc) {
+        const ulonglong2 me = s_cand[tid];
+        int r = 0;
+        for (int q = 0; q < nc; q++) {
+            const ulonglong2 o = s_cand[q];
+            r += (o.x > me.x || (o.x == me.x && o.y < me.y)) ? 1 : 0;
+        }
+        if (r < k) idx_out[r] = (int)me.y;
+    }
+    __syncthreads();
+}
+
+__global__ void topk_bench(const double *logits, unsigned long long *out, int32_t *idx_a, int32_t *idx_b) {
+    __shared__ double lg[256];
+    __shared__ int32_t s_idx[8];
+    __shared__ ulonglong2 cand[256];
+    __shared__ __align__(16) uint32_t s_gm[32];
+    __shared__ int s_nc;
+    for (int rep = 0; rep < kReps; rep++) {
+        if (threadIdx.x < 256) lg[threadIdx.x] = logits[rep * 256 + threadIdx.x];
+        __syncthreads();
+        unsigned long long t0 = clock64();
+        if (threadIdx.x < 32) warp_topk_filter(lg, 256, 8, s_idx, cand);
+        __syncthreads();
+        unsigned long long t1 = clock64();
+        if (threadIdx.x < 8) idx_a[rep * 8 + threadIdx.x] = s_idx[threadIdx.x];
+        if (threadIdx.x == 0) out[2 * rep] = t1 - t0;
+        __syncthreads();
+        t0 = clock64();
+        block_filter(lg, 256, 8, s_idx, s_gm, &s_nc, cand);
+        t1 = clock64();
+        if (threadIdx.x < 8) idx_b[rep * 8 + threadIdx.x] = s_idx[threadIdx.x];
+        if (threadIdx.x == 0) out[2 * rep + 1] = t1 - t0;
+        __syncthreads();
+    }
+}
+
+// bulk copies of `bytes` each from src into shared memory: mode 0 = n copies from lane 0 of
+// warp 0, mode 1 = one copy from lane 0 of each of n warps.
+__global__ void bulk_issue(const uint8_t *src, int n, int bytes, int mode, unsigned long long *out, int *status) {
+    extern __shared__ __align__(128) uint8_t sm[];
+    __shared__ __align__(8) uint64_t mb;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(&mb, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    for (int rep = 0; rep < 8; rep++) {
+        if (threadIdx.x == 0) mbar_expect_tx(&mb, (uint32_t)(n * bytes));
+        __syncthreads();
+        const unsigned long long t0 = clock64();
+        const uint8_t *s = src + (size_t)rep * n * bytes;
+        if (mode == 0) {
+            if (threadIdx.x == 0)
+                for (int i = 0; i < n; i++) bulk_g2s(sm + (size_t)i * bytes, s + (size_t)i * bytes, (uint32_t)bytes, &mb);
+        } else if (warp < n && lane == 0) {
+            bulk_g2s(sm + (size_t)warp * bytes, s + (size_t)warp * bytes, (uint32_t)bytes, &mb);
+        }
+        __syncthreads();
+        const unsigned long long t1 = clock64();
+        mbar_wait(&mb, (uint32_t)(rep & 1), 1000000000ll, status);
+        const unsigned long long t2 = clock64();
+        if (threadIdx.x == 0) {
+            out[2 * rep] = t1 - t0;
+            out[2 * rep + 1] = t2 - t0;
+        }
+        __syncthreads();
+    }
+}
+
+static double median(std::vector<double> v) {
+    std::sort(v.begin(), v.end());
+    return v.empty() ? 0.0 : v[v.size() / 2];
+}
+
+#define CK(x)                                                                                         \
+    do {                                                                                              \
+        cudaError_t e_ = (x);                                                                         \
+        if (e_ != cudaSuccess) {                                                                      \
+            printf("{\"error\": \"%s: %s\"}\n", #x, cudaGetErrorString(e_));                          \
+            return 1;                                                                                 \
+        }                                                                                             \
+    } while (0)
+
+int main() {
+    CK(cudaSetDevice(0));
+    unsigned long long *d_out;
+    double *d_lg;
+    int *d_st, *d_i;
+    int32_t *d_ia, *d_ib;
+    uint8_t *d_src;
+    CK(cudaMalloc(&d_out, 4096 * 8));
+    CK(cudaMalloc(&d_lg, kReps * 256 * 8));
+    CK(cudaMalloc(&d_st, 4));
+    CK(cudaMalloc(&d_i, 4096));
+    CK(cudaMalloc(&d_ia, kReps * 8 * 4));
+    CK(cudaMalloc(&d_ib, kReps * 8 * 4));
+    CK(cudaMalloc(&d_src, 64 << 20));
+    CK(cudaMemset(d_src, 1, 64 << 20));
+    CK(cudaMemset(d_st, 0, 4));
+    // logits: N(0, 1)-like values from a small LCG, a few exact ties
+    std::vector<double> h(kReps * 256);
+    unsigned long long z = 0x1234567ull;
+    for (auto &x : h) {
+        z = z * 6364136223846793005ull + 1442695040888963407ull;
+        x = ((double)(z >> 11) / 9007199254740992.0 - 0.5) * 4.0;
+    }
+    for (int r = 0; r < kReps; r += 8) h[r * 256 + 17] = h[r * 256 + 200];
+    CK(cudaMemcpy(d_lg, h.data(), h.size() * 8, cudaMemcpyHostToDevice));
+    std::vector<unsigned long long> o(4096);
+
+    printf("{");
+    chains<<<1, 128>>>(d_out, d_lg, d_i);
+    CK(cudaDeviceSynchronize());
+    CK(cudaMemcpy(o.data(), d_out, 8 * 8, cudaMemcpyDeviceToHost));
+    const char *names[] = {"chain_shfl", "chain_lds", "chain_dfma", "chain_f64_div", "chain_redux_max",
+                           "chain_f32_f64_f32", "chain_int_alu"};
+    for (int i = 0; i < 7; i++) printf("\"%s\": %.1f, ", names[i], o[i] / 256.0);
+
+    barriers<<<1, 512>>>(d_out);
+    CK(cudaDeviceSynchronize());
+    CK(cudaMemcpy(o.data(), d_out, 2 * 8, cudaMemcpyDeviceToHost));
+    printf("\"bar_cta512\": %.1f, \"bar_named256\": %.1f, ", o[0] / 256.0, o[1] / 256.0);
+
+    topk_bench<<<1, 512>>>(d_lg, d_out, d_ia, d_ib);
+    CK(cudaDeviceSynchronize());
+    CK(cudaMemcpy(o.data(), d_out, 2 * kReps * 8, cudaMemcpyDeviceToHost));
+    std::vector<double> ta, tb;
+    for (int r = 1; r < kReps; r++) {
+        ta.push_back((double)o[2 * r]);
+        tb.push_back((double)o[2 * r + 1]);
+    }
+    std::vector<int32_t> ia(kReps * 8), ib(kReps * 8);
+    CK(cudaMemcpy(ia.data(), d_ia, ia.size() * 4, cudaMemcpyDeviceToHost));
+    CK(cudaMemcpy(ib.data(), d_ib, ib.size() * 4, cudaMemcpyDeviceToHost));
+    // check both against a host selection (larger first, ties to the lower index)
+    int bad = 0;
+    for (int r = 0; r < kReps; r++) {
+        std::vector<int> ord(256);
+        for (int i = 0; i < 256; i++) ord[i] = i;
+        std::stable_sort(ord.begin(), ord.end(), [&](int a, int b) { return h[r * 256 + a] > h[r * 256 + b]; });
+        for (int j = 0; j < 8; j++) bad += (ia[r * 8 + j] != ord[j]) + (ib[r * 8 + j] != ord[j]);
+    }
+    printf("\"topk_warp_filter\": %.0f, \"topk_block_filter\": %.0f, \"topk_mismatches\": %d, ", median(ta), median(tb),
+           bad);
+
+    CK(cudaFuncSetAttribute(bulk_issue, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024));
+    for (int mode = 0; mode < 2; mode++) {
+        for (int n : {1, 4, 8}) {
+            bulk_issue<<<1, 512, 128 * 1024>>>(d_src, n, 8192, mode, d_out, d_st);
+            CK(cudaDeviceSynchronize());
+            CK(cudaMemcpy(o.data(), d_out, 16 * 8, cudaMemcpyDeviceToHost));
+            std::vector<double> iss, land;
+            for (int r = 1; r < 8; r++) {
+                iss.push_back((double)o[2 * r]);
+                land.push_back((double)o[2 * r + 1]);
+            }
+            printf("\"bulk_%s_%d_issue\": %.0f, \"bulk_%s_%d_landed\": %.0f, ", mode ? "warps" : "lane", n, median(iss),
+                   mode ? "warps" : "lane", n, median(land));
+        }
+    }
+    int st = 0;
+    CK(cudaMemcpy(&st, d_st, 4, cudaMemcpyDeviceToHost));
+    int clk = 0;
+    cudaDeviceGetAttribute(&clk, cudaDevAttrClockRate, 0);
+    printf("\"status\": %d, \"clock_khz\": %d}\n", st, clk);
+    return 0;
+}
