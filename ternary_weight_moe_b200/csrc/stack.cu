@@ -68,8 +68,9 @@ constexpr int kMaxGroup = 32;       // CTAs per slot group
 constexpr int kMaxGU = 32;          // gate/up rows per CTA (two chunks of 16)
 constexpr int kMaxDN = 128;         // down rows per CTA
 constexpr int kMaxRouterRows = 8;   // router rows per CTA
-constexpr int kPredTop = 12;        // predicted next-layer experts prefetched to L2
+constexpr int kPredTop = 10;        // at least this many predicted next-layer experts go to L2
 constexpr int kTracePoints = 24;
+constexpr int kRouterWarps = 4;     // warps that compute the router rows (16 columns per thread)
 constexpr long long kPredictWaitCycles = 10000;  // the prediction exchange is a hint: give up after ~5 us
 constexpr unsigned kPollSleepNs = 32;           // sleep between two polls of a tagged word
 constexpr int kTraceExtra = 8;                  // stamps inside the layer's phases (15 .. 22)
@@ -133,7 +134,7 @@ __device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool pred) {
 
 // ------------------------------------------------------------------ shared memory map
 struct SmemMap {
-    uint32_t gbuf, ubuf, dbuf, rbuf0, rbuf1, xs, ns, xl, hl, lg, plg, hv, yv, cand, total;
+    uint32_t gbuf, ubuf, dbuf, rbuf0, rbuf1, xs, ns, xl, hl, lg, hv, yv, cand, total;
 };
 
 __host__ __device__ inline uint32_t align128(uint32_t v) { return (v + 127u) & ~127u; }
@@ -156,7 +157,6 @@ __host__ __device__ inline SmemMap smem_map(int d, int f, int k, int gu_max, int
     m.xl = take((uint32_t)NL * (d / 64) * kSegPad * 4);
     m.hl = take((uint32_t)NL * (f / 64) * kSegPad * 4);
     m.lg = take(256 * 8);
-    m.plg = take(256 * 8);
     m.hv = take((uint32_t)f * 4);
     m.yv = take((uint32_t)k * kMaxDN * 4);
     m.cand = take(256 * 16);
@@ -199,7 +199,6 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
     __shared__ double s_xss[kMaxGroup];
     __shared__ float s_xam[kMaxGroup];
     __shared__ int32_t s_idx[kSK];
-    __shared__ int32_t s_pidx[kPredTop];
     __shared__ double s_gate[kSK];
     __shared__ long long s_S[kMaxGU][2];
     // scales of this CTA's rows, bulk-copied with the rows: a 16-byte aligned superset of the
@@ -230,7 +229,6 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
     uint32_t *xl = reinterpret_cast<uint32_t *>(smem + sm.xl);
     uint32_t *hl = reinterpret_cast<uint32_t *>(smem + sm.hl);
     double *lg = reinterpret_cast<double *>(smem + sm.lg);
-    double *plg = reinterpret_cast<double *>(smem + sm.plg);
     float *hv = reinterpret_cast<float *>(smem + sm.hv);
     float *yv = reinterpret_cast<float *>(smem + sm.yv);
     ulonglong2 *cand = reinterpret_cast<ulonglong2 *>(smem + sm.cand);
@@ -345,10 +343,18 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                     ta = fmaxf(ta, s_redf[w]);
                 }
             } else {
-                for (int q = 0; q < G; q++) {
-                    ts += s_xss[q];
-                    ta = fmaxf(ta, s_xam[q]);
+                // pairwise tree over the (up to 32) parts, the same order in every thread and CTA
+                double v[kMaxGroup];
+#pragma unroll
+                for (int q = 0; q < kMaxGroup; q++) {
+                    v[q] = q < G ? s_xss[q] : 0.0;
+                    ta = fmaxf(ta, q < G ? s_xam[q] : 0.0f);
                 }
+#pragma unroll
+                for (int w = kMaxGroup / 2; w > 0; w >>= 1)
+#pragma unroll
+                    for (int q = 0; q < w; q++) v[q] += v[q + w];
+                ts = v[0];
             }
             r = sqrt(ts / (double)d + p.eps);
             amax = ta;
@@ -360,68 +366,72 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
         const float amax_n = bf16_to_f32(f64_to_bf16_rne((double)amax / r));
         const float s_nq = (NL == 1) ? (amax_n > 0.0f ? __fdiv_rn(amax_n, 127.0f) : 0.0f) : 0.0f;
         const int sh_n = (NL == 1) ? 0 : fixed_shift(amax_n);
-        double nd[4];
-        float nf[4];
         {
             uint16_t nb[4];
             const double rinv = 1.0 / r;
 #pragma unroll
-            for (int e = 0; e < 4; e++) {
-                nb[e] = bf16_of_quotient((double)xv[e], r, rinv);
-                nf[e] = bf16_to_f32(nb[e]);
-                nd[e] = (double)nf[e];
-            }
+            for (int e = 0; e < 4; e++) nb[e] = bf16_of_quotient((double)xv[e], r, rinv);
             reinterpret_cast<uint2 *>(ns)[tid] =
                 make_uint2((uint32_t)nb[0] | ((uint32_t)nb[1] << 16), (uint32_t)nb[2] | ((uint32_t)nb[3] << 16));
         }
+        __syncthreads();  // n (shared) complete
         TSTAMP(l, 16)  // n known
-        // router rows of this layer: thread t multiplies columns 4t..4t+3; bf16 x bf16 has at
-        // most 16 significant bits, so each product is exact in fp64 and the fma adds it with
-        // one rounding (the sums are exact at these magnitudes: the order does not matter)
-        if (nr > 0) {
-            if (!mbar_wait_sleep(&mb_r[par], (uint32_t)((l >> 1) & 1), lim, p.status)) alive = false;
-            const uint16_t *rb = par ? rbuf1 : rbuf0;
-#pragma unroll 1
-            for (int q = 0; q < nr; q += 2) {
-                // rows q and q + 1 together (two independent chains); a missing second row is 0
-                const uint2 w0 = reinterpret_cast<const uint2 *>(rb + (size_t)q * d)[tid];
-                const uint2 w1 = q + 1 < nr ? reinterpret_cast<const uint2 *>(rb + (size_t)(q + 1) * d)[tid]
-                                            : make_uint2(0u, 0u);
-                double a0 = 0.0, a1 = 0.0;
-                a0 = fma(bf16_to_f64((uint16_t)(w0.x & 0xFFFFu)), nd[0], a0);
-                a1 = fma(bf16_to_f64((uint16_t)(w1.x & 0xFFFFu)), nd[0], a1);
-                a0 = fma(bf16_to_f64((uint16_t)(w0.x >> 16)), nd[1], a0);
-                a1 = fma(bf16_to_f64((uint16_t)(w1.x >> 16)), nd[1], a1);
-                a0 = fma(bf16_to_f64((uint16_t)(w0.y & 0xFFFFu)), nd[2], a0);
-                a1 = fma(bf16_to_f64((uint16_t)(w1.y & 0xFFFFu)), nd[2], a1);
-                a0 = fma(bf16_to_f64((uint16_t)(w0.y >> 16)), nd[3], a0);
-                a1 = fma(bf16_to_f64((uint16_t)(w1.y >> 16)), nd[3], a1);
+        // Router rows of this layer on warps 0..3: thread t (< 128) multiplies columns
+        // 16t..16t+15 (n from shared memory); bf16 x bf16 has at most 16 significant bits, so
+        // each product is exact in fp64 and every fma adds it with one rounding (the sums are
+        // exact at these magnitudes: the order does not matter).  Warps 4..15 meanwhile build
+        // the activation limbs of the gate/up dots.
+        if (warp < kRouterWarps) {
+            if (nr > 0) {
+                if (!mbar_wait_sleep(&mb_r[par], (uint32_t)((l >> 1) & 1), lim, p.status)) alive = false;
+                double nv[16];
+                {
+                    const uint4 *np4 = reinterpret_cast<const uint4 *>(ns) + 2 * tid;
+                    const uint4 n0v = np4[0], n1v = np4[1];
+                    const uint32_t nw[8] = {n0v.x, n0v.y, n0v.z, n0v.w, n1v.x, n1v.y, n1v.z, n1v.w};
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    a0 += __shfl_xor_sync(0xFFFFFFFFu, a0, o);
-                    a1 += __shfl_xor_sync(0xFFFFFFFFu, a1, o);
+                    for (int z = 0; z < 8; z++) {
+                        nv[2 * z] = bf16_to_f64((uint16_t)(nw[z] & 0xFFFFu));
+                        nv[2 * z + 1] = bf16_to_f64((uint16_t)(nw[z] >> 16));
+                    }
                 }
-                if (lane == 0) {
-                    s_rp[warp][q] = a0;
-                    if (q + 1 < nr) s_rp[warp][q + 1] = a1;
+                const uint16_t *rb = par ? rbuf1 : rbuf0;
+#pragma unroll 1
+                for (int q = 0; q < nr; q++) {
+                    const uint4 *wp = reinterpret_cast<const uint4 *>(rb + (size_t)q * d) + 2 * tid;
+                    const uint4 w0v = wp[0], w1v = wp[1];
+                    const uint32_t ww[8] = {w0v.x, w0v.y, w0v.z, w0v.w, w1v.x, w1v.y, w1v.z, w1v.w};
+                    double a[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+                    for (int z = 0; z < 8; z++) {
+                        a[(2 * z) & 3] = fma(bf16_to_f64((uint16_t)(ww[z] & 0xFFFFu)), nv[2 * z], a[(2 * z) & 3]);
+                        a[(2 * z + 1) & 3] = fma(bf16_to_f64((uint16_t)(ww[z] >> 16)), nv[2 * z + 1], a[(2 * z + 1) & 3]);
+                    }
+                    double t = (a[0] + a[1]) + (a[2] + a[3]);
+                    t = warp_sum_f64(t);
+                    if (lane == 0) s_rp[warp][q] = t;
                 }
+            }
+        } else {
+            // limbs of elements 4u..4u+3 for u = tid - 128 and u + 384 (all 512 quads)
+            const float inv = (NL == 1 && amax_n > 0.0f) ? quant_inv(amax_n) : 0.0f;
+            for (int u = tid - kRouterWarps * 32; u < d / 4; u += kStackThreads - kRouterWarps * 32) {
+                const uint2 nb2 = reinterpret_cast<const uint2 *>(ns)[u];
+                const float v4[4] = {bf16_to_f32((uint16_t)(nb2.x & 0xFFFFu)), bf16_to_f32((uint16_t)(nb2.x >> 16)),
+                                     bf16_to_f32((uint16_t)(nb2.y & 0xFFFFu)), bf16_to_f32((uint16_t)(nb2.y >> 16))};
+                store_limbs4<NL>(xl, xlp, u, v4, sh_n, inv, amax_n > 0.0f);
             }
         }
         TSTAMP(l, 17)  // this warp's router partials written
         if (!__syncthreads_and(alive ? 1 : 0)) break;  // router partials (and n) visible
         if (tid < nr) {
             double sum = 0.0;
-            for (int w = 0; w < kStackWarps; w++) sum += s_rp[w][tid];
+            for (int w = 0; w < kRouterWarps; w++) sum += s_rp[w][tid];
             const unsigned long long b = (unsigned long long)__double_as_longlong(sum);
             st_relaxed_v2(p.lb + ((size_t)par * E + e0 + tid) * 2, tagged((uint32_t)(b >> 32), tag),
                           tagged((uint32_t)b, tag));
         }
         TSTAMP(l, 2)
-        // activation limbs for the gate/up dots (needed only after top-k and the row copies)
-        {
-            const float inv = (NL == 1 && amax_n > 0.0f) ? quant_inv(amax_n) : 0.0f;
-            store_limbs4<NL>(xl, xlp, tid, nf, sh_n, inv, amax_n > 0.0f);
-        }
         // rbuf[par] is free (this layer's rows are used): fetch the rows of layer l + 2 into it
         if (tid == 0 && nr > 0 && l + 2 < p.n_layers) {
             mbar_expect_tx(&mb_r[par], (uint32_t)(nr * d * 2));
@@ -448,8 +458,8 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
         if (warp == 0) {
             warp_topk_filter(lg, E, k, s_idx, cand);
             TSTAMP(l, 18)  // top-k known
-            // copies of expert idx[s]: first gate/up chunk, second chunk, down rows; thread 0
-            // registers the byte counts first (counted here, so only issued phases are drained)
+            // thread 0 registers the byte counts of this CTA's copies (counted here, so only
+            // issued phases are drained after a timeout); warps 0..7 issue them below
             const size_t e = (size_t)s_idx[s];
             // scales: aligned supersets [ga, ga + gn) of rows j0..j1 and [da, da + dn) of i0..i1
             const size_t ga = (e * f + j0) & ~(size_t)3, da = (e * d + i0) & ~(size_t)3;
@@ -462,22 +472,31 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                 n_gu++;
                 n_dn++;
             }
-            __syncwarp();
-            if (lane < 8) {
-                const uint32_t rowg = (uint32_t)(d / 4), rowd = (uint32_t)(f / 4);
-                if (lane == 0 && n0 > 0) bulk_g2s(gbuf, Ly.gate + (e * f + j0) * rowg, (uint32_t)n0 * rowg, &mb_gu0);
-                if (lane == 1 && n0 > 0) bulk_g2s(ubuf, Ly.up + (e * f + j0) * rowg, (uint32_t)n0 * rowg, &mb_gu0);
-                if (lane == 2 && n1 > 0)
-                    bulk_g2s(gbuf + (size_t)n0 * rowg, Ly.gate + (e * f + j0 + n0) * rowg, (uint32_t)n1 * rowg, &mb_gu1);
-                if (lane == 3 && n1 > 0)
-                    bulk_g2s(ubuf + (size_t)n0 * rowg, Ly.up + (e * f + j0 + n0) * rowg, (uint32_t)n1 * rowg, &mb_gu1);
-                if (lane == 4 && ndn > 0) bulk_g2s(dbuf, Ly.down + (e * d + i0) * rowd, (uint32_t)ndn * rowd, &mb_dn);
-                if (lane == 5) bulk_g2s(s_sgb, Ly.sg + ga, 4u * gn, &mb_gu0);
-                if (lane == 6) bulk_g2s(s_sub, Ly.su + ga, 4u * gn, &mb_gu0);
-                if (lane == 7 && dn > 0) bulk_g2s(s_sdb, Ly.sd + da, 4u * dn, &mb_dn);
-            }
-            TSTAMP(l, 5)
         }
+
+        // the copies, one per warp (a warp issues a bulk copy in ~250 cycles; eight from one
+        // thread take ~700): warps 0..7 meet at hardware barrier 3 once warp 0 has the experts
+        if (warp < 8) {
+            named_bar_sync(3, 256);
+            if (lane == 0) {
+                const size_t e = (size_t)s_idx[s];
+                const size_t ga = (e * f + j0) & ~(size_t)3, da = (e * d + i0) & ~(size_t)3;
+                const uint32_t gn = (uint32_t)((((e * f + j1) + 3) & ~(size_t)3) - ga);
+                const uint32_t dn = ndn > 0 ? (uint32_t)((((e * d + i1) + 3) & ~(size_t)3) - da) : 0u;
+                const uint32_t rowg = (uint32_t)(d / 4), rowd = (uint32_t)(f / 4);
+                if (warp == 0 && n0 > 0) bulk_g2s(gbuf, Ly.gate + (e * f + j0) * rowg, (uint32_t)n0 * rowg, &mb_gu0);
+                if (warp == 1 && n0 > 0) bulk_g2s(ubuf, Ly.up + (e * f + j0) * rowg, (uint32_t)n0 * rowg, &mb_gu0);
+                if (warp == 2 && n1 > 0)
+                    bulk_g2s(gbuf + (size_t)n0 * rowg, Ly.gate + (e * f + j0 + n0) * rowg, (uint32_t)n1 * rowg, &mb_gu1);
+                if (warp == 3 && n1 > 0)
+                    bulk_g2s(ubuf + (size_t)n0 * rowg, Ly.up + (e * f + j0 + n0) * rowg, (uint32_t)n1 * rowg, &mb_gu1);
+                if (warp == 4 && ndn > 0) bulk_g2s(dbuf, Ly.down + (e * d + i0) * rowd, (uint32_t)ndn * rowd, &mb_dn);
+                if (warp == 5) bulk_g2s(s_sgb, Ly.sg + ga, 4u * gn, &mb_gu0);
+                if (warp == 6) bulk_g2s(s_sub, Ly.su + ga, 4u * gn, &mb_gu0);
+                if (warp == 7 && dn > 0) bulk_g2s(s_sdb, Ly.sd + da, 4u * dn, &mb_dn);
+            }
+        }
+        TSTAMP(l, 5)
         // ------------------------------------------------------------ C: gate/up -> h
         {
             // activation limbs of this lane's segment (d / 64 = 32 segments: lane = segment)
@@ -694,40 +713,69 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
         }
         TSTAMP(l, 13)
         if (warp == kStackWarps - 1 && p.predict && has_next) {
-            // predicted experts of the next layer -> L2 prefetch of this CTA's rows of
-            // predictions s and s + 8 (what it would copy if one of them lands in its slot).
-            // Only a hint: if the predictions are not all there within a few microseconds, skip.
-            // This warp runs it while warps 0..3 combine; it joins the CTA again at the next
-            // layer's first barrier.
+            // The experts predicted for the next layer -> L2 prefetch.  No exact ranking (a hint
+            // needs none): tau = the kPredTop-th largest of the 32 lane maxima of the predicted
+            // logits (lane l holds experts l, l+32, ...), so at least kPredTop experts have a
+            // predicted logit >= tau; the c-th of them (lane-major order) is prefetched by slot
+            // group c mod k, each CTA its own rows (what it copies if that expert lands in its
+            // group).  Only a hint: if the predictions are not all there within a few
+            // microseconds, nothing is prefetched.  This warp runs it while warps 0..3 combine;
+            // it joins the CTA again at the next layer's first barrier.
             bool ok = true;
+            float pv[8];
             const long long t0 = clock64();
-            for (int e = lane; e < E && ok; e += 32) {
-                unsigned long long w;
-                while (true) {
-                    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(p.pb + (size_t)par * E + e) : "memory");
-                    if ((uint32_t)(w >> 32) == tag) break;
-                    if (clock64() - t0 > kPredictWaitCycles) {
-                        ok = false;
-                        break;
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                const int e = lane + 32 * j;
+                pv[j] = -INFINITY;
+                if (e < E && ok) {
+                    unsigned long long w;
+                    while (true) {
+                        asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(p.pb + (size_t)par * E + e) : "memory");
+                        if ((uint32_t)(w >> 32) == tag) break;
+                        if (clock64() - t0 > kPredictWaitCycles) {
+                            ok = false;
+                            break;
+                        }
+                        __nanosleep(kPollSleepNs);
                     }
-                    __nanosleep(kPollSleepNs);
+                    pv[j] = __uint_as_float((uint32_t)w);
                 }
-                plg[e] = (double)__uint_as_float((uint32_t)w);
             }
             if (__all_sync(0xFFFFFFFFu, ok)) {
+                float mx = pv[0];
+#pragma unroll
+                for (int j = 1; j < 8; j++) mx = fmaxf(mx, pv[j]);
+                int above = 0;
+#pragma unroll
+                for (int i = 0; i < 32; i++) {
+                    const float o = __shfl_sync(0xFFFFFFFFu, mx, i);
+                    above += (o > mx || (o == mx && i < lane)) ? 1 : 0;
+                }
                 const int np = E < kPredTop ? E : kPredTop;
-                warp_topk_filter(plg, E, np, s_pidx, cand);
+                const unsigned who = __ballot_sync(0xFFFFFFFFu, above == np - 1);
+                const float tau = __shfl_sync(0xFFFFFFFFu, mx, __ffs(who) - 1);
                 const StackLayerDev &Ln = s_layer[l + 1];
                 const uint32_t rowg = (uint32_t)(d / 4), rowd = (uint32_t)(f / 4);
-                for (int q = s; q < np; q += kSK) {
-                    const size_t e = (size_t)s_pidx[q];
-                    if (lane == 0 && ngu > 0) prefetch_l2_bulk(Ln.gate + (e * f + j0) * rowg, (uint32_t)ngu * rowg);
-                    if (lane == 1 && ngu > 0) prefetch_l2_bulk(Ln.up + (e * f + j0) * rowg, (uint32_t)ngu * rowg);
-                    if (lane == 2 && ndn > 0) prefetch_l2_bulk(Ln.down + (e * d + i0) * rowd, (uint32_t)ndn * rowd);
-                    if (lane == 3) asm volatile("prefetch.global.L2 [%0];" ::"l"(Ln.sg + e * f + j0));
-                    if (lane == 4) asm volatile("prefetch.global.L2 [%0];" ::"l"(Ln.su + e * f + j0));
-                    if (lane >= 5 && lane < 9 && 32 * (lane - 5) < ndn)
-                        asm volatile("prefetch.global.L2 [%0];" ::"l"(Ln.sd + e * d + i0 + 32 * (lane - 5)));
+                int count = 0;
+#pragma unroll
+                for (int j = 0; j < 8; j++) {
+                    const int e = lane + 32 * j;
+                    const bool take = e < E && pv[j] >= tau;
+                    const unsigned msk = __ballot_sync(0xFFFFFFFFu, take);
+                    const int cidx = count + __popc(msk & ((1u << lane) - 1u));
+                    if (take && cidx % k == s) {
+                        const size_t ee = (size_t)e;
+                        if (ngu > 0) {
+                            prefetch_l2_bulk(Ln.gate + (ee * f + j0) * rowg, (uint32_t)ngu * rowg);
+                            prefetch_l2_bulk(Ln.up + (ee * f + j0) * rowg, (uint32_t)ngu * rowg);
+                        }
+                        if (ndn > 0) prefetch_l2_bulk(Ln.down + (ee * d + i0) * rowd, (uint32_t)ndn * rowd);
+                        asm volatile("prefetch.global.L2 [%0];" ::"l"(Ln.sg + ee * f + j0));
+                        asm volatile("prefetch.global.L2 [%0];" ::"l"(Ln.su + ee * f + j0));
+                        for (int o = 0; o < ndn; o += 32) asm volatile("prefetch.global.L2 [%0];" ::"l"(Ln.sd + ee * d + i0 + o));
+                    }
+                    count += __popc(msk);
                 }
             }
         }
@@ -740,8 +788,13 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             double sq = 0.0;
             float am = 0.0f;
             if (tid < ndn) {
+                double yq[kSK];
+#pragma unroll
+                for (int q = 0; q < kSK; q++) yq[q] = q < k ? (double)yv[q * kMaxDN + tid] : 0.0;
                 double y = 0.0;
-                for (int q = 0; q < k; q++) y += s_gate[q] * (double)yv[q * kMaxDN + tid];
+#pragma unroll
+                for (int q = 0; q < kSK; q++)
+                    if (q < k) y += s_gate[q] * yq[q];  // top-k order
                 const uint16_t yb = f64_to_bf16_rne(y);
                 xo = f64_to_bf16_rne((double)bf16_to_f32(xs[i0 + tid]) + (double)bf16_to_f32(yb));
                 const double xv2 = (double)bf16_to_f32(xo);
