@@ -69,8 +69,8 @@ constexpr int kMaxGU = 32;          // gate/up rows per CTA (two chunks of 16)
 constexpr int kMaxDN = 128;         // down rows per CTA
 constexpr int kMaxRouterRows = 8;   // router rows per CTA
 constexpr int kPredTop = 10;        // at least this many predicted next-layer experts go to L2
+constexpr int kMaxPrefetch = 2;     // predicted experts one slot group prefetches (3 warps each)
 constexpr int kTracePoints = 24;
-constexpr int kRouterWarps = 4;     // warps that compute the router rows (16 columns per thread)
 constexpr long long kPredictWaitCycles = 10000;  // the prediction exchange is a hint: give up after ~5 us
 constexpr unsigned kPollSleepNs = 32;           // sleep between two polls of a tagged word
 constexpr int kTraceExtra = 8;                  // stamps inside the layer's phases (15 .. 22)
@@ -205,6 +205,8 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
     // range, so entry q is at [q + offset], offset < 4
     __shared__ __align__(16) float s_sgb[kMaxGU + 8], s_sub[kMaxGU + 8], s_sdb[kMaxDN + 8];
     __shared__ float s_hmax[kStackWarps];
+    __shared__ int32_t s_pf[kMaxPrefetch];  // next-layer experts this CTA prefetches
+    __shared__ int s_npf;
     // the layers' pointers, copied once: a dynamically indexed kernel parameter is a constant
     // cache line fetched from L2 on the critical path of every layer
     __shared__ StackLayerDev s_layer[kMaxLayers];
@@ -374,64 +376,61 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             reinterpret_cast<uint2 *>(ns)[tid] =
                 make_uint2((uint32_t)nb[0] | ((uint32_t)nb[1] << 16), (uint32_t)nb[2] | ((uint32_t)nb[3] << 16));
         }
-        __syncthreads();  // n (shared) complete
         TSTAMP(l, 16)  // n known
-        // Router rows of this layer on warps 0..3: thread t (< 128) multiplies columns
-        // 16t..16t+15 (n from shared memory); bf16 x bf16 has at most 16 significant bits, so
-        // each product is exact in fp64 and every fma adds it with one rounding (the sums are
-        // exact at these magnitudes: the order does not matter).  Warps 4..15 meanwhile build
-        // the activation limbs of the gate/up dots.
-        if (warp < kRouterWarps) {
-            if (nr > 0) {
-                if (!mbar_wait_sleep(&mb_r[par], (uint32_t)((l >> 1) & 1), lim, p.status)) alive = false;
-                double nv[16];
-                {
-                    const uint4 *np4 = reinterpret_cast<const uint4 *>(ns) + 2 * tid;
-                    const uint4 n0v = np4[0], n1v = np4[1];
-                    const uint32_t nw[8] = {n0v.x, n0v.y, n0v.z, n0v.w, n1v.x, n1v.y, n1v.z, n1v.w};
-#pragma unroll
-                    for (int z = 0; z < 8; z++) {
-                        nv[2 * z] = bf16_to_f64((uint16_t)(nw[z] & 0xFFFFu));
-                        nv[2 * z + 1] = bf16_to_f64((uint16_t)(nw[z] >> 16));
-                    }
-                }
-                const uint16_t *rb = par ? rbuf1 : rbuf0;
+        // router rows of this layer: thread t multiplies columns 4t..4t+3 (n from shared memory);
+        // bf16 x bf16 has at most 16 significant bits, so each product is exact in fp64 and the
+        // fma adds it with one rounding (the sums are exact at these magnitudes: the order does
+        // not matter)
+        if (nr > 0) {
+            if (!mbar_wait_sleep(&mb_r[par], (uint32_t)((l >> 1) & 1), lim, p.status)) alive = false;
+            const uint2 n2 = reinterpret_cast<const uint2 *>(ns)[tid];
+            const double nd[4] = {bf16_to_f64((uint16_t)(n2.x & 0xFFFFu)), bf16_to_f64((uint16_t)(n2.x >> 16)),
+                                  bf16_to_f64((uint16_t)(n2.y & 0xFFFFu)), bf16_to_f64((uint16_t)(n2.y >> 16))};
+            const uint16_t *rb = par ? rbuf1 : rbuf0;
 #pragma unroll 1
-                for (int q = 0; q < nr; q++) {
-                    const uint4 *wp = reinterpret_cast<const uint4 *>(rb + (size_t)q * d) + 2 * tid;
-                    const uint4 w0v = wp[0], w1v = wp[1];
-                    const uint32_t ww[8] = {w0v.x, w0v.y, w0v.z, w0v.w, w1v.x, w1v.y, w1v.z, w1v.w};
-                    double a[4] = {0.0, 0.0, 0.0, 0.0};
+            for (int q = 0; q < nr; q += 2) {
+                // rows q and q + 1 together (two independent chains); a missing second row is 0
+                const uint2 w0 = reinterpret_cast<const uint2 *>(rb + (size_t)q * d)[tid];
+                const uint2 w1 = q + 1 < nr ? reinterpret_cast<const uint2 *>(rb + (size_t)(q + 1) * d)[tid]
+                                            : make_uint2(0u, 0u);
+                double a0 = 0.0, a1 = 0.0;
+                a0 = fma(bf16_to_f64((uint16_t)(w0.x & 0xFFFFu)), nd[0], a0);
+                a1 = fma(bf16_to_f64((uint16_t)(w1.x & 0xFFFFu)), nd[0], a1);
+                a0 = fma(bf16_to_f64((uint16_t)(w0.x >> 16)), nd[1], a0);
+                a1 = fma(bf16_to_f64((uint16_t)(w1.x >> 16)), nd[1], a1);
+                a0 = fma(bf16_to_f64((uint16_t)(w0.y & 0xFFFFu)), nd[2], a0);
+                a1 = fma(bf16_to_f64((uint16_t)(w1.y & 0xFFFFu)), nd[2], a1);
+                a0 = fma(bf16_to_f64((uint16_t)(w0.y >> 16)), nd[3], a0);
+                a1 = fma(bf16_to_f64((uint16_t)(w1.y >> 16)), nd[3], a1);
 #pragma unroll
-                    for (int z = 0; z < 8; z++) {
-                        a[(2 * z) & 3] = fma(bf16_to_f64((uint16_t)(ww[z] & 0xFFFFu)), nv[2 * z], a[(2 * z) & 3]);
-                        a[(2 * z + 1) & 3] = fma(bf16_to_f64((uint16_t)(ww[z] >> 16)), nv[2 * z + 1], a[(2 * z + 1) & 3]);
-                    }
-                    double t = (a[0] + a[1]) + (a[2] + a[3]);
-                    t = warp_sum_f64(t);
-                    if (lane == 0) s_rp[warp][q] = t;
+                for (int o = 16; o > 0; o >>= 1) {
+                    a0 += __shfl_xor_sync(0xFFFFFFFFu, a0, o);
+                    a1 += __shfl_xor_sync(0xFFFFFFFFu, a1, o);
                 }
-            }
-        } else {
-            // limbs of elements 4u..4u+3 for u = tid - 128 and u + 384 (all 512 quads)
-            const float inv = (NL == 1 && amax_n > 0.0f) ? quant_inv(amax_n) : 0.0f;
-            for (int u = tid - kRouterWarps * 32; u < d / 4; u += kStackThreads - kRouterWarps * 32) {
-                const uint2 nb2 = reinterpret_cast<const uint2 *>(ns)[u];
-                const float v4[4] = {bf16_to_f32((uint16_t)(nb2.x & 0xFFFFu)), bf16_to_f32((uint16_t)(nb2.x >> 16)),
-                                     bf16_to_f32((uint16_t)(nb2.y & 0xFFFFu)), bf16_to_f32((uint16_t)(nb2.y >> 16))};
-                store_limbs4<NL>(xl, xlp, u, v4, sh_n, inv, amax_n > 0.0f);
+                if (lane == 0) {
+                    s_rp[warp][q] = a0;
+                    if (q + 1 < nr) s_rp[warp][q + 1] = a1;
+                }
             }
         }
         TSTAMP(l, 17)  // this warp's router partials written
         if (!__syncthreads_and(alive ? 1 : 0)) break;  // router partials (and n) visible
         if (tid < nr) {
             double sum = 0.0;
-            for (int w = 0; w < kRouterWarps; w++) sum += s_rp[w][tid];
+            for (int w = 0; w < kStackWarps; w++) sum += s_rp[w][tid];
             const unsigned long long b = (unsigned long long)__double_as_longlong(sum);
             st_relaxed_v2(p.lb + ((size_t)par * E + e0 + tid) * 2, tagged((uint32_t)(b >> 32), tag),
                           tagged((uint32_t)b, tag));
         }
         TSTAMP(l, 2)
+        // activation limbs of the gate/up dots (needed only after top-k and the row copies)
+        {
+            const float inv = (NL == 1 && amax_n > 0.0f) ? quant_inv(amax_n) : 0.0f;
+            const uint2 n2 = reinterpret_cast<const uint2 *>(ns)[tid];
+            const float v4[4] = {bf16_to_f32((uint16_t)(n2.x & 0xFFFFu)), bf16_to_f32((uint16_t)(n2.x >> 16)),
+                                 bf16_to_f32((uint16_t)(n2.y & 0xFFFFu)), bf16_to_f32((uint16_t)(n2.y >> 16))};
+            store_limbs4<NL>(xl, xlp, tid, v4, sh_n, inv, amax_n > 0.0f);
+        }
         // rbuf[par] is free (this layer's rows are used): fetch the rows of layer l + 2 into it
         if (tid == 0 && nr > 0 && l + 2 < p.n_layers) {
             mbar_expect_tx(&mb_r[par], (uint32_t)(nr * d * 2));
@@ -712,70 +711,91 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             }
         }
         TSTAMP(l, 13)
-        if (warp == kStackWarps - 1 && p.predict && has_next) {
-            // The experts predicted for the next layer -> L2 prefetch.  No exact ranking (a hint
-            // needs none): tau = the kPredTop-th largest of the 32 lane maxima of the predicted
-            // logits (lane l holds experts l, l+32, ...), so at least kPredTop experts have a
-            // predicted logit >= tau; the c-th of them (lane-major order) is prefetched by slot
-            // group c mod k, each CTA its own rows (what it copies if that expert lands in its
-            // group).  Only a hint: if the predictions are not all there within a few
-            // microseconds, nothing is prefetched.  This warp runs it while warps 0..3 combine;
-            // it joins the CTA again at the next layer's first barrier.
-            bool ok = true;
-            float pv[8];
-            const long long t0 = clock64();
-#pragma unroll
-            for (int j = 0; j < 8; j++) {
-                const int e = lane + 32 * j;
-                pv[j] = -INFINITY;
-                if (e < E && ok) {
-                    unsigned long long w;
-                    while (true) {
-                        asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(p.pb + (size_t)par * E + e) : "memory");
-                        if ((uint32_t)(w >> 32) == tag) break;
-                        if (clock64() - t0 > kPredictWaitCycles) {
-                            ok = false;
-                            break;
-                        }
-                        __nanosleep(kPollSleepNs);
-                    }
-                    pv[j] = __uint_as_float((uint32_t)w);
-                }
-            }
-            if (__all_sync(0xFFFFFFFFu, ok)) {
-                float mx = pv[0];
-#pragma unroll
-                for (int j = 1; j < 8; j++) mx = fmaxf(mx, pv[j]);
-                int above = 0;
-#pragma unroll
-                for (int i = 0; i < 32; i++) {
-                    const float o = __shfl_sync(0xFFFFFFFFu, mx, i);
-                    above += (o > mx || (o == mx && i < lane)) ? 1 : 0;
-                }
-                const int np = E < kPredTop ? E : kPredTop;
-                const unsigned who = __ballot_sync(0xFFFFFFFFu, above == np - 1);
-                const float tau = __shfl_sync(0xFFFFFFFFu, mx, __ffs(who) - 1);
-                const StackLayerDev &Ln = s_layer[l + 1];
-                const uint32_t rowg = (uint32_t)(d / 4), rowd = (uint32_t)(f / 4);
-                int count = 0;
+        if (warp >= kStackWarps / 2 && p.predict && has_next) {
+            // The experts predicted for the next layer -> L2 prefetch, by warps 8..15 while warps
+            // 0..3 combine.  No exact ranking (a hint needs none): warp 15 takes tau = the
+            // kPredTop-th largest of the 32 lane maxima of the predicted logits (lane l holds
+            // experts l, l+32, ...), so at least kPredTop experts have a predicted logit >= tau;
+            // the c-th of them (lane-major order) belongs to slot group c mod k, and this CTA
+            // prefetches its own rows of its group's experts (what it copies if one of them lands
+            // in its group).  Warps 8..13 then issue one bulk prefetch each (a warp issues a
+            // bulk operation in ~250 cycles; several from one thread serialise).  Only a hint: if
+            // the predictions are not all there within a few microseconds, nothing is prefetched.
+            // These warps join the CTA again at the next layer's first barrier.
+            if (warp == kStackWarps - 1) {
+                bool ok = true;
+                float pv[8];
+                const long long t0 = clock64();
 #pragma unroll
                 for (int j = 0; j < 8; j++) {
                     const int e = lane + 32 * j;
-                    const bool take = e < E && pv[j] >= tau;
-                    const unsigned msk = __ballot_sync(0xFFFFFFFFu, take);
-                    const int cidx = count + __popc(msk & ((1u << lane) - 1u));
-                    if (take && cidx % k == s) {
-                        const size_t ee = (size_t)e;
-                        if (ngu > 0) {
-                            prefetch_l2_bulk(Ln.gate + (ee * f + j0) * rowg, (uint32_t)ngu * rowg);
-                            prefetch_l2_bulk(Ln.up + (ee * f + j0) * rowg, (uint32_t)ngu * rowg);
+                    pv[j] = -INFINITY;
+                    if (e < E && ok) {
+                        unsigned long long w;
+                        while (true) {
+                            asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(p.pb + (size_t)par * E + e) : "memory");
+                            if ((uint32_t)(w >> 32) == tag) break;
+                            if (clock64() - t0 > kPredictWaitCycles) {
+                                ok = false;
+                                break;
+                            }
+                            __nanosleep(kPollSleepNs);
                         }
-                        if (ndn > 0) prefetch_l2_bulk(Ln.down + (ee * d + i0) * rowd, (uint32_t)ndn * rowd);
-                        asm volatile("prefetch.global.L2 [%0];" ::"l"(Ln.sg + ee * f + j0));
-                        asm volatile("prefetch.global.L2 [%0];" ::"l"(Ln.su + ee * f + j0));
-                        for (int o = 0; o < ndn; o += 32) asm volatile("prefetch.global.L2 [%0];" ::"l"(Ln.sd + ee * d + i0 + o));
+                        pv[j] = __uint_as_float((uint32_t)w);
                     }
-                    count += __popc(msk);
+                }
+                int npf = 0;
+                if (__all_sync(0xFFFFFFFFu, ok)) {
+                    float mx = pv[0];
+#pragma unroll
+                    for (int j = 1; j < 8; j++) mx = fmaxf(mx, pv[j]);
+                    int above4[4] = {0, 0, 0, 0};
+#pragma unroll
+                    for (int i = 0; i < 32; i++) {
+                        const float o = __shfl_sync(0xFFFFFFFFu, mx, i);
+                        above4[i & 3] += (o > mx || (o == mx && i < lane)) ? 1 : 0;
+                    }
+                    const int above = (above4[0] + above4[1]) + (above4[2] + above4[3]);
+                    const int np = E < kPredTop ? E : kPredTop;
+                    const unsigned who = __ballot_sync(0xFFFFFFFFu, above == np - 1);
+                    const float tau = __shfl_sync(0xFFFFFFFFu, mx, __ffs(who) - 1);
+                    unsigned msk[8];
+#pragma unroll
+                    for (int j = 0; j < 8; j++) msk[j] = __ballot_sync(0xFFFFFFFFu, lane + 32 * j < E && pv[j] >= tau);
+                    int count = 0;
+#pragma unroll
+                    for (int j = 0; j < 8; j++) {
+                        const int cidx = count + __popc(msk[j] & ((1u << lane) - 1u));
+                        if (((msk[j] >> lane) & 1u) && cidx % k == s) {
+                            const int slot = cidx / k;
+                            if (slot < kMaxPrefetch) s_pf[slot] = lane + 32 * j;
+                        }
+                        count += __popc(msk[j]);
+                    }
+                    npf = (count - s + k - 1) / k;  // candidates c < count with c mod k == s
+                    if (npf > kMaxPrefetch) npf = kMaxPrefetch;
+                    if (npf < 0) npf = 0;
+                }
+                if (lane == 0) s_npf = npf;
+            }
+            named_bar_sync(4, kStackThreads / 2);
+            const int task = warp - kStackWarps / 2;  // 0..5: expert task / 3, array task % 3
+            if (task < 3 * s_npf && lane == 0) {
+                const StackLayerDev &Ln = s_layer[l + 1];
+                const size_t ee = (size_t)s_pf[task / 3];
+                const uint32_t rowg = (uint32_t)(d / 4), rowd = (uint32_t)(f / 4);
+                const int a = task % 3;
+                if (a == 0 && ngu > 0) {
+                    prefetch_l2_bulk(Ln.gate + (ee * f + j0) * rowg, (uint32_t)ngu * rowg);
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(Ln.sg + ee * f + j0));
+                }
+                if (a == 1 && ngu > 0) {
+                    prefetch_l2_bulk(Ln.up + (ee * f + j0) * rowg, (uint32_t)ngu * rowg);
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(Ln.su + ee * f + j0));
+                }
+                if (a == 2 && ndn > 0) {
+                    prefetch_l2_bulk(Ln.down + (ee * d + i0) * rowd, (uint32_t)ndn * rowd);
+                    for (int o = 0; o < ndn; o += 32) asm volatile("prefetch.global.L2 [%0];" ::"l"(Ln.sd + ee * d + i0 + o));
                 }
             }
         }

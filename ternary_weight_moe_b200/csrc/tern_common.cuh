@@ -479,41 +479,57 @@ __device__ __forceinline__ void block_topk_select(double mine, int E, int k, int
 // cand: shared scratch of 256 entries; idx_out: shared memory.  No CTA barrier: only the
 // calling warp takes part, and it ends with __syncwarp.
 static __device__ __noinline__ void warp_topk_filter(const double *lg, int E, int k, int32_t *idx_out,
-                                              ulonglong2 *cand) {
+                                                     ulonglong2 *cand) {
+    // Written for a short dependency chain (every step a few dependent operations): counts are
+    // split over independent partial sums, the eight ballots are issued before their prefix sums,
+    // and the candidate ranking loads four candidates per step.
     const int lane = threadIdx.x & 31;
     unsigned long long key[8];
-    uint32_t m = 0;
+    uint32_t hi[8];
 #pragma unroll
     for (int j = 0; j < 8; j++) {
         const int e = lane + 32 * j;
         key[j] = e < E ? f64_order_key(lg[e]) : 0ull;  // 0 = below every finite logit
-        m = max(m, (uint32_t)(key[j] >> 32));
+        hi[j] = (uint32_t)(key[j] >> 32);
     }
-    int above = 0;
+    const uint32_t m = max(max(max(hi[0], hi[1]), max(hi[2], hi[3])), max(max(hi[4], hi[5]), max(hi[6], hi[7])));
+    int above4[4] = {0, 0, 0, 0};
 #pragma unroll
     for (int i = 0; i < 32; i++) {
         const uint32_t v = __shfl_sync(0xFFFFFFFFu, m, i);
-        above += (v > m || (v == m && i < lane)) ? 1 : 0;
+        above4[i & 3] += (v > m || (v == m && i < lane)) ? 1 : 0;
     }
+    const int above = (above4[0] + above4[1]) + (above4[2] + above4[3]);
     const unsigned who = __ballot_sync(0xFFFFFFFFu, above == k - 1);
     const uint32_t tau = __shfl_sync(0xFFFFFFFFu, m, __ffs(who) - 1);
-    int nc = 0;
+    unsigned msk[8];
+#pragma unroll
+    for (int j = 0; j < 8; j++) msk[j] = __ballot_sync(0xFFFFFFFFu, lane + 32 * j < E && hi[j] >= tau);
+    const unsigned below = (1u << lane) - 1u;
+    int base = 0;
 #pragma unroll
     for (int j = 0; j < 8; j++) {
-        const int e = lane + 32 * j;
-        const bool take = e < E && (uint32_t)(key[j] >> 32) >= tau;
-        const unsigned mask = __ballot_sync(0xFFFFFFFFu, take);
-        if (take) cand[nc + __popc(mask & ((1u << lane) - 1u))] = make_ulonglong2(key[j], (unsigned long long)e);
-        nc += __popc(mask);
+        if ((msk[j] >> lane) & 1u) cand[base + __popc(msk[j] & below)] = make_ulonglong2(key[j], (unsigned long long)(lane + 32 * j));
+        base += __popc(msk[j]);
     }
+    const int nc = base;
     __syncwarp();
     for (int i = lane; i < nc; i += 32) {
         const ulonglong2 me = cand[i];
-        int r = 0;
-        for (int q = 0; q < nc; q++) {
-            const ulonglong2 o = cand[q];
-            r += (o.x > me.x || (o.x == me.x && o.y < me.y)) ? 1 : 0;
+        int r4[4] = {0, 0, 0, 0};
+        int q = 0;
+        for (; q + 4 <= nc; q += 4) {
+#pragma unroll
+            for (int z = 0; z < 4; z++) {
+                const ulonglong2 o = cand[q + z];
+                r4[z] += (o.x > me.x || (o.x == me.x && o.y < me.y)) ? 1 : 0;
+            }
         }
+        for (; q < nc; q++) {
+            const ulonglong2 o = cand[q];
+            r4[0] += (o.x > me.x || (o.x == me.x && o.y < me.y)) ? 1 : 0;
+        }
+        const int r = (r4[0] + r4[1]) + (r4[2] + r4[3]);
         if (r < k) idx_out[r] = (int)me.y;
     }
     __syncwarp();
