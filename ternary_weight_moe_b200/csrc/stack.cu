@@ -72,7 +72,6 @@ constexpr int kPredTop = 10;        // at least this many predicted next-layer e
 constexpr int kMaxPrefetch = 2;     // predicted experts one slot group prefetches (3 warps each)
 constexpr int kTracePoints = 24;
 constexpr long long kPredictWaitCycles = 10000;  // the prediction exchange is a hint: give up after ~5 us
-constexpr unsigned kPollSleepNs = 32;           // sleep between two polls of a tagged word
 constexpr int kTraceExtra = 8;                  // stamps inside the layer's phases (15 .. 22)
 
 struct StackParams {
@@ -109,15 +108,13 @@ __device__ __forceinline__ void st_word(unsigned long long *p, uint32_t payload,
 }
 
 // Poll the pair of tagged words at src until both carry `tag`; false once `limit` SM cycles
-// have passed since t0 (clock64).  Between polls the thread sleeps briefly, so polling warps
-// leave the issue slots to the warps that compute.
+// have passed since t0 (clock64, cheaper than %globaltimer inside a poll loop).
 __device__ __forceinline__ bool poll_pair(const unsigned long long *src, uint32_t tag, long long t0, long long limit,
                                           ulonglong2 &out) {
     while (true) {
         out = ld_relaxed_v2(src);
         if ((uint32_t)(out.x >> 32) == tag && (uint32_t)(out.y >> 32) == tag) return true;
         if (clock64() - t0 > limit) return false;
-        __nanosleep(kPollSleepNs);
     }
 }
 
@@ -723,27 +720,36 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             // the predictions are not all there within a few microseconds, nothing is prefetched.
             // These warps join the CTA again at the next layer's first barrier.
             if (warp == kStackWarps - 1) {
+                // the eight words of a lane are loaded together (a global load is a ~700-cycle
+                // round trip); only words not yet published are loaded again
                 bool ok = true;
                 float pv[8];
+                unsigned pending = 0;
                 const long long t0 = clock64();
+                do {
+                    unsigned long long w[8];
 #pragma unroll
-                for (int j = 0; j < 8; j++) {
-                    const int e = lane + 32 * j;
-                    pv[j] = -INFINITY;
-                    if (e < E && ok) {
-                        unsigned long long w;
-                        while (true) {
-                            asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(p.pb + (size_t)par * E + e) : "memory");
-                            if ((uint32_t)(w >> 32) == tag) break;
-                            if (clock64() - t0 > kPredictWaitCycles) {
-                                ok = false;
-                                break;
-                            }
-                            __nanosleep(kPollSleepNs);
-                        }
-                        pv[j] = __uint_as_float((uint32_t)w);
+                    for (int j = 0; j < 8; j++) {
+                        const int e = lane + 32 * j;
+                        w[j] = 0ull;
+                        if (e < E && ((pending >> j) & 1u || pending == 0u))
+                            asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w[j]) : "l"(p.pb + (size_t)par * E + e) : "memory");
                     }
-                }
+                    unsigned still = 0;
+#pragma unroll
+                    for (int j = 0; j < 8; j++) {
+                        const int e = lane + 32 * j;
+                        if (e >= E) {
+                            pv[j] = -INFINITY;
+                        } else if ((pending >> j) & 1u || pending == 0u) {
+                            if ((uint32_t)(w[j] >> 32) == tag) pv[j] = __uint_as_float((uint32_t)w[j]);
+                            else still |= 1u << j;
+                        }
+                    }
+                    pending = still ? still : 0u;
+                    if (still && clock64() - t0 > kPredictWaitCycles) ok = false;
+                    if (!still) break;
+                } while (ok);
                 int npf = 0;
                 if (__all_sync(0xFFFFFFFFu, ok)) {
                     float mx = pv[0];

@@ -150,6 +150,85 @@ __device__ void block_filter(const double *lg, int E, int k, int32_t *idx_out, u
     __syncthreads();
 }
 
+// The library's one-warp filter, step by step (the same operations as warp_topk_filter in
+// tern_common.cuh, with a clock64 stamp after each step): st[0..5] = keys, tau, ballots,
+// compaction, ranking, total.
+__global__ void topk_steps(const double *logits, unsigned long long *out) {
+    __shared__ double lg[256];
+    __shared__ ulonglong2 cand[256];
+    __shared__ int32_t idx_out[8];
+    const int lane = threadIdx.x & 31;
+    const int E = 256, k = 8;
+    for (int rep = 0; rep < kReps; rep++) {
+        for (int i = threadIdx.x; i < 256; i += blockDim.x) lg[i] = logits[rep * 256 + i];
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            unsigned long long c0 = clock64();
+            unsigned long long key[8];
+            uint32_t hi[8];
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                const int e = lane + 32 * j;
+                key[j] = f64_order_key(lg[e]);
+                hi[j] = (uint32_t)(key[j] >> 32);
+            }
+            const uint32_t m = max(max(max(hi[0], hi[1]), max(hi[2], hi[3])), max(max(hi[4], hi[5]), max(hi[6], hi[7])));
+            __syncwarp();
+            unsigned long long c1 = clock64();
+            int above4[4] = {0, 0, 0, 0};
+#pragma unroll
+            for (int i = 0; i < 32; i++) {
+                const uint32_t v = __shfl_sync(0xFFFFFFFFu, m, i);
+                above4[i & 3] += (v > m || (v == m && i < lane)) ? 1 : 0;
+            }
+            const int above = (above4[0] + above4[1]) + (above4[2] + above4[3]);
+            const unsigned who = __ballot_sync(0xFFFFFFFFu, above == k - 1);
+            const uint32_t tau = __shfl_sync(0xFFFFFFFFu, m, __ffs(who) - 1);
+            unsigned long long c2 = clock64();
+            unsigned msk[8];
+#pragma unroll
+            for (int j = 0; j < 8; j++) msk[j] = __ballot_sync(0xFFFFFFFFu, hi[j] >= tau);
+            unsigned long long c3 = clock64();
+            const unsigned below = (1u << lane) - 1u;
+            int base = 0;
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                if ((msk[j] >> lane) & 1u) cand[base + __popc(msk[j] & below)] = make_ulonglong2(key[j], (unsigned long long)(lane + 32 * j));
+                base += __popc(msk[j]);
+            }
+            const int nc = base;
+            __syncwarp();
+            unsigned long long c4 = clock64();
+            for (int i = lane; i < nc; i += 32) {
+                const ulonglong2 me = cand[i];
+                int r4[4] = {0, 0, 0, 0};
+                int q = 0;
+                for (; q + 4 <= nc; q += 4) {
+#pragma unroll
+                    for (int z = 0; z < 4; z++) {
+                        const ulonglong2 o = cand[q + z];
+                        r4[z] += (o.x > me.x || (o.x == me.x && o.y < me.y)) ? 1 : 0;
+                    }
+                }
+                for (; q < nc; q++) {
+                    const ulonglong2 o = cand[q];
+                    r4[0] += (o.x > me.x || (o.x == me.x && o.y < me.y)) ? 1 : 0;
+                }
+                const int r = (r4[0] + r4[1]) + (r4[2] + r4[3]);
+                if (r < k) idx_out[r] = (int)me.y;
+            }
+            __syncwarp();
+            unsigned long long c5 = clock64();
+            if (lane == 0) {
+                unsigned long long *o = out + rep * 8;
+                o[0] = c1 - c0; o[1] = c2 - c1; o[2] = c3 - c2; o[3] = c4 - c3; o[4] = c5 - c4; o[5] = c5 - c0;
+                o[6] = (unsigned long long)nc;
+            }
+        }
+        __syncthreads();
+    }
+}
+
 __global__ void topk_bench(const double *logits, unsigned long long *out, int32_t *idx_a, int32_t *idx_b) {
     __shared__ double lg[256];
     __shared__ int32_t s_idx[8];
@@ -284,6 +363,18 @@ int main() {
     }
     printf("\"topk_warp_filter\": %.0f, \"topk_block_filter\": %.0f, \"topk_mismatches\": %d, ", median(ta), median(tb),
            bad);
+
+    topk_steps<<<1, 512>>>(d_lg, d_out);
+    CK(cudaDeviceSynchronize());
+    CK(cudaMemcpy(o.data(), d_out, kReps * 8 * 8, cudaMemcpyDeviceToHost));
+    {
+        const char *sn[] = {"keys", "tau", "ballots", "compact", "rank", "total", "candidates"};
+        for (int st = 0; st < 7; st++) {
+            std::vector<double> v;
+            for (int r = 1; r < kReps; r++) v.push_back((double)o[r * 8 + st]);
+            printf("\"topk_step_%s\": %.0f, ", sn[st], median(v));
+        }
+    }
 
     CK(cudaFuncSetAttribute(bulk_issue, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024));
     for (int mode = 0; mode < 2; mode++) {
