@@ -1035,9 +1035,10 @@ tern_status launch_stack_persistent(const tern_moe_layer *layers, int n_layers, 
     // phase stamps cost a %globaltimer read and a store each: only when TERNMOE_TRACE=1
     const char *tenv = getenv("TERNMOE_TRACE");
     prm.ttrace = (tenv && tenv[0] == '1') ? reinterpret_cast<unsigned long long *>(b + o.ttrace) : nullptr;
-    // L2 prefetch of predicted next-layer experts: on unless TERNMOE_PREDICT=0
+    // L2 prefetch of predicted next-layer experts: only when TERNMOE_PREDICT=1 (measured: the
+    // prediction's own cost still exceeds the row-wait time it saves)
     const char *penv = getenv("TERNMOE_PREDICT");
-    prm.predict = (penv && penv[0] == '0') ? 0 : 1;
+    prm.predict = (penv && penv[0] == '1') ? 1 : 0;
     prm.status = status;
     prm.limit_ns = limit_ns;
     prm.P = pl.P;

@@ -476,13 +476,15 @@ __device__ __forceinline__ void block_topk_select(double mine, int E, int k, int
 //  3. the logits with h >= tau (typically a few more than k) are compacted into `cand`;
 //  4. each candidate's rank = the number of candidates ordered before it (full 64-bit key, then
 //     index); ranks below k land in idx_out.
-// cand: shared scratch of 256 entries; idx_out: shared memory.  No CTA barrier: only the
-// calling warp takes part, and it ends with __syncwarp.
+// cand: shared scratch of 256 entries; idx_out: shared memory; k <= 32.  No CTA barrier: only
+// the calling warp takes part, and it ends with __syncwarp.  It keeps 128 bytes of static shared
+// scratch, so at most one warp of a block may be inside it at a time.
 static __device__ __noinline__ void warp_topk_filter(const double *lg, int E, int k, int32_t *idx_out,
                                                      ulonglong2 *cand) {
-    // Written for a short dependency chain (every step a few dependent operations): counts are
-    // split over independent partial sums, the eight ballots are issued before their prefix sums,
-    // and the candidate ranking loads four candidates per step.
+    // Written for a short dependency chain: tau from the 32 lane maxima read back from shared
+    // memory as broadcasts (eight 16-byte loads instead of 32 shuffles), the eight ballots issued
+    // before their prefix sums, and the candidate ranking loading four candidates per step.
+    __shared__ __align__(16) uint32_t s_m[32];
     const int lane = threadIdx.x & 31;
     unsigned long long key[8];
     uint32_t hi[8];
@@ -493,15 +495,20 @@ static __device__ __noinline__ void warp_topk_filter(const double *lg, int E, in
         hi[j] = (uint32_t)(key[j] >> 32);
     }
     const uint32_t m = max(max(max(hi[0], hi[1]), max(hi[2], hi[3])), max(max(hi[4], hi[5]), max(hi[6], hi[7])));
+    s_m[lane] = m;
+    __syncwarp();
     int above4[4] = {0, 0, 0, 0};
 #pragma unroll
-    for (int i = 0; i < 32; i++) {
-        const uint32_t v = __shfl_sync(0xFFFFFFFFu, m, i);
-        above4[i & 3] += (v > m || (v == m && i < lane)) ? 1 : 0;
+    for (int q4 = 0; q4 < 8; q4++) {
+        const uint4 v = reinterpret_cast<const uint4 *>(s_m)[q4];
+        above4[0] += (v.x > m || (v.x == m && 4 * q4 + 0 < lane)) ? 1 : 0;
+        above4[1] += (v.y > m || (v.y == m && 4 * q4 + 1 < lane)) ? 1 : 0;
+        above4[2] += (v.z > m || (v.z == m && 4 * q4 + 2 < lane)) ? 1 : 0;
+        above4[3] += (v.w > m || (v.w == m && 4 * q4 + 3 < lane)) ? 1 : 0;
     }
     const int above = (above4[0] + above4[1]) + (above4[2] + above4[3]);
     const unsigned who = __ballot_sync(0xFFFFFFFFu, above == k - 1);
-    const uint32_t tau = __shfl_sync(0xFFFFFFFFu, m, __ffs(who) - 1);
+    const uint32_t tau = s_m[__ffs(who) - 1];
     unsigned msk[8];
 #pragma unroll
     for (int j = 0; j < 8; j++) msk[j] = __ballot_sync(0xFFFFFFFFu, lane + 32 * j < E && hi[j] >= tau);

@@ -150,9 +150,8 @@ __device__ void block_filter(const double *lg, int E, int k, int32_t *idx_out, u
     __syncthreads();
 }
 
-// The library's one-warp filter, step by step (the same operations as warp_topk_filter in
-// tern_common.cuh, with a clock64 stamp after each step): st[0..5] = keys, tau, ballots,
-// compaction, ranking, total.
+// The one-warp filter with tau taken by 32 shuffles, step by step (a clock64 stamp after each
+// step): st[0..5] = keys, tau, ballots, compaction, ranking, total.
 __global__ void topk_steps(const double *logits, unsigned long long *out) {
     __shared__ double lg[256];
     __shared__ ulonglong2 cand[256];
@@ -251,6 +250,124 @@ __global__ void topk_bench(const double *logits, unsigned long long *out, int32_
         if (threadIdx.x < 8) idx_b[rep * 8 + threadIdx.x] = s_idx[threadIdx.x];
         if (threadIdx.x == 0) out[2 * rep + 1] = t1 - t0;
         __syncthreads();
+    }
+}
+
+// Two other formulations of the one-warp filter, timed beside the library's (which reads tau
+// from shared memory and compacts by ballots): V == 0 takes tau by 32 shuffles; V == 2 reads
+// tau like the library but compacts by per-lane counts and a prefix read from shared memory.
+template <int V>
+static __device__ __noinline__ void topk_variant(const double *lg, int k, int32_t *idx_out, ulonglong2 *cand) {
+    __shared__ __align__(16) uint32_t s_m[32];
+    __shared__ __align__(16) int s_c[32];
+    const int lane = threadIdx.x & 31;
+    unsigned long long key[8];
+    uint32_t hi[8];
+#pragma unroll
+    for (int j = 0; j < 8; j++) {
+        key[j] = f64_order_key(lg[lane + 32 * j]);
+        hi[j] = (uint32_t)(key[j] >> 32);
+    }
+    const uint32_t m = max(max(max(hi[0], hi[1]), max(hi[2], hi[3])), max(max(hi[4], hi[5]), max(hi[6], hi[7])));
+    int above4[4] = {0, 0, 0, 0};
+    uint32_t tau;
+    if (V == 0) {
+#pragma unroll
+        for (int i = 0; i < 32; i++) {
+            const uint32_t v = __shfl_sync(0xFFFFFFFFu, m, i);
+            above4[i & 3] += (v > m || (v == m && i < lane)) ? 1 : 0;
+        }
+        const int above = (above4[0] + above4[1]) + (above4[2] + above4[3]);
+        const unsigned who = __ballot_sync(0xFFFFFFFFu, above == k - 1);
+        tau = __shfl_sync(0xFFFFFFFFu, m, __ffs(who) - 1);
+    } else {
+        s_m[lane] = m;
+        __syncwarp();
+#pragma unroll
+        for (int q4 = 0; q4 < 8; q4++) {
+            const uint4 v = reinterpret_cast<const uint4 *>(s_m)[q4];
+            above4[0] += (v.x > m || (v.x == m && 4 * q4 + 0 < lane)) ? 1 : 0;
+            above4[1] += (v.y > m || (v.y == m && 4 * q4 + 1 < lane)) ? 1 : 0;
+            above4[2] += (v.z > m || (v.z == m && 4 * q4 + 2 < lane)) ? 1 : 0;
+            above4[3] += (v.w > m || (v.w == m && 4 * q4 + 3 < lane)) ? 1 : 0;
+        }
+        const int above = (above4[0] + above4[1]) + (above4[2] + above4[3]);
+        const unsigned who = __ballot_sync(0xFFFFFFFFu, above == k - 1);
+        tau = s_m[__ffs(who) - 1];
+    }
+    int nc = 0;
+    if (V == 2) {
+        int c = 0;
+#pragma unroll
+        for (int j = 0; j < 8; j++) c += hi[j] >= tau ? 1 : 0;
+        s_c[lane] = c;
+        __syncwarp();
+        int pre = 0;
+#pragma unroll
+        for (int q4 = 0; q4 < 8; q4++) {
+            const int4 v = reinterpret_cast<const int4 *>(s_c)[q4];
+            pre += (4 * q4 + 0 < lane ? v.x : 0) + (4 * q4 + 1 < lane ? v.y : 0);
+            pre += (4 * q4 + 2 < lane ? v.z : 0) + (4 * q4 + 3 < lane ? v.w : 0);
+            nc += (v.x + v.y) + (v.z + v.w);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            if (hi[j] >= tau) cand[pre++] = make_ulonglong2(key[j], (unsigned long long)(lane + 32 * j));
+        }
+    } else {
+        unsigned msk[8];
+#pragma unroll
+        for (int j = 0; j < 8; j++) msk[j] = __ballot_sync(0xFFFFFFFFu, hi[j] >= tau);
+        const unsigned below = (1u << lane) - 1u;
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            if ((msk[j] >> lane) & 1u) cand[nc + __popc(msk[j] & below)] = make_ulonglong2(key[j], (unsigned long long)(lane + 32 * j));
+            nc += __popc(msk[j]);
+        }
+    }
+    __syncwarp();
+    for (int i = lane; i < nc; i += 32) {
+        const ulonglong2 me = cand[i];
+        int r4[4] = {0, 0, 0, 0};
+        int q = 0;
+        for (; q + 4 <= nc; q += 4) {
+#pragma unroll
+            for (int z = 0; z < 4; z++) {
+                const ulonglong2 o = cand[q + z];
+                r4[z] += (o.x > me.x || (o.x == me.x && o.y < me.y)) ? 1 : 0;
+            }
+        }
+        for (; q < nc; q++) {
+            const ulonglong2 o = cand[q];
+            r4[0] += (o.x > me.x || (o.x == me.x && o.y < me.y)) ? 1 : 0;
+        }
+        const int r = (r4[0] + r4[1]) + (r4[2] + r4[3]);
+        if (r < k) idx_out[r] = (int)me.y;
+    }
+    __syncwarp();
+}
+
+// out[3 * rep + v]: cycles of variant v (0: shuffles, 1: the library's, 2: count prefix);
+// idx[(3 * rep + v) * 8 + j]: its selection
+__global__ void topk_variants(const double *logits, unsigned long long *out, int32_t *idx) {
+    __shared__ double lg[256];
+    __shared__ int32_t s_idx[8];
+    __shared__ ulonglong2 cand[256];
+    for (int rep = 0; rep < kReps; rep++) {
+        if (threadIdx.x < 256) lg[threadIdx.x] = logits[rep * 256 + threadIdx.x];
+        __syncthreads();
+        for (int v = 0; v < 3; v++) {
+            if (threadIdx.x < 32) {
+                const unsigned long long t0 = clock64();
+                if (v == 0) topk_variant<0>(lg, 8, s_idx, cand);
+                else if (v == 1) warp_topk_filter(lg, 256, 8, s_idx, cand);
+                else topk_variant<2>(lg, 8, s_idx, cand);
+                const unsigned long long t1 = clock64();
+                if (threadIdx.x < 8) idx[(3 * rep + v) * 8 + threadIdx.x] = s_idx[threadIdx.x];
+                if (threadIdx.x == 0) out[3 * rep + v] = t1 - t0;
+            }
+            __syncthreads();
+        }
     }
 }
 
@@ -374,6 +491,30 @@ int main() {
             for (int r = 1; r < kReps; r++) v.push_back((double)o[r * 8 + st]);
             printf("\"topk_step_%s\": %.0f, ", sn[st], median(v));
         }
+    }
+
+    {
+        int32_t *d_iv;
+        CK(cudaMalloc(&d_iv, kReps * 3 * 8 * 4));
+        topk_variants<<<1, 512>>>(d_lg, d_out, d_iv);
+        CK(cudaDeviceSynchronize());
+        CK(cudaMemcpy(o.data(), d_out, kReps * 3 * 8, cudaMemcpyDeviceToHost));
+        std::vector<int32_t> iv(kReps * 3 * 8);
+        CK(cudaMemcpy(iv.data(), d_iv, iv.size() * 4, cudaMemcpyDeviceToHost));
+        const char *vn[] = {"shuffle_tau", "shared_tau", "count_prefix"};
+        for (int v = 0; v < 3; v++) {
+            std::vector<double> tv;
+            for (int r = 1; r < kReps; r++) tv.push_back((double)o[3 * r + v]);
+            int badv = 0;
+            for (int r = 0; r < kReps; r++) {
+                std::vector<int> ord(256);
+                for (int i = 0; i < 256; i++) ord[i] = i;
+                std::stable_sort(ord.begin(), ord.end(), [&](int a, int b) { return h[r * 256 + a] > h[r * 256 + b]; });
+                for (int j = 0; j < 8; j++) badv += iv[(3 * r + v) * 8 + j] != ord[j];
+            }
+            printf("\"topk_variant_%s\": %.0f, \"topk_variant_%s_mismatches\": %d, ", vn[v], median(tv), vn[v], badv);
+        }
+        CK(cudaFree(d_iv));
     }
 
     CK(cudaFuncSetAttribute(bulk_issue, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024));
