@@ -216,7 +216,7 @@ def cpu_baseline(act_oracle, n_tokens=4):
                       "expert regeneration excluded"}
 
 
-PHASES = [("x_wait", 0, 1), ("norm_router", 1, 2), ("predict_next", 2, 3), ("logits_wait", 3, 4),
+PHASES = [("x_wait", 0, 1), ("norm_router", 1, 2), ("limbs_predict", 2, 3), ("logits_wait", 3, 4),
           ("topk_issue", 4, 5), ("gate_up_rows_wait", 5, 6), ("gate_up_dots", 6, 7), ("swiglu", 7, 8),
           ("h_wait", 8, 9), ("h_limbs", 9, 10), ("down_rows_wait", 10, 11), ("down_dots", 11, 12),
           ("y_wait", 12, 13), ("combine", 13, 14)]

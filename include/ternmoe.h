@@ -274,8 +274,8 @@ tern_status flash_head(const uint8_t *C4, const double *c_scale, const uint16_t 
  *           slots' outputs of this CTA's rows received, 14 x' published; inside the phases
  *           (CTA thread 0): 15 r known, 16 n known, 17 own router partials written, 18 top-k
  *           known (before the copies are issued); 19..23 unused.
- * The persistent kernel prefetches the experts it predicts for the next layer into L2 (a hint
- * that changes no value); TERNMOE_PREDICT=0 in the environment turns that off. */
+ * With TERNMOE_PREDICT=1 in the environment the persistent kernel also prefetches the experts
+ * it predicts for the next layer into L2 (a hint that changes no value; off by default). */
 typedef struct {
     int64_t hist, idx, gates64, y32, h32, trace, total;
 } tern_stack_layout;

@@ -60,11 +60,22 @@ def test_phase_summary_and_aggregate_single_rank():
     import bench
 
     assert bench.aggregate(3.5, "max", 1) == 3.5
+    # P = 4 CTAs in k = 2 slot groups; stamp j of CTA c at layer l: 10 us * l + 0.1 us * j + c ns
     L, P = 3, 4
-    tr = np.zeros((L, P, 16), np.int64)
+    tr = np.zeros((L, P, 24), np.int64)
     for l in range(L):
         for c in range(P):
             tr[l, c, :15] = 10000 * l + 100 * np.arange(15) + c
-    s = bench.phase_summary(tr)
+    s = bench.phase_summary(tr, k=2)
     assert s["layer_total"] == 10.0
     assert abs(s["x_wait"] - 0.1) < 1e-9
+    assert abs(s["combine"] - 0.1) < 1e-9
+    # logits, all CTAs: first receipt (CTA 0, stamp 4) - last publish (CTA 3, stamp 2) = 200 - 3 ns
+    assert abs(s["exchange_latency"]["logits"] - 0.197) < 1e-9
+    # h inside a slot group {0, 1} / {2, 3}: 100 ns - 1 ns
+    assert abs(s["exchange_latency"]["h"] - 0.099) < 1e-9
+    # y among the CTAs of one part (CTAs 0 and 2): 100 ns - 2 ns
+    assert abs(s["exchange_latency"]["y"] - 0.098) < 1e-9
+    # x from layer l's last publish (stamp 14) to layer l + 1's first receipt (stamp 1): 10 us
+    # + 100 ns - 1,400 ns - 1 ns
+    assert abs(s["exchange_latency"]["x"] - 8.699) < 1e-9
