@@ -438,6 +438,96 @@ def run_batch_sweep(args):
     return 0
 
 
+def run_stack_batch(args):
+    """Extra output: the 24-layer stack through moe_stack_decode with T = 1, 2, 4, 8, 16 tokens
+    per call (T = 1: the batch-1 kernel; 2 <= T <= 16: the one-launch small-batch kernel), L2
+    flushed before every call; one JSON line per (T, activations).  Algorithmic bytes per call
+    = sum over layers of (U_l * 798,720 + 1,048,576), U_l = the distinct experts of layer l
+    (from the call's per-layer record)."""
+    import torch
+
+    import synth
+    import ternary_weight_moe_b200 as tm
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peak, peak_kind = peaks()
+    shape, layers, st = build_stack(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for T in ([int(v) for v in args.batch_T.split(",")] if args.batch_T else (1, 2, 4, 8, 16)):
+        xs_host = synth.tokens_bf16(WID, 95000 + 1000 * T, args.steps + 3, T * shape.d).reshape(-1, T, shape.d)
+        xs = torch.from_numpy(xs_host.view(np.int16)).to(dev)
+        for act_name, act in (("bf16", tm.TERN_ACT_BF16), ("int8", tm.TERN_ACT_INT8)):
+            if args.act_only and act_name != args.act:
+                continue
+            ws = tm.workspace(tm.moe_stack_workspace_bytes(layers[0], T, act), dev)
+            lay = tm.moe_stack_workspace_layout(layers[0], T, act)
+            launches = tm.moe_stack_kernel_launches(layers[0], N_LAYERS, T, act)
+            buf = xs[0].clone()
+            for i in range(3):
+                buf.copy_(xs[i])
+                tm.moe_stack_decode(st, buf, act=act, ws=ws)
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+            uniq = []
+            torch.cuda.synchronize(dev)
+            for i in range(args.steps):
+                buf.copy_(xs[3 + i])
+                flush.fill_(i & 0xFF)
+                evs[i][0].record(stream)
+                tm.moe_stack_decode(st, buf, act=act, ws=ws)
+                evs[i][1].record(stream)
+                if i < 4 and launches == 1:
+                    idx = ws[lay["idx"]:lay["idx"] + 4 * N_LAYERS * T * shape.k].view(torch.int32)
+                    idx = idx.view(N_LAYERS, T * shape.k).cpu().numpy()
+                    uniq.append([len(np.unique(r)) for r in idx])
+            torch.cuda.synchronize(dev)
+            if tm.tern_stream_status() != 0:
+                raise RuntimeError("device status set during the stack batch sweep")
+            ms = [a.elapsed_time(b) for a, b in evs]
+            med = statistics.median(ms)
+            phases = None
+            if launches == 1 and T >= 2:
+                # one extra traced call (not timed): clock64 stamps per layer and CTA
+                os.environ["TERNMOE_TRACE"] = "1"
+                buf.copy_(xs[3])
+                tm.moe_stack_decode(st, buf, act=act, ws=ws)
+                torch.cuda.synchronize(dev)
+                os.environ["TERNMOE_TRACE"] = "0"
+                P = torch.cuda.get_device_properties(dev).multi_processor_count
+                tr = ws[lay["trace"]:lay["trace"] + 8 * N_LAYERS * P * 16].view(torch.int64)
+                tr = tr.view(N_LAYERS, P, 16).cpu().numpy().astype(np.float64) / 1965.0
+                phases = batch_phase_summary(tr)
+            U = float(np.mean(uniq)) if uniq else float("nan")
+            nbytes = N_LAYERS * (U * 798720 + 1048576)
+            gbs = nbytes / (med * 1e-3) / 1e9
+            print(json.dumps({"moe_stack_decode": f"T={T}", "act": act_name, "layers": N_LAYERS, "launches": launches,
+                              "us_per_call": med * 1e3, "us_per_layer": med * 1e3 / N_LAYERS,
+                              "us_p10": float(np.percentile(ms, 10)) * 1e3, "tokens_per_s": T / (med * 1e-3),
+                              "unique_experts_per_layer": U, "bytes": nbytes, "GB/s": gbs, "frac": gbs / peak,
+                              "peak": peak, "peak_kind": peak_kind, "steps": args.steps,
+                              "layer_phase_us_traced_call": phases}), flush=True)
+    return 0
+
+
+BATCH_PHASES = [("A_sum_sq", 0, 8), ("A_fold", 8, 9), ("A_limbs_router", 9, 10), ("A_publish", 10, 1),
+                ("barrier1_load_logits", 1, 11), ("B_topk_gates", 11, 12), ("B_group", 12, 2), ("C_gate_up", 2, 3),
+                ("barrier2", 3, 4), ("D_down", 4, 5), ("barrier3", 5, 6), ("E_combine", 6, 7)]
+
+
+def batch_phase_summary(tr):
+    """Small-batch kernel trace [layers][P][16] (us from SM clock stamps): median over CTAs and
+    layers of each phase, the slowest CTA's C and D, and the layer time (start to start)."""
+    out = {name: round(float(np.median(tr[:, :, b] - tr[:, :, a])), 3) for name, a, b in BATCH_PHASES}
+    out["C_copy_wait"] = round(float(np.median(tr[:, :, 13])), 3)  # stored as durations
+    out["D_copy_wait"] = round(float(np.median(tr[:, :, 14])), 3)
+    out["C_gate_up_max"] = round(float(np.median((tr[:, :, 3] - tr[:, :, 2]).max(1))), 3)
+    out["D_down_max"] = round(float(np.median((tr[:, :, 5] - tr[:, :, 4]).max(1))), 3)
+    out["layer_total"] = round(float(np.median(np.diff(tr[:, :, 0].min(1)))), 3)
+    return out
+
+
 def run_head(args):
     """Extra output: the approximate output head (151,936 tokens in 4,748 clusters of 32,
     d = 2048, top 512 clusters) against the full head (every cluster kept), one token per
@@ -500,6 +590,8 @@ def main():
     ap.add_argument("--batch-sweep", action="store_true",
                     help="extra output: time one MoE FFN layer at T = 1, 4, 16, 64 tokens per step")
     ap.add_argument("--batch-T", default=None, help="with --batch-sweep: comma-separated T values only")
+    ap.add_argument("--stack-batch", action="store_true",
+                    help="time the 24-layer stack at T = 1, 2, 4, 8, 16 tokens per call (one launch each)")
     ap.add_argument("--latency-probe", action="store_true",
                     help="compile and run the on-chip latency probe (probes/latency_probe.cu) and print its JSON")
     ap.add_argument("--head", action="store_true",
@@ -515,6 +607,8 @@ def main():
         return run_gemv_sweep(args)
     if args.batch_sweep:
         return run_batch_sweep(args)
+    if args.stack_batch:
+        return run_stack_batch(args)
     if args.head:
         return run_head(args)
 

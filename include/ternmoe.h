@@ -50,7 +50,7 @@
 extern "C" {
 #endif
 
-#define TERNMOE_ABI_VERSION 2
+#define TERNMOE_ABI_VERSION 3
 
 typedef enum {
     TERN_OK = 0,
@@ -216,12 +216,18 @@ tern_status moe_ffn_decode(const tern_moe_layer *L, const uint16_t *x, int64_t T
 /* A stack of n_layers residual MoE FFN layers, applied in place to x [T][d] (bf16):
  *   n = bf16(x / sqrt(mean(x^2) + rms_eps))   (fp64, no learned gain)
  *   x = bf16(x + moe_ffn_decode(n))            (exact sum, one rounding)
- * All layers must share d, f, E, k.  1 <= n_layers <= 64.  For T == 1 the whole stack runs
- * as ONE persistent kernel (one CTA per SM, cooperative launch; the CTAs exchange data
- * through tagged words in the workspace and every in-kernel wait is bounded);
- * otherwise layer by layer.  A timed-out in-kernel wait sets the device status word to
- * TERN_ETIMEOUT (read it with tern_stream_status); x is then unspecified, and the workspace
- * can be used again as it is. */
+ * All layers must share d, f, E, k.  1 <= n_layers <= 64.  The whole stack runs in ONE
+ * cooperative launch (one CTA per SM, every in-kernel wait bounded) when
+ *   T == 1: the batch-1 kernel (the CTAs exchange data through tagged words in the
+ *           workspace); needs d == 2048, f % 64 == 0 with f / 64 a power of two, E <= 256,
+ *           k <= 8, 16-byte aligned scale arrays;
+ *   2 <= T <= 16: the small-batch kernel (grid-wide barriers between the stages of a layer;
+ *           every selected expert's rows are read once per layer and applied to all of its
+ *           tokens); needs d == 2048, f in {128, 256, 512}, E <= 256, k <= 8;
+ * otherwise it runs layer by layer, kernel per stage.  Every path gives each token the same
+ * bits, whatever else is in its batch.  A timed-out in-kernel wait sets the device status
+ * word to TERN_ETIMEOUT (read it with tern_stream_status); x is then unspecified, and the
+ * workspace can be used again as it is. */
 size_t moe_stack_workspace_bytes(const tern_moe_layer *L0, int64_t T_max, tern_act act);
 tern_status moe_stack_decode(const tern_moe_layer *layers, int32_t n_layers, uint16_t *x, int64_t T,
                              float rms_eps, tern_act act, void *workspace, size_t ws_bytes,
@@ -254,21 +260,23 @@ tern_status flash_head(const uint8_t *C4, const double *c_scale, const uint16_t 
                        double *scores, int32_t *sel_clusters, int32_t *cand_ids, double *cand_logits,
                        int32_t *best_id, void *stream);
 
-/* Where, inside a moe_stack_decode workspace, a T == 1 call (the persistent kernel) leaves
- * its per-layer record, for inspection and parity checks (byte offsets):
- *   hist    uint16 [n_layers+1][d]  bf16 x entering each layer, and the final x;
- *   idx     int32  [n_layers][k]    experts chosen at each layer (descending logit);
- *   gates64 double [n_layers][k]    their renormalised gates;
- *   y32     float  [n_layers][d]    each layer's FFN output y before its bf16 cast (the value
- *                                   the residual adds), for parity checks of every layer;
- *   h32     float  [n_layers][k][f] each layer's SwiGLU output h of every slot (the down
- *                                   projection's input, before its limbs or int8 codes);
+/* Where, inside a moe_stack_decode workspace, a one-launch call with T tokens leaves its
+ * per-layer record, for inspection and parity checks (byte offsets; pass T_max = T, and a
+ * workspace of at least moe_stack_workspace_bytes(L0, T, act) bytes):
+ *   hist    uint16 [n_layers+1][T][d]  bf16 x entering each layer, and the final x;
+ *   idx     int32  [n_layers][T][k]    experts chosen at each layer (descending logit);
+ *   gates64 double [n_layers][T][k]    their renormalised gates;
+ *   y32     float  [n_layers][T][d]    each layer's FFN output y before its bf16 cast (the
+ *                                      value the residual adds), for parity checks;
+ *   h32     float  [n_layers][T][k][f] each layer's SwiGLU output h of every slot (the down
+ *                                      projection's input, before its limbs or int8 codes);
+ *   (T == 1 only:)
  *   trace   uint64 [2][n_layers][P][24]: %globaltimer (ns), then clock64 (SM cycles), stamped
  *           by each of the P CTAs (one per SM, P = moe_stack_persistent_ctas(), P <= 256) at
  *           phase boundaries, written only when
  *           the environment variable TERNMOE_TRACE is "1" at the time of the call: 0 layer
- *           start, 1 x received, 2 router logits published, 3 predicted next-layer logits
- *           published, 4 all logits received, 5 top-k done and row copies issued, 6 first
+ *           start, 1 x received, 2 router logits published, 3 activation limbs built (with
+ *           TERNMOE_PREDICT=1: predicted next-layer logits published), 4 all logits received, 5 top-k done and row copies issued, 6 first
  *           gate/up rows landed, 7 gate/up dots done, 8 h published, 9 slot's h received,
  *           10 h limbs built, 11 down rows landed, 12 down dots done and published, 13 the
  *           slots' outputs of this CTA's rows received, 14 x' published; inside the phases
@@ -287,7 +295,7 @@ tern_status moe_stack_workspace_layout(const tern_moe_layer *L0, int64_t T_max, 
 int32_t moe_stack_persistent_ctas(const tern_moe_layer *L0, int32_t n_layers, tern_act act);
 
 /* Number of kernel launches one moe_stack_decode call with these arguments makes on the
- * current device (1 on the persistent T == 1 path), or -1 if the arguments are invalid. */
+ * current device (1 on the one-launch paths), or -1 if the arguments are invalid. */
 int32_t moe_stack_kernel_launches(const tern_moe_layer *L0, int32_t n_layers, int64_t T, tern_act act);
 
 /* Waits for `stream`, then returns and clears the device status word of the current device

@@ -1,6 +1,8 @@
 // api.cu -- the extern "C" entry points of libternmoe.so: argument checks, workspace
 // carving and dispatch to the sm_100a kernels.  See include/ternmoe.h for the contract.
 #include <cuda_runtime.h>
+
+#include <algorithm>
 #include <stdint.h>
 
 #include "../../include/ternmoe.h"
@@ -237,12 +239,19 @@ tern_status moe_ffn_decode(const tern_moe_layer *L, const uint16_t *x, int64_t T
     return cuda_status(launch_ffn_stages(L, x, (int)T, act, w, y, y_f32, nullptr, nullptr, S(stream)));
 }
 
+// One-launch regions after the stage path's workspace and the layer input copy: the batch-1
+// persistent kernel's region, then (T_max >= 2) the small-batch kernel's, sized for
+// min(T_max, 16) tokens.  The two never overlap, so neither kernel sees the other's words.
+static int64_t batch_region_bytes(const tern_moe_layer *L0, int64_t T_max) {
+    return T_max >= 2 ? up256((int64_t)stack_batch_ws_bytes(L0, std::min<int64_t>(T_max, kBatchMaxT))) : 0;
+}
+
 size_t moe_stack_workspace_bytes(const tern_moe_layer *L0, int64_t T_max, tern_act act) {
     if (check_layer(L0) != TERN_OK || T_max < 1 || T_max > kMaxT) return 0;
     const Layout o = make_layout(L0->d, L0->f, L0->E, L0->k, T_max, act);
     int64_t tot = o.total + up256(T_max * L0->d * 2);
     const int64_t pers = (int64_t)stack_persistent_ws_bytes(L0);
-    return (size_t)(tot + up256(pers));
+    return (size_t)(tot + up256(pers) + batch_region_bytes(L0, T_max));
 }
 
 tern_status moe_stack_decode(const tern_moe_layer *layers, int32_t n_layers, uint16_t *x, int64_t T, float rms_eps,
@@ -270,6 +279,13 @@ tern_status moe_stack_decode(const tern_moe_layer *layers, int32_t n_layers, uin
                                                  status_word(), -1, kStackWaitLimitNs, S(stream));
         if (st != TERN_EUNSUPPORTED) return st;
     }
+    if (T >= 2 && T <= kBatchMaxT) {
+        const int64_t at = o.total + up256(T * layers[0].d * 2) + up256((int64_t)stack_persistent_ws_bytes(&layers[0]));
+        tern_status st = launch_stack_batch(layers, n_layers, x, T, rms_eps, act, b + at,
+                                            (size_t)batch_region_bytes(&layers[0], T), status_word(),
+                                            kStackWaitLimitNs, S(stream));
+        if (st != TERN_EUNSUPPORTED) return st;
+    }
     const FfnWs w = carve(workspace, o, act);
     uint16_t *n = reinterpret_cast<uint16_t *>(b + o.total);
     for (int l = 0; l < n_layers; l++) {
@@ -289,12 +305,23 @@ tern_status moe_stack_workspace_layout(const tern_moe_layer *L0, int64_t T_max, 
     const int64_t base = o.total + up256(T_max * L0->d * 2);
     int64_t hist, idx, g, y32, h32, tr;
     stack_persistent_offsets(L0, &hist, &idx, &g, &y32, &h32, &tr);
+    out->trace = base + tr;
+    if (T_max >= 2) {
+        // the small-batch kernel's record (a call with T = T_max tokens writes it)
+        const int64_t bb = base + up256((int64_t)stack_persistent_ws_bytes(L0));
+        stack_batch_offsets(L0, std::min<int64_t>(T_max, kBatchMaxT), &hist, &idx, &g, &y32, &h32, &tr);
+        out->trace = bb + tr;
+        hist += bb - base;
+        idx += bb - base;
+        g += bb - base;
+        y32 += bb - base;
+        h32 += bb - base;
+    }
     out->hist = base + hist;
     out->idx = base + idx;
     out->gates64 = base + g;
     out->y32 = base + y32;
     out->h32 = base + h32;
-    out->trace = base + tr;
     out->total = (int64_t)moe_stack_workspace_bytes(L0, T_max, act);
     return TERN_OK;
 }
@@ -302,6 +329,7 @@ tern_status moe_stack_workspace_layout(const tern_moe_layer *L0, int64_t T_max, 
 int32_t moe_stack_kernel_launches(const tern_moe_layer *L0, int32_t n_layers, int64_t T, tern_act act) {
     if (check_layer(L0) != TERN_OK || n_layers < 1 || n_layers > kMaxLayers || T < 1 || T > kMaxT) return -1;
     if (T == 1 && stack_persistent_supported(L0, n_layers, act)) return 1;
+    if (T >= 2 && T <= kBatchMaxT && stack_batch_supported(L0, n_layers, T, act)) return 1;
     return 8 * n_layers;  // rmsnorm, logits, select, prep, gate/up, prep, down, combine
 }
 

@@ -72,7 +72,6 @@ constexpr int kPredTop = 10;        // at least this many predicted next-layer e
 constexpr int kMaxPrefetch = 2;     // predicted experts one slot group prefetches (3 warps each)
 constexpr int kTracePoints = 24;
 constexpr long long kPredictWaitCycles = 10000;  // the prediction exchange is a hint: give up after ~5 us
-constexpr int kTraceExtra = 8;                  // stamps inside the layer's phases (15 .. 22)
 
 struct StackParams {
     StackLayerDev layer[kMaxLayers];
@@ -161,29 +160,6 @@ __host__ __device__ inline SmemMap smem_map(int d, int f, int k, int gu_max, int
     return m;
 }
 
-// Limb bytes of four consecutive values v[0..3] (elements 4t..4t+3 of a vector whose limbs go
-// to `limbs`, laid out [NL][segments][kSegPad words], position-major inside each segment):
-// element 4t+e lands in byte (t & 3) of word 4 * ((t >> 2) & 3) + e of segment t >> 4.
-template <int NL>
-__device__ __forceinline__ void store_limbs4(uint32_t *limbs, int seg_words_per_limb, int t, const float (&v)[4], int sh,
-                                             float inv, bool nonzero) {
-    uint8_t *lb = reinterpret_cast<uint8_t *>(limbs);
-    const int g = t >> 4, q = (t >> 2) & 3, b = t & 3;
-#pragma unroll
-    for (int e = 0; e < 4; e++) {
-        const int w = g * kSegPad + 4 * q + e;
-        if (NL == 1) {
-            lb[4 * w + b] = (uint8_t)((nonzero ? quant_one(v[e], inv) : 0) & 0xFF);
-        } else {
-            uint32_t hi, mid, lo;
-            fixed_limbs(v[e], sh, hi, mid, lo);
-            lb[4 * w + b] = (uint8_t)hi;
-            lb[4 * (seg_words_per_limb + w) + b] = (uint8_t)mid;
-            lb[4 * (2 * seg_words_per_limb + w) + b] = (uint8_t)lo;
-        }
-    }
-}
-
 // ------------------------------------------------------------------ the kernel
 template <int NL>
 __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_constant__ StackParams p) {
@@ -196,6 +172,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
     __shared__ double s_xss[kMaxGroup];
     __shared__ float s_xam[kMaxGroup];
     __shared__ int32_t s_idx[kSK];
+    __shared__ __align__(16) uint32_t s_tkm[32];  // top-k scratch
     __shared__ double s_gate[kSK];
     __shared__ long long s_S[kMaxGU][2];
     // scales of this CTA's rows, bulk-copied with the rows: a 16-byte aligned superset of the
@@ -452,7 +429,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
         }
         TSTAMP(l, 4)
         if (warp == 0) {
-            warp_topk_filter(lg, E, k, s_idx, cand);
+            warp_topk_filter(lg, E, k, s_idx, cand, s_tkm);
             TSTAMP(l, 18)  // top-k known
             // thread 0 registers the byte counts of this CTA's copies (counted here, so only
             // issued phases are drained after a timeout); warps 0..7 issue them below

@@ -70,14 +70,18 @@ __device__ __forceinline__ double pow2_f64(int e) {
 // the normal bf16 range); those take the exact division.  The rounding itself is integer
 // arithmetic on q's bits: the top 19 bits (sign, exponent, 7 mantissa bits) plus one when the
 // 45 bits below exceed the halfway point or equal it with an odd last kept bit.
+// the exact path, out of line: it is rare, and an inlined fp64 division per call site would
+// multiply the code of loops that call this many times
+static __device__ __noinline__ uint16_t bf16_of_exact_quotient(double x, double r) { return f64_to_bf16_rne(x / r); }
+
 __device__ __forceinline__ uint16_t bf16_of_quotient(double x, double r, double rinv) {
     const double q = x * rinv;
     const unsigned long long b = (unsigned long long)__double_as_longlong(q);
     const unsigned long long low = b & ((1ull << 45) - 1), half = 1ull << 44;
     const long long dist = (long long)low - (long long)half;
     const uint32_t e11 = (uint32_t)(b >> 52) & 0x7FFu;
-    if (dist >= -8 && dist <= 8) return f64_to_bf16_rne(x / r);        // near a tie: exact path
-    if (e11 < 1023 - 126 + 1 || e11 > 1023 + 127 - 1) return f64_to_bf16_rne(x / r);  // not a normal bf16
+    if (dist >= -8 && dist <= 8) return bf16_of_exact_quotient(x, r);  // near a tie: exact path
+    if (e11 < 1023 - 126 + 1 || e11 > 1023 + 127 - 1) return bf16_of_exact_quotient(x, r);  // not a normal bf16
     uint32_t t = (uint32_t)(b >> 45);                                   // sign | e11 | 7 mantissa bits
     t += (dist > 0) ? 1u : 0u;                                          // no ties here (|dist| > 8)
     const uint32_t sign = (t >> 18) & 1u, e = (t >> 7) & 0x7FFu, m = t & 0x7Fu;
@@ -476,15 +480,14 @@ __device__ __forceinline__ void block_topk_select(double mine, int E, int k, int
 //  3. the logits with h >= tau (typically a few more than k) are compacted into `cand`;
 //  4. each candidate's rank = the number of candidates ordered before it (full 64-bit key, then
 //     index); ranks below k land in idx_out.
-// cand: shared scratch of 256 entries; idx_out: shared memory; k <= 32.  No CTA barrier: only
-// the calling warp takes part, and it ends with __syncwarp.  It keeps 128 bytes of static shared
-// scratch, so at most one warp of a block may be inside it at a time.
+// cand: shared scratch of 256 entries; s_m: 32 words of shared scratch, 16-byte aligned (both
+// private to the calling warp, so several warps may run it at once); idx_out: shared memory;
+// k <= 32.  No CTA barrier: only the calling warp takes part, and it ends with __syncwarp.
 static __device__ __noinline__ void warp_topk_filter(const double *lg, int E, int k, int32_t *idx_out,
-                                                     ulonglong2 *cand) {
+                                                     ulonglong2 *cand, uint32_t *s_m) {
     // Written for a short dependency chain: tau from the 32 lane maxima read back from shared
     // memory as broadcasts (eight 16-byte loads instead of 32 shuffles), the eight ballots issued
     // before their prefix sums, and the candidate ranking loading four candidates per step.
-    __shared__ __align__(16) uint32_t s_m[32];
     const int lane = threadIdx.x & 31;
     unsigned long long key[8];
     uint32_t hi[8];
@@ -577,18 +580,44 @@ __device__ __forceinline__ float swiglu_f32(double g, double u) {
     return (float)(g / (1.0 + exp(-g)) * u);
 }
 
+// Limb bytes of four consecutive values v[0..3] (elements 4t..4t+3 of a vector whose limbs go
+// to `limbs`, laid out [NL][segments][kSegPad words], position-major inside each segment):
+// element 4t+e lands in byte (t & 3) of word 4 * ((t >> 2) & 3) + e of segment t >> 4.
+template <int NL>
+__device__ __forceinline__ void store_limbs4(uint32_t *limbs, int seg_words_per_limb, int t, const float (&v)[4], int sh,
+                                             float inv, bool nonzero) {
+    uint8_t *lb = reinterpret_cast<uint8_t *>(limbs);
+    const int g = t >> 4, q = (t >> 2) & 3, b = t & 3;
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+        const int w = g * kSegPad + 4 * q + e;
+        if (NL == 1) {
+            lb[4 * w + b] = (uint8_t)((nonzero ? quant_one(v[e], inv) : 0) & 0xFF);
+        } else {
+            uint32_t hi, mid, lo;
+            fixed_limbs(v[e], sh, hi, mid, lo);
+            lb[4 * w + b] = (uint8_t)hi;
+            lb[4 * (seg_words_per_limb + w) + b] = (uint8_t)mid;
+            lb[4 * (2 * seg_words_per_limb + w) + b] = (uint8_t)lo;
+        }
+    }
+}
+
 // --------------------------------------------------------- bounded grid-wide barrier
 // Monotonic arrival counter: barrier number n waits until the counter reaches n * nblocks.
 // The counter is reset to zero by the last block to leave the kernel (see grid_exit), so it
-// is zero at every launch.  Waits give up after `limit` polls: the status word is set to
-// TERN_ETIMEOUT and false is returned; the caller then leaves the kernel.
+// is zero at every launch.  Waits give up after `limit` SM cycles (clock64): the status word
+// is set to TERN_ETIMEOUT and false is returned; the caller then leaves the kernel.  Stores a
+// block made before the barrier are visible to every block after it: the block barrier orders
+// them before thread 0's release add, and each block's thread 0 acquires before its block
+// barrier releases the other threads.
 struct GridSync {
     unsigned int *arrive;   // monotonic arrivals
     unsigned int *leave;    // blocks that finished
     int *status;            // device status word
     unsigned int nblocks;
     unsigned int epoch;     // barriers passed by this block
-    long long limit;
+    long long limit;        // SM cycles
 };
 
 __device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int *p) {
@@ -607,10 +636,10 @@ __device__ __forceinline__ bool grid_sync(GridSync &gs, int *flag_smem) {
         gs.epoch++;
         const unsigned int target = gs.epoch * gs.nblocks;
         red_release_gpu_add(gs.arrive, 1u);
-        long long n = 0;
+        const long long t0 = clock64();
         int ok = 1;
         while ((int)(ld_acquire_gpu(gs.arrive) - target) < 0) {
-            if (++n > gs.limit) {
+            if (clock64() - t0 > gs.limit) {
                 ok = 0;
                 set_status(gs.status, TERN_ETIMEOUT);
                 break;

@@ -233,13 +233,14 @@ __global__ void topk_bench(const double *logits, unsigned long long *out, int32_
     __shared__ double lg[256];
     __shared__ int32_t s_idx[8];
     __shared__ ulonglong2 cand[256];
+    __shared__ __align__(16) uint32_t s_tkm[32];
     __shared__ __align__(16) uint32_t s_gm[32];
     __shared__ int s_nc;
     for (int rep = 0; rep < kReps; rep++) {
         if (threadIdx.x < 256) lg[threadIdx.x] = logits[rep * 256 + threadIdx.x];
         __syncthreads();
         unsigned long long t0 = clock64();
-        if (threadIdx.x < 32) warp_topk_filter(lg, 256, 8, s_idx, cand);
+        if (threadIdx.x < 32) warp_topk_filter(lg, 256, 8, s_idx, cand, s_tkm);
         __syncthreads();
         unsigned long long t1 = clock64();
         if (threadIdx.x < 8) idx_a[rep * 8 + threadIdx.x] = s_idx[threadIdx.x];
@@ -354,6 +355,7 @@ __global__ void topk_variants(const double *logits, unsigned long long *out, int
     __shared__ double lg[256];
     __shared__ int32_t s_idx[8];
     __shared__ ulonglong2 cand[256];
+    __shared__ __align__(16) uint32_t s_tkm[32];
     for (int rep = 0; rep < kReps; rep++) {
         if (threadIdx.x < 256) lg[threadIdx.x] = logits[rep * 256 + threadIdx.x];
         __syncthreads();
@@ -361,7 +363,7 @@ __global__ void topk_variants(const double *logits, unsigned long long *out, int
             if (threadIdx.x < 32) {
                 const unsigned long long t0 = clock64();
                 if (v == 0) topk_variant<0>(lg, 8, s_idx, cand);
-                else if (v == 1) warp_topk_filter(lg, 256, 8, s_idx, cand);
+                else if (v == 1) warp_topk_filter(lg, 256, 8, s_idx, cand, s_tkm);
                 else topk_variant<2>(lg, 8, s_idx, cand);
                 const unsigned long long t1 = clock64();
                 if (threadIdx.x < 8) idx[(3 * rep + v) * 8 + threadIdx.x] = s_idx[threadIdx.x];

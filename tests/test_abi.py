@@ -14,7 +14,7 @@ def test_library_exports_every_header_function():
     L = tm.lib()
     for n in names:
         assert hasattr(L, n), n
-    assert tm.abi_version() == 2
+    assert tm.abi_version() == 3
 
 
 def test_status_strings():

@@ -42,6 +42,20 @@ def _bf16_ulp_close(a_bits, b_bits):
     return np.abs(a - b) <= ulp * 1.0001
 
 
+def _x_out_close(got_bits, ref_bits, y64):
+    """x_out = bf16(x + bf16(y)) from a y within its tolerance of the oracle's y64: where
+    bf16(y) matches the oracle's the result is identical; where it rounds to the neighbouring
+    bf16 (y within tolerance of a rounding boundary) the sum moves by that one ulp of bf16(y)
+    before its own rounding.  So each element is within one ulp of x_out plus one ulp of
+    bf16(y64).  (With x and y of opposite signs and nearly equal, one ulp of y is many ulps of
+    the small x_out, so a plain one-ulp check of x_out would not hold.)"""
+    a = synth.bf16_bits_to_f64(got_bits)
+    b = synth.bf16_bits_to_f64(ref_bits)
+    ulp = lambda v: np.exp2(np.floor(np.log2(np.maximum(np.abs(v), 1e-30))) - 7)
+    yb = synth.bf16_bits_to_f64(_oracle_bf16(y64))
+    return np.abs(a - b) <= (ulp(b) + ulp(yb)) * 1.0001
+
+
 def _check_bf16_output(y_bits, y32, ref_y64, ref_bits):
     """The GPU's bf16 output is the nearest bf16 of its own fp32-accurate value (checked
     against the fp64 oracle by the tolerance tests), so it may differ from the oracle's
@@ -183,30 +197,45 @@ def test_stack_teacher_forced_per_layer(stack3, act):
         ref = oracle.stack_layer(H.oracle_layer(), xin, eps=1e-6, act=act)
         tm.moe_stack_decode(tm.Stack([L]), cur, eps=1e-6, act=act)
         got = host_u16(cur)
-        close = _bf16_ulp_close(got, ref["x_out"])
+        close = _x_out_close(got, ref["x_out"], ref["y64"])
         assert close.all(), (l, np.argwhere(~close)[:5])
         mismatched += int((got != ref["x_out"]).sum())
     assert mismatched <= 3 * 2048 * 5e-3
     assert torch.equal(full.view(torch.int16), cur.view(torch.int16))
 
 
-def test_persistent_matches_stage_path_bit_exact(stack3):
-    """The one-launch T=1 stack and the kernel-per-stage path (taken for T=2) do the same
-    arithmetic in the same order, so a token gives identical bits on both."""
+def test_one_launch_paths_match_stage_path_bit_exact(stack3):
+    """Three ways through the same stack do the same arithmetic in the same order, so every
+    token gives identical bits on all of them, whatever else is in its batch:
+      * T = 17 distinct tokens: the kernel-per-stage path (24 launches);
+      * the first 16 and the first 4 of them: the one-launch small-batch kernel;
+      * single tokens: the one-launch batch-1 kernel."""
     shape, layers, hosts = stack3
     dev = layers[0].gate.device
     st = tm.Stack(layers)
     for act in (tm.TERN_ACT_BF16, tm.TERN_ACT_INT8):
         assert tm.moe_stack_kernel_launches(layers[0], 3, 1, act) == 1
-        assert tm.moe_stack_kernel_launches(layers[0], 3, 2, act) == 24
-        x = synth.tokens_bf16(WID_STACK, 8, 1, shape.d)
-        one = dev_u16(x, dev)
-        two = dev_u16(np.concatenate([x, x]), dev)
-        tm.moe_stack_decode(st, one, act=act)
-        tm.moe_stack_decode(st, two, act=act)
+        assert tm.moe_stack_kernel_launches(layers[0], 3, 2, act) == 1
+        assert tm.moe_stack_kernel_launches(layers[0], 3, 16, act) == 1
+        assert tm.moe_stack_kernel_launches(layers[0], 3, 17, act) == 24
+        x = synth.tokens_bf16(WID_STACK, 8, 17, shape.d)
+        stage = dev_u16(x, dev)
+        tm.moe_stack_decode(st, stage, act=act)
+        b16 = dev_u16(x[:16], dev)
+        tm.moe_stack_decode(st, b16, act=act)
+        b4 = dev_u16(x[:4], dev)
+        tm.moe_stack_decode(st, b4, act=act)
+        b2 = dev_u16(np.concatenate([x[5:6], x[5:6]]), dev)  # one token twice: one expert list of two
+        tm.moe_stack_decode(st, b2, act=act)
         assert tm.tern_stream_status() == 0
-        assert torch.equal(one.view(torch.int16)[0], two.view(torch.int16)[0])
-        assert torch.equal(two.view(torch.int16)[0], two.view(torch.int16)[1])
+        s16 = stage.view(torch.int16)
+        assert torch.equal(b16.view(torch.int16), s16[:16])
+        assert torch.equal(b4.view(torch.int16), s16[:4])
+        assert torch.equal(b2.view(torch.int16)[0], s16[5]) and torch.equal(b2.view(torch.int16)[1], s16[5])
+        for i in (0, 3, 16):
+            one = dev_u16(x[i:i + 1], dev)
+            tm.moe_stack_decode(st, one, act=act)
+            assert torch.equal(one.view(torch.int16)[0], s16[i]), i
 
 
 @pytest.fixture(scope="module")
@@ -226,7 +255,8 @@ def test_stack24_persistent_teacher_forced(stack24, act, steps):
         max-abs 1e-4 * ||n||_2 of the oracle (n = the layer's normalised input); int8 path
         within 1e-6 of the largest |y| of the oracle teacher-forced on the kernel's own h
         (its int8 codes), so the int32 down sums are the same integers;
-      * x_out = bf16(x + bf16(y)) within one bf16 ulp (at most 0.5% differ)."""
+      * x_out = bf16(x + bf16(y)) within one bf16 ulp of itself plus one of bf16(y) (at most
+        0.5% differ)."""
     shape, layers = stack24
     dev = layers[0].gate.device
     st = tm.Stack(layers)
@@ -270,7 +300,7 @@ def test_stack24_persistent_teacher_forced(stack24, act, steps):
                 y64 = oracle.moe_ffn(L, n, act, qh_in=qh, sh_in=sh)["y64"][0]
                 assert np.abs(y32[l] - y64).max() <= 1e-6 * np.abs(y64).max(), l
             x_out = _oracle_bf16(synth.bf16_bits_to_f64(hist[l]) + synth.bf16_bits_to_f64(_oracle_bf16(y64)))
-            close = _bf16_ulp_close(hist[l + 1], x_out)
+            close = _x_out_close(hist[l + 1], x_out, y64)
             assert close.all(), (l, np.argwhere(~close)[:5])
             mism += int((hist[l + 1] != x_out).sum())
         assert mism <= 24 * d * 5e-3
@@ -303,3 +333,65 @@ def test_stack_kernel_waits_time_out_and_the_next_call_recovers(stack3, act):
     tm.moe_stack_decode(st, b, act=act)  # fresh workspace
     assert tm.tern_stream_status() == 0
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+@pytest.mark.parametrize("act", [tm.TERN_ACT_BF16, tm.TERN_ACT_INT8])
+def test_stack24_small_batch_teacher_forced(stack24, act):
+    """The 24-layer stack for T = 4 tokens in one launch (the small-batch kernel).  Its
+    per-layer record is checked token by token against the oracle run on the kernel's own
+    input to that layer, with the batch-1 test's tolerances: experts bit-exact, gates within
+    1e-12, h within 1e-5 of the largest, y within rel-L2 1e-5 and max-abs 1e-4 * ||n||_2
+    (bf16; int8: within 1e-6 of the largest, teacher-forced on the kernel's h), x_out within
+    one bf16 ulp of itself plus one of bf16(y)."""
+    shape, layers = stack24
+    dev = layers[0].gate.device
+    st = tm.Stack(layers)
+    T = 4
+    assert tm.moe_stack_kernel_launches(layers[0], 24, T, act) == 1
+    ws = tm.workspace(tm.moe_stack_workspace_bytes(layers[0], T, act), dev)
+    lay = tm.moe_stack_workspace_layout(layers[0], T, act)
+    k, d, f = shape.k, shape.d, shape.f
+    hosts = [HostLayer(WID_STACK, l, shape) for l in range(24)]
+    x = synth.tokens_bf16(WID_STACK, 2000 + act, T, d)
+    xd = dev_u16(x, dev)
+    tm.moe_stack_decode(st, xd, eps=1e-6, act=act, ws=ws)
+    assert tm.tern_stream_status() == 0
+    hist = host_u16(ws_view(ws, lay["hist"], torch.int16, 25 * T * d).view(25, T, d))
+    idx = ws_view(ws, lay["idx"], torch.int32, 24 * T * k).view(24, T, k).cpu().numpy()
+    g64 = ws_view(ws, lay["gates64"], torch.float64, 24 * T * k).view(24, T, k).cpu().numpy()
+    y32 = ws_view(ws, lay["y32"], torch.float32, 24 * T * d).view(24, T, d).cpu().numpy().astype(np.float64)
+    h32 = ws_view(ws, lay["h32"], torch.float32, 24 * T * k * f).view(24, T, k, f).cpu().numpy()
+    assert (hist[0] == x).all()
+    assert (hist[24] == host_u16(xd)).all()
+    mism = 0
+    for l in range(24):
+        n, _ = oracle.rmsnorm(hist[l], 1e-6)
+        _, idx_ref, _, _ = hosts[l].route(n)
+        hosts[l].fill(idx_ref)
+        L = hosts[l].oracle_layer()
+        ref = oracle.moe_ffn(L, n, act)
+        assert (idx[l] == ref["idx"]).all(), l
+        assert np.abs(g64[l] - ref["gates"]).max() <= 1e-12
+        for t in range(T):
+            hmax = np.abs(ref["h"][t]).max()
+            assert np.abs(h32[l, t] - ref["h"][t]).max() <= 1e-5 * hmax, (l, t)
+        if act == tm.TERN_ACT_BF16:
+            y64 = ref["y64"]
+            for t in range(T):
+                nn = np.linalg.norm(synth.bf16_bits_to_f64(n[t]))
+                assert np.linalg.norm(y32[l, t] - y64[t]) <= 1e-5 * np.linalg.norm(y64[t]), (l, t)
+                assert np.abs(y32[l, t] - y64[t]).max() <= 1e-4 * nn, (l, t)
+        else:
+            qh = np.empty((T, k, f), np.int8)
+            sh = np.empty((T, k), np.float32)
+            for t in range(T):
+                for q in range(k):
+                    qh[t, q], sh[t, q] = oracle.quant_absmax(h32[l, t, q])
+            y64 = oracle.moe_ffn(L, n, act, qh_in=qh, sh_in=sh)["y64"]
+            for t in range(T):
+                assert np.abs(y32[l, t] - y64[t]).max() <= 1e-6 * np.abs(y64[t]).max(), (l, t)
+        x_out = _oracle_bf16(synth.bf16_bits_to_f64(hist[l]) + synth.bf16_bits_to_f64(_oracle_bf16(y64)))
+        close = _x_out_close(hist[l + 1], x_out, y64)
+        assert close.all(), (l, np.argwhere(~close)[:5])
+        mism += int((hist[l + 1] != x_out).sum())
+    assert mism <= 24 * T * d * 5e-3
