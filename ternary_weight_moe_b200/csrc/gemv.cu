@@ -9,7 +9,8 @@
 //     so activations are read once per CTA, never per row;
 //   - K > 2048 is split across the warps of a CTA (split-K) and combined in shared memory
 //     in a fixed order;
-//   - every byte of weights is decoded with one table read and consumed by one dp4a per limb.
+//   - large calls: every byte of weights is decoded with one table read and consumed by one
+//     dp4a per limb (ring kernel); small one-token calls: decoded without a table (lean kernel).
 #include <cuda_runtime.h>
 
 #include "kernels.h"
@@ -363,10 +364,187 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     }
 }
 
+// ------------------------------------------------------------ the lean GEMV (small calls)
+// For one token and a few MB of weights the ring kernel's fixed costs dominate: a 64 KB
+// decode-table fill per CTA, a producer warp, and for bf16 two passes over x before the
+// first dot.  This kernel has none of them:
+//   - the weights are decoded without a table (decode.cuh);
+//   - every warp first puts the loads of all its rows' segments in flight (<= kLnMaxIter per
+//     lane, ld.global.nc), so their HBM latency overlaps the work on x;
+//   - the activations go to each lane in position-major order (word 4q + j of a limb holds
+//     the activations of position j of packed word q: 16q + j, 16q + 4 + j, 16q + 8 + j,
+//     16q + 12 + j): int8 by a byte transpose of the lane's own 64 values; bf16 limbs are
+//     built once per CTA in shared memory (four values per thread, after a CTA-wide absmax)
+//     and each lane loads its segment's;
+//   - K <= 2048: G = K/64 lanes per row, 32/G rows per warp pass; K > 2048: NS = K/2048
+//     slices, warp w takes slice w % NS of rows w / NS, w / NS + 16/NS, ...; the exact slice
+//     partials meet in shared memory and are added in slice order.
+// The integers are the ring kernel's, so y is identical.
+constexpr int kLnWarps = 16;
+constexpr int kLnThreads = kLnWarps * 32;
+constexpr int kLnMaxIter = 8;    // row segments per lane kept in flight
+constexpr int kLnMaxRows = 256;  // rows per CTA when K > 2048 (slice partials in shared memory)
+constexpr int kLnMaxSlices = 8;
+constexpr int64_t kLnMaxBytes = 16ll << 20;
+constexpr int kLnMaxXPass = 8;   // groups of four activations per thread (K <= 16384)
+
+// bytes 4x4 transpose: P_j holds byte j of N0, N1, N2, N3 (in that byte order)
+__device__ __forceinline__ void bytes_transpose4(uint32_t n0, uint32_t n1, uint32_t n2, uint32_t n3, uint32_t &p0,
+                                                 uint32_t &p1, uint32_t &p2, uint32_t &p3) {
+    const uint32_t t0 = __byte_perm(n0, n1, 0x5140u), t1 = __byte_perm(n2, n3, 0x5140u);
+    const uint32_t t2 = __byte_perm(n0, n1, 0x7362u), t3 = __byte_perm(n2, n3, 0x7362u);
+    p0 = __byte_perm(t0, t1, 0x5410u);
+    p1 = __byte_perm(t0, t1, 0x7632u);
+    p2 = __byte_perm(t2, t3, 0x5410u);
+    p3 = __byte_perm(t2, t3, 0x7632u);
+}
+
+template <int NL, int G>
+__global__ void __launch_bounds__(kLnThreads, 1)
+    gemv_lean_kernel(const uint8_t *__restrict__ Wp, const float *__restrict__ rs, int M, int K, int NS, int Rc,
+                     const void *__restrict__ x, const float *__restrict__ xs, int32_t *__restrict__ acc_out,
+                     float *__restrict__ y) {
+    __shared__ float s_red[kLnWarps];
+    __shared__ long long s_part[kLnMaxRows * kLnMaxSlices];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int RB = K / 4;
+    const int r0c = (int)blockIdx.x * Rc, nrc = min(Rc, M - r0c);  // this CTA's rows
+    constexpr int RPW = 32 / G;                                     // rows per warp pass
+    const int sub = lane / G, gl = lane % G;
+    const int slice = (G == 32) ? warp % NS : 0;
+    const int rg = (G == 32) ? warp / NS : 0, ngroups = (G == 32) ? kLnWarps / NS : 1;
+    const int seg = (G == 32) ? slice * 32 + lane : gl;  // this lane's 64 codes
+    auto row_of = [&](int i) { return (G == 32) ? rg + i * ngroups : (warp + i * kLnWarps) * RPW + sub; };
+
+    // 1. this lane's segment of every row it will take, all loads in flight
+    uint4 wv[kLnMaxIter];
+#pragma unroll
+    for (int i = 0; i < kLnMaxIter; i++) {
+        const int r = row_of(i);
+        wv[i] = r < nrc ? __ldg(reinterpret_cast<const uint4 *>(Wp + (size_t)(r0c + r) * RB) + seg)
+                        : make_uint4(0u, 0u, 0u, 0u);
+    }
+    // scales of the rows this thread writes, early as well
+    const bool split = (G == 32) && NS > 1;
+    float scp[kLnMaxIter];
+#pragma unroll
+    for (int i = 0; i < kLnMaxIter; i++) {
+        const int r = split ? tid + i * kLnThreads : row_of(i);
+        scp[i] = (r < nrc && (split || gl == 0)) ? __ldg(rs + r0c + r) : 0.0f;
+    }
+
+    // 2. the activations of this lane's segment, as limbs in position-major order
+    SegX<NL> X;
+    int sh = 0;
+    if constexpr (NL == 1) {
+        const uint4 *xp = reinterpret_cast<const uint4 *>(static_cast<const int8_t *>(x) + (size_t)seg * 64);
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+            const uint4 t = __ldg(xp + q);
+            bytes_transpose4(t.x, t.y, t.z, t.w, X.w[0][4 * q], X.w[0][4 * q + 1], X.w[0][4 * q + 2], X.w[0][4 * q + 3]);
+        }
+    } else {
+        // bf16: the CTA builds the limbs of x once, four values per thread and pass
+        // (position-major, padded: store_limbs4), then each lane loads its segment's
+        const uint16_t *xb = static_cast<const uint16_t *>(x);
+        const int ng = K / 4, xlp = (K / 64) * kSegPad;
+        uint2 xg[kLnMaxXPass];
+        float am = 0.0f;
+#pragma unroll
+        for (int u = 0; u < kLnMaxXPass; u++) {
+            const int g = tid + u * kLnThreads;
+            xg[u] = g < ng ? __ldg(reinterpret_cast<const uint2 *>(xb) + g) : make_uint2(0u, 0u);
+            am = fmaxf(am, fmaxf(fmaxf(fabsf(bf16_to_f32((uint16_t)(xg[u].x & 0xFFFFu))),
+                                       fabsf(bf16_to_f32((uint16_t)(xg[u].x >> 16)))),
+                                 fmaxf(fabsf(bf16_to_f32((uint16_t)(xg[u].y & 0xFFFFu))),
+                                       fabsf(bf16_to_f32((uint16_t)(xg[u].y >> 16))))));
+        }
+        am = warp_max_f32(am);
+        if (lane == 0) s_red[warp] = am;
+        __syncthreads();
+        float amax = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kLnWarps; w++) amax = fmaxf(amax, s_red[w]);
+        sh = fixed_shift(amax);
+        extern __shared__ __align__(16) uint32_t ln_xl[];  // [3][K/64 segments][kSegPad words]
+#pragma unroll
+        for (int u = 0; u < kLnMaxXPass; u++) {
+            const int g = tid + u * kLnThreads;
+            if (g < ng) {
+                const float v4[4] = {bf16_to_f32((uint16_t)(xg[u].x & 0xFFFFu)), bf16_to_f32((uint16_t)(xg[u].x >> 16)),
+                                     bf16_to_f32((uint16_t)(xg[u].y & 0xFFFFu)), bf16_to_f32((uint16_t)(xg[u].y >> 16))};
+                store_limbs4<NL>(ln_xl, xlp, g, v4, sh, 0.0f, true);
+            }
+        }
+        __syncthreads();
+        seg_load_x_padded<NL>(X, ln_xl, xlp, seg);
+    }
+    auto finish = [&](int r, float sc, long long S) {
+        const int row = r0c + r;
+        if (NL == 1) {
+            if (acc_out) acc_out[row] = (int32_t)S;
+            float v = __fmul_rn(__int2float_rn((int)S), sc);
+            if (xs != nullptr) v = __fmul_rn(v, xs[0]);
+            y[row] = v;
+        } else {
+            y[row] = (float)(ldexp((double)S, -sh) * (double)sc);
+        }
+    };
+
+    // 3. the dots
+#pragma unroll
+    for (int i = 0; i < kLnMaxIter; i++) {
+        const int r = row_of(i);
+        if (!__any_sync(0xFFFFFFFFu, r < nrc)) break;
+        int acc[NL];
+#pragma unroll
+        for (int z = 0; z < NL; z++) acc[z] = 0;
+        seg_dot_alu<NL>(wv[i], X, acc);
+        int a, b;
+        acc_to_pair_x64<NL>(acc, a, b);
+        a = group_sum<G>(a);
+        if (NL > 1) b = group_sum<G>(b);
+        if (r < nrc && gl == 0) {
+            if (split) {
+                if (lane == 0) s_part[r * kLnMaxSlices + slice] = pair_value(NL, a, b);
+            } else {
+                finish(r, scp[i], pair_value(NL, a, b));
+            }
+        }
+    }
+    if (split) {
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < kLnMaxIter; i++) {
+            const int r = tid + i * kLnThreads;
+            if (r < nrc) {
+                long long S = 0;
+                for (int sl = 0; sl < NS; sl++) S += s_part[r * kLnMaxSlices + sl];
+                finish(r, scp[i], S);
+            }
+        }
+    }
+}
+
 static int device_sms() {
     int dev = 0, n = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
     return n > 0 ? n : 148;
+}
+
+// The lean kernel's plan for one token: rows per CTA Rc over the SMs; false when the call is
+// too large for it (more row segments per lane than kLnMaxIter, or more bytes than kLnMaxBytes)
+static bool lean_plan(int64_t M, int64_t K, int64_t T, int sms, int &Rc, int &grid) {
+    if (T != 1 || M * K / 4 > kLnMaxBytes) return false;
+    const int NS = K > 2048 ? (int)(K / 2048) : 1;
+    const int G = NS > 1 ? 32 : (int)(K / 64);
+    if (NS > kLnMaxSlices || NS > kLnWarps) return false;
+    Rc = (int)((M + sms - 1) / sms);
+    grid = (int)((M + Rc - 1) / Rc);
+    const int per_iter = G == 32 ? kLnWarps / NS : kLnWarps * (32 / G);  // rows per CTA per iteration
+    if ((Rc + per_iter - 1) / per_iter > kLnMaxIter) return false;
+    if (NS > 1 && (Rc > kLnMaxRows || Rc > kLnMaxIter * kLnThreads)) return false;
+    return true;
 }
 
 template <int NL>
@@ -376,6 +554,27 @@ static cudaError_t gemv_dispatch(const uint8_t *Wp, const float *rs, int M, int 
     const int NS = K > 2048 ? K / 2048 : 1;
     const int G = NS > 1 ? 32 : RB / 16;
     const int sms = device_sms();
+    int Rl = 0, gl = 0;
+    if (lean_plan(M, K, T, sms, Rl, gl)) {
+        const int lsm = NL == 1 ? 0 : 3 * (K / 64) * kSegPad * 4;  // bf16 limbs of x
+#define TERN_LEAN_CASE(GG)                                                                           \
+    case GG:                                                                                         \
+        if (lsm > 48 * 1024)                                                                         \
+            cudaFuncSetAttribute(gemv_lean_kernel<NL, GG>, cudaFuncAttributeMaxDynamicSharedMemorySize, lsm); \
+        gemv_lean_kernel<NL, GG><<<gl, kLnThreads, lsm, s>>>(Wp, rs, M, K, NS, Rl, x, xs, acc, y);   \
+        break;
+        switch (G) {
+            TERN_LEAN_CASE(1)
+            TERN_LEAN_CASE(2)
+            TERN_LEAN_CASE(4)
+            TERN_LEAN_CASE(8)
+            TERN_LEAN_CASE(16)
+            TERN_LEAN_CASE(32)
+            default: return cudaErrorInvalidValue;
+        }
+#undef TERN_LEAN_CASE
+        return cudaGetLastError();
+    }
     // rows per chunk: a full stage, fewer when that would leave SMs without a chunk; always a
     // multiple of 4 so that every chunk's scales start on a 16-byte boundary
     int R = (kGvStageBytes / RB) & ~3;  // >= 4: RB <= 4096

@@ -100,6 +100,39 @@ def test_gemv_bf16_ragged_tolerance(cuda_dev, M, K, T):
     assert _rel_l2(y.cpu().numpy(), y_ref) <= 1e-5
 
 
+@pytest.mark.parametrize("M,K", [(77, 64), (130, 128), (1000, 256), (333, 1024), (517, 2048), (16384, 2048),
+                                 (300, 8192), (64, 16384), (40000, 2048)])
+def test_gemv_lean_and_ring_kernels_agree_bit_exact(cuda_dev, M, K):
+    """One token takes the lean kernel (no decode table, rows loaded straight into registers)
+    when the call is small; two tokens always take the ring kernel.  Both form the same exact
+    integer sums and the same epilogue, so the token's outputs (and int32 sums) must be
+    identical bit for bit; the largest case here is too big for the lean kernel and checks
+    the switch.  Also against the oracle (int8: bit-exact)."""
+    w = synth.ternary_codes(M * 5 + K, 0, M * K, synth.P0_SPARSE).reshape(M, K)
+    s = synth.uniform_f32(M + 7, 0, M, 0.01, 0.05)
+    Wp, _ = oracle.pack(w)
+    Wd, sd = torch.from_numpy(Wp).to(cuda_dev), torch.from_numpy(s).to(cuda_dev)
+    xb = synth.normal_bf16(K + 8, 0, K, 1.0).reshape(1, K)
+    y1 = tm.tern_gemv(Wd, sd, dev_u16(xb, cuda_dev))
+    y2 = tm.tern_gemv(Wd, sd, dev_u16(np.concatenate([xb, xb]), cuda_dev))
+    assert torch.equal(y1[0], y2[0]) and torch.equal(y2[0], y2[1])
+    q = synth.int8_uniform(K + 9, 0, K).reshape(1, K)
+    xs = np.array([0.004], np.float32)
+    acc1 = torch.empty((1, M), dtype=torch.int32, device=cuda_dev)
+    acc2 = torch.empty((2, M), dtype=torch.int32, device=cuda_dev)
+    z1 = tm.tern_gemv(Wd, sd, torch.from_numpy(q).to(cuda_dev), act=tm.TERN_ACT_INT8,
+                      x_scale=torch.from_numpy(xs).to(cuda_dev), acc=acc1)
+    z2 = tm.tern_gemv(Wd, sd, torch.from_numpy(np.concatenate([q, q])).to(cuda_dev), act=tm.TERN_ACT_INT8,
+                      x_scale=torch.from_numpy(np.concatenate([xs, xs])).to(cuda_dev), acc=acc2)
+    assert torch.equal(acc1[0], acc2[0]) and torch.equal(z1[0], z2[0])
+    acc_ref, y_ref = oracle.gemv_i8(Wp, s, q, x_scale=xs)
+    assert (acc1.cpu().numpy() == acc_ref).all()
+    assert (z1.cpu().numpy() == y_ref).all()
+    if M * K <= 4 << 20:
+        y_ref, _ = oracle.gemv_bf16(Wp, s, xb)
+        assert _rel_l2(y1.cpu().numpy(), y_ref) <= 1e-5
+
+
 def test_gemv_bf16_zero_and_tiny_inputs(cuda_dev):
     M, K = 64, 512
     w = synth.ternary_codes(99, 0, M * K, synth.P0_SPARSE).reshape(M, K)
