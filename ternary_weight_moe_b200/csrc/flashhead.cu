@@ -11,8 +11,9 @@
 // fp64 scale = absmax / 7.  Scores and candidate logits are fp64 sums of exact products
 // (int4 x bf16 and bf16 x bf16 products fit fp64), one fused multiply-add each.
 //
-// Kernels: centroid (offline preparation), score (warp per cluster), select (one CTA,
-// bitonic sort of the scores by (score desc, index asc)), logits (warp per candidate token),
+// Kernels: centroid (offline preparation), score (warp per cluster), select (one CTA: radix
+// select of the top clusters then their ranks, or for more than 1,024 of them a bitonic sort
+// by (score desc, index asc)), logits (warp per candidate token),
 // best (one CTA, candidate with the largest logit, ties to the lower token id).
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -133,27 +134,146 @@ __global__ void __launch_bounds__(kFhSelectThreads) fh_select_kernel(const doubl
     for (int q = threadIdx.x; q < top_c; q += blockDim.x) sel[q] = si[q];
 }
 
+// Top top_c clusters (top_c <= kFhRadixMax) without sorting all of them, one CTA:
+//  1. tau = the top_c-th largest order key: MSB-first radix select, 8 passes of 8-bit digits,
+//     each a 256-bin histogram (shared atomics) of the keys that match the digits chosen so
+//     far, then one warp finds the bin where the count from the top reaches the rank sought;
+//  2. every key above tau is kept, and of the keys equal to tau the `need` ones with the
+//     lowest indices (a block scan in index order);
+//  3. each kept cluster's output position = how many kept clusters come before it (larger
+//     key, or the same key and a lower index).
+constexpr int kFhRadixMax = 1024;
+
+__global__ void __launch_bounds__(kFhSelectThreads) fh_select_radix_kernel(const double *__restrict__ scores, int nc,
+                                                                            int top_c, int32_t *__restrict__ sel) {
+    constexpr int J = kFhMaxClusters / kFhSelectThreads;  // clusters per thread
+    __shared__ int s_hist[256];
+    __shared__ int s_bin, s_need, s_cnt;
+    __shared__ int s_wsum[kFhSelectThreads / 32];
+    __shared__ unsigned long long s_k[kFhRadixMax];
+    __shared__ int s_i[kFhRadixMax];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    unsigned long long key[J];
+#pragma unroll
+    for (int j = 0; j < J; j++) {
+        const int i = tid + j * kFhSelectThreads;
+        key[j] = i < nc ? f64_order_key(scores[i]) : 0ull;
+    }
+    unsigned long long prefix = 0ull, mask = 0ull;
+    int need = top_c;  // rank sought among the keys that match the prefix (1 = largest)
+    for (int shift = 56; shift >= 0; shift -= 8) {
+        if (tid < 256) s_hist[tid] = 0;
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < J; j++)
+            if (tid + j * kFhSelectThreads < nc && (key[j] & mask) == prefix)
+                atomicAdd(&s_hist[(int)((key[j] >> shift) & 255ull)], 1);
+        __syncthreads();
+        if (warp == 0) {
+            // lane l holds bins 255 - 8l .. 248 - 8l (from the top)
+            int c[8], tot = 0;
+#pragma unroll
+            for (int q = 0; q < 8; q++) {
+                c[q] = s_hist[255 - 8 * lane - q];
+                tot += c[q];
+            }
+            int incl = tot;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            const int excl = incl - tot;
+            if (excl < need && need <= incl) {
+                int cum = excl;
+#pragma unroll
+                for (int q = 0; q < 8; q++) {
+                    if (cum < need && cum + c[q] >= need) {
+                        s_bin = 255 - 8 * lane - q;
+                        s_need = need - cum;
+                    }
+                    cum += c[q];
+                }
+            }
+        }
+        __syncthreads();
+        prefix |= (unsigned long long)s_bin << shift;
+        mask |= 255ull << shift;
+        need = s_need;
+        __syncthreads();
+    }
+    const unsigned long long tau = prefix;  // need = clusters with key tau to keep
+    if (tid == 0) s_cnt = 0;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < J; j++) {
+        const int i = tid + j * kFhSelectThreads;
+        if (i < nc && key[j] > tau) s_i[atomicAdd(&s_cnt, 1)] = i;
+    }
+    // the ties, in index order (item (tid, j) has index j * threads + tid)
+    int base = 0;
+#pragma unroll
+    for (int j = 0; j < J; j++) {
+        const int i = tid + j * kFhSelectThreads;
+        const bool eq = i < nc && key[j] == tau;
+        const unsigned bal = __ballot_sync(0xFFFFFFFFu, eq);
+        if (lane == 0) s_wsum[warp] = __popc(bal);
+        __syncthreads();
+        int before = 0, all = 0;
+        for (int w = 0; w < kFhSelectThreads / 32; w++) {
+            before += w < warp ? s_wsum[w] : 0;
+            all += s_wsum[w];
+        }
+        const int r = base + before + __popc(bal & ((1u << lane) - 1u));
+        if (eq && r < need) s_i[atomicAdd(&s_cnt, 1)] = i;
+        base += all;
+        __syncthreads();
+    }
+    for (int t = tid; t < top_c; t += kFhSelectThreads) s_k[t] = f64_order_key(scores[s_i[t]]);
+    __syncthreads();
+    for (int t = tid; t < top_c; t += kFhSelectThreads) {
+        const unsigned long long kt = s_k[t];
+        const int it = s_i[t];
+        int r = 0;
+        for (int u = 0; u < top_c; u++) r += fh_before(s_k[u], s_i[u], kt, it) ? 1 : 0;
+        sel[r] = it;
+    }
+}
+
+// acc + w * x for bf16 w and x, with one rounding (as fma in fp64): the product of two bf16
+// values (8 significant bits each) is exact in fp32 unless it leaves fp32's normal range, so it
+// is formed there and added in fp64; the rare product outside that range takes the fp64 path
+__device__ __forceinline__ double fh_add_prod(double acc, float w, float x) {
+    const float p = __fmul_rn(w, x);
+    const float ap = fabsf(p);
+    if ((ap >= 1.17549435e-38f && ap <= 3.40282347e38f) || w == 0.0f || x == 0.0f) return acc + (double)p;
+    return fma((double)w, (double)x, acc);
+}
+
 __global__ void __launch_bounds__(kFhWarps * 32) fh_logits_kernel(const uint16_t *__restrict__ W,
                                                                    const uint16_t *__restrict__ x, int64_t d, int cs,
                                                                    const int32_t *__restrict__ sel, int ncand,
                                                                    int32_t *__restrict__ ids,
                                                                    double *__restrict__ logits) {
-    extern __shared__ double xs[];
-    stage_x64(x, d, xs);
+    // x in fp32 (exact): each lane reads four consecutive values per step, one 16-byte load,
+    // consecutive lanes consecutive addresses (no bank conflict)
+    extern __shared__ float xsf[];
+    for (int64_t k = threadIdx.x; k < d; k += blockDim.x) xsf[k] = bf16_to_f32(x[k]);
+    __syncthreads();
     const int lane = threadIdx.x & 31;
     const int q = blockIdx.x * kFhWarps + (threadIdx.x >> 5);
     if (q >= ncand) return;
     const int v = sel[q / cs] * cs + q % cs;
-    const uint4 *row = reinterpret_cast<const uint4 *>(W + (int64_t)v * d);
+    const uint2 *row = reinterpret_cast<const uint2 *>(W + (int64_t)v * d);
+    const float4 *x4 = reinterpret_cast<const float4 *>(xsf);
     double acc = 0.0;
-    for (int64_t ch = lane; ch < d / 8; ch += 32) {
-        const uint4 wv = __ldg(row + ch);
-        const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-        for (int e = 0; e < 4; e++) {
-            acc = fma(bf16_f64((uint16_t)(ww[e] & 0xFFFFu)), xs[8 * ch + 2 * e], acc);
-            acc = fma(bf16_f64((uint16_t)(ww[e] >> 16)), xs[8 * ch + 2 * e + 1], acc);
-        }
+    for (int64_t ch = lane; ch < d / 4; ch += 32) {
+        const uint2 wv = __ldg(row + ch);
+        const float4 xv = x4[ch];
+        acc = fh_add_prod(acc, bf16_to_f32((uint16_t)(wv.x & 0xFFFFu)), xv.x);
+        acc = fh_add_prod(acc, bf16_to_f32((uint16_t)(wv.x >> 16)), xv.y);
+        acc = fh_add_prod(acc, bf16_to_f32((uint16_t)(wv.y & 0xFFFFu)), xv.z);
+        acc = fh_add_prod(acc, bf16_to_f32((uint16_t)(wv.y >> 16)), xv.w);
     }
     acc = warp_sum_f64(acc);
     if (lane == 0) {
@@ -233,18 +353,22 @@ extern "C" tern_status flash_head(const uint8_t *C4, const double *c_scale, cons
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const size_t xs_bytes = (size_t)d * sizeof(double);  // x as fp64, up to 64 KB
     cudaFuncSetAttribute(fh_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)xs_bytes);
-    cudaFuncSetAttribute(fh_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)xs_bytes);
+
     fh_score_kernel<<<(n_clusters + kFhWarps - 1) / kFhWarps, kFhWarps * 32, xs_bytes, s>>>(C4, c_scale, x, d,
                                                                                            n_clusters, scores);
     if (cudaGetLastError() != cudaSuccess) return TERN_ECUDA;
-    int N = 1;
-    while (N < n_clusters) N <<= 1;
-    const size_t sel_bytes = (size_t)N * (sizeof(unsigned long long) + sizeof(int));
-    cudaFuncSetAttribute(fh_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_bytes);
-    fh_select_kernel<<<1, kFhSelectThreads, sel_bytes, s>>>(scores, n_clusters, N, top_c, sel_clusters);
+    if (top_c <= kFhRadixMax) {
+        fh_select_radix_kernel<<<1, kFhSelectThreads, 0, s>>>(scores, n_clusters, top_c, sel_clusters);
+    } else {
+        int N = 1;
+        while (N < n_clusters) N <<= 1;
+        const size_t sel_bytes = (size_t)N * (sizeof(unsigned long long) + sizeof(int));
+        cudaFuncSetAttribute(fh_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_bytes);
+        fh_select_kernel<<<1, kFhSelectThreads, sel_bytes, s>>>(scores, n_clusters, N, top_c, sel_clusters);
+    }
     if (cudaGetLastError() != cudaSuccess) return TERN_ECUDA;
     const int ncand = top_c * cluster_size;
-    fh_logits_kernel<<<(ncand + kFhWarps - 1) / kFhWarps, kFhWarps * 32, xs_bytes, s>>>(W, x, d, cluster_size,
+    fh_logits_kernel<<<(ncand + kFhWarps - 1) / kFhWarps, kFhWarps * 32, (size_t)d * sizeof(float), s>>>(W, x, d, cluster_size,
                                                                                        sel_clusters, ncand, cand_ids,
                                                                                        cand_logits);
     if (cudaGetLastError() != cudaSuccess) return TERN_ECUDA;

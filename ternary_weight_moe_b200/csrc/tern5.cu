@@ -115,8 +115,11 @@ __global__ void __launch_bounds__(kT5Warps * 32) gemv5_kernel(const uint8_t *__r
                                                               int32_t *__restrict__ acc_out, float *__restrict__ y) {
     extern __shared__ __align__(16) uint32_t smem[];
     uint2 *lut = reinterpret_cast<uint2 *>(smem);                 // [256][32] lane-private 8-byte entries
-    uint32_t *xa = smem + 256 * 32 * 2;                           // [NL][rb]   activations 5b..5b+3
-    uint32_t *xb = xa + NL * rb;                                  // [NL][rb/4] fifth activations
+    // activations 5b..5b+3 of byte b: [NL][segments][kSegPad words] (16 used per segment; the
+    // padding puts the 16-byte loads of 8 lanes reading 8 segments in 8 different bank groups)
+    const int nseg = rb / 16, xap = nseg * kSegPad;
+    uint32_t *xa = smem + 256 * 32 * 2;
+    uint32_t *xb = xa + NL * xap;                                 // [NL][rb/4] fifth activations
     uint8_t *xbb = reinterpret_cast<uint8_t *>(xb);
     __shared__ float red[32];
     __shared__ int s_sh;
@@ -124,7 +127,6 @@ __global__ void __launch_bounds__(kT5Warps * 32) gemv5_kernel(const uint8_t *__r
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint32_t lane8 = (uint32_t)lane << 3;
     const char *lbase = reinterpret_cast<const char *>(lut);
-    const int nseg = rb / 16;
     for (int t = 0; t < T; t++) {
         const void *xt;
         int sh = 0;
@@ -153,7 +155,7 @@ __global__ void __launch_bounds__(kT5Warps * 32) gemv5_kernel(const uint8_t *__r
             limbs_at<NL>(xt, 5 * (int64_t)b + 4, K, sh, l5);
 #pragma unroll
             for (int l = 0; l < NL; l++) {
-                xa[l * rb + b] = w4[l];
+                xa[l * xap + (b >> 4) * kSegPad + (b & 15)] = w4[l];
                 xbb[l * rb + b] = (uint8_t)l5[l];
             }
         }
@@ -166,6 +168,9 @@ __global__ void __launch_bounds__(kT5Warps * 32) gemv5_kernel(const uint8_t *__r
             for (int seg = lane; seg < nseg; seg += 32) {
                 const uint4 wv = __ldg(reinterpret_cast<const uint4 *>(W5 + (int64_t)row * rb) + seg);
                 const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
+                uint4 x5v[NL];  // fifth activations of the segment's 16 bytes, one 16-byte load per limb
+#pragma unroll
+                for (int l = 0; l < NL; l++) x5v[l] = *reinterpret_cast<const uint4 *>(xb + l * (rb / 4) + seg * 4);
 #pragma unroll
                 for (int q = 0; q < 4; q++) {
                     uint2 e[4];
@@ -176,11 +181,11 @@ __global__ void __launch_bounds__(kT5Warps * 32) gemv5_kernel(const uint8_t *__r
                     const uint32_t c01 = __byte_perm(e[0].y, e[1].y, 0x1140u);
                     const uint32_t c23 = __byte_perm(e[2].y, e[3].y, 0x1140u);
                     const uint32_t c5 = __byte_perm(c01, c23, 0x5410u);
-                    const int bq = seg * 16 + 4 * q;
 #pragma unroll
                     for (int l = 0; l < NL; l++) {
-                        const uint32_t *xl = xa + l * rb + bq;
-                        const uint32_t x5 = xb[l * (rb / 4) + seg * 4 + q];
+                        const uint4 xv = *reinterpret_cast<const uint4 *>(xa + l * xap + seg * kSegPad + 4 * q);
+                        const uint32_t xl[4] = {xv.x, xv.y, xv.z, xv.w};
+                        const uint32_t x5 = q == 0 ? x5v[l].x : q == 1 ? x5v[l].y : q == 2 ? x5v[l].z : x5v[l].w;
                         if (l == 0) {
 #pragma unroll
                             for (int i = 0; i < 4; i++) acc[l] = dp4a_ss(e[i].x, xl[i], acc[l]);
@@ -246,7 +251,8 @@ template <int NL>
 cudaError_t gemv5_launch(const uint8_t *W5, const float *rs, int M, int K, const void *x, const float *xs, int T,
                          int32_t *acc, float *y, cudaStream_t s) {
     const int rb = (int)row_bytes5(K);
-    const size_t smem = (size_t)256 * 32 * 8 + (size_t)NL * rb * 4 + (size_t)NL * rb;
+    // table, padded activation words (kSegPad per 16 bytes of row), fifth activations
+    const size_t smem = (size_t)256 * 32 * 8 + (size_t)NL * (rb / 16) * kSegPad * 4 + (size_t)NL * rb;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     int grid = (M + kT5Warps - 1) / kT5Warps;

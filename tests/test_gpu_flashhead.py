@@ -54,6 +54,25 @@ def test_flash_head_ties_go_to_the_lower_index(cuda_dev):
     assert int(out["best"][0]) == ref["best"]
 
 
+@pytest.mark.parametrize("nc,top_c,equal", [(100, 37, True), (3000, 1024, False), (2000, 1500, False),
+                                             (3000, 700, True)])
+def test_flash_head_selection_paths(cuda_dev, nc, top_c, equal):
+    """The selection against the oracle on both of its paths: top_c <= 1,024 (radix select of
+    the cutoff, then ranks) and more (a full sort).  With every cluster equal, all scores tie
+    and the top_c lowest cluster indices must come out in order."""
+    d, cs = 64, 4
+    W = synth.normal_bf16(25 + nc, 0, nc * cs * d, 0.02).reshape(nc * cs, d)
+    if equal:
+        W[:] = W[:cs].reshape(1, cs, d).repeat(nc, 0).reshape(nc * cs, d)
+    x = synth.normal_bf16(26 + nc, 0, d, 1.0)
+    Wd = torch.from_numpy(W.view(np.int16)).to(cuda_dev)
+    C4, sc, out = _run(Wd, x, cs, top_c)
+    assert (out["sel"] == fh.select(out["scores"], top_c)).all()
+    if equal:
+        assert (out["sel"] == np.arange(top_c)).all()
+    assert int(out["best"][0]) == fh.best(out["ids"], out["logits"])
+
+
 def test_flash_head_full_size_sampled(cuda_dev):
     """151,936 tokens x 2,048, top 512 of 4,748 clusters: sampled centroids, scores and logits
     against the oracle, the selection and the answer against the oracle on the device's values."""
