@@ -30,6 +30,7 @@ __device__ unsigned long long g_code5_errors = 0;
 
 constexpr int kT5Warps = 8;
 constexpr int64_t kT5MaxK = 16384;
+constexpr int kT5Pre = 7;  // row segments per lane loaded ahead: ceil(row_bytes5(kT5MaxK) / 16 / 32)
 constexpr int64_t kT5MaxT = 64;
 
 __host__ __device__ inline int64_t row_bytes5(int64_t K) { return ((K + 4) / 5 + 15) / 16 * 16; }
@@ -165,8 +166,21 @@ __global__ void __launch_bounds__(kT5Warps * 32) gemv5_kernel(const uint8_t *__r
             int acc[NL];
 #pragma unroll
             for (int l = 0; l < NL; l++) acc[l] = 0;
-            for (int seg = lane; seg < nseg; seg += 32) {
-                const uint4 wv = __ldg(reinterpret_cast<const uint4 *>(W5 + (int64_t)row * rb) + seg);
+            // every segment of the row this lane takes, all loads in flight before any decode
+            // (K <= 16384: at most 205 segments, kT5Pre per lane)
+            uint4 wpre[kT5Pre];
+#pragma unroll
+            for (int u = 0; u < kT5Pre; u++) {
+                const int sg = lane + 32 * u;
+                wpre[u] = sg < nseg ? __ldg(reinterpret_cast<const uint4 *>(W5 + (int64_t)row * rb) + sg)
+                                    : make_uint4(0u, 0u, 0u, 0u);
+            }
+            const float rsv = lane == 0 ? rs[row] : 0.0f;
+#pragma unroll
+            for (int u = 0; u < kT5Pre; u++) {
+                const int seg = lane + 32 * u;
+                if (seg >= nseg) break;
+                const uint4 wv = wpre[u];
                 const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
                 uint4 x5v[NL];  // fifth activations of the segment's 16 bytes, one 16-byte load per limb
 #pragma unroll
@@ -207,11 +221,11 @@ __global__ void __launch_bounds__(kT5Warps * 32) gemv5_kernel(const uint8_t *__r
                 const int64_t o = (int64_t)t * M + row;
                 if (NL == 1) {
                     if (acc_out) acc_out[o] = (int32_t)S;
-                    float v = __fmul_rn(__int2float_rn((int)S), rs[row]);
+                    float v = __fmul_rn(__int2float_rn((int)S), rsv);
                     if (xs != nullptr) v = __fmul_rn(v, xscale);
                     y[o] = v;
                 } else {
-                    y[o] = (float)(ldexp((double)S, -sh) * (double)rs[row]);
+                    y[o] = (float)(ldexp((double)S, -sh) * (double)rsv);
                 }
             }
         }
