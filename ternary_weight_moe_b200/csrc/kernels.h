@@ -57,6 +57,12 @@ struct FfnWs {           // device pointers carved from the caller's workspace
     double *ye;          // [T*k][d]
 };
 
+// grouped gate/up (phase 0) and down (phase 1) on tcgen05 tensor cores (moe_tc.cu), for the
+// >= 32-token path; d and f multiples of 128
+bool tc_grouped_supported(int d, int f);
+template <int NL>
+cudaError_t launch_grouped_tc(const tern_moe_layer *L, int T, const FfnWs &w, cudaStream_t s, int phase);
+
 cudaError_t launch_route(const uint16_t *Wg, const uint16_t *x, int T, int d, int E, int k, double *logits,
                          int32_t *idx, float *g32, double *g64, unsigned int *counter, bool dispatch,
                          int32_t *n_unique, int32_t *uexp, int32_t *uoff, int32_t *ent, cudaStream_t s);

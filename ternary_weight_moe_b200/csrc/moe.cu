@@ -678,7 +678,19 @@ static cudaError_t ffn_stages_nl(const tern_moe_layer *L, const uint16_t *x, int
     if (err != cudaSuccess) return err;
     const int umax = (E < T * k) ? E : T * k;
     const int Gd = d / 64, Gf = f / 64;
-    if (T >= kMmaGroupedMinT) {  // grouped path on int8 tensor cores
+    if (T >= kMmaGroupedMinT && tc_grouped_supported(d, f)) {  // grouped path on tcgen05 tensor cores
+        err = launch_grouped_tc<NL>(L, T, w, s, 0);
+        if (err != cudaSuccess) return err;
+        err = launch_k(prep_kernel<NL>, dim3(T * k), dim3(128), 0, s, (const uint16_t *)nullptr,
+                       (const float *)w.h, f, w.hw, w.hsc, (const int32_t *)nullptr);
+        if (err != cudaSuccess) return err;
+        err = launch_grouped_tc<NL>(L, T, w, s, 1);
+        if (err != cudaSuccess) return err;
+        int cg = (T * d + 255) / 256;
+        return launch_k(combine_kernel, dim3(cg), dim3(256), 0, s, (const double *)w.g64, (const double *)w.ye, T,
+                        d, k, y, y32, resid, x_out);
+    }
+    if (T >= kMmaGroupedMinT) {  // grouped path on mma.sync (other shapes)
         const dim3 m1(umax, (f + kMmaRows - 1) / kMmaRows), m2(umax, (d + kMmaRows - 1) / kMmaRows);
         const size_t sm1 = 1024 + (size_t)kMmaTok * NL * (d / 4 + kMmaPad) * 4;
         const size_t sm2 = 1024 + (size_t)kMmaTok * NL * (f / 4 + kMmaPad) * 4;
