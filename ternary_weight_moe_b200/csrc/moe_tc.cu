@@ -28,7 +28,9 @@ namespace tern {
 
 constexpr int kTcM = 128;        // rows per CTA (the MMA's M)
 constexpr int kTcN = 16;         // tokens per pass (the MMA's N)
-constexpr int kTcKT = 128;       // codes per K-tile (bytes of int8)
+constexpr int kTcKT = 64;        // codes per K-tile (bytes of int8): 38 KB of shared memory per CTA
+constexpr int kTcKW = kTcKT / 64; // 16-byte packed words per row and tile
+constexpr int kTcBChunks = kTcN * (kTcKT / 16);  // 16-byte limb chunks per limb and tile
 constexpr int kTcThreads = 128;  // warp w reads accumulator lanes 32w .. 32w + 31
 constexpr int kTcABytes = kTcM * kTcKT;
 constexpr int kTcBBytes = kTcN * kTcKT;
@@ -109,10 +111,12 @@ __device__ __forceinline__ uint4 tc_decode_word(uint32_t w) {
 // One K-tile's global data for this thread, loaded one tile ahead of its use: the 32 packed bytes
 // of row `threadIdx.x` of each matrix, and NL chunks of 16 limb bytes (chunk i = threadIdx.x +
 // j * threads: limb l, token row n, 16-byte chunk c of the tile).
+constexpr int kTcBPerThread(int NL) { return (NL * kTcBChunks + kTcThreads - 1) / kTcThreads; }
+
 template <int NM, int NL>
 struct TcTile {
-    uint4 a[NM][2];
-    uint4 b[NL];
+    uint4 a[NM][kTcKW];
+    uint4 b[kTcBPerThread(NL)];
 };
 
 template <int NM, int NL>
@@ -122,20 +126,18 @@ __device__ __forceinline__ void tc_load(TcTile<NM, NL> &p, const uint8_t *const 
     const int r = threadIdx.x;
 #pragma unroll
     for (int m = 0; m < NM; m++) {
-        if (r < nrows) {
-            const uint4 *q = reinterpret_cast<const uint4 *>(mats[m] + (int64_t)r * rowb + (int64_t)t * (kTcKT / 4));
-            p.a[m][0] = __ldg(q);
-            p.a[m][1] = __ldg(q + 1);
-        } else {
-            p.a[m][0] = p.a[m][1] = make_uint4(0u, 0u, 0u, 0u);
-        }
-    }
+        const uint4 *q = reinterpret_cast<const uint4 *>(mats[m] + (int64_t)r * rowb + (int64_t)t * (kTcKT / 4));
 #pragma unroll
-    for (int j = 0; j < NL; j++) {
-        const int i = threadIdx.x + j * kTcThreads;  // < NL * kTcN * (kTcKT / 16) = NL * 128
-        const int c = i % (kTcKT / 16), n = (i / (kTcKT / 16)) % kTcN, l = i / ((kTcKT / 16) * kTcN);
+        for (int w = 0; w < kTcKW; w++) p.a[m][w] = r < nrows ? __ldg(q + w) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    // chunk i: token row n = i % kTcN (fastest: 8 consecutive threads fill one 128-byte row of
+    // core matrices without a bank conflict), 16-byte chunk c, limb l
+#pragma unroll
+    for (int j = 0; j < kTcBPerThread(NL); j++) {
+        const int i = threadIdx.x + j * kTcThreads;
+        const int n = i % kTcN, c = (i / kTcN) % (kTcKT / 16), l = i / kTcBChunks;
         p.b[j] = make_uint4(0u, 0u, 0u, 0u);
-        if (n < nb) {
+        if (l < NL && n < nb) {
             const int64_t vec = ent[q0 + n] / div;
             p.b[j] = __ldg(reinterpret_cast<const uint4 *>(src + (vec * NL + l) * K4 + (int64_t)t * (kTcKT / 4)) + c);
         }
@@ -148,17 +150,20 @@ __device__ __forceinline__ void tc_store(const TcTile<NM, NL> &p, unsigned char 
     const int r = threadIdx.x;
 #pragma unroll
     for (int m = 0; m < NM; m++) {
-        const uint32_t pw[8] = {p.a[m][0].x, p.a[m][0].y, p.a[m][0].z, p.a[m][0].w,
-                                p.a[m][1].x, p.a[m][1].y, p.a[m][1].z, p.a[m][1].w};
 #pragma unroll
-        for (int c = 0; c < 8; c++)  // 16 codes per packed word = one 16-byte chunk of the tile
-            *reinterpret_cast<uint4 *>(A + (size_t)m * kTcABytes + tc_off(r, 16 * c)) = tc_decode_word(pw[c]);
+        for (int w = 0; w < kTcKW; w++) {
+            const uint32_t pw[4] = {p.a[m][w].x, p.a[m][w].y, p.a[m][w].z, p.a[m][w].w};
+#pragma unroll
+            for (int c = 0; c < 4; c++)  // 16 codes per packed word = one 16-byte chunk of the tile
+                *reinterpret_cast<uint4 *>(A + (size_t)m * kTcABytes + tc_off(r, 16 * (4 * w + c))) =
+                    tc_decode_word(pw[c]);
+        }
     }
 #pragma unroll
-    for (int j = 0; j < NL; j++) {
+    for (int j = 0; j < kTcBPerThread(NL); j++) {
         const int i = threadIdx.x + j * kTcThreads;
-        const int c = i % (kTcKT / 16), n = (i / (kTcKT / 16)) % kTcN, l = i / ((kTcKT / 16) * kTcN);
-        *reinterpret_cast<uint4 *>(B + (size_t)l * kTcBBytes + tc_off(n, 16 * c)) = p.b[j];
+        const int n = i % kTcN, c = (i / kTcN) % (kTcKT / 16), l = i / kTcBChunks;
+        if (l < NL) *reinterpret_cast<uint4 *>(B + (size_t)l * kTcBBytes + tc_off(n, 16 * c)) = p.b[j];
     }
 }
 
