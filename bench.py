@@ -222,6 +222,10 @@ PHASES = [("x_wait", 0, 1), ("norm_router", 1, 2), ("limbs_predict", 2, 3), ("lo
           ("y_wait", 12, 13), ("combine", 13, 14)]
 
 
+INNER_PHASES = [("r", 1, 15), ("n", 15, 16), ("router_rows", 16, 17), ("router_publish", 17, 2),
+                ("topk", 4, 18), ("copy_issue", 18, 5)]
+
+
 def phase_summary(tr, clk=None, mhz=1965.0, k=8):
     """Median over CTAs and layers of each phase (us; from SM clock stamps when given, else
     from %globaltimer), the exchange latencies, and the layer time.  CTA p is part p % G of
@@ -231,6 +235,9 @@ def phase_summary(tr, clk=None, mhz=1965.0, k=8):
     else:
         d = lambda a, b: np.median((tr[:, :, b] - tr[:, :, a]).astype(np.float64)) / 1e3
     out = {name: round(float(d(a, b)), 3) for name, a, b in PHASES}
+    # inside phases (CTA thread 0): r known (15), n known (16), own router partials (17), top-k
+    # known (18)
+    out["inner"] = {name: round(float(d(a, b)), 3) for name, a, b in INNER_PHASES}
     L, P, _ = tr.shape
     G = P // k
     by_slot = tr.reshape(L, k, G, -1)            # [layer, slot group, part, stamp]

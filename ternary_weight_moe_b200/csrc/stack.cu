@@ -338,13 +338,14 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
         TSTAMP(l, 1)
         TSTAMP(l, 15)  // r known
         if (l == 0 && pid == 0) reinterpret_cast<uint2 *>(p.hist)[tid] = reinterpret_cast<const uint2 *>(xs)[tid];
-        // rounding is monotone, so max |bf16(x_k / r)| = bf16(max |x_k| / r)
-        const float amax_n = bf16_to_f32(f64_to_bf16_rne((double)amax / r));
+        // 1 / r correctly rounded (the same bits as 1.0 / r, without the division routine); rounding
+        // is monotone, so max |bf16(x_k / r)| = bf16(max |x_k| / r)
+        const double rinv = __drcp_rn(r);
+        const float amax_n = bf16_to_f32(bf16_of_quotient((double)amax, r, rinv));
         const float s_nq = (NL == 1) ? (amax_n > 0.0f ? __fdiv_rn(amax_n, 127.0f) : 0.0f) : 0.0f;
         const int sh_n = (NL == 1) ? 0 : fixed_shift(amax_n);
         {
             uint16_t nb[4];
-            const double rinv = 1.0 / r;
 #pragma unroll
             for (int e = 0; e < 4; e++) nb[e] = bf16_of_quotient((double)xv[e], r, rinv);
             reinterpret_cast<uint2 *>(ns)[tid] =

@@ -240,9 +240,10 @@ __global__ void __launch_bounds__(kBThreads, 1) stack_batch_kernel(const __grid_
             }
             const double r = sqrt(ts / (double)d + p.eps);
             s_r[tid] = r;
-            s_rinv[tid] = 1.0 / r;
+            const double rinv = __drcp_rn(r);  // correctly rounded: the same bits as 1.0 / r
+            s_rinv[tid] = rinv;
             // rounding is monotone, so max |bf16(x_k / r)| = bf16(max |x_k| / r)
-            const float amax_n = bf16_to_f32(f64_to_bf16_rne((double)ta / r));
+            const float amax_n = bf16_to_f32(bf16_of_quotient((double)ta, r, rinv));
             s_tam[tid] = amax_n;
             s_tsh[tid] = (NL == 1) ? 0 : fixed_shift(amax_n);
             s_tsc[tid] = (NL == 1 && amax_n > 0.0f) ? __fdiv_rn(amax_n, 127.0f) : 0.0f;
