@@ -315,6 +315,17 @@ tern_status tern_test_stack_stall(const tern_moe_layer *layers, int32_t n_layers
                                   tern_act act, int32_t stall_layer, int64_t limit_ns, void *workspace,
                                   size_t ws_bytes, void *stream);
 
+/* Test hook for the small-batch stack kernel's own bounded waits (2 <= T <= 16): the same
+ * launch as moe_stack_decode with T tokens, except that at layer `stall_layer` CTA 0 waits at
+ * the grid barrier after the gate/up stage without arriving there, and every in-kernel wait
+ * gives up after limit_ns (1 us .. 1 s).  Every CTA then gives up at that barrier and leaves;
+ * the last one out resets the barrier counters, so the next moe_stack_decode call on the same
+ * workspace runs normally.  tern_stream_status reports TERN_ETIMEOUT; x is left unspecified.
+ * Returns TERN_EUNSUPPORTED when the arguments would not take the small-batch path. */
+tern_status tern_test_stack_batch_stall(const tern_moe_layer *layers, int32_t n_layers, uint16_t *x, int64_t T,
+                                        float rms_eps, tern_act act, int32_t stall_layer, int64_t limit_ns,
+                                        void *workspace, size_t ws_bytes, void *stream);
+
 /* Test hook for the bounded waits: launches one block that waits on a flag nobody sets,
  * for at most `spin_limit` polls, then sets TERN_ETIMEOUT in the device status word and
  * returns.  `flag` is a device int the caller owns (must stay 0). */

@@ -99,6 +99,8 @@ def lib():
             "moe_stack_persistent_ctas": (i32, [ctypes.POINTER(MoELayerC), i32, st]),
             "tern_test_stack_stall": (st, [ctypes.POINTER(MoELayerC), i32, vp, ctypes.c_float, st, i32, i64, vp, sz,
                                            vp]),
+            "tern_test_stack_batch_stall": (st, [ctypes.POINTER(MoELayerC), i32, vp, i64, ctypes.c_float, st, i32,
+                                                 i64, vp, sz, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -441,6 +443,21 @@ def tern_test_stack_stall(stack: Stack, x, stall_layer: int, limit_ns: int, eps=
         ws = workspace(moe_stack_workspace_bytes(stack.layers[0], 1, act), xb.device)
     _check(lib().tern_test_stack_stall(stack.c, len(stack.layers), _ptr(xb), float(eps), act, int(stall_layer),
                                        int(limit_ns), _ptr(ws), ws.numel(), _stream(stream)), "tern_test_stack_stall")
+    return ws
+
+
+def tern_test_stack_batch_stall(stack: Stack, x, stall_layer: int, limit_ns: int, eps=1e-6, act=TERN_ACT_BF16,
+                                ws=None, stream=None):
+    """The small-batch stack launch (x [T, d], 2 <= T <= 16) with CTA 0 not arriving at the grid
+    barrier after the gate/up stage of layer stall_layer, and every in-kernel wait bounded by
+    limit_ns; the kernel must give up by itself and leave TERN_ETIMEOUT in the status word."""
+    xb = _bits16(x, "x")
+    T = xb.shape[0]
+    if ws is None:
+        ws = workspace(moe_stack_workspace_bytes(stack.layers[0], T, act), xb.device)
+    _check(lib().tern_test_stack_batch_stall(stack.c, len(stack.layers), _ptr(xb), T, float(eps), act,
+                                             int(stall_layer), int(limit_ns), _ptr(ws), ws.numel(), _stream(stream)),
+           "tern_test_stack_batch_stall")
     return ws
 
 

@@ -374,6 +374,33 @@ tern_status tern_test_stack_stall(const tern_moe_layer *layers, int32_t n_layers
                                    (long long)limit_ns, S(stream));
 }
 
+tern_status tern_test_stack_batch_stall(const tern_moe_layer *layers, int32_t n_layers, uint16_t *x, int64_t T,
+                                        float rms_eps, tern_act act, int32_t stall_layer, int64_t limit_ns,
+                                        void *workspace, size_t ws_bytes, void *stream) {
+    if (!layers || n_layers < 1 || n_layers > kMaxLayers || !x || T < 2 || T > kBatchMaxT || stall_layer < 0 ||
+        stall_layer >= n_layers || limit_ns < 1000 || limit_ns > kStackWaitLimitNs)
+        return TERN_EINVAL;
+    if (act != TERN_ACT_INT8 && act != TERN_ACT_BF16) return TERN_EINVAL;
+    for (int i = 0; i < n_layers; i++) {
+        tern_status st = check_layer(&layers[i]);
+        if (st != TERN_OK) return st;
+        if (layers[i].d != layers[0].d || layers[i].f != layers[0].f || layers[i].E != layers[0].E ||
+            layers[i].k != layers[0].k)
+            return TERN_EINVAL;
+    }
+    if (!aligned(x, 16)) return TERN_EALIGN;
+    const size_t need = moe_stack_workspace_bytes(&layers[0], T, act);
+    if (!workspace || ws_bytes < need) return TERN_EWORKSPACE;
+    if (!aligned(workspace, 256)) return TERN_EALIGN;
+    const Layout o = make_layout(layers[0].d, layers[0].f, layers[0].E, layers[0].k, T, act);
+    char *b = static_cast<char *>(workspace);
+    int *st = status_word();
+    if (!st) return TERN_ECUDA;
+    const int64_t at = o.total + up256(T * layers[0].d * 2) + up256((int64_t)stack_persistent_ws_bytes(&layers[0]));
+    return launch_stack_batch(layers, n_layers, x, T, rms_eps, act, b + at, (size_t)batch_region_bytes(&layers[0], T), st,
+                              (long long)limit_ns, S(stream), stall_layer);
+}
+
 tern_status tern_test_bounded_wait(int32_t *flag, int64_t spin_limit, void *stream) {
     if (!flag || spin_limit < 1) return TERN_EINVAL;
     if (!aligned(flag, 4)) return TERN_EALIGN;

@@ -96,9 +96,11 @@ size_t stack_batch_ws_bytes(const tern_moe_layer *L0, int64_t T);
 bool stack_batch_supported(const tern_moe_layer *L0, int n_layers, int64_t T, tern_act act);
 void stack_batch_offsets(const tern_moe_layer *L0, int64_t T, int64_t *hist, int64_t *idx, int64_t *gates,
                          int64_t *y32, int64_t *h32, int64_t *trace);
+// stall_layer: -1, or a layer at which CTA 0 does not arrive at the barrier after phase C (the
+// timeout test); limit_ns: bound on every in-kernel wait
 tern_status launch_stack_batch(const tern_moe_layer *layers, int n_layers, uint16_t *x, int64_t T, float eps,
                                tern_act act, void *ws, size_t ws_bytes, int *status, long long limit_ns,
-                               cudaStream_t s);
+                               cudaStream_t s, int stall_layer = -1);
 
 // ---- bounded-wait test hook
 cudaError_t launch_test_wait(int32_t *flag, long long limit, int *status, cudaStream_t s);

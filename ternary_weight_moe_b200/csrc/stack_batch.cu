@@ -72,6 +72,7 @@ struct BatchParams {
     long long limit_ns;     // the same bound for mbarrier waits (%globaltimer)
     unsigned long long *ttrace;  // [n_layers][P][kBTracePoints] clock64 stamps, or null
     int P;                  // CTAs
+    int stall_layer;        // test hook: at this layer CTA 0 does not arrive at the barrier after phase C
     int stages;             // ring stages
     uint32_t stage_bytes;
 };
@@ -522,7 +523,7 @@ __global__ void __launch_bounds__(kBThreads, 1) stack_batch_kernel(const __grid_
         }
         if (!alive) break;
         BSTAMP(l, 3)
-        if (!grid_sync(gs, &s_flag)) {
+        if (!grid_sync(gs, &s_flag, !(l == p.stall_layer && pid == 0))) {
             alive = false;
             break;
         }
@@ -777,7 +778,7 @@ bool stack_batch_supported(const tern_moe_layer *L0, int n_layers, int64_t T, te
 
 tern_status launch_stack_batch(const tern_moe_layer *layers, int n_layers, uint16_t *x, int64_t T, float eps,
                                tern_act act, void *ws, size_t ws_bytes, int *status, long long limit_ns,
-                               cudaStream_t s) {
+                               cudaStream_t s, int stall_layer) {
     const tern_moe_layer &L0 = layers[0];
     BatchPlan pl;
     const tern_status pst = batch_plan(L0, n_layers, T, act, pl);
@@ -824,6 +825,7 @@ tern_status launch_stack_batch(const tern_moe_layer *layers, int n_layers, uint1
     prm.limit_cycles = 2 * limit_ns;  // SM clocks <= 2 GHz
     prm.P = pl.P;
     prm.stages = pl.stages;
+    prm.stall_layer = stall_layer;
     prm.stage_bytes = pl.stage_bytes;
     void *args[] = {&prm};
     const cudaError_t e = cudaLaunchCooperativeKernel(pl.fn, dim3(pl.P), dim3(kBThreads), args, pl.sm.total, s);

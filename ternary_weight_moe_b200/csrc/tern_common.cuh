@@ -629,13 +629,14 @@ __device__ __forceinline__ void red_release_gpu_add(unsigned int *p, unsigned in
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// returns false on timeout (all threads of the block get the same answer)
-__device__ __forceinline__ bool grid_sync(GridSync &gs, int *flag_smem) {
+// returns false on timeout (all threads of the block get the same answer); arrive = false (a
+// test hook) waits without arriving, so this barrier and every block waiting at it time out
+__device__ __forceinline__ bool grid_sync(GridSync &gs, int *flag_smem, bool arrive = true) {
     __syncthreads();
     if (threadIdx.x == 0) {
         gs.epoch++;
         const unsigned int target = gs.epoch * gs.nblocks;
-        red_release_gpu_add(gs.arrive, 1u);
+        if (arrive) red_release_gpu_add(gs.arrive, 1u);
         const long long t0 = clock64();
         int ok = 1;
         while ((int)(ld_acquire_gpu(gs.arrive) - target) < 0) {

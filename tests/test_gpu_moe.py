@@ -395,3 +395,29 @@ def test_stack24_small_batch_teacher_forced(stack24, act):
         assert close.all(), (l, np.argwhere(~close)[:5])
         mism += int((hist[l + 1] != x_out).sum())
     assert mism <= 24 * T * d * 5e-3
+
+
+@pytest.mark.parametrize("act", [tm.TERN_ACT_BF16, tm.TERN_ACT_INT8])
+def test_small_batch_kernel_waits_time_out_and_the_next_call_recovers(stack3, act):
+    """The small-batch kernel's own bounded waits: CTA 0 does not arrive at the grid barrier
+    after the gate/up stage of layer 1, and every wait is bounded by 200 us.  All CTAs give up at
+    that barrier and leave by themselves; the status word reads TERN_ETIMEOUT; the last CTA out
+    resets the barrier counters, so the same workspace then decodes 4 tokens bit for bit as a
+    fresh one.  Nothing faults or hangs: every wait ends on its own."""
+    shape, layers, hosts = stack3
+    dev = layers[0].gate.device
+    st = tm.Stack(layers)
+    T = 4
+    ws = tm.workspace(tm.moe_stack_workspace_bytes(layers[0], T, act), dev)
+    assert tm.tern_stream_status() == 0
+    xs = dev_u16(synth.tokens_bf16(WID_STACK, 31, T, shape.d), dev)
+    tm.tern_test_stack_batch_stall(st, xs, stall_layer=1, limit_ns=200_000, act=act, ws=ws)
+    assert tm.tern_stream_status() == 5  # TERN_ETIMEOUT
+    assert tm.tern_stream_status() == 0  # read and cleared
+    x = synth.tokens_bf16(WID_STACK, 32, T, shape.d)
+    a = dev_u16(x, dev)
+    tm.moe_stack_decode(st, a, act=act, ws=ws)
+    b = dev_u16(x, dev)
+    tm.moe_stack_decode(st, b, act=act)  # fresh workspace
+    assert tm.tern_stream_status() == 0
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
