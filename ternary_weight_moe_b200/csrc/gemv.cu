@@ -388,17 +388,6 @@ constexpr int kLnMaxSlices = 8;
 constexpr int64_t kLnMaxBytes = 16ll << 20;
 constexpr int kLnMaxXPass = 8;   // groups of four activations per thread (K <= 16384)
 
-// bytes 4x4 transpose: P_j holds byte j of N0, N1, N2, N3 (in that byte order)
-__device__ __forceinline__ void bytes_transpose4(uint32_t n0, uint32_t n1, uint32_t n2, uint32_t n3, uint32_t &p0,
-                                                 uint32_t &p1, uint32_t &p2, uint32_t &p3) {
-    const uint32_t t0 = __byte_perm(n0, n1, 0x5140u), t1 = __byte_perm(n2, n3, 0x5140u);
-    const uint32_t t2 = __byte_perm(n0, n1, 0x7362u), t3 = __byte_perm(n2, n3, 0x7362u);
-    p0 = __byte_perm(t0, t1, 0x5410u);
-    p1 = __byte_perm(t0, t1, 0x7632u);
-    p2 = __byte_perm(t2, t3, 0x5410u);
-    p3 = __byte_perm(t2, t3, 0x7632u);
-}
-
 template <int NL, int G>
 __global__ void __launch_bounds__(kLnThreads, 1)
     gemv_lean_kernel(const uint8_t *__restrict__ Wp, const float *__restrict__ rs, int M, int K, int NS, int Rc,

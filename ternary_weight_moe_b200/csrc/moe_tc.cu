@@ -4,19 +4,25 @@
 // At 32 or more tokens the selected experts each serve a few tokens ("iPhone Runs a 20B Model at
 // 120 tok/s", "What Makes 120 tok/s So Fast?": batched work turns the matrix-vector products of
 // decode into small matrix products), so every expert's rows are decoded once and multiplied
-// against all of its tokens at once:
-//   * one CTA of 128 threads per (distinct expert, 128 rows); per K-tile of 128 codes each thread
-//     decodes one row's 32 packed bytes into int8 weights (a byte permutation of a four-entry
-//     table, no memory lookup) and writes them into shared memory in the tensor core's K-major
-//     layout; the staged activation limbs of up to 16 tokens (the expert's entries) go beside
-//     them;
-//   * one thread issues the MMAs, one accumulator per (matrix, limb) in tensor memory: A = the
-//     weights (signed int8), B = a limb (hi: signed, mid and lo: unsigned), M = 128, N = 16,
-//     K = 32 per instruction; tcgen05.commit signals an mbarrier per buffer, so the next tile is
-//     decoded into the other buffer while the tensor core works;
-//   * the epilogue reads the accumulators with tcgen05.ld (thread = row) and recombines the
-//     limbs exactly in int64, S = hi * 65536 + mid * 256 + lo: the same integers as the dp4a and
-//     mma.sync kernels, so the outputs are identical.
+// against all of its tokens at once.  One CTA per (distinct expert, 128 rows), 160 threads:
+//   * four decoder warps, thread = row: per K-tile of 64 codes each thread decodes its row's 16
+//     packed bytes by integer logic into int8 lanes of 64 * w (the table-free decode of
+//     decode.cuh, position-major order) and writes them into shared memory in the tensor core's
+//     K-major layout.  Beside them go the B rows: every activation limb of every token of the
+//     pass (the expert's entries), put into the same order by a byte transpose.  Each thread
+//     keeps the global loads of the next kTcDepth tiles in flight, and decoding runs ahead of the
+//     tensor core by kTcStages buffers;
+//   * one MMA warp: its lane 0 waits for a buffer's decoders (mbarrier), issues one MMA per
+//     matrix and K step (M = 128, K = 32, N = the pass's B rows rounded up to 16; A = the weights,
+//     signed int8) and commits to the buffer's second mbarrier, which frees it for the decoders.
+//     With bf16 activations the three limbs of a token are three B rows, all unsigned: the hi
+//     limb carries an offset of 128, and a row of ones gives the weights' row sums that take it
+//     out again;
+//   * the epilogue reads the accumulators with tcgen05.ld (thread = row), divides out the 64
+//     exactly and recombines the limbs in int64, S = hi * 65536 + mid * 256 + lo: the same
+//     integers as the dp4a and mma.sync kernels, so the outputs are identical.
+// Every wait is bounded; after a timeout (status set) both sides keep the barrier protocol but
+// skip their work, so no thread is left waiting.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -27,13 +33,23 @@
 namespace tern {
 
 constexpr int kTcM = 128;        // rows per CTA (the MMA's M)
-constexpr int kTcN = 16;         // tokens per pass (the MMA's N)
-constexpr int kTcKT = 64;        // codes per K-tile (bytes of int8): 38 KB of shared memory per CTA
-constexpr int kTcKW = kTcKT / 64; // 16-byte packed words per row and tile
-constexpr int kTcBChunks = kTcN * (kTcKT / 16);  // 16-byte limb chunks per limb and tile
-constexpr int kTcThreads = 128;  // warp w reads accumulator lanes 32w .. 32w + 31
+constexpr int kTcKT = 64;        // codes per K-tile: one 16-byte packed word per row
+constexpr int kTcBRows = 64;     // rows of the B operand (limb rows of the pass's tokens): the largest N
+constexpr int kTcBChunks = kTcBRows * (kTcKT / 16);  // 16-byte chunks of B per tile
+constexpr int kTcDec = 128;      // decoder threads (thread = row); warp w reads accumulator lanes 32w .. 32w + 31
+constexpr int kTcThreads = kTcDec + 32;  // and the MMA warp
+constexpr int kTcStages = 2;     // operand buffers: 40 KB of shared memory per gate/up CTA
+constexpr int kTcDepth = 4;      // K-tiles of global loads in flight per decoder thread
 constexpr int kTcABytes = kTcM * kTcKT;
-constexpr int kTcBBytes = kTcN * kTcKT;
+constexpr int kTcBBytes = kTcBRows * kTcKT;
+// Tokens per pass.  One int8 limb (int8 activations, signed): one B row per token.  Three limbs
+// (bf16 activations): limb l of token n is B row l * NBp + n (NBp = the pass's tokens rounded up
+// to 4), and row 3 * NBp is all ones: it accumulates the row sums of the weights, which turn
+// the hi limb stored with an offset of 128 (so that every B row is unsigned) back into the signed
+// limb.  So one MMA per matrix and K step covers every limb of every token of the pass, and the
+// tensor core reads each weight tile from shared memory once.
+template <int NL>
+constexpr int kTcTokens() { return NL == 1 ? kTcBRows : (kTcBRows - 1) / 3 / 4 * 4; }
 constexpr long long kTcWaitNs = 1000000000ll;
 
 // K-major operand without swizzle: 8 rows x 16 bytes make a contiguous 128-byte core matrix,
@@ -57,8 +73,8 @@ __device__ __forceinline__ uint64_t tc_desc(uint32_t saddr) {
 // instruction descriptor: s32 accumulators (bits 4-5 = 2), A signed 8-bit (bits 7-9 = 1), B
 // signed (1) or unsigned (0) 8-bit (bits 10-12), both K-major (bits 15, 16 = 0), N / 8 in bits
 // 17-22, M / 16 in bits 24-28
-__device__ __forceinline__ uint32_t tc_idesc(bool b_signed) {
-    return (2u << 4) | (1u << 7) | ((b_signed ? 1u : 0u) << 10) | ((uint32_t)(kTcN >> 3) << 17) |
+__device__ __forceinline__ uint32_t tc_idesc(bool b_signed, int n) {
+    return (2u << 4) | (1u << 7) | ((b_signed ? 1u : 0u) << 10) | ((uint32_t)(n >> 3) << 17) |
            ((uint32_t)(kTcM >> 4) << 24);
 }
 
@@ -75,12 +91,15 @@ __device__ __forceinline__ void tc_commit(uint64_t *bar) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-__device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t (&v)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
-          "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-        : "r"(taddr));
+__device__ __forceinline__ void tc_ld4(uint32_t taddr, uint32_t (&v)[4]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+                 : "r"(taddr));
+}
+__device__ __forceinline__ void tc_ld8(uint32_t taddr, uint32_t (&v)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+                 : "r"(taddr));
 }
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tc_alloc(uint32_t *dst, uint32_t ncols) {  // one full warp
@@ -92,289 +111,377 @@ __device__ __forceinline__ void tc_dealloc(uint32_t taddr, uint32_t ncols) {  //
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
 
-// The 16 int8 weights of a packed word w (codes 0..15, two bits each: 00 = 0, 01 = +1, 10 = -1,
-// 11 reads as 0) as four words of four int8, codes in order: each 2-bit code selects a byte of the
-// table {0, +1, -1, 0} through __byte_perm (its selector nibbles are the codes).
-__device__ __forceinline__ uint4 tc_decode_word(uint32_t w) {
-    const uint32_t T = 0x00FF0100u;  // byte c = the weight of code c
-    uint32_t lo = w & 0xFFFFu, hi = w >> 16;
-    lo = (lo | (lo << 8)) & 0x00FF00FFu;
-    hi = (hi | (hi << 8)) & 0x00FF00FFu;
-    lo = (lo | (lo << 4)) & 0x0F0F0F0Fu;
-    hi = (hi | (hi << 4)) & 0x0F0F0F0Fu;
-    lo = (lo | (lo << 2)) & 0x33333333u;  // code j of the low half in nibble j
-    hi = (hi | (hi << 2)) & 0x33333333u;
-    return make_uint4(__byte_perm(T, 0u, lo), __byte_perm(T, 0u, lo >> 16), __byte_perm(T, 0u, hi),
-                      __byte_perm(T, 0u, hi >> 16));
-}
+// One K-tile of global data for a decoder thread: the packed 16 bytes (64 codes) of row
+// threadIdx.x of each matrix, and two of the tile's B chunks (chunk i = threadIdx.x + j * kTcDec:
+// B row i % 64, 16-byte chunk i / 64 of the tile).
+constexpr int kTcBPer = kTcBChunks / kTcDec;
 
-// One K-tile's global data for this thread, loaded one tile ahead of its use: the 32 packed bytes
-// of row `threadIdx.x` of each matrix, and NL chunks of 16 limb bytes (chunk i = threadIdx.x +
-// j * threads: limb l, token row n, 16-byte chunk c of the tile).
-constexpr int kTcBPerThread(int NL) { return (NL * kTcBChunks + kTcThreads - 1) / kTcThreads; }
-
-template <int NM, int NL>
+template <int NM>
 struct TcTile {
-    uint4 a[NM][kTcKW];
-    uint4 b[kTcBPerThread(NL)];
+    uint4 a[NM];
+    uint4 b[kTcBPer];
 };
 
+// Where a decoder thread's data of tile 0 sits; tile t is t uint4 further on for rows and 4t
+// for limbs.  A null pointer reads as zero (a row past the end, a B row of no token).  Each B
+// chunk is then XORed with bx[j]: 0x80 in every byte of a hi limb (the offset of 128), 0x01 in
+// every byte of the ones row.
+template <int NM>
+struct TcSrc {
+    const uint4 *a[NM];
+    const uint4 *b[kTcBPer];
+    uint32_t bx[kTcBPer];
+};
+
+// B rows of a pass of nb tokens with NL limbs, and its MMA's N (a multiple of 16)
+template <int NL>
+__device__ __forceinline__ int tc_nbp(int nb) { return NL == 1 ? nb : (nb + 3) & ~3; }
+template <int NL>
+__device__ __forceinline__ int tc_n(int nb) {
+    const int rows = NL == 1 ? nb : 3 * tc_nbp<NL>(nb) + 1;
+    return (rows + 15) & ~15;
+}
+
 template <int NM, int NL>
-__device__ __forceinline__ void tc_load(TcTile<NM, NL> &p, const uint8_t *const (&mats)[NM], int64_t rowb, int nrows,
-                                        const uint32_t *__restrict__ src, int K4, const int32_t *__restrict__ ent,
-                                        int q0, int nb, int div, int t) {
+__device__ __forceinline__ void tc_src(TcSrc<NM> &p, const uint8_t *const (&mats)[NM], int64_t rowb, int nrows,
+                                       const uint32_t *__restrict__ src, int K4, const int32_t *__restrict__ ent,
+                                       int q0, int nb, int div) {
     const int r = threadIdx.x;
 #pragma unroll
-    for (int m = 0; m < NM; m++) {
-        const uint4 *q = reinterpret_cast<const uint4 *>(mats[m] + (int64_t)r * rowb + (int64_t)t * (kTcKT / 4));
+    for (int m = 0; m < NM; m++)
+        p.a[m] = r < nrows ? reinterpret_cast<const uint4 *>(mats[m] + (int64_t)r * rowb) : nullptr;
+    const int nbp = tc_nbp<NL>(nb);
 #pragma unroll
-        for (int w = 0; w < kTcKW; w++) p.a[m][w] = r < nrows ? __ldg(q + w) : make_uint4(0u, 0u, 0u, 0u);
-    }
-    // chunk i: token row n = i % kTcN (fastest: 8 consecutive threads fill one 128-byte row of
-    // core matrices without a bank conflict), 16-byte chunk c, limb l
-#pragma unroll
-    for (int j = 0; j < kTcBPerThread(NL); j++) {
-        const int i = threadIdx.x + j * kTcThreads;
-        const int n = i % kTcN, c = (i / kTcN) % (kTcKT / 16), l = i / kTcBChunks;
-        p.b[j] = make_uint4(0u, 0u, 0u, 0u);
+    for (int j = 0; j < kTcBPer; j++) {
+        const int i = threadIdx.x + j * kTcDec;
+        const int row = i % kTcBRows, c = i / kTcBRows;
+        int l = 0, n = row;
+        if (NL > 1) {
+            l = row / nbp;
+            n = row - l * nbp;
+        }
+        p.b[j] = nullptr;
+        p.bx[j] = 0u;
         if (l < NL && n < nb) {
             const int64_t vec = ent[q0 + n] / div;
-            p.b[j] = __ldg(reinterpret_cast<const uint4 *>(src + (vec * NL + l) * K4 + (int64_t)t * (kTcKT / 4)) + c);
+            p.b[j] = reinterpret_cast<const uint4 *>(src + (vec * NL + l) * K4) + c;
+            if (NL > 1 && l == 0) p.bx[j] = 0x80808080u;
+        } else if (NL > 1 && row == 3 * nbp) {
+            p.bx[j] = 0x01010101u;
         }
     }
 }
 
-// the tile into shared memory: weights decoded into A (K-major layout), limbs into B
-template <int NM, int NL>
-__device__ __forceinline__ void tc_store(const TcTile<NM, NL> &p, unsigned char *A, unsigned char *B) {
+template <int NM>
+__device__ __forceinline__ void tc_load(TcTile<NM> &p, const TcSrc<NM> &q, int t) {
+#pragma unroll
+    for (int m = 0; m < NM; m++) p.a[m] = q.a[m] ? __ldg(q.a[m] + t) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int j = 0; j < kTcBPer; j++) {
+        const uint4 v = q.b[j] ? __ldg(q.b[j] + (kTcKT / 16) * t) : make_uint4(0u, 0u, 0u, 0u);
+        p.b[j] = make_uint4(v.x ^ q.bx[j], v.y ^ q.bx[j], v.z ^ q.bx[j], v.w ^ q.bx[j]);
+    }
+}
+
+// The tile into one operand buffer.  Packed word q of the row (codes 16q .. 16q + 15) becomes
+// 16-byte chunk q of the row in the table-free decode's position-major order: byte 4j + b
+// holds 64 times the weight of code 16q + 4b + j (decode.cuh).  The B chunks take the same
+// order by a 4x4 byte transpose, so A and B agree on every K index of the tile.
+template <int NM>
+__device__ __forceinline__ void tc_store(const TcTile<NM> &p, unsigned char *A, unsigned char *B) {
     const int r = threadIdx.x;
 #pragma unroll
     for (int m = 0; m < NM; m++) {
+        const uint32_t pw[4] = {p.a[m].x, p.a[m].y, p.a[m].z, p.a[m].w};
 #pragma unroll
-        for (int w = 0; w < kTcKW; w++) {
-            const uint32_t pw[4] = {p.a[m][w].x, p.a[m][w].y, p.a[m][w].z, p.a[m][w].w};
-#pragma unroll
-            for (int c = 0; c < 4; c++)  // 16 codes per packed word = one 16-byte chunk of the tile
-                *reinterpret_cast<uint4 *>(A + (size_t)m * kTcABytes + tc_off(r, 16 * (4 * w + c))) =
-                    tc_decode_word(pw[c]);
+        for (int q = 0; q < 4; q++) {
+            const uint32_t sf = tern_signed_fields(pw[q]);
+            *reinterpret_cast<uint4 *>(A + (size_t)m * kTcABytes + tc_off(r, 16 * q)) =
+                make_uint4(tern_position_lanes(sf, 0), tern_position_lanes(sf, 1), tern_position_lanes(sf, 2),
+                           tern_position_lanes(sf, 3));
         }
     }
 #pragma unroll
-    for (int j = 0; j < kTcBPerThread(NL); j++) {
-        const int i = threadIdx.x + j * kTcThreads;
-        const int n = i % kTcN, c = (i / kTcN) % (kTcKT / 16), l = i / kTcBChunks;
-        if (l < NL) *reinterpret_cast<uint4 *>(B + (size_t)l * kTcBBytes + tc_off(n, 16 * c)) = p.b[j];
+    for (int j = 0; j < kTcBPer; j++) {
+        const int i = threadIdx.x + j * kTcDec;
+        uint4 v;
+        bytes_transpose4(p.b[j].x, p.b[j].y, p.b[j].z, p.b[j].w, v.x, v.y, v.z, v.w);
+        *reinterpret_cast<uint4 *>(B + tc_off(i % kTcBRows, 16 * (i / kTcBRows))) = v;
     }
 }
 
-// The K loop of one token pass: NM matrices x NL limbs accumulate into tensor-memory columns
-// (m * NL + l) * kTcN .. + kTcN.  `it` counts tiles across passes (buffer it & 1; mbarrier b
-// completes once per tile issued on it).  Tile t + 1's global loads are in flight while tile t is
-// decoded, stored and multiplied.  Returns false on a timed-out wait.
-template <int NM, int NL>
-__device__ __forceinline__ bool tc_pass(unsigned char *A, unsigned char *B, uint64_t *mb, uint32_t tmem,
-                                        const uint8_t *const (&mats)[NM], int64_t rowb, int nrows, int ntile,
-                                        const uint32_t *__restrict__ src, int K4, const int32_t *__restrict__ ent,
-                                        int q0, int nb, int div, unsigned &it, int *status) {
-    TcTile<NM, NL> cur, nxt;
-    tc_load<NM, NL>(nxt, mats, rowb, nrows, src, K4, ent, q0, nb, div, 0);
-    for (int t = 0; t < ntile; t++, it++) {
-        cur = nxt;
-        if (t + 1 < ntile) tc_load<NM, NL>(nxt, mats, rowb, nrows, src, K4, ent, q0, nb, div, t + 1);
-        const int b = (int)(it & 1u);
-        // the buffer's previous tile (two tiles back) must be consumed by the tensor core
-        if (it >= 2 && !mbar_wait(&mb[b], ((it - 2) >> 1) & 1u, kTcWaitNs, status)) return false;
-        unsigned char *Ab = A + (size_t)b * NM * kTcABytes;
-        unsigned char *Bb = B + (size_t)b * NL * kTcBBytes;
-        tc_store<NM, NL>(cur, Ab, Bb);
-        fence_async_smem();  // the generic-proxy writes above, visible to the tensor core
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            tc_fence_after();
+// Shared state of one CTA's pipeline: operand buffers, their mbarriers and the tile counter.
+// Tile g (counted over the CTA's passes) goes to buffer g % kTcStages as that buffer's use
+// g / kTcStages.  mb_full[b] completes a phase when the four decoder warps have stored a tile
+// into buffer b; mb_done[b] when the MMAs reading it have finished (tcgen05.commit).
+struct TcPipe {
+    unsigned char *A, *B;
+    uint64_t *full, *done;
+    uint32_t tmem;
+    unsigned it;
+    bool failed;  // a wait timed out (status set): the pipeline keeps its protocol but skips work
+};
+
+// Decoder side of one pass (warps 0..3): tiles 0 .. ntile-1 of the pass, kTcDepth tiles of global
+// loads in flight, each tile decoded into the next buffer once the tensor core has finished with
+// that buffer's previous tile.  Returns once every MMA of the pass has completed.
+template <int NM>
+__device__ __forceinline__ void tc_decode_pass(TcPipe &pp, const TcSrc<NM> &src, int ntile, int *status) {
+    const int lane = threadIdx.x & 31;
+    TcTile<NM> buf[kTcDepth];
+#pragma unroll
+    for (int j = 0; j < kTcDepth; j++)
+        if (j < ntile) tc_load<NM>(buf[j], src, j);
+    for (int t0 = 0; t0 < ntile; t0 += kTcDepth) {
+#pragma unroll
+        for (int j = 0; j < kTcDepth; j++) {
+            const int t = t0 + j;
+            if (t < ntile) {
+                const unsigned g = pp.it + (unsigned)t;
+                const int b = (int)(g % kTcStages);
+                if (g >= kTcStages && !pp.failed &&
+                    !mbar_wait(&pp.done[b], ((g / kTcStages) - 1u) & 1u, kTcWaitNs, status))
+                    pp.failed = true;
+                if (!pp.failed) tc_store<NM>(buf[j], pp.A + (size_t)b * NM * kTcABytes, pp.B + (size_t)b * kTcBBytes);
+                if (t + kTcDepth < ntile) tc_load<NM>(buf[j], src, t + kTcDepth);
+                fence_async_smem();  // the generic-proxy stores above, visible to the tensor core
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&pp.full[b]);
+            }
+        }
+    }
+    const unsigned last = pp.it + (unsigned)ntile - 1u;
+    if (!pp.failed && !mbar_wait(&pp.done[last % kTcStages], (last / kTcStages) & 1u, kTcWaitNs, status))
+        pp.failed = true;
+    tc_fence_after();
+    pp.it += (unsigned)ntile;
+}
+
+// MMA side of one pass (lane 0 of warp 4): per tile, wait for the decoders, issue NM x (kTcKT /
+// 32) MMAs (M = 128, N = n, K = 32) into accumulator columns m * kTcBRows .. + n, and commit to
+// the buffer's mbarrier.  The descriptors of buffer 0 are built once; a buffer, matrix or K step
+// is an offset added to the start-address field.
+template <int NM>
+__device__ __forceinline__ void tc_mma_pass(TcPipe &pp, int ntile, uint32_t idesc, int *status) {
+    const uint64_t a0 = tc_desc(smem_u32(pp.A)), b0 = tc_desc(smem_u32(pp.B));
+    for (int t = 0; t < ntile; t++) {
+        const unsigned g = pp.it + (unsigned)t;
+        const int b = (int)(g % kTcStages);
+        if (!pp.failed && !mbar_wait(&pp.full[b], (g / kTcStages) & 1u, kTcWaitNs, status)) pp.failed = true;
+        tc_fence_after();
+        if (!pp.failed) {
 #pragma unroll
             for (int s = 0; s < kTcKT / 32; s++)
 #pragma unroll
                 for (int m = 0; m < NM; m++)
-#pragma unroll
-                    for (int l = 0; l < NL; l++)
-                        tc_mma(tmem + (uint32_t)((m * NL + l) * kTcN),
-                               tc_desc(smem_u32(Ab + (size_t)m * kTcABytes + s * 256)),
-                               tc_desc(smem_u32(Bb + (size_t)l * kTcBBytes + s * 256)), tc_idesc(l == 0),
-                               (t > 0 || s > 0) ? 1u : 0u);
-            tc_commit(&mb[b]);
+                    tc_mma(pp.tmem + (uint32_t)(m * kTcBRows), a0 + (uint64_t)((((b * NM + m) * kTcABytes) + s * 256) >> 4),
+                           b0 + (uint64_t)(((b * kTcBBytes) + s * 256) >> 4), idesc, (t > 0 || s > 0) ? 1u : 0u);
         }
+        tc_commit(&pp.done[b]);
     }
-    // every MMA of the pass done (the last commit covers all earlier ones)
-    const unsigned last = it - 1;
-    if (!mbar_wait(&mb[last & 1u], (last >> 1) & 1u, kTcWaitNs, status)) return false;
+    pp.it += (unsigned)ntile;
+}
+
+// The CTA's set-up: mbarriers, tensor memory (warp 0), then one barrier.
+__device__ __forceinline__ void tc_setup(TcPipe &pp, unsigned char *smem, int a_bytes, uint64_t *full, uint64_t *done,
+                                         uint32_t *s_tmem, uint32_t ncols) {
+    pp.A = smem;
+    pp.B = smem + a_bytes;
+    pp.full = full;
+    pp.done = done;
+    pp.it = 0;
+    pp.failed = false;
+    if (threadIdx.x == 0) {
+        for (int b = 0; b < kTcStages; b++) {
+            mbar_init(&full[b], kTcDec / 32);
+            mbar_init(&done[b], 1);
+        }
+        fence_mbar_init();
+    }
+    if (threadIdx.x < 32) tc_alloc(s_tmem, ncols);
+    tc_fence_before();
+    __syncthreads();
     tc_fence_after();
-    return true;
+    pp.tmem = *s_tmem;
+}
+
+// The end: the MMA thread waits for its last commit, then warp 0 frees the tensor memory.
+__device__ __forceinline__ void tc_teardown(TcPipe &pp, uint32_t ncols, int *status) {
+    if (threadIdx.x == kTcDec && pp.it > 0 && !pp.failed) {
+        const unsigned last = pp.it - 1u;
+        mbar_wait(&pp.done[last % kTcStages], (last / kTcStages) & 1u, kTcWaitNs, status);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (threadIdx.x < 32) tc_dealloc(pp.tmem, ncols);
+}
+
+// an accumulator column read back: 64 times the exact sum (the weights are 64 * w)
+__device__ __forceinline__ long long tc_acc(uint32_t v) { return (long long)((int32_t)v >> 6); }
+
+// The exact integer sums of tokens n0 .. n0 + 3 (pass of nbp B rows per limb) for the matrix
+// whose accumulators start at column `col` of this thread's lane: three limbs recombined, the
+// hi limb's offset of 128 taken out with the row sum R of the ones row.
+template <int NL>
+__device__ __forceinline__ void tc_sums4(uint32_t ta, int col, int nbp, int n0, long long R, long long (&S)[4]) {
+    if (NL == 1) {
+        uint32_t v[4];
+        tc_ld4(ta + (uint32_t)(col + n0), v);
+        tc_wait_ld();
+#pragma unroll
+        for (int z = 0; z < 4; z++) S[z] = tc_acc(v[z]);
+    } else {
+        uint32_t v0[4], v1[4], v2[4];
+        tc_ld4(ta + (uint32_t)(col + n0), v0);
+        tc_ld4(ta + (uint32_t)(col + nbp + n0), v1);
+        tc_ld4(ta + (uint32_t)(col + 2 * nbp + n0), v2);
+        tc_wait_ld();
+#pragma unroll
+        for (int z = 0; z < 4; z++) S[z] = (tc_acc(v0[z]) - 128 * R) * 65536 + tc_acc(v1[z]) * 256 + tc_acc(v2[z]);
+    }
+}
+
+// row sum of the weights over K (the ones row of a three-limb pass), for the matrix at `col`
+template <int NL>
+__device__ __forceinline__ long long tc_rowsum(uint32_t ta, int col, int nbp) {
+    if (NL == 1) return 0;
+    uint32_t v[4];
+    tc_ld4(ta + (uint32_t)(col + 3 * nbp), v);
+    tc_wait_ld();
+    return tc_acc(v[0]);
 }
 
 // grid: (distinct experts bound, f / 128); 128 rows of gate and up per CTA
 template <int NL>
-__global__ void __launch_bounds__(kTcThreads) gateup_tc_kernel(
+__global__ void __launch_bounds__(kTcThreads, 3) gateup_tc_kernel(
     const uint8_t *__restrict__ gate, const uint8_t *__restrict__ up, const float *__restrict__ sg,
     const float *__restrict__ su, int d, int f, int k, const int32_t *__restrict__ n_unique,
     const int32_t *__restrict__ uexp, const int32_t *__restrict__ uoff, const int32_t *__restrict__ ent,
     const uint32_t *__restrict__ xw, const float *__restrict__ xsc, float *__restrict__ h,
     int32_t *__restrict__ acc_g, int32_t *__restrict__ acc_u, int *status) {
     extern __shared__ __align__(128) unsigned char smem[];
-    __shared__ __align__(8) uint64_t mb[2];
+    __shared__ __align__(8) uint64_t mb_full[kTcStages], mb_done[kTcStages];
     __shared__ uint32_t s_tmem;
     const int u = blockIdx.x;
     if (u >= *n_unique) return;  // before any tensor memory is held
-    constexpr int NCOL = 2 * NL * kTcN;
-    constexpr uint32_t ALLOC = NCOL <= 32 ? 32u : (NCOL <= 64 ? 64u : 128u);
+    constexpr uint32_t ALLOC = 2 * kTcBRows;
+    constexpr int NBMAX = kTcTokens<NL>();
     const int tid = threadIdx.x, warp = tid >> 5;
     const int e = uexp[u], e0 = uoff[u], e1 = uoff[u + 1];
     const int row0 = blockIdx.y * kTcM, nrows = min(kTcM, f - row0);
     const int64_t rowb = d / 4;
+    const int ntile = d / kTcKT;
     const uint8_t *const mats[2] = {gate + ((int64_t)e * f + row0) * rowb, up + ((int64_t)e * f + row0) * rowb};
-    unsigned char *A = smem;                                // [2 buffers][2 matrices][kTcABytes]
-    unsigned char *B = smem + 2 * 2 * kTcABytes;            // [2 buffers][NL][kTcBBytes]
-    if (tid == 0) {
-        mbar_init(&mb[0], 1);
-        mbar_init(&mb[1], 1);
-        fence_mbar_init();
-    }
-    if (warp == 0) tc_alloc(&s_tmem, ALLOC);
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = s_tmem;
-    unsigned it = 0;
-    bool ok = true;
-    for (int q0 = e0; q0 < e1 && ok; q0 += kTcN) {
-        const int nb = min(kTcN, e1 - q0);
-        ok = tc_pass<2, NL>(A, B, mb, tmem, mats, rowb, nrows, d / kTcKT, xw, d / 4, ent, q0, nb, k, it, status);
-        if (!ok) break;
-        // thread = row of this tile; the accumulators of token n are column n of each block
-        const int j = row0 + tid;
-        const uint32_t ta = tmem + ((uint32_t)(32 * warp) << 16);
-        long long Sg[kTcN], Su[kTcN];
-#pragma unroll
-        for (int n = 0; n < kTcN; n++) Sg[n] = Su[n] = 0;
-#pragma unroll
-        for (int l = 0; l < NL; l++) {
-            const long long wgt = (NL == 1) ? 1ll : (l == 0 ? 65536ll : (l == 1 ? 256ll : 1ll));
-            uint32_t vg[16], vu[16];
-            tc_ld16(ta + (uint32_t)((0 * NL + l) * kTcN), vg);
-            tc_ld16(ta + (uint32_t)((1 * NL + l) * kTcN), vu);
-            tc_wait_ld();
-#pragma unroll
-            for (int n = 0; n < kTcN; n++) {
-                Sg[n] += (long long)(int32_t)vg[n] * wgt;
-                Su[n] += (long long)(int32_t)vu[n] * wgt;
-            }
+    TcPipe pp;
+    tc_setup(pp, smem, kTcStages * 2 * kTcABytes, mb_full, mb_done, &s_tmem, ALLOC);
+    for (int q0 = e0; q0 < e1; q0 += NBMAX) {
+        const int nb = min(NBMAX, e1 - q0), nbp = tc_nbp<NL>(nb);
+        if (warp == kTcDec / 32) {  // the MMA warp
+            if ((tid & 31) == 0) tc_mma_pass<2>(pp, ntile, tc_idesc(NL == 1, tc_n<NL>(nb)), status);
+            continue;
         }
-        if (j < f) {
-            const int64_t o = (int64_t)e * f + j;
-            const float sgv = sg[o], suv = su[o];
+        TcSrc<2> src;
+        tc_src<2, NL>(src, mats, rowb, nrows, xw, d / 4, ent, q0, nb, k);
+        tc_decode_pass<2>(pp, src, ntile, status);
+        // thread = row of this tile; nb is the same in every thread, so the accumulator loads
+        // stay collective
+        const int j = row0 + tid;
+        const uint32_t ta = pp.tmem + ((uint32_t)(32 * warp) << 16);
+        const bool live = j < f && !pp.failed;
+        const float sgv = live ? sg[(int64_t)e * f + j] : 0.0f, suv = live ? su[(int64_t)e * f + j] : 0.0f;
+        const long long Rg = tc_rowsum<NL>(ta, 0, nbp), Ru = tc_rowsum<NL>(ta, kTcBRows, nbp);
+#pragma unroll 1
+        for (int n0 = 0; n0 < nb; n0 += 4) {
+            long long Sg[4], Su[4];
+            tc_sums4<NL>(ta, 0, nbp, n0, Rg, Sg);
+            tc_sums4<NL>(ta, kTcBRows, nbp, n0, Ru, Su);
 #pragma unroll
-            for (int n = 0; n < kTcN; n++) {
-                if (n >= nb) continue;
+            for (int z = 0; z < 4; z++) {
+                const int n = n0 + z;
+                if (!live || n >= nb) continue;
                 const int entry = ent[q0 + n];
                 const float xsv = xsc[entry / k];
                 float hv;
                 if (NL == 1) {
-                    acc_g[(int64_t)entry * f + j] = (int32_t)Sg[n];
-                    acc_u[(int64_t)entry * f + j] = (int32_t)Su[n];
-                    const float gv = __fmul_rn(__fmul_rn(__int2float_rn((int)Sg[n]), sgv), xsv);
-                    const float uv = __fmul_rn(__fmul_rn(__int2float_rn((int)Su[n]), suv), xsv);
+                    acc_g[(int64_t)entry * f + j] = (int32_t)Sg[z];
+                    acc_u[(int64_t)entry * f + j] = (int32_t)Su[z];
+                    const float gv = __fmul_rn(__fmul_rn(__int2float_rn((int)Sg[z]), sgv), xsv);
+                    const float uv = __fmul_rn(__fmul_rn(__int2float_rn((int)Su[z]), suv), xsv);
                     hv = swiglu_f32((double)gv, (double)uv);
                 } else {
                     const int sh = __float_as_int(xsv);
-                    hv = swiglu_f32(ldexp((double)Sg[n], -sh) * (double)sgv, ldexp((double)Su[n], -sh) * (double)suv);
+                    hv = swiglu_f32(ldexp((double)Sg[z], -sh) * (double)sgv, ldexp((double)Su[z], -sh) * (double)suv);
                 }
                 h[(int64_t)entry * f + j] = hv;
             }
         }
-        // every thread's reads of the accumulators are done before the next pass overwrites them
+        // every read of the accumulators done before this warp's next arrival lets the MMA
+        // thread overwrite them
         tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
     }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) tc_dealloc(tmem, ALLOC);
+    tc_teardown(pp, ALLOC, status);
 }
 
 // grid: (distinct experts bound, d / 128); 128 output rows per CTA
 template <int NL>
-__global__ void __launch_bounds__(kTcThreads) down_tc_kernel(
+__global__ void __launch_bounds__(kTcThreads, 3) down_tc_kernel(
     const uint8_t *__restrict__ down, const float *__restrict__ sd, int d, int f, const int32_t *__restrict__ n_unique,
     const int32_t *__restrict__ uexp, const int32_t *__restrict__ uoff, const int32_t *__restrict__ ent,
     const uint32_t *__restrict__ hw, const float *__restrict__ hsc, double *__restrict__ ye,
     int32_t *__restrict__ acc_d, int *status) {
     extern __shared__ __align__(128) unsigned char smem[];
-    __shared__ __align__(8) uint64_t mb[2];
+    __shared__ __align__(8) uint64_t mb_full[kTcStages], mb_done[kTcStages];
     __shared__ uint32_t s_tmem;
     const int u = blockIdx.x;
     if (u >= *n_unique) return;
-    constexpr int NCOL = NL * kTcN;
-    constexpr uint32_t ALLOC = NCOL <= 32 ? 32u : (NCOL <= 64 ? 64u : 128u);
+    constexpr uint32_t ALLOC = kTcBRows;
+    constexpr int NBMAX = kTcTokens<NL>();
     const int tid = threadIdx.x, warp = tid >> 5;
     const int e = uexp[u], e0 = uoff[u], e1 = uoff[u + 1];
     const int row0 = blockIdx.y * kTcM, nrows = min(kTcM, d - row0);
     const int64_t rowb = f / 4;
+    const int ntile = f / kTcKT;
     const uint8_t *const mats[1] = {down + ((int64_t)e * d + row0) * rowb};
-    unsigned char *A = smem;                            // [2 buffers][kTcABytes]
-    unsigned char *B = smem + 2 * kTcABytes;            // [2 buffers][NL][kTcBBytes]
-    if (tid == 0) {
-        mbar_init(&mb[0], 1);
-        mbar_init(&mb[1], 1);
-        fence_mbar_init();
-    }
-    if (warp == 0) tc_alloc(&s_tmem, ALLOC);
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = s_tmem;
-    unsigned it = 0;
-    bool ok = true;
-    for (int q0 = e0; q0 < e1 && ok; q0 += kTcN) {
-        const int nb = min(kTcN, e1 - q0);
-        ok = tc_pass<1, NL>(A, B, mb, tmem, mats, rowb, nrows, f / kTcKT, hw, f / 4, ent, q0, nb, 1, it, status);
-        if (!ok) break;
-        const int i = row0 + tid;
-        const uint32_t ta = tmem + ((uint32_t)(32 * warp) << 16);
-        long long S[kTcN];
-#pragma unroll
-        for (int n = 0; n < kTcN; n++) S[n] = 0;
-#pragma unroll
-        for (int l = 0; l < NL; l++) {
-            const long long wgt = (NL == 1) ? 1ll : (l == 0 ? 65536ll : (l == 1 ? 256ll : 1ll));
-            uint32_t v[16];
-            tc_ld16(ta + (uint32_t)(l * kTcN), v);
-            tc_wait_ld();
-#pragma unroll
-            for (int n = 0; n < kTcN; n++) S[n] += (long long)(int32_t)v[n] * wgt;
+    TcPipe pp;
+    tc_setup(pp, smem, kTcStages * kTcABytes, mb_full, mb_done, &s_tmem, ALLOC);
+    for (int q0 = e0; q0 < e1; q0 += NBMAX) {
+        const int nb = min(NBMAX, e1 - q0), nbp = tc_nbp<NL>(nb);
+        if (warp == kTcDec / 32) {
+            if ((tid & 31) == 0) tc_mma_pass<1>(pp, ntile, tc_idesc(NL == 1, tc_n<NL>(nb)), status);
+            continue;
         }
-        if (i < d) {
-            const float sdv = sd[(int64_t)e * d + i];
+        TcSrc<1> src;
+        tc_src<1, NL>(src, mats, rowb, nrows, hw, f / 4, ent, q0, nb, 1);
+        tc_decode_pass<1>(pp, src, ntile, status);
+        const int i = row0 + tid;
+        const uint32_t ta = pp.tmem + ((uint32_t)(32 * warp) << 16);
+        const bool live = i < d && !pp.failed;
+        const float sdv = live ? sd[(int64_t)e * d + i] : 0.0f;
+        const long long R = tc_rowsum<NL>(ta, 0, nbp);
+#pragma unroll 1
+        for (int n0 = 0; n0 < nb; n0 += 4) {
+            long long S[4];
+            tc_sums4<NL>(ta, 0, nbp, n0, R, S);
 #pragma unroll
-            for (int n = 0; n < kTcN; n++) {
-                if (n >= nb) continue;
+            for (int z = 0; z < 4; z++) {
+                const int n = n0 + z;
+                if (!live || n >= nb) continue;
                 const int entry = ent[q0 + n];
                 const float hs = hsc[entry];
                 double v;
                 if (NL == 1) {
-                    acc_d[(int64_t)entry * d + i] = (int32_t)S[n];
-                    v = (double)__fmul_rn(__fmul_rn(__int2float_rn((int)S[n]), sdv), hs);
+                    acc_d[(int64_t)entry * d + i] = (int32_t)S[z];
+                    v = (double)__fmul_rn(__fmul_rn(__int2float_rn((int)S[z]), sdv), hs);
                 } else {
-                    v = ldexp((double)S[n], -__float_as_int(hs)) * (double)sdv;
+                    v = ldexp((double)S[z], -__float_as_int(hs)) * (double)sdv;
                 }
                 ye[(int64_t)entry * d + i] = v;
             }
         }
         tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
     }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) tc_dealloc(tmem, ALLOC);
+    tc_teardown(pp, ALLOC, status);
 }
 
 bool tc_grouped_supported(int d, int f) { return d % kTcKT == 0 && f % kTcKT == 0; }
@@ -385,13 +492,13 @@ cudaError_t launch_grouped_tc(const tern_moe_layer *L, int T, const FfnWs &w, cu
     const int umax = (E < T * k) ? E : T * k;
     int *st = status_word();
     if (phase == 0) {
-        const size_t sm = (size_t)2 * 2 * kTcABytes + (size_t)2 * NL * kTcBBytes;
+        const size_t sm = (size_t)kTcStages * (2 * kTcABytes + kTcBBytes);
         cudaFuncSetAttribute(gateup_tc_kernel<NL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
         gateup_tc_kernel<NL><<<dim3(umax, (f + kTcM - 1) / kTcM), kTcThreads, sm, s>>>(
             L->gate, L->up, L->gate_scale, L->up_scale, d, f, k, w.n_unique, w.uexp, w.uoff, w.ent,
             (const uint32_t *)w.xw, (const float *)w.xsc, w.h, w.acc_g, w.acc_u, st);
     } else {
-        const size_t sm = (size_t)2 * kTcABytes + (size_t)2 * NL * kTcBBytes;
+        const size_t sm = (size_t)kTcStages * (kTcABytes + kTcBBytes);
         cudaFuncSetAttribute(down_tc_kernel<NL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
         down_tc_kernel<NL><<<dim3(umax, (d + kTcM - 1) / kTcM), kTcThreads, sm, s>>>(
             L->down, L->down_scale, d, f, w.n_unique, w.uexp, w.uoff, w.ent, (const uint32_t *)w.hw,

@@ -580,6 +580,18 @@ __device__ __forceinline__ float swiglu_f32(double g, double u) {
     return (float)(g / (1.0 + exp(-g)) * u);
 }
 
+// 4x4 byte transpose, into the position-major order of the table-free decode: P_j holds byte j
+// of N0, N1, N2, N3 (in that byte order)
+__device__ __forceinline__ void bytes_transpose4(uint32_t n0, uint32_t n1, uint32_t n2, uint32_t n3, uint32_t &p0,
+                                                 uint32_t &p1, uint32_t &p2, uint32_t &p3) {
+    const uint32_t t0 = __byte_perm(n0, n1, 0x5140u), t1 = __byte_perm(n2, n3, 0x5140u);
+    const uint32_t t2 = __byte_perm(n0, n1, 0x7362u), t3 = __byte_perm(n2, n3, 0x7362u);
+    p0 = __byte_perm(t0, t1, 0x5410u);
+    p1 = __byte_perm(t0, t1, 0x7632u);
+    p2 = __byte_perm(t2, t3, 0x5410u);
+    p3 = __byte_perm(t2, t3, 0x7632u);
+}
+
 // Limb bytes of four consecutive values v[0..3] (elements 4t..4t+3 of a vector whose limbs go
 // to `limbs`, laid out [NL][segments][kSegPad words], position-major inside each segment):
 // element 4t+e lands in byte (t & 3) of word 4 * ((t >> 2) & 3) + e of segment t >> 4.

@@ -157,6 +157,25 @@ def test_moe_layer_batch_invariance(layer_pair, act):
         assert torch.equal(y132, yb32[t:t + 1])
 
 
+@pytest.mark.parametrize("act", [tm.TERN_ACT_BF16, tm.TERN_ACT_INT8])
+def test_moe_layer_grouped_multi_pass(layer_pair, act):
+    """An expert with more tokens than one tensor-core pass takes with bf16 activations (20):
+    50 copies of one token send 50 tokens to each of its experts (passes of 20, 20 and 10; with
+    int8 activations one pass of 50 takes all); every token's output still equals its batch-1
+    output bit for bit."""
+    shape, dl, hl = layer_pair
+    dev = dl.gate.device
+    x = synth.tokens_bf16(WID_LAYER, 310, 64, shape.d)
+    x[:50] = x[0]
+    yb32 = torch.empty((64, shape.d), dtype=torch.float32, device=dev)
+    yb = tm.moe_ffn_decode(dl, dev_u16(x, dev), act=act, y_f32=yb32)
+    for t in (0, 21, 49, 50, 63):
+        y132 = torch.empty((1, shape.d), dtype=torch.float32, device=dev)
+        y1 = tm.moe_ffn_decode(dl, dev_u16(x[t:t + 1], dev), act=act, y_f32=y132)
+        assert torch.equal(y1.view(torch.int16), yb[t:t + 1].view(torch.int16))
+        assert torch.equal(y132, yb32[t:t + 1])
+
+
 def test_moe_layer_repeat_is_deterministic(layer_pair):
     shape, dl, hl = layer_pair
     dev = dl.gate.device
