@@ -40,6 +40,7 @@ constexpr int kTcDec = 128;      // decoder threads (thread = row); warp w reads
 constexpr int kTcThreads = kTcDec + 32;  // and the MMA warp
 constexpr int kTcStages = 2;     // operand buffers: 40 KB of shared memory per gate/up CTA
 constexpr int kTcDepth = 4;      // K-tiles of global loads in flight per decoder thread
+constexpr int kTcDownRB = 2;     // blocks of 128 rows per down CTA
 constexpr int kTcABytes = kTcM * kTcKT;
 constexpr int kTcBBytes = kTcBRows * kTcKT;
 // Tokens per pass.  One int8 limb (int8 activations, signed): one B row per token.  Three limbs
@@ -122,15 +123,25 @@ struct TcTile {
     uint4 b[kTcBPer];
 };
 
-// Where a decoder thread's data of tile 0 sits; tile t is t uint4 further on for rows and 4t
-// for limbs.  A null pointer reads as zero (a row past the end, a B row of no token).  Each B
-// chunk is then XORed with bx[j]: 0x80 in every byte of a hi limb (the offset of 128), 0x01 in
+// Where a decoder thread's data of tile 0 sits.  A CTA takes NRB blocks of 128 rows one after
+// another, ntk K-tiles each: tile t is K-tile t % ntk of row block t / ntk, t % ntk uint4 into the
+// row and rbstep uint4 on per row block; for the limbs 4 (t % ntk) uint4 on.  A null pointer, or
+// a row block at or past nrb (the blocks in which this thread's row exists), reads as zero.  Each
+// B chunk is then XORed with bx[j]: 0x80 in every byte of a hi limb (the offset of 128), 0x01 in
 // every byte of the ones row.
+// row block of tile t (ntk tiles per block)
+template <int NRB>
+__device__ __forceinline__ int tc_rb(int t, int ntk) {
+    return NRB == 1 ? 0 : (NRB == 2 ? (t >= ntk ? 1 : 0) : t / ntk);
+}
+
 template <int NM>
 struct TcSrc {
     const uint4 *a[NM];
     const uint4 *b[kTcBPer];
     uint32_t bx[kTcBPer];
+    int64_t rbstep;
+    int ntk, nrb;
 };
 
 // B rows of a pass of nb tokens with NL limbs, and its MMA's N (a multiple of 16)
@@ -142,14 +153,18 @@ __device__ __forceinline__ int tc_n(int nb) {
     return (rows + 15) & ~15;
 }
 
-template <int NM, int NL>
+// mats[m]: row 0 of the CTA's first row block; nrows: the CTA's rows that exist (from row 0 on)
+template <int NM, int NL, int NRB>
 __device__ __forceinline__ void tc_src(TcSrc<NM> &p, const uint8_t *const (&mats)[NM], int64_t rowb, int nrows,
-                                       const uint32_t *__restrict__ src, int K4, const int32_t *__restrict__ ent,
-                                       int q0, int nb, int div) {
+                                       int ntk, const uint32_t *__restrict__ src, int K4,
+                                       const int32_t *__restrict__ ent, int q0, int nb, int div) {
     const int r = threadIdx.x;
 #pragma unroll
     for (int m = 0; m < NM; m++)
         p.a[m] = r < nrows ? reinterpret_cast<const uint4 *>(mats[m] + (int64_t)r * rowb) : nullptr;
+    p.rbstep = (int64_t)kTcM * rowb / 16;
+    p.ntk = ntk;
+    p.nrb = r < nrows ? min(NRB, (nrows - r + kTcM - 1) / kTcM) : 0;
     const int nbp = tc_nbp<NL>(nb);
 #pragma unroll
     for (int j = 0; j < kTcBPer; j++) {
@@ -172,13 +187,15 @@ __device__ __forceinline__ void tc_src(TcSrc<NM> &p, const uint8_t *const (&mats
     }
 }
 
-template <int NM>
+template <int NM, int NRB>
 __device__ __forceinline__ void tc_load(TcTile<NM> &p, const TcSrc<NM> &q, int t) {
+    const int rb = tc_rb<NRB>(t, q.ntk), kt = t - rb * q.ntk;
 #pragma unroll
-    for (int m = 0; m < NM; m++) p.a[m] = q.a[m] ? __ldg(q.a[m] + t) : make_uint4(0u, 0u, 0u, 0u);
+    for (int m = 0; m < NM; m++)
+        p.a[m] = rb < q.nrb ? __ldg(q.a[m] + rb * q.rbstep + kt) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
     for (int j = 0; j < kTcBPer; j++) {
-        const uint4 v = q.b[j] ? __ldg(q.b[j] + (kTcKT / 16) * t) : make_uint4(0u, 0u, 0u, 0u);
+        const uint4 v = q.b[j] ? __ldg(q.b[j] + (kTcKT / 16) * kt) : make_uint4(0u, 0u, 0u, 0u);
         p.b[j] = make_uint4(v.x ^ q.bx[j], v.y ^ q.bx[j], v.z ^ q.bx[j], v.w ^ q.bx[j]);
     }
 }
@@ -225,13 +242,13 @@ struct TcPipe {
 // Decoder side of one pass (warps 0..3): tiles 0 .. ntile-1 of the pass, kTcDepth tiles of global
 // loads in flight, each tile decoded into the next buffer once the tensor core has finished with
 // that buffer's previous tile.  Returns once every MMA of the pass has completed.
-template <int NM>
+template <int NM, int NRB>
 __device__ __forceinline__ void tc_decode_pass(TcPipe &pp, const TcSrc<NM> &src, int ntile, int *status) {
     const int lane = threadIdx.x & 31;
     TcTile<NM> buf[kTcDepth];
 #pragma unroll
     for (int j = 0; j < kTcDepth; j++)
-        if (j < ntile) tc_load<NM>(buf[j], src, j);
+        if (j < ntile) tc_load<NM, NRB>(buf[j], src, j);
     for (int t0 = 0; t0 < ntile; t0 += kTcDepth) {
 #pragma unroll
         for (int j = 0; j < kTcDepth; j++) {
@@ -240,10 +257,10 @@ __device__ __forceinline__ void tc_decode_pass(TcPipe &pp, const TcSrc<NM> &src,
                 const unsigned g = pp.it + (unsigned)t;
                 const int b = (int)(g % kTcStages);
                 if (g >= kTcStages && !pp.failed &&
-                    !mbar_wait(&pp.done[b], ((g / kTcStages) - 1u) & 1u, kTcWaitNs, status))
+                    !mbar_wait_sleep(&pp.done[b], ((g / kTcStages) - 1u) & 1u, kTcWaitNs, status))
                     pp.failed = true;
                 if (!pp.failed) tc_store<NM>(buf[j], pp.A + (size_t)b * NM * kTcABytes, pp.B + (size_t)b * kTcBBytes);
-                if (t + kTcDepth < ntile) tc_load<NM>(buf[j], src, t + kTcDepth);
+                if (t + kTcDepth < ntile) tc_load<NM, NRB>(buf[j], src, t + kTcDepth);
                 fence_async_smem();  // the generic-proxy stores above, visible to the tensor core
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&pp.full[b]);
@@ -251,31 +268,33 @@ __device__ __forceinline__ void tc_decode_pass(TcPipe &pp, const TcSrc<NM> &src,
         }
     }
     const unsigned last = pp.it + (unsigned)ntile - 1u;
-    if (!pp.failed && !mbar_wait(&pp.done[last % kTcStages], (last / kTcStages) & 1u, kTcWaitNs, status))
+    if (!pp.failed && !mbar_wait_sleep(&pp.done[last % kTcStages], (last / kTcStages) & 1u, kTcWaitNs, status))
         pp.failed = true;
     tc_fence_after();
     pp.it += (unsigned)ntile;
 }
 
 // MMA side of one pass (lane 0 of warp 4): per tile, wait for the decoders, issue NM x (kTcKT /
-// 32) MMAs (M = 128, N = n, K = 32) into accumulator columns m * kTcBRows .. + n, and commit to
-// the buffer's mbarrier.  The descriptors of buffer 0 are built once; a buffer, matrix or K step
-// is an offset added to the start-address field.
-template <int NM>
-__device__ __forceinline__ void tc_mma_pass(TcPipe &pp, int ntile, uint32_t idesc, int *status) {
+// 32) MMAs (M = 128, N = n, K = 32) into accumulator columns (rb * NM + m) * kTcBRows .. + n of
+// the tile's row block rb, and commit to the buffer's mbarrier.  The descriptors of buffer 0 are
+// built once; a buffer, matrix or K step is an offset added to the start-address field.
+template <int NM, int NRB>
+__device__ __forceinline__ void tc_mma_pass(TcPipe &pp, int ntile, int ntk, uint32_t idesc, int *status) {
     const uint64_t a0 = tc_desc(smem_u32(pp.A)), b0 = tc_desc(smem_u32(pp.B));
     for (int t = 0; t < ntile; t++) {
         const unsigned g = pp.it + (unsigned)t;
         const int b = (int)(g % kTcStages);
-        if (!pp.failed && !mbar_wait(&pp.full[b], (g / kTcStages) & 1u, kTcWaitNs, status)) pp.failed = true;
+        const int rb = tc_rb<NRB>(t, ntk), kt = t - rb * ntk;
+        if (!pp.failed && !mbar_wait_sleep(&pp.full[b], (g / kTcStages) & 1u, kTcWaitNs, status)) pp.failed = true;
         tc_fence_after();
         if (!pp.failed) {
 #pragma unroll
             for (int s = 0; s < kTcKT / 32; s++)
 #pragma unroll
                 for (int m = 0; m < NM; m++)
-                    tc_mma(pp.tmem + (uint32_t)(m * kTcBRows), a0 + (uint64_t)((((b * NM + m) * kTcABytes) + s * 256) >> 4),
-                           b0 + (uint64_t)(((b * kTcBBytes) + s * 256) >> 4), idesc, (t > 0 || s > 0) ? 1u : 0u);
+                    tc_mma(pp.tmem + (uint32_t)((rb * NM + m) * kTcBRows),
+                           a0 + (uint64_t)((((b * NM + m) * kTcABytes) + s * 256) >> 4),
+                           b0 + (uint64_t)(((b * kTcBBytes) + s * 256) >> 4), idesc, (kt > 0 || s > 0) ? 1u : 0u);
         }
         tc_commit(&pp.done[b]);
     }
@@ -363,6 +382,8 @@ __global__ void __launch_bounds__(kTcThreads, 3) gateup_tc_kernel(
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t mb_full[kTcStages], mb_done[kTcStages];
     __shared__ uint32_t s_tmem;
+    __shared__ int s_ent[2][kTcTokens<NL>()];
+    __shared__ float s_sc[2][kTcTokens<NL>()];
     const int u = blockIdx.x;
     if (u >= *n_unique) return;  // before any tensor memory is held
     constexpr uint32_t ALLOC = 2 * kTcBRows;
@@ -375,15 +396,25 @@ __global__ void __launch_bounds__(kTcThreads, 3) gateup_tc_kernel(
     const uint8_t *const mats[2] = {gate + ((int64_t)e * f + row0) * rowb, up + ((int64_t)e * f + row0) * rowb};
     TcPipe pp;
     tc_setup(pp, smem, kTcStages * 2 * kTcABytes, mb_full, mb_done, &s_tmem, ALLOC);
-    for (int q0 = e0; q0 < e1; q0 += NBMAX) {
+    for (int q0 = e0, pass = 0; q0 < e1; q0 += NBMAX, pass++) {
         const int nb = min(NBMAX, e1 - q0), nbp = tc_nbp<NL>(nb);
         if (warp == kTcDec / 32) {  // the MMA warp
-            if ((tid & 31) == 0) tc_mma_pass<2>(pp, ntile, tc_idesc(NL == 1, tc_n<NL>(nb)), status);
+            if ((tid & 31) == 0) tc_mma_pass<2, 1>(pp, ntile, ntile, tc_idesc(NL == 1, tc_n<NL>(nb)), status);
             continue;
         }
+        // the pass's entries and activation scales, for the epilogue (two copies by pass parity:
+        // a copy is written again only after every decoder thread has passed the barrier below
+        // in the pass between)
+        int *const te = s_ent[pass & 1];
+        float *const tsc = s_sc[pass & 1];
+        if (tid < nb) {
+            te[tid] = ent[q0 + tid];
+            tsc[tid] = xsc[te[tid] / k];
+        }
         TcSrc<2> src;
-        tc_src<2, NL>(src, mats, rowb, nrows, xw, d / 4, ent, q0, nb, k);
-        tc_decode_pass<2>(pp, src, ntile, status);
+        tc_src<2, NL, 1>(src, mats, rowb, nrows, ntile, xw, d / 4, ent, q0, nb, k);
+        tc_decode_pass<2, 1>(pp, src, ntile, status);
+        named_bar_sync(1, kTcDec);
         // thread = row of this tile; nb is the same in every thread, so the accumulator loads
         // stay collective
         const int j = row0 + tid;
@@ -400,8 +431,8 @@ __global__ void __launch_bounds__(kTcThreads, 3) gateup_tc_kernel(
             for (int z = 0; z < 4; z++) {
                 const int n = n0 + z;
                 if (!live || n >= nb) continue;
-                const int entry = ent[q0 + n];
-                const float xsv = xsc[entry / k];
+                const int entry = te[n];
+                const float xsv = tsc[n];
                 float hv;
                 if (NL == 1) {
                     acc_g[(int64_t)entry * f + j] = (int32_t)Sg[z];
@@ -423,9 +454,10 @@ __global__ void __launch_bounds__(kTcThreads, 3) gateup_tc_kernel(
     tc_teardown(pp, ALLOC, status);
 }
 
-// grid: (distinct experts bound, d / 128); 128 output rows per CTA
+// grid: (distinct experts bound, d / (128 kTcDownRB)); kTcDownRB blocks of 128 output rows per
+// CTA, streamed as one run of tiles (the K of a down row is short: f / 64 tiles per block)
 template <int NL>
-__global__ void __launch_bounds__(kTcThreads, 3) down_tc_kernel(
+__global__ void __launch_bounds__(kTcThreads, 4) down_tc_kernel(
     const uint8_t *__restrict__ down, const float *__restrict__ sd, int d, int f, const int32_t *__restrict__ n_unique,
     const int32_t *__restrict__ uexp, const int32_t *__restrict__ uoff, const int32_t *__restrict__ ent,
     const uint32_t *__restrict__ hw, const float *__restrict__ hsc, double *__restrict__ ye,
@@ -433,50 +465,64 @@ __global__ void __launch_bounds__(kTcThreads, 3) down_tc_kernel(
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t mb_full[kTcStages], mb_done[kTcStages];
     __shared__ uint32_t s_tmem;
+    __shared__ int s_ent[2][kTcTokens<NL>()];
+    __shared__ float s_sc[2][kTcTokens<NL>()];
     const int u = blockIdx.x;
     if (u >= *n_unique) return;
-    constexpr uint32_t ALLOC = kTcBRows;
+    constexpr int NRB = kTcDownRB;
+    constexpr uint32_t ALLOC = NRB * kTcBRows;
     constexpr int NBMAX = kTcTokens<NL>();
     const int tid = threadIdx.x, warp = tid >> 5;
     const int e = uexp[u], e0 = uoff[u], e1 = uoff[u + 1];
-    const int row0 = blockIdx.y * kTcM, nrows = min(kTcM, d - row0);
+    const int row0 = blockIdx.y * NRB * kTcM, nrows = min(NRB * kTcM, d - row0);
     const int64_t rowb = f / 4;
-    const int ntile = f / kTcKT;
+    const int ntk = f / kTcKT, ntile = NRB * ntk;
     const uint8_t *const mats[1] = {down + ((int64_t)e * d + row0) * rowb};
     TcPipe pp;
     tc_setup(pp, smem, kTcStages * kTcABytes, mb_full, mb_done, &s_tmem, ALLOC);
-    for (int q0 = e0; q0 < e1; q0 += NBMAX) {
+    for (int q0 = e0, pass = 0; q0 < e1; q0 += NBMAX, pass++) {
         const int nb = min(NBMAX, e1 - q0), nbp = tc_nbp<NL>(nb);
         if (warp == kTcDec / 32) {
-            if ((tid & 31) == 0) tc_mma_pass<1>(pp, ntile, tc_idesc(NL == 1, tc_n<NL>(nb)), status);
+            if ((tid & 31) == 0) tc_mma_pass<1, NRB>(pp, ntile, ntk, tc_idesc(NL == 1, tc_n<NL>(nb)), status);
             continue;
         }
+        int *const te = s_ent[pass & 1];
+        float *const tsc = s_sc[pass & 1];
+        if (tid < nb) {
+            te[tid] = ent[q0 + tid];
+            tsc[tid] = hsc[te[tid]];
+        }
         TcSrc<1> src;
-        tc_src<1, NL>(src, mats, rowb, nrows, hw, f / 4, ent, q0, nb, 1);
-        tc_decode_pass<1>(pp, src, ntile, status);
-        const int i = row0 + tid;
+        tc_src<1, NL, NRB>(src, mats, rowb, nrows, ntk, hw, f / 4, ent, q0, nb, 1);
+        tc_decode_pass<1, NRB>(pp, src, ntile, status);
+        named_bar_sync(1, kTcDec);
         const uint32_t ta = pp.tmem + ((uint32_t)(32 * warp) << 16);
-        const bool live = i < d && !pp.failed;
-        const float sdv = live ? sd[(int64_t)e * d + i] : 0.0f;
-        const long long R = tc_rowsum<NL>(ta, 0, nbp);
 #pragma unroll 1
-        for (int n0 = 0; n0 < nb; n0 += 4) {
-            long long S[4];
-            tc_sums4<NL>(ta, 0, nbp, n0, R, S);
+        for (int rb = 0; rb < NRB; rb++) {
+            const int i = row0 + rb * kTcM + tid;
+            const bool live = i < d && !pp.failed;
+            const float sdv = live ? sd[(int64_t)e * d + i] : 0.0f;
+            const int col = rb * kTcBRows;
+            const long long R = tc_rowsum<NL>(ta, col, nbp);
+#pragma unroll 1
+            for (int n0 = 0; n0 < nb; n0 += 4) {
+                long long S[4];
+                tc_sums4<NL>(ta, col, nbp, n0, R, S);
 #pragma unroll
-            for (int z = 0; z < 4; z++) {
-                const int n = n0 + z;
-                if (!live || n >= nb) continue;
-                const int entry = ent[q0 + n];
-                const float hs = hsc[entry];
-                double v;
-                if (NL == 1) {
-                    acc_d[(int64_t)entry * d + i] = (int32_t)S[z];
-                    v = (double)__fmul_rn(__fmul_rn(__int2float_rn((int)S[z]), sdv), hs);
-                } else {
-                    v = ldexp((double)S[z], -__float_as_int(hs)) * (double)sdv;
+                for (int z = 0; z < 4; z++) {
+                    const int n = n0 + z;
+                    if (!live || n >= nb) continue;
+                    const int entry = te[n];
+                    const float hs = tsc[n];
+                    double v;
+                    if (NL == 1) {
+                        acc_d[(int64_t)entry * d + i] = (int32_t)S[z];
+                        v = (double)__fmul_rn(__fmul_rn(__int2float_rn((int)S[z]), sdv), hs);
+                    } else {
+                        v = ldexp((double)S[z], -__float_as_int(hs)) * (double)sdv;
+                    }
+                    ye[(int64_t)entry * d + i] = v;
                 }
-                ye[(int64_t)entry * d + i] = v;
             }
         }
         tc_fence_before();
@@ -500,7 +546,7 @@ cudaError_t launch_grouped_tc(const tern_moe_layer *L, int T, const FfnWs &w, cu
     } else {
         const size_t sm = (size_t)kTcStages * (kTcABytes + kTcBBytes);
         cudaFuncSetAttribute(down_tc_kernel<NL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-        down_tc_kernel<NL><<<dim3(umax, (d + kTcM - 1) / kTcM), kTcThreads, sm, s>>>(
+        down_tc_kernel<NL><<<dim3(umax, (d + kTcDownRB * kTcM - 1) / (kTcDownRB * kTcM)), kTcThreads, sm, s>>>(
             L->down, L->down_scale, d, f, w.n_unique, w.uexp, w.uoff, w.ent, (const uint32_t *)w.hw,
             (const float *)w.hsc, w.ye, w.acc_d, st);
     }
