@@ -35,41 +35,53 @@ static cudaError_t launch_k(void (*kern)(K...), dim3 grid, dim3 block, size_t sm
 
 
 // ------------------------------------------------------------------------- route kernels
-// logits_kernel: one warp per expert row, 16 experts x 8 tokens per CTA.  The tokens' x is
-// converted to fp64 once per CTA, 512 elements at a time, into shared memory.  Each product of
-// two bf16 values is exact in fp64 (at most 16 significant bits), so one fp64 fma per product
-// adds the exact product with one rounding; the sums are exact for the router's magnitudes
-// (checked by the oracle), so the summation order does not change the logits.
-constexpr int kRouteTok = 8;
-constexpr int kLogitWarps = 16;
+// logits_kernel: each warp takes 4 expert rows and each CTA 4 tokens (8 warps: 32 experts x 4
+// tokens).  The tokens' x is converted to fp64 once per CTA, 512 elements at a time, into shared
+// memory; a lane reads two adjacent columns of x per load and applies them to the 4 rows of its
+// warp, so every shared-memory read feeds 8 products per token.  Each product of two bf16 values
+// is exact in fp64 (at most 16 significant bits), so one fp64 fma per product adds the exact
+// product with one rounding; the sums are exact for the router's magnitudes (checked by the
+// oracle), so the summation order does not change the logits.
+constexpr int kRouteTok = 4;
+constexpr int kLogitWarps = 8;
+constexpr int kLogitEPW = 4;  // expert rows per warp
 constexpr int kLogitChunk = 512;
 
 __global__ void __launch_bounds__(kLogitWarps * 32) logits_kernel(const uint16_t *__restrict__ Wg,
                                                                    const uint16_t *__restrict__ x, int T, int d,
                                                                    int E, double *__restrict__ logits) {
-    __shared__ double s_x[kRouteTok][kLogitChunk];
+    __shared__ __align__(16) double s_x[kRouteTok][kLogitChunk];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int e = blockIdx.x * kLogitWarps + warp;
+    const int eb = (blockIdx.x * kLogitWarps + warp) * kLogitEPW;  // first expert row of this warp
     const int t0 = blockIdx.y * kRouteTok;
     const int nt = min(kRouteTok, T - t0);
-    const uint16_t *wr = Wg + (int64_t)(e < E ? e : 0) * d;
-    double acc[kRouteTok];
+    double acc[kLogitEPW][kRouteTok];
 #pragma unroll
-    for (int tt = 0; tt < kRouteTok; tt++) acc[tt] = 0.0;
-    constexpr int WPL = kLogitChunk / 32;                             // weights per lane per chunk
+    for (int q = 0; q < kLogitEPW; q++)
+#pragma unroll
+        for (int tt = 0; tt < kRouteTok; tt++) acc[q][tt] = 0.0;
+    constexpr int PPL = kLogitChunk / 64;                               // column pairs per lane per chunk
     constexpr int XPT = kRouteTok * kLogitChunk / (kLogitWarps * 32);  // x values per thread per chunk
-    uint16_t wv[WPL], xv[XPT];
-    // loads of chunk c0 into registers (all issued before any is used)
+    uint32_t wv[kLogitEPW][PPL];
+    uint16_t xv[XPT];
+    // loads of chunk c0 into registers (all issued before any is used); pair i of a lane is
+    // columns 2 * lane + 64 * i and the next one
     auto fetch = [&](int c0) {
         const int n = min(kLogitChunk, d - c0);
 #pragma unroll
-        for (int i = 0; i < WPL; i++) {
-            const int j = lane + 32 * i;
-            wv[i] = (e < E && j < n) ? __ldg(wr + c0 + j) : (uint16_t)0;
+        for (int q = 0; q < kLogitEPW; q++) {
+            const int e = eb + q;
+#pragma unroll
+            for (int i = 0; i < PPL; i++) {
+                const int j = 2 * lane + 64 * i;
+                wv[q][i] = (e < E && j < n)
+                               ? __ldg(reinterpret_cast<const uint32_t *>(Wg + (int64_t)e * d + c0 + j))
+                               : 0u;
+            }
         }
 #pragma unroll
         for (int i = 0; i < XPT; i++) {
-            const int q = threadIdx.x + i * kLogitWarps * 32, tt = q / kLogitChunk, j = q % kLogitChunk;
+            const int qq = threadIdx.x + i * kLogitWarps * 32, tt = qq / kLogitChunk, j = qq % kLogitChunk;
             xv[i] = (tt < nt && j < n) ? __ldg(x + (int64_t)(t0 + tt) * d + c0 + j) : (uint16_t)0;
         }
     };
@@ -78,28 +90,40 @@ __global__ void __launch_bounds__(kLogitWarps * 32) logits_kernel(const uint16_t
         __syncthreads();  // previous chunk consumed
 #pragma unroll
         for (int i = 0; i < XPT; i++) {
-            const int q = threadIdx.x + i * kLogitWarps * 32;
-            s_x[q / kLogitChunk][q % kLogitChunk] = bf16_to_f64(xv[i]);
+            const int qq = threadIdx.x + i * kLogitWarps * 32;
+            s_x[qq / kLogitChunk][qq % kLogitChunk] = bf16_to_f64(xv[i]);
         }
-        double w[WPL];
+        uint32_t w[kLogitEPW][PPL];
 #pragma unroll
-        for (int i = 0; i < WPL; i++) w[i] = bf16_to_f64(wv[i]);
+        for (int q = 0; q < kLogitEPW; q++)
+#pragma unroll
+            for (int i = 0; i < PPL; i++) w[q][i] = wv[q][i];
         if (c0 + kLogitChunk < d) fetch(c0 + kLogitChunk);  // next chunk's loads fly during this one
         __syncthreads();
-        if (e < E) {
 #pragma unroll
-            for (int i = 0; i < WPL; i++) {
-                const int j = lane + 32 * i;
+        for (int i = 0; i < PPL; i++) {
+            const int j = 2 * lane + 64 * i;
+            double2 xs[kRouteTok];
 #pragma unroll
-                for (int tt = 0; tt < kRouteTok; tt++) acc[tt] = fma(w[i], s_x[tt][j], acc[tt]);
+            for (int tt = 0; tt < kRouteTok; tt++) xs[tt] = *reinterpret_cast<const double2 *>(&s_x[tt][j]);
+#pragma unroll
+            for (int q = 0; q < kLogitEPW; q++) {
+                const double w0 = bf16_to_f64((uint16_t)(w[q][i] & 0xFFFFu)), w1 = bf16_to_f64((uint16_t)(w[q][i] >> 16));
+#pragma unroll
+                for (int tt = 0; tt < kRouteTok; tt++) {
+                    acc[q][tt] = fma(w0, xs[tt].x, acc[q][tt]);
+                    acc[q][tt] = fma(w1, xs[tt].y, acc[q][tt]);
+                }
             }
         }
     }
-    if (e < E) {
+#pragma unroll
+    for (int q = 0; q < kLogitEPW; q++) {
+        const int e = eb + q;
 #pragma unroll
         for (int tt = 0; tt < kRouteTok; tt++) {
-            const double v = warp_sum_f64(acc[tt]);
-            if (lane == 0 && tt < nt) logits[(int64_t)(t0 + tt) * E + e] = v;
+            const double v = warp_sum_f64(acc[q][tt]);
+            if (lane == 0 && tt < nt && e < E) logits[(int64_t)(t0 + tt) * E + e] = v;
         }
     }
 }
@@ -228,7 +252,7 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(
 cudaError_t launch_route(const uint16_t *Wg, const uint16_t *x, int T, int d, int E, int k, double *logits,
                          int32_t *idx, float *g32, double *g64, unsigned int *counter, bool dispatch,
                          int32_t *n_unique, int32_t *uexp, int32_t *uoff, int32_t *ent, cudaStream_t s) {
-    const dim3 g1((E + kLogitWarps - 1) / kLogitWarps, (T + kRouteTok - 1) / kRouteTok);
+    const dim3 g1((E + kLogitWarps * kLogitEPW - 1) / (kLogitWarps * kLogitEPW), (T + kRouteTok - 1) / kRouteTok);
     cudaError_t err = launch_k(logits_kernel, g1, dim3(kLogitWarps * 32), 0, s, Wg, x, T, d, E, logits);
     if (err != cudaSuccess) return err;
     return launch_k(select_kernel, dim3(T), dim3(kSelectThreads), 0, s, (const double *)logits, T, E, k, idx,
