@@ -41,6 +41,7 @@ constexpr int kTcThreads = kTcDec + 32;  // and the MMA warp
 constexpr int kTcStages = 2;     // operand buffers: 40 KB of shared memory per gate/up CTA
 constexpr int kTcDepth = 4;      // K-tiles of global loads in flight per decoder thread
 constexpr int kTcDownRB = 2;     // blocks of 128 rows per down CTA
+constexpr int kTcBWholeMax = 512;  // largest K whose whole B operand (64 rows) a down CTA stages once per pass
 constexpr int kTcABytes = kTcM * kTcKT;
 constexpr int kTcBBytes = kTcBRows * kTcKT;
 // Tokens per pass.  One int8 limb (int8 activations, signed): one B row per token.  Three limbs
@@ -65,8 +66,8 @@ __device__ __forceinline__ uint32_t tc_off(int r, int b) {
 // shared-memory matrix descriptor: start >> 4 in bits 0-13, leading byte offset >> 4 in bits
 // 16-29, stride byte offset >> 4 in bits 32-45, version 1 in bits 46-47, base offset 0, layout
 // type 0 (no swizzle) in bits 61-63
-__device__ __forceinline__ uint64_t tc_desc(uint32_t saddr) {
-    const uint64_t lbo = 128u, sbo = (uint64_t)(kTcKT / 16) * 128u;
+__device__ __forceinline__ uint64_t tc_desc(uint32_t saddr, uint32_t sbo_bytes = (kTcKT / 16) * 128) {
+    const uint64_t lbo = 128u, sbo = sbo_bytes;
     return (uint64_t)((saddr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFull) << 16) | (((sbo >> 4) & 0x3FFFull) << 32) |
            (1ull << 46);
 }
@@ -117,10 +118,11 @@ __device__ __forceinline__ void tc_dealloc(uint32_t taddr, uint32_t ncols) {  //
 // B row i % 64, 16-byte chunk i / 64 of the tile).
 constexpr int kTcBPer = kTcBChunks / kTcDec;
 
-template <int NM>
+// BW: the B operand of the whole K is staged once per pass instead (tiles carry no B chunks)
+template <int NM, bool BW>
 struct TcTile {
     uint4 a[NM];
-    uint4 b[kTcBPer];
+    uint4 b[BW ? 1 : kTcBPer];
 };
 
 // Where a decoder thread's data of tile 0 sits.  A CTA takes NRB blocks of 128 rows one after
@@ -187,12 +189,13 @@ __device__ __forceinline__ void tc_src(TcSrc<NM> &p, const uint8_t *const (&mats
     }
 }
 
-template <int NM, int NRB>
-__device__ __forceinline__ void tc_load(TcTile<NM> &p, const TcSrc<NM> &q, int t) {
+template <int NM, int NRB, bool BW>
+__device__ __forceinline__ void tc_load(TcTile<NM, BW> &p, const TcSrc<NM> &q, int t) {
     const int rb = tc_rb<NRB>(t, q.ntk), kt = t - rb * q.ntk;
 #pragma unroll
     for (int m = 0; m < NM; m++)
         p.a[m] = rb < q.nrb ? __ldg(q.a[m] + rb * q.rbstep + kt) : make_uint4(0u, 0u, 0u, 0u);
+    if (BW) return;
 #pragma unroll
     for (int j = 0; j < kTcBPer; j++) {
         const uint4 v = q.b[j] ? __ldg(q.b[j] + (kTcKT / 16) * kt) : make_uint4(0u, 0u, 0u, 0u);
@@ -204,8 +207,8 @@ __device__ __forceinline__ void tc_load(TcTile<NM> &p, const TcSrc<NM> &q, int t
 // 16-byte chunk q of the row in the table-free decode's position-major order: byte 4j + b
 // holds 64 times the weight of code 16q + 4b + j (decode.cuh).  The B chunks take the same
 // order by a 4x4 byte transpose, so A and B agree on every K index of the tile.
-template <int NM>
-__device__ __forceinline__ void tc_store(const TcTile<NM> &p, unsigned char *A, unsigned char *B) {
+template <int NM, bool BW>
+__device__ __forceinline__ void tc_store(const TcTile<NM, BW> &p, unsigned char *A, unsigned char *B) {
     const int r = threadIdx.x;
 #pragma unroll
     for (int m = 0; m < NM; m++) {
@@ -218,12 +221,38 @@ __device__ __forceinline__ void tc_store(const TcTile<NM> &p, unsigned char *A, 
                            tern_position_lanes(sf, 3));
         }
     }
+    if (BW) return;
 #pragma unroll
     for (int j = 0; j < kTcBPer; j++) {
         const int i = threadIdx.x + j * kTcDec;
         uint4 v;
         bytes_transpose4(p.b[j].x, p.b[j].y, p.b[j].z, p.b[j].w, v.x, v.y, v.z, v.w);
         *reinterpret_cast<uint4 *>(B + tc_off(i % kTcBRows, 16 * (i / kTcBRows))) = v;
+    }
+}
+
+// The B operand of the whole K (kb bytes per row) for one pass, in the K-major layout with a
+// stride of kb / 16 core matrices between 8-row groups.  B row r is staged by threads r and r + 64
+// (chunk i = threadIdx.x + j * kTcDec keeps row threadIdx.x % 64 for every j): chunk c = c0 + 2j
+// of the row, c0 = threadIdx.x / 64, from the pointer tc_src set for j = 0.
+template <int NM>
+__device__ __forceinline__ void tc_stage_b_whole(const TcSrc<NM> &q, unsigned char *B, int kb) {
+    const int row = threadIdx.x % kTcBRows, c0 = threadIdx.x / kTcBRows;
+    const int nch = kb / 32;  // chunks of this thread
+    const uint32_t x = q.bx[0];
+    for (int j0 = 0; j0 < nch; j0 += 8) {
+        uint4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; u++)
+            v[u] = (q.b[0] && j0 + u < nch) ? __ldg(q.b[0] + 2 * (j0 + u)) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int u = 0; u < 8; u++) {
+            if (j0 + u >= nch) continue;
+            const int c = c0 + 2 * (j0 + u);
+            uint4 w;
+            bytes_transpose4(v[u].x ^ x, v[u].y ^ x, v[u].z ^ x, v[u].w ^ x, w.x, w.y, w.z, w.w);
+            *reinterpret_cast<uint4 *>(B + ((((row >> 3) * (kb / 16) + c) << 7) + ((row & 7) << 4))) = w;
+        }
     }
 }
 
@@ -242,13 +271,15 @@ struct TcPipe {
 // Decoder side of one pass (warps 0..3): tiles 0 .. ntile-1 of the pass, kTcDepth tiles of global
 // loads in flight, each tile decoded into the next buffer once the tensor core has finished with
 // that buffer's previous tile.  Returns once every MMA of the pass has completed.
-template <int NM, int NRB>
-__device__ __forceinline__ void tc_decode_pass(TcPipe &pp, const TcSrc<NM> &src, int ntile, int *status) {
+template <int NM, int NRB, bool BW>
+__device__ __forceinline__ void tc_decode_pass(TcPipe &pp, const TcSrc<NM> &src, int ntile, int kb, int *status) {
     const int lane = threadIdx.x & 31;
-    TcTile<NM> buf[kTcDepth];
+    TcTile<NM, BW> buf[kTcDepth];
 #pragma unroll
     for (int j = 0; j < kTcDepth; j++)
-        if (j < ntile) tc_load<NM, NRB>(buf[j], src, j);
+        if (j < ntile) tc_load<NM, NRB, BW>(buf[j], src, j);
+    // the whole B while the first tiles' loads are in flight; the previous pass's MMAs are done
+    if (BW) tc_stage_b_whole<NM>(src, pp.B, kb);
     for (int t0 = 0; t0 < ntile; t0 += kTcDepth) {
 #pragma unroll
         for (int j = 0; j < kTcDepth; j++) {
@@ -259,8 +290,9 @@ __device__ __forceinline__ void tc_decode_pass(TcPipe &pp, const TcSrc<NM> &src,
                 if (g >= kTcStages && !pp.failed &&
                     !mbar_wait_sleep(&pp.done[b], ((g / kTcStages) - 1u) & 1u, kTcWaitNs, status))
                     pp.failed = true;
-                if (!pp.failed) tc_store<NM>(buf[j], pp.A + (size_t)b * NM * kTcABytes, pp.B + (size_t)b * kTcBBytes);
-                if (t + kTcDepth < ntile) tc_load<NM, NRB>(buf[j], src, t + kTcDepth);
+                if (!pp.failed)
+                    tc_store<NM, BW>(buf[j], pp.A + (size_t)b * NM * kTcABytes, pp.B + (size_t)b * kTcBBytes);
+                if (t + kTcDepth < ntile) tc_load<NM, NRB, BW>(buf[j], src, t + kTcDepth);
                 fence_async_smem();  // the generic-proxy stores above, visible to the tensor core
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&pp.full[b]);
@@ -278,9 +310,9 @@ __device__ __forceinline__ void tc_decode_pass(TcPipe &pp, const TcSrc<NM> &src,
 // 32) MMAs (M = 128, N = n, K = 32) into accumulator columns (rb * NM + m) * kTcBRows .. + n of
 // the tile's row block rb, and commit to the buffer's mbarrier.  The descriptors of buffer 0 are
 // built once; a buffer, matrix or K step is an offset added to the start-address field.
-template <int NM, int NRB>
-__device__ __forceinline__ void tc_mma_pass(TcPipe &pp, int ntile, int ntk, uint32_t idesc, int *status) {
-    const uint64_t a0 = tc_desc(smem_u32(pp.A)), b0 = tc_desc(smem_u32(pp.B));
+template <int NM, int NRB, bool BW>
+__device__ __forceinline__ void tc_mma_pass(TcPipe &pp, int ntile, int ntk, int kb, uint32_t idesc, int *status) {
+    const uint64_t a0 = tc_desc(smem_u32(pp.A)), b0 = tc_desc(smem_u32(pp.B), BW ? (uint32_t)(kb / 16) * 128u : (kTcKT / 16) * 128u);
     for (int t = 0; t < ntile; t++) {
         const unsigned g = pp.it + (unsigned)t;
         const int b = (int)(g % kTcStages);
@@ -294,7 +326,8 @@ __device__ __forceinline__ void tc_mma_pass(TcPipe &pp, int ntile, int ntk, uint
                 for (int m = 0; m < NM; m++)
                     tc_mma(pp.tmem + (uint32_t)((rb * NM + m) * kTcBRows),
                            a0 + (uint64_t)((((b * NM + m) * kTcABytes) + s * 256) >> 4),
-                           b0 + (uint64_t)(((b * kTcBBytes) + s * 256) >> 4), idesc, (kt > 0 || s > 0) ? 1u : 0u);
+                           b0 + (uint64_t)((BW ? (kt * (kTcKT / 16) + 2 * s) * 128 : (b * kTcBBytes) + s * 256) >> 4),
+                           idesc, (kt > 0 || s > 0) ? 1u : 0u);
         }
         tc_commit(&pp.done[b]);
     }
@@ -399,7 +432,7 @@ __global__ void __launch_bounds__(kTcThreads, 3) gateup_tc_kernel(
     for (int q0 = e0, pass = 0; q0 < e1; q0 += NBMAX, pass++) {
         const int nb = min(NBMAX, e1 - q0), nbp = tc_nbp<NL>(nb);
         if (warp == kTcDec / 32) {  // the MMA warp
-            if ((tid & 31) == 0) tc_mma_pass<2, 1>(pp, ntile, ntile, tc_idesc(NL == 1, tc_n<NL>(nb)), status);
+            if ((tid & 31) == 0) tc_mma_pass<2, 1, false>(pp, ntile, ntile, d, tc_idesc(NL == 1, tc_n<NL>(nb)), status);
             continue;
         }
         // the pass's entries and activation scales, for the epilogue (two copies by pass parity:
@@ -413,7 +446,7 @@ __global__ void __launch_bounds__(kTcThreads, 3) gateup_tc_kernel(
         }
         TcSrc<2> src;
         tc_src<2, NL, 1>(src, mats, rowb, nrows, ntile, xw, d / 4, ent, q0, nb, k);
-        tc_decode_pass<2, 1>(pp, src, ntile, status);
+        tc_decode_pass<2, 1, false>(pp, src, ntile, d, status);
         named_bar_sync(1, kTcDec);
         // thread = row of this tile; nb is the same in every thread, so the accumulator loads
         // stay collective
@@ -455,8 +488,10 @@ __global__ void __launch_bounds__(kTcThreads, 3) gateup_tc_kernel(
 }
 
 // grid: (distinct experts bound, d / (128 kTcDownRB)); kTcDownRB blocks of 128 output rows per
-// CTA, streamed as one run of tiles (the K of a down row is short: f / 64 tiles per block)
-template <int NL>
+// CTA, streamed as one run of tiles (the K of a down row is short: f / 64 tiles per block).  BW:
+// the B rows of the whole K (f bytes each) staged once per pass, for f <= kTcBWholeMax; the row
+// blocks then share them instead of restaging them per tile
+template <int NL, bool BW>
 __global__ void __launch_bounds__(kTcThreads, 4) down_tc_kernel(
     const uint8_t *__restrict__ down, const float *__restrict__ sd, int d, int f, const int32_t *__restrict__ n_unique,
     const int32_t *__restrict__ uexp, const int32_t *__restrict__ uoff, const int32_t *__restrict__ ent,
@@ -483,7 +518,7 @@ __global__ void __launch_bounds__(kTcThreads, 4) down_tc_kernel(
     for (int q0 = e0, pass = 0; q0 < e1; q0 += NBMAX, pass++) {
         const int nb = min(NBMAX, e1 - q0), nbp = tc_nbp<NL>(nb);
         if (warp == kTcDec / 32) {
-            if ((tid & 31) == 0) tc_mma_pass<1, NRB>(pp, ntile, ntk, tc_idesc(NL == 1, tc_n<NL>(nb)), status);
+            if ((tid & 31) == 0) tc_mma_pass<1, NRB, BW>(pp, ntile, ntk, f, tc_idesc(NL == 1, tc_n<NL>(nb)), status);
             continue;
         }
         int *const te = s_ent[pass & 1];
@@ -494,7 +529,7 @@ __global__ void __launch_bounds__(kTcThreads, 4) down_tc_kernel(
         }
         TcSrc<1> src;
         tc_src<1, NL, NRB>(src, mats, rowb, nrows, ntk, hw, f / 4, ent, q0, nb, 1);
-        tc_decode_pass<1, NRB>(pp, src, ntile, status);
+        tc_decode_pass<1, NRB, BW>(pp, src, ntile, f, status);
         named_bar_sync(1, kTcDec);
         const uint32_t ta = pp.tmem + ((uint32_t)(32 * warp) << 16);
 #pragma unroll 1
@@ -544,9 +579,18 @@ cudaError_t launch_grouped_tc(const tern_moe_layer *L, int T, const FfnWs &w, cu
             L->gate, L->up, L->gate_scale, L->up_scale, d, f, k, w.n_unique, w.uexp, w.uoff, w.ent,
             (const uint32_t *)w.xw, (const float *)w.xsc, w.h, w.acc_g, w.acc_u, st);
     } else {
+        const dim3 grid(umax, (d + kTcDownRB * kTcM - 1) / (kTcDownRB * kTcM));
+        if (f <= kTcBWholeMax) {
+            const size_t sm = (size_t)kTcStages * kTcABytes + (size_t)kTcBRows * f;
+            cudaFuncSetAttribute(down_tc_kernel<NL, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+            down_tc_kernel<NL, true><<<grid, kTcThreads, sm, s>>>(
+                L->down, L->down_scale, d, f, w.n_unique, w.uexp, w.uoff, w.ent, (const uint32_t *)w.hw,
+                (const float *)w.hsc, w.ye, w.acc_d, st);
+            return cudaGetLastError();
+        }
         const size_t sm = (size_t)kTcStages * (kTcABytes + kTcBBytes);
-        cudaFuncSetAttribute(down_tc_kernel<NL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-        down_tc_kernel<NL><<<dim3(umax, (d + kTcDownRB * kTcM - 1) / (kTcDownRB * kTcM)), kTcThreads, sm, s>>>(
+        cudaFuncSetAttribute(down_tc_kernel<NL, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        down_tc_kernel<NL, false><<<grid, kTcThreads, sm, s>>>(
             L->down, L->down_scale, d, f, w.n_unique, w.uexp, w.uoff, w.ent, (const uint32_t *)w.hw,
             (const float *)w.hsc, w.ye, w.acc_d, st);
     }
