@@ -737,7 +737,7 @@ def main():
         "config": dict(_config(args.act, world, "flushed before every timed step (256 MB write, not timed)"),
                        layers=N_LAYERS),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": traffic, "kernel": f"stack_kernel<{1 if args.act == 'int8' else 3}>",
+                     "traffic": traffic, "kernel": f"stack_kernel<{1 if args.act == 'int8' else 3}, 0>",
                      "bytes_per_launch": BYTES_PER_TOKEN // launches, "peak_kind": peak_kind},
         "e2e": {"value": tokens_all / (e2e_ms_max / 1e3), "unit": UNIT, "h2d_bytes_per_step": 2 * shape.d,
                 "d2h_bytes_per_step": 2 * shape.d},

@@ -161,7 +161,9 @@ __host__ __device__ inline SmemMap smem_map(int d, int f, int k, int gu_max, int
 }
 
 // ------------------------------------------------------------------ the kernel
-template <int NL>
+// PRED: the next-layer prediction side task is compiled in (an option, off by default); the
+// default instantiation carries none of its code, which keeps the per-layer code smaller
+template <int NL, bool PRED>
 __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_constant__ StackParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t mb_r[2], mb_gu0, mb_gu1, mb_dn;
@@ -547,7 +549,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
                 p.gate_hist[l * k + lane] = s_gate[lane];
             }
         }
-        const bool predict = p.predict && has_next && nr > 0;
+        const bool predict = PRED && p.predict && has_next && nr > 0;
         if (predict && warp >= kStackWarps / 2) {
             const uint32_t npar = (uint32_t)((l + 1) & 1);
             const bool okr =
@@ -686,7 +688,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) stack_kernel(const __grid_co
             }
         }
         TSTAMP(l, 13)
-        if (warp >= kStackWarps / 2 && p.predict && has_next) {
+        if (PRED && warp >= kStackWarps / 2 && p.predict && has_next) {
             // The experts predicted for the next layer -> L2 prefetch, by warps 8..15 while warps
             // 0..3 combine.  No exact ranking (a hint needs none): warp 15 takes tau = the
             // kPredTop-th largest of the 32 lane maxima of the predicted logits (lane l holds
@@ -919,7 +921,7 @@ static int sm_count() {
 struct StackPlan {
     int P, G;
     SmemMap sm;
-    const void *fn;
+    const void *fn, *fn_pred;  // without / with the next-layer prediction code
 };
 
 static tern_status stack_plan(const tern_moe_layer &L0, int n_layers, tern_act act, StackPlan &pl) {
@@ -944,13 +946,16 @@ static tern_status stack_plan(const tern_moe_layer &L0, int n_layers, tern_act a
     pl.G = G;
     const int NL = act == TERN_ACT_INT8 ? 1 : 3;
     pl.sm = smem_map(d, f, k, (f + G - 1) / G, 2 * ((d / 2 + G - 1) / G), (E + P - 1) / P, NL);
-    pl.fn = act == TERN_ACT_INT8 ? (const void *)stack_kernel<1> : (const void *)stack_kernel<3>;
-    if (cudaFuncSetAttribute(pl.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.sm.total) != cudaSuccess)
-        return TERN_ECUDA;
-    int nb = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, pl.fn, kStackThreads, pl.sm.total) != cudaSuccess)
-        return TERN_ECUDA;
-    if (nb < 1 || nb * sms < P) return TERN_EUNSUPPORTED;
+    pl.fn = act == TERN_ACT_INT8 ? (const void *)stack_kernel<1, false> : (const void *)stack_kernel<3, false>;
+    pl.fn_pred = act == TERN_ACT_INT8 ? (const void *)stack_kernel<1, true> : (const void *)stack_kernel<3, true>;
+    for (const void *fn : {pl.fn, pl.fn_pred}) {
+        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.sm.total) != cudaSuccess)
+            return TERN_ECUDA;
+        int nb = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, kStackThreads, pl.sm.total) != cudaSuccess)
+            return TERN_ECUDA;
+        if (nb < 1 || nb * sms < P) return TERN_EUNSUPPORTED;
+    }
     return TERN_OK;
 }
 
@@ -1024,7 +1029,8 @@ tern_status launch_stack_persistent(const tern_moe_layer *layers, int n_layers, 
     prm.stall_layer = stall_layer;
 
     void *args[] = {&prm};
-    const cudaError_t e = cudaLaunchCooperativeKernel(pl.fn, dim3(pl.P), dim3(kStackThreads), args, pl.sm.total, s);
+    const cudaError_t e = cudaLaunchCooperativeKernel(prm.predict ? pl.fn_pred : pl.fn, dim3(pl.P), dim3(kStackThreads),
+                                                      args, pl.sm.total, s);
     return e == cudaSuccess ? TERN_OK : TERN_ECUDA;
 }
 

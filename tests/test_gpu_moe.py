@@ -223,6 +223,27 @@ def test_stack_teacher_forced_per_layer(stack3, act):
     assert torch.equal(full.view(torch.int16), cur.view(torch.int16))
 
 
+def test_stack_next_layer_prediction_changes_no_value(stack3, monkeypatch):
+    """With TERNMOE_PREDICT=1 the batch-1 kernel built with the next-layer prediction side task
+    runs (L2 prefetches of predicted experts' rows): a hint only, so every token's output is
+    the same bits as without it."""
+    shape, layers, hosts = stack3
+    dev = layers[0].gate.device
+    st = tm.Stack(layers)
+    x = synth.tokens_bf16(WID_STACK, 9, 3, shape.d)
+    for act in (tm.TERN_ACT_BF16, tm.TERN_ACT_INT8):
+        for t in range(3):
+            monkeypatch.delenv("TERNMOE_PREDICT", raising=False)
+            plain = dev_u16(x[t:t + 1], dev)
+            tm.moe_stack_decode(st, plain, act=act)
+            monkeypatch.setenv("TERNMOE_PREDICT", "1")
+            pred = dev_u16(x[t:t + 1], dev)
+            tm.moe_stack_decode(st, pred, act=act)
+            monkeypatch.delenv("TERNMOE_PREDICT", raising=False)
+            assert tm.tern_stream_status() == 0
+            assert torch.equal(plain.view(torch.int16), pred.view(torch.int16)), (act, t)
+
+
 def test_one_launch_paths_match_stage_path_bit_exact(stack3):
     """Three ways through the same stack do the same arithmetic in the same order, so every
     token gives identical bits on all of them, whatever else is in its batch:
