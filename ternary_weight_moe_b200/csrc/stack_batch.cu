@@ -343,11 +343,9 @@ __global__ void __launch_bounds__(kBThreads, 1) stack_batch_kernel(const __grid_
             __syncthreads();
             BSTAMP(l, 12)
             // how many (token, slot) pairs chose each expert
-            if (tid < E) {
-                int c = 0;
-                for (int q = 0; q < npair; q++) c += s_idx[q] == tid ? 1 : 0;
-                s_cnt[tid] = c;
-            }
+            if (tid < E) s_cnt[tid] = 0;
+            __syncthreads();
+            if (tid < npair) atomicAdd(&s_cnt[s_idx[tid]], 1);
             __syncthreads();
             // the distinct experts in ascending order and where their pair lists start: lane l
             // of warp 0 takes experts 8l .. 8l + 7 (E <= 256), then an exclusive scan
@@ -388,12 +386,26 @@ __global__ void __launch_bounds__(kBThreads, 1) stack_batch_kernel(const __grid_
                 }
             }
             __syncthreads();
-            // each expert's pairs in pair order (token-major)
-            if (tid < npair) {
-                const int e = s_idx[tid];
-                int pos = 0;
-                for (int q = 0; q < tid; q++) pos += s_idx[q] == e ? 1 : 0;
-                s_plist[s_ustart[s_rank[e]] + pos] = tid;
+            // each expert's pairs in pair order (token-major): warp 0 walks the pairs 32 at a time;
+            // equal experts within a chunk are ranked by lane, and s_cnt (no longer needed as a
+            // count) carries each expert's running fill across chunks
+            if (warp == 0) {
+                for (int e = lane; e < E; e += 32) s_cnt[e] = 0;
+                __syncwarp();
+                for (int q0 = 0; q0 < npair; q0 += 32) {
+                    const int q = q0 + lane;
+                    const bool v = q < npair;
+                    const int e = v ? s_idx[q] : -1 - lane;  // distinct values for lanes past the end
+                    const unsigned m = __match_any_sync(0xFFFFFFFFu, e);
+                    const int before = __popc(m & ((1u << lane) - 1u));
+                    const int base = v ? s_cnt[e] : 0;
+                    __syncwarp();
+                    if (v) {
+                        s_plist[s_ustart[s_rank[e]] + base + before] = q;
+                        if (lane == __ffs(m) - 1) s_cnt[e] = base + __popc(m);
+                    }
+                    __syncwarp();
+                }
             }
             // this CTA's work items in phases C and D: contiguous ranges of equal weight, an
             // item weighing 1 + the pairs of its expert (its rows' load and decode, then one dot
