@@ -205,6 +205,10 @@ tern_status moe_route_topk_static(const uint16_t *Wg, const uint16_t *x, int64_t
  *   act = TERN_ACT_INT8: x is absmax-quantised per token and h per (token, slot); the dots
  *     are exact int32; g = ((float)acc_g * s_g) * s_x, u likewise, h = fp32 of the fp64
  *     SwiGLU, y_e = ((float)acc_d * s_d) * s_h.
+ * From 32 tokens on (d and f multiples of 64), the grouped gate/up and down stages run on the
+ * fifth-generation tensor cores (int8 MMAs on decoded weight tiles, accumulators in tensor
+ * memory); their integer sums are the same as those of the other kernels, so a token's output
+ * does not depend on the batch it is in.
  * x [T][d] bf16, y [T][d] bf16, y_f32 [T][d] or NULL.  1 <= T <= T_max <= 64. */
 size_t moe_ffn_workspace_bytes(const tern_moe_layer *L, int64_t T_max, tern_act act);
 tern_status moe_ffn_workspace_layout(const tern_moe_layer *L, int64_t T_max, tern_act act,
