@@ -4,7 +4,9 @@
 // At 32 or more tokens the selected experts each serve a few tokens ("iPhone Runs a 20B Model at
 // 120 tok/s", "What Makes 120 tok/s So Fast?": batched work turns the matrix-vector products of
 // decode into small matrix products), so every expert's rows are decoded once and multiplied
-// against all of its tokens at once.  One CTA per (distinct expert, 128 rows), 160 threads:
+// against all of its tokens at once.  One CTA per (distinct expert, 128 rows) for gate/up, and per
+// (distinct expert, 2 x 128 rows) for down, whose short K (f) lets it stage the B rows of the
+// whole K once per pass for both row blocks.  160 threads:
 //   * four decoder warps, thread = row: per K-tile of 64 codes each thread decodes its row's 16
 //     packed bytes by integer logic into int8 lanes of 64 * w (the table-free decode of
 //     decode.cuh, position-major order) and writes them into shared memory in the tensor core's
