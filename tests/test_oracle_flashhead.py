@@ -1,11 +1,21 @@
 """Pins of the FlashHead oracle against arithmetic that does not go through it."""
 from fractions import Fraction
+import importlib.util
 import itertools
+import os
 
 import numpy as np
 
 import synth
-from oracle import flashhead as fh
+
+# The mutant test runs these pins against planted-mistake copies of the module.
+_SRC = os.environ.get("TERNMOE_FLASHHEAD_SRC")
+if _SRC:
+    _spec = importlib.util.spec_from_file_location("flashhead_under_test", _SRC)
+    fh = importlib.util.module_from_spec(_spec)
+    _spec.loader.exec_module(fh)
+else:
+    from oracle import flashhead as fh
 
 
 def _bits(vals):
@@ -79,3 +89,10 @@ def test_all_clusters_selected_is_the_exact_full_head():
     assert r["best"] == int(np.lexsort((np.arange(V), -full))[0])
     # the candidates are exactly the selected clusters' rows, in selection order
     assert (r["ids"].reshape(-1, cs)[:, 0] // cs == r["sel"]).all()
+
+
+def test_best_breaks_ties_to_the_lower_token_id():
+    ids = np.array([5, 3, 9, 1], np.int32)
+    assert fh.best(ids, np.array([1.0, 1.0, 0.5, -2.0])) == 3
+    assert fh.best(ids, np.array([0.0, -1.0, 2.0, 2.0])) == 1
+    assert fh.best(ids[:1], np.array([-7.0])) == 5

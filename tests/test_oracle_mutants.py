@@ -30,6 +30,18 @@ MUTANTS = {
 }
 
 
+def test_pins_pass_on_the_oracle_built_the_same_way(tmp_path):
+    """Control: the unmutated source, built and loaded exactly as the mutants are, passes."""
+    so = tmp_path / "orig.so"
+    subprocess.check_call(["gcc", "-O2", "-std=gnu11", "-fPIC", "-shared", "-ffp-contract=off",
+                           "-o", str(so), SRC, "-lm"])
+    env = dict(os.environ, TERNMOE_ORACLE_LIB=str(so))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-2000:]
+
+
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_pins_catch_mutant(name, tmp_path):
     old, new = MUTANTS[name]
@@ -43,5 +55,43 @@ def test_pins_catch_mutant(name, tmp_path):
     env = dict(os.environ, TERNMOE_ORACLE_LIB=str(so))
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
                         os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, "pins did not catch mutant " + name + "\n" + r.stdout[-2000:]
+
+
+# The same for the approximate-head oracle (plain numpy): each planted mistake must fail one of
+# its pins in tests/test_oracle_flashhead.py.
+FH_SRC = os.path.join(ROOT, "oracle", "flashhead.py")
+FH_MUTANTS = {
+    "mean_off_by_one": (".sum(axis=1) / cluster_size", ".sum(axis=1) / (cluster_size - 1)"),
+    "int4_scale_over_8": ("scale = absmax / 7.0", "scale = absmax / 8.0"),
+    "int4_ties_away_from_zero": ("np.rint(C[nz] / scale[nz, None])", "np.trunc(C[nz] / scale[nz, None] + np.copysign(0.5, C[nz]))"),
+    "nibbles_swapped": ("return (lo | (hi << 4)).astype(np.uint8)", "return (hi | (lo << 4)).astype(np.uint8)"),
+    "score_scale_dropped": ("return (q @ x) * np.asarray(scale, dtype=np.float64)", "return q @ x"),
+    "clusters_ties_to_higher": ("order = np.lexsort((np.arange(sc.size), -sc))", "order = np.lexsort((-np.arange(sc.size), -sc))"),
+    "cluster_rows_misplaced": ("[:, None] * cluster_size + np.arange(cluster_size)", "[:, None] * (cluster_size - 1) + np.arange(cluster_size)"),
+    "best_ties_to_higher": ("order = np.lexsort((ids, -logits))", "order = np.lexsort((-ids, -logits))"),
+}
+
+
+def test_flashhead_pins_pass_on_the_oracle_loaded_the_same_way():
+    """Control: the unmutated module, loaded exactly as the mutants are, passes."""
+    env = dict(os.environ, TERNMOE_FLASHHEAD_SRC=FH_SRC)
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_flashhead.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-2000:]
+
+
+@pytest.mark.parametrize("name", sorted(FH_MUTANTS))
+def test_flashhead_pins_catch_mutant(name, tmp_path):
+    old, new = FH_MUTANTS[name]
+    src = open(FH_SRC).read()
+    assert src.count(old) == 1, "mutation site vanished: " + name
+    mut = tmp_path / "flashhead_mut.py"
+    mut.write_text(src.replace(old, new))
+    env = dict(os.environ, TERNMOE_FLASHHEAD_SRC=str(mut))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_flashhead.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, "pins did not catch mutant " + name + "\n" + r.stdout[-2000:]
