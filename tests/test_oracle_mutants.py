@@ -19,6 +19,9 @@ MUTANTS = {
     "down_scale_dropped": ("tern_dot_f64(drow, hd, f, &bad, &unchecked) * (double)sd",
                            "tern_dot_f64(drow, hd, f, &bad, &unchecked)"),
     "rms_sum_not_mean": ("sqrt(ss / (double)d + eps)", "sqrt(ss + eps)"),
+    "rms_eps_outside_root": ("sqrt(ss / (double)d + eps)", "sqrt(ss / (double)d) + eps"),
+    "residual_unrounded_ffn": ("bad += or_moe_ffn(L, n, T, act, y, y64, tr, NULL, NULL, NULL);\n    for (int64_t i = 0; i < T * d; i++) x_out[i] = f64_to_bf16(bf16_to_f64(x[i]) + bf16_to_f64(y[i]));",
+                               "double *yy = (double *)malloc(sizeof(double) * (size_t)(T * d));\n    bad += or_moe_ffn(L, n, T, act, y, yy, tr, NULL, NULL, NULL);\n    for (int64_t i = 0; i < T * d; i++) x_out[i] = f64_to_bf16(bf16_to_f64(x[i]) + yy[i]);\n    if (y64) memcpy(y64, yy, sizeof(double) * (size_t)(T * d));\n    free(yy);"),
     "quant_truncates": ("float r = rintf(p);", "float r = truncf(p);"),
     "residual_dropped": ("f64_to_bf16(bf16_to_f64(x[i]) + bf16_to_f64(y[i]))", "y[i]"),
     "gate_up_swapped": ("h[j] = (float)silu_times(g, u);", "h[j] = (float)silu_times(u, g);"),

@@ -193,6 +193,11 @@ def test_rmsnorm_closed_forms():
     # zero vector with eps > 0 -> zeros
     n, _ = oracle.rmsnorm(_bf16(np.zeros(d)), eps=1e-6)
     assert (n[0] == 0).all()
+    # eps inside the root: constant c with mean c^2 + eps a perfect square
+    n, _ = oracle.rmsnorm(_bf16(np.full(d, 1.0)), eps=3.0)       # 1 / sqrt(1 + 3) = 0.5
+    assert (n[0] == 0x3F00).all()
+    n, _ = oracle.rmsnorm(_bf16(np.full(d, -2.0)), eps=12.0)     # -2 / sqrt(4 + 12) = -0.5
+    assert (n[0] == 0xBF00).all()
     # scale invariance under x -> 2x (eps = 0) is exact
     x = synth.normal_bf16(31, 0, 2048, 1.0)
     n1, _ = oracle.rmsnorm(x, eps=0.0)
