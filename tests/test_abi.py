@@ -45,6 +45,28 @@ def test_workspace_queries_are_host_only():
     assert tm.lib().moe_route_workspace_bytes(1, 256) > 256 * 8
 
 
+@pytest.mark.parametrize("T", [1, 2, 4, 16])
+@pytest.mark.parametrize("act", [tm.TERN_ACT_BF16, tm.TERN_ACT_INT8])
+def test_stack_record_layout_holds_the_documented_shapes(T, act):
+    """The per-layer record of a one-launch stack call: regions in header order, 16-byte
+    aligned, each large enough for the shapes the header documents at the largest stack (64
+    layers), and the layout's total equal to the workspace size query."""
+    L = _fake_layer()
+    d, f, k, nl = 2048, 512, 8, 64
+    out = tm.StackLayoutC()
+    assert tm.lib().moe_stack_workspace_layout(ctypes.byref(L), T, act, ctypes.byref(out)) == 0
+    assert out.total == tm.lib().moe_stack_workspace_bytes(ctypes.byref(L), T, act)
+    offs = [out.hist, out.idx, out.gates64, out.y32, out.h32, out.trace, out.total]
+    assert all(o % 16 == 0 for o in offs) and offs == sorted(offs)
+    assert out.idx - out.hist >= (nl + 1) * T * d * 2
+    assert out.gates64 - out.idx >= nl * T * k * 4
+    assert out.y32 - out.gates64 >= nl * T * k * 8
+    assert out.h32 - out.y32 >= nl * T * d * 4
+    assert out.trace - out.h32 >= nl * T * k * f * 4
+    if T == 1:
+        assert out.total - out.trace >= 2 * nl * 256 * 24 * 8
+
+
 @pytest.mark.parametrize("bad", [dict(d=100), dict(f=0), dict(E=0), dict(k=9), dict(k=300, E=256), dict(E=2000),
                                  dict(d=4096)])
 def test_layer_validation(bad):
