@@ -104,6 +104,35 @@ __global__ void barriers(unsigned long long *out) {
     }
 }
 
+// A 16-byte shared store followed by fence.proxy.async.shared::cta (what a thread does before
+// the tensor core may read what it stored), against the store alone: cycles per iteration.
+__global__ void proxy_fence(unsigned long long *out) {
+    __shared__ uint4 buf[128];
+    uint4 v = make_uint4(threadIdx.x, 1u, 2u, 3u);
+    __syncthreads();
+    unsigned long long t0 = clock64();
+#pragma unroll 1
+    for (int i = 0; i < 256; i++) {
+        buf[threadIdx.x] = v;
+        v.x += 1u;
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    unsigned long long t1 = clock64();
+#pragma unroll 1
+    for (int i = 0; i < 256; i++) {
+        buf[threadIdx.x] = v;
+        v.x += 1u;
+        asm volatile("" ::: "memory");
+    }
+    unsigned long long t2 = clock64();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        out[0] = t1 - t0;
+        out[1] = t2 - t1;
+        out[2] = buf[7].x;  // keeps the stores
+    }
+}
+
 // CTA-wide filter: thread t < E holds logit t; result in idx_out (shared); all threads call.
 __device__ void block_filter(const double *lg, int E, int k, int32_t *idx_out, uint32_t *s_gm, int *s_nc,
                              ulonglong2 *s_cand) {
@@ -461,6 +490,11 @@ int main() {
     CK(cudaDeviceSynchronize());
     CK(cudaMemcpy(o.data(), d_out, 2 * 8, cudaMemcpyDeviceToHost));
     printf("\"bar_cta512\": %.1f, \"bar_named256\": %.1f, ", o[0] / 256.0, o[1] / 256.0);
+
+    proxy_fence<<<1, 128>>>(d_out);
+    CK(cudaDeviceSynchronize());
+    CK(cudaMemcpy(o.data(), d_out, 2 * 8, cudaMemcpyDeviceToHost));
+    printf("\"sts16_proxy_fence\": %.1f, \"sts16_alone\": %.1f, ", o[0] / 256.0, o[1] / 256.0);
 
     topk_bench<<<1, 512>>>(d_lg, d_out, d_ia, d_ib);
     CK(cudaDeviceSynchronize());
