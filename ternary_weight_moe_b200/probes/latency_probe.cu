@@ -11,6 +11,10 @@
 //   bulk_*       issuing bulk copies (cp.async.bulk global -> shared): n copies from one lane,
 //                or one copy from each of n warps; cycles until the issuing returns / until all
 //                copies have landed
+//   sts16_*      a 16-byte shared store with and without the async-proxy fence after it
+//   mma_*        n tcgen05 kind::i8 MMAs (M = 128, N = 16, K = 32, operands in shared memory)
+//                issued by one thread and committed to an mbarrier: cycles from the first issue
+//                to the mbarrier's completion seen by the issuing thread
 // Every wait is bounded; nothing here waits on another CTA.
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -437,6 +441,66 @@ __global__ void bulk_issue(const uint8_t *src, int n, int bytes, int mode, unsig
     }
 }
 
+// tcgen05 pieces (the forms the grouped kernels use): K-major operands without swizzle, 64
+// bytes of K per row, core matrices of 8 rows x 16 bytes
+__device__ __forceinline__ uint64_t pr_desc(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(128u >> 4) << 16) | ((uint64_t)(512u >> 4) << 32) |
+           (1ull << 46);
+}
+__global__ void mma_commit(unsigned long long *out, int *status) {
+    __shared__ __align__(1024) unsigned char A[128 * 64];
+    __shared__ __align__(1024) unsigned char B[16 * 64];
+    __shared__ __align__(8) uint64_t mb;
+    __shared__ uint32_t s_tmem;
+    for (int i = threadIdx.x; i < 128 * 64 / 16; i += blockDim.x) reinterpret_cast<uint4 *>(A)[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = threadIdx.x; i < 16 * 64 / 16; i += blockDim.x) reinterpret_cast<uint4 *>(B)[i] = make_uint4(1u, 1u, 1u, 1u);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    if (threadIdx.x == 0) {
+        mbar_init(&mb, 1);
+        fence_mbar_init();
+    }
+    if (threadIdx.x < 32) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
+                     "r"(64u)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = s_tmem;
+    const uint32_t idesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(16 >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+    if (threadIdx.x == 0) {
+        const uint64_t a0 = pr_desc(smem_u32(A)), b0 = pr_desc(smem_u32(B));
+        unsigned ph = 0;
+        for (int v = 0; v < 3; v++) {
+            const int n = 1 << v;  // 1, 2, 4 MMAs (4: one gate/up tile of the grouped kernel)
+            for (int r = 0; r < kReps; r++) {
+                const unsigned long long t0 = clock64();
+                for (int q = 0; q < n; q++) {
+                    const uint64_t off = (uint64_t)((q & 1) * 256) >> 4;  // K step 0 or 1
+                    const uint32_t acc = q > 0 ? 1u : 0u;
+                    asm volatile(
+                        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+                        " tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n}\n" ::"r"(tmem),
+                        "l"(a0 + off), "l"(b0 + off), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
+                }
+                asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                                 smem_u32(&mb))
+                             : "memory");
+                mbar_wait(&mb, ph & 1u, 1000000000ll, status);
+                ph++;
+                const unsigned long long t1 = clock64();
+                out[v * kReps + r] = t1 - t0;
+            }
+        }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (threadIdx.x < 32)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(64u) : "memory");
+}
+
 static double median(std::vector<double> v) {
     std::sort(v.begin(), v.end());
     return v.empty() ? 0.0 : v[v.size() / 2];
@@ -495,6 +559,25 @@ int main() {
     CK(cudaDeviceSynchronize());
     CK(cudaMemcpy(o.data(), d_out, 2 * 8, cudaMemcpyDeviceToHost));
     printf("\"sts16_proxy_fence\": %.1f, \"sts16_alone\": %.1f, ", o[0] / 256.0, o[1] / 256.0);
+
+    {
+        int *d_st;
+        CK(cudaMalloc(&d_st, sizeof(int)));
+        CK(cudaMemset(d_st, 0, sizeof(int)));
+        mma_commit<<<1, 128>>>(d_out, d_st);
+        CK(cudaDeviceSynchronize());
+        std::vector<unsigned long long> m(3 * kReps);
+        CK(cudaMemcpy(m.data(), d_out, 3 * kReps * 8, cudaMemcpyDeviceToHost));
+        int mst = 0;
+        CK(cudaMemcpy(&mst, d_st, sizeof(int), cudaMemcpyDeviceToHost));
+        for (int v = 0; v < 3; v++) {
+            std::vector<double> t;
+            for (int r = 1; r < kReps; r++) t.push_back((double)m[v * kReps + r]);
+            printf("\"mma_%d_commit\": %.0f, ", 1 << v, median(t));
+        }
+        printf("\"mma_status\": %d, ", mst);
+        CK(cudaFree(d_st));
+    }
 
     topk_bench<<<1, 512>>>(d_lg, d_out, d_ia, d_ib);
     CK(cudaDeviceSynchronize());
